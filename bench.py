@@ -1,0 +1,388 @@
+"""Benchmark of one absorbed-MLA decode step on the DeepSeek-V2-scale workload.
+
+A step is the whole hot path over one batch: append the new token's latent (RMSNorm + RoPE), absorb
+the queries into the latent (W_UK), attend over the latent cache (fused split-KV decode), project
+(W_UV, W_O). Workload: batch 64, 128 heads, d_c 512, d_r 64, qk_nope 128, v_head 128, d_model
+5120, 4096 cached positions per sequence, bf16 storage, fp32 accumulation. Inputs are seeded and
+synthetic; the per-step traffic (302 MB of cache + 201 MB of weights) is larger than the 126 MB L2,
+so no separate flush is needed between steps.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). Under torchrun every rank runs an independent replica (the path
+shards over sequences with no exchange step), and the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA absorbed decode tokens/s and latent-cache HBM GB/s, % of B200 roofline"
+WORKLOAD = dict(batch=64, n_heads=128, kv_lora_rank=512, rope_dim=64, qk_nope=128, v_head=128,
+                d_model=5120, seqlen=4096, q_lora_rank=1536)
+SEED = 1003
+CONFIG = {
+    "workload": "DeepSeek-V2-scale absorbed MLA decode step: append + absorb + split-KV decode + "
+                "W_UV/W_O projection; B64 H128 d_c512 d_r64 qk_nope128 v_head128 d_model5120 "
+                "T4096 per sequence, bf16 storage, fp32 accumulate",
+    "batch": 64, "n_heads": 128, "kv_lora_rank": 512, "rope_dim": 64, "qk_nope": 128,
+    "v_head": 128, "d_model": 5120, "seq_len": 4096, "n_q": 1,
+    "l2": "no flush: every step streams 302 MB of latent cache + 201 MB of weights (> 126 MB L2)",
+    "parallelism": "replicas (one independent decode per GPU, no collective)",
+}
+DECODE_SOURCES = ("head_latent_attention_08_b200/csrc/tc_decode.cu",
+                  "head_latent_attention_08_b200/csrc/generic.cu")
+
+
+def cache_bytes() -> int:
+    w = WORKLOAD
+    return w["batch"] * w["seqlen"] * (w["kv_lora_rank"] + w["rope_dim"]) * 2
+
+
+def decode_flops() -> int:
+    w = WORKLOAD
+    return w["batch"] * w["n_heads"] * w["seqlen"] * (2 * (w["kv_lora_rank"] + w["rope_dim"]) +
+                                                      2 * w["kv_lora_rank"])
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in DECODE_SOURCES:
+        p = os.path.join(ROOT, rel)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on the current
+    decode sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "decode_c3_traffic.json")
+    if not os.path.exists(p):
+        return None
+    j = json.load(open(p))
+    if j.get("source_hash") != source_hash():
+        return None
+    return j.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        load = [r for r in rows if r["power"] > 300.0] or rows
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": rows[0]["smax"],
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load)}
+
+
+# --------------------------------------------------------------------------------------------
+# CPU oracle legs (the oracle as it stands, timed on the host cores)
+# --------------------------------------------------------------------------------------------
+
+def oracle_problem(n_seqs: int, seed: int = SEED):
+    from head_latent_attention_08_b200 import inputs as I
+    w = WORKLOAD
+    return I.decode_problem(batch=n_seqs, n_heads=w["n_heads"], kv_lora_rank=w["kv_lora_rank"],
+                            rope_dim=w["rope_dim"], qk_nope=w["qk_nope"], v_head=w["v_head"],
+                            d_model=w["d_model"], seqlens=[w["seqlen"]] * n_seqs, dtype="bf16",
+                            seed=seed)
+
+
+def oracle_sample(p):
+    """The full step of the sequences of ``p`` through the oracle; returns (seconds, threads)."""
+    from oracle import mla_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = 1
+    t0 = time.perf_counter()
+    cache = O.append_latent(p.cache, p.row_idx, p.c_new, p.kpe_new, p.positions, norm=True, rope=True,
+                            dtype="bf16")
+    q_abs = O.absorb_query(p.q_nope, p.q_pe, p.w_uk)
+    out_lat, _ = O.decode_absorbed(q_abs, cache, p.cu_seqlens, 1, p.kv_lora_rank, p.kq_scale, True)
+    O.out_project(out_lat, p.w_uv, p.w_o)
+    return time.perf_counter() - t0, threads
+
+
+def cpu_baseline(target_s: float = 12.0):
+    secs, threads = oracle_sample(oracle_problem(1))
+    n = max(1, min(WORKLOAD["batch"], int(target_s / max(secs, 1e-3))))
+    if n > 1:
+        secs, threads = oracle_sample(oracle_problem(n))
+    return {"value": n / secs, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"full step (append, absorb, decode, W_UV/W_O) of {n} of the 64 sequences, "
+                      f"float64 numpy oracle, {secs:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    per_step = 1
+    p = oracle_problem(per_step)
+    for _ in range(args.warmup):
+        oracle_sample(p)
+    secs, threads = 0.0, 1
+    for k in range(args.steps):
+        s, threads = oracle_sample(p)
+        secs += s
+    value = args.steps * per_step / secs
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": CONFIG,
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{per_step} of the 64 sequences per step (full step)"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------------------------
+# the GPU arm
+# --------------------------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from head_latent_attention_08_b200 import build, inputs as I, mla as M
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    M.lib()
+
+    w = WORKLOAD
+    B, H, dc, dr, T = w["batch"], w["n_heads"], w["kv_lora_rank"], w["rope_dim"], w["seqlen"]
+    p = I.decode_problem(batch=B, n_heads=H, kv_lora_rank=dc, rope_dim=dr, qk_nope=w["qk_nope"],
+                         v_head=w["v_head"], d_model=w["d_model"], seqlens=[T] * B, dtype="bf16",
+                         seed=SEED + rank)
+    bf = torch.bfloat16
+    dev = torch.device("cuda", local)
+
+    def d_(x, dt=bf):
+        return torch.from_numpy(np.ascontiguousarray(x)).to(device=dev, dtype=dt)
+
+    cache = d_(p.cache)
+    cu = torch.from_numpy(p.cu_seqlens.astype(np.int32)).to(dev)
+    d = M.dims(H, dc, dr, w["qk_nope"], w["v_head"], w["d_model"])
+    step = M.DecodeStep(d, bf, B, 1, T, cache, cu, d_(p.w_uk), d_(p.w_uv), d_(p.w_o))
+    q_nope, q_pe = d_(p.q_nope), d_(p.q_pe)
+    c_new, kpe_new = d_(p.c_new, torch.float32), d_(p.kpe_new, torch.float32)
+    row_idx = torch.from_numpy(p.row_idx).to(dev)
+    positions = torch.from_numpy(p.positions).to(dev)
+    del p
+    stream = torch.cuda.current_stream()
+
+    # ---- device-resident timing -------------------------------------------------------------
+    for _ in range(args.warmup):
+        step(q_nope, q_pe, c_new, kpe_new, row_idx, positions)
+    torch.cuda.synchronize()
+    if M.mla_check_status() != 0:
+        raise SystemExit("device status word reports a timeout")
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    nq = B
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = M.mla_launch_count()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            M.mla_append_latent(d, cache, row_idx, c_new, kpe_new, positions, step.append_flags)
+            M.mla_absorb_weights(d, M.MLA_ABSORB_QUERY, q_nope, q_pe, step.w_uk, nq, step.q_abs)
+            ev_dec[k][0].record(stream)
+            M.mla_decode_absorbed(d, step.q_abs, cache, cu, B, 1, T, step.flags, step.out_lat, step.lse,
+                                  step.ws_dec)
+            ev_dec[k][1].record(stream)
+            M.mla_out_project(d, step.out_lat, step.w_uv, step.w_o, None, nq, step.y, step.ws_out)
+        stop.record(stream)
+        torch.cuda.synchronize()
+    launches = M.mla_launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(stop)
+    dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    status = M.mla_check_status()
+
+    # ---- end to end through the public API with host buffers --------------------------------
+    h_q_nope = q_nope.cpu().pin_memory()
+    h_q_pe = q_pe.cpu().pin_memory()
+    h_c_new = c_new.cpu().pin_memory()
+    h_kpe = kpe_new.cpu().pin_memory()
+    h_y = torch.empty(step.y.shape, dtype=bf).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q_nope, h_q_pe, h_c_new, h_kpe))
+    d2h = h_y.numel() * h_y.element_size()
+
+    def e2e_step():
+        q_nope.copy_(h_q_nope, non_blocking=True)
+        q_pe.copy_(h_q_pe, non_blocking=True)
+        c_new.copy_(h_c_new, non_blocking=True)
+        kpe_new.copy_(h_kpe, non_blocking=True)
+        y = step(q_nope, q_pe, c_new, kpe_new, row_idx, positions)
+        h_y.copy_(y, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    cpu = cpu_baseline() if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        hbm, tflops, src = peaks()
+        dec_avg_s = statistics.mean(dec_ms) / 1e3
+        achieved = cache_bytes() / dec_avg_s / 1e9
+        tokens = world * nq * args.steps
+        line = {
+            "metric": METRIC, "value": tokens / (elapsed_ms / 1e3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": CONFIG,
+            "roofline": {
+                "kernel": "mla_decode_absorbed (split-KV decode + combine)",
+                "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": recorded_traffic(),
+                "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback",
+                "algorithmic_bytes_per_launch": cache_bytes(),
+                "decode_ms": statistics.mean(dec_ms),
+                "tensor_tflops": decode_flops() / dec_avg_s / 1e12,
+                "tensor_frac_of_measured_bf16": decode_flops() / dec_avg_s / 1e12 / tflops,
+                "roofline_time_ms": 1e3 * max(cache_bytes() / (hbm * 1e9), decode_flops() / (tflops * 1e12)),
+            },
+            "cpu_baseline": cpu,
+            "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": int(launches),
+            "clocks": clk.summary(),
+            "device_status": status,
+        }
+        line["roofline"]["frac_of_roofline_time"] = line["roofline"]["roofline_time_ms"] / line["roofline"]["decode_ms"]
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

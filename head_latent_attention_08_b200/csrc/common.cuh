@@ -1,0 +1,96 @@
+// common.cuh -- small device/host helpers shared by the library's kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/mla.h"
+
+namespace mla {
+
+// ---------------------------------------------------------------------------------------------
+// element conversion
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// ---------------------------------------------------------------------------------------------
+// device status word: set by bounded waits that gave up; read and cleared by mla_check_status
+// ---------------------------------------------------------------------------------------------
+// Kernels with bounded waits receive the word's device address and the spin limit as parameters.
+int* device_status_ptr();        // device address of the status word on the current device
+long long wait_limit();          // spins before a bounded wait gives up
+void set_wait_limit(long long);  // 0 restores the default
+
+__device__ __forceinline__ void report_timeout(int* status) {
+  if (status) atomicExch(status, (int)MLA_ERR_TIMEOUT);
+}
+
+// ---------------------------------------------------------------------------------------------
+// host helpers
+// ---------------------------------------------------------------------------------------------
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t round_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+inline size_t dtype_bytes(int32_t dt) { return dt == MLA_BF16 ? 2 : 4; }
+
+int sm_count();          // multiprocessors of the current device (cached per device)
+int current_device();
+
+void count_launch();      // one more kernel launched by this library (see mla_launch_count)
+long long launch_count();
+
+// after every kernel launch: count it and turn a launch error into MLA_ERR_CUDA
+#define MLA_LAUNCH_CHECK()                                   \
+  do {                                                       \
+    ::mla::count_launch();                                   \
+    if (cudaPeekAtLastError() != cudaSuccess) {              \
+      (void)cudaGetLastError();                              \
+      return MLA_ERR_CUDA;                                   \
+    }                                                        \
+  } while (0)
+
+// ---------------------------------------------------------------------------------------------
+// CUDA-core kernels (any dims; fp32 accumulate). Launchers return an mla status.
+// ---------------------------------------------------------------------------------------------
+struct GemmArgs {
+  // C[b][m][n] = epi( sum_k A[b][m][k] * B[b](n, k) ) (* G[b][m][n] when G != nullptr)
+  const void* A; int64_t sa_b, sa_m, sa_k;
+  const void* B; int64_t sb_b, sb_n, sb_k;
+  void* C;       int64_t sc_b, sc_m, sc_n;
+  const void* G; int64_t sg_b, sg_m, sg_n;
+  int64_t M, N, K, batch;
+  int sigmoid;
+};
+
+// a_dt / b_dt / c_dt / g_dt: MLA_F32 or MLA_BF16 for each operand
+int gemm_generic(const GemmArgs& args, int32_t a_dt, int32_t b_dt, int32_t c_dt, int32_t g_dt,
+                 cudaStream_t stream);
+
+int copy_rows_strided(const void* src, int64_t src_stride, void* dst, int64_t dst_stride,
+                      int64_t rows, int64_t cols, int32_t dt, cudaStream_t stream);
+
+int append_latent_launch(const mla_dims& d, int32_t cache_dtype, void* cache, int64_t cache_rows,
+                         const int64_t* row_idx, const float* c_new, const float* kpe_new,
+                         const int32_t* positions, int64_t n_new, uint32_t flags, float eps,
+                         float theta, cudaStream_t stream);
+
+struct DecodeArgs {
+  const void* q_abs; const void* cache; const int32_t* cu_seqlens;
+  int32_t batch, n_q, H, dc, dr; int64_t max_seqlen, total_rows;
+  float scale; bool causal;
+  float* out_lat; float* lse;
+  void* workspace; size_t workspace_bytes;
+};
+
+size_t decode_generic_workspace(const DecodeArgs& a);
+int decode_generic_launch(const DecodeArgs& a, int32_t dtype, cudaStream_t stream);
+
+}  // namespace mla

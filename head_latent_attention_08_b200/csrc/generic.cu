@@ -1,0 +1,516 @@
+// generic.cu -- CUDA-core kernels of the library: any dims, fp32 or bf16 storage, fp32 arithmetic.
+//
+// These carry the fp32 workloads (where tensor-core tf32 would not meet a 1e-4 tolerance) and
+// every shape the tensor-core kernels do not take:
+//   * gemm_generic: a strided, batched C = A . B^T with fp32 accumulation (query absorption,
+//     weight folding, value/output projection, dense linear);
+//   * append_latent_kernel: the latent-cache append with optional RMSNorm and RoPE;
+//   * decode_generic_kernel + decode_combine_kernel: split-KV absorbed decode with an online
+//     softmax held per head by one warp (shuffle max/sum), and the log-sum-exp merge of splits.
+#include <math.h>
+
+#include <atomic>
+
+#include "common.cuh"
+
+namespace mla {
+
+// device status word (one per device that loads the library)
+static __device__ int g_device_status = 0;
+static long long g_wait_limit_host = 0;
+constexpr long long kDefaultWaitLimit = 1LL << 26;
+
+int* device_status_ptr() {
+  static int* cached[64] = {nullptr};
+  const int d = current_device();
+  if (d < 0 || d >= 64) return nullptr;
+  if (!cached[d]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return nullptr;
+    }
+    cached[d] = static_cast<int*>(p);
+  }
+  return cached[d];
+}
+
+static std::atomic<long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+long long launch_count() { return g_launches.load(std::memory_order_relaxed); }
+
+long long wait_limit() { return g_wait_limit_host > 0 ? g_wait_limit_host : kDefaultWaitLimit; }
+void set_wait_limit(long long v) { g_wait_limit_host = v > 0 ? v : 0; }
+
+int current_device() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return d;
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int d = current_device();
+  if (d < 0 || d >= 64) return 148;
+  if (cached[d] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0) n = 148;
+    cached[d] = n;
+  }
+  return cached[d];
+}
+
+// ---------------------------------------------------------------------------------------------
+// strided batched GEMM, 64 x 64 tile, 256 threads, 4 x 4 outputs per thread
+// ---------------------------------------------------------------------------------------------
+template <typename TA, typename TB, typename TC, typename TG>
+__global__ void __launch_bounds__(256) gemm_generic_kernel(GemmArgs a) {
+  __shared__ float As[16][68];
+  __shared__ float Bs[16][68];
+  const int64_t bz = blockIdx.z;
+  const int64_t m0 = (int64_t)blockIdx.y * 64, n0 = (int64_t)blockIdx.x * 64;
+  const TA* A = static_cast<const TA*>(a.A) + bz * a.sa_b;
+  const TB* B = static_cast<const TB*>(a.B) + bz * a.sb_b;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+  for (int64_t k0 = 0; k0 < a.K; k0 += 16) {
+    for (int i = threadIdx.x; i < 1024; i += 256) {
+      const int r = i >> 4, kk = i & 15;
+      const int64_t k = k0 + kk;
+      const int64_t m = m0 + r, n = n0 + r;
+      As[kk][r] = (m < a.M && k < a.K) ? to_f32(A[m * a.sa_m + k * a.sa_k]) : 0.f;
+      Bs[kk][r] = (n < a.N && k < a.K) ? to_f32(B[n * a.sb_n + k * a.sb_k]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) av[i] = As[kk][ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  TC* C = static_cast<TC*>(a.C) + bz * a.sc_b;
+  const TG* G = a.G ? static_cast<const TG*>(a.G) + bz * a.sg_b : nullptr;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t m = m0 + ty + 16 * i;
+    if (m >= a.M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t n = n0 + tx + 16 * j;
+      if (n >= a.N) continue;
+      float v = acc[i][j];
+      if (a.sigmoid) v = 1.f / (1.f + expf(-v));
+      if (G) v *= to_f32(G[m * a.sg_m + n * a.sg_n]);
+      C[m * a.sc_m + n * a.sc_n] = from_f32<TC>(v);
+    }
+  }
+}
+
+template <typename TA, typename TB, typename TC, typename TG>
+static int gemm_launch_t(const GemmArgs& a, cudaStream_t s) {
+  if (a.M <= 0 || a.N <= 0 || a.batch <= 0) return MLA_OK;
+  dim3 grid((unsigned)ceil_div(a.N, 64), (unsigned)ceil_div(a.M, 64), (unsigned)a.batch);
+  if (grid.y > 65535u || grid.z > 65535u) return MLA_ERR_UNSUPPORTED;
+  gemm_generic_kernel<TA, TB, TC, TG><<<grid, 256, 0, s>>>(a);
+  MLA_LAUNCH_CHECK();
+  return MLA_OK;
+}
+
+template <typename TA, typename TB, typename TC>
+static int gemm_launch_g(const GemmArgs& a, int32_t g_dt, cudaStream_t s) {
+  if (g_dt == MLA_BF16) return gemm_launch_t<TA, TB, TC, __nv_bfloat16>(a, s);
+  return gemm_launch_t<TA, TB, TC, float>(a, s);
+}
+
+template <typename TA, typename TB>
+static int gemm_launch_c(const GemmArgs& a, int32_t c_dt, int32_t g_dt, cudaStream_t s) {
+  if (c_dt == MLA_BF16) return gemm_launch_g<TA, TB, __nv_bfloat16>(a, g_dt, s);
+  return gemm_launch_g<TA, TB, float>(a, g_dt, s);
+}
+
+int gemm_generic(const GemmArgs& a, int32_t a_dt, int32_t b_dt, int32_t c_dt, int32_t g_dt,
+                 cudaStream_t s) {
+  if (a_dt == MLA_BF16 && b_dt == MLA_BF16) return gemm_launch_c<__nv_bfloat16, __nv_bfloat16>(a, c_dt, g_dt, s);
+  if (a_dt == MLA_F32 && b_dt == MLA_BF16) return gemm_launch_c<float, __nv_bfloat16>(a, c_dt, g_dt, s);
+  if (a_dt == MLA_BF16 && b_dt == MLA_F32) return gemm_launch_c<__nv_bfloat16, float>(a, c_dt, g_dt, s);
+  return gemm_launch_c<float, float>(a, c_dt, g_dt, s);
+}
+
+// ---------------------------------------------------------------------------------------------
+// strided row copy (e.g. q_pe into the tail of each absorbed query row)
+// ---------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void copy_rows_kernel(const T* __restrict__ src, int64_t ss, T* __restrict__ dst, int64_t ds,
+                                 int64_t rows, int64_t cols) {
+  const int64_t total = rows * cols;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / cols, c = e - r * cols;
+    dst[r * ds + c] = src[r * ss + c];
+  }
+}
+
+int copy_rows_strided(const void* src, int64_t ss, void* dst, int64_t ds, int64_t rows, int64_t cols,
+                      int32_t dt, cudaStream_t s) {
+  if (rows <= 0 || cols <= 0) return MLA_OK;
+  const int64_t total = rows * cols;
+  const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(total, 256), 4 * 148);
+  if (dt == MLA_BF16)
+    copy_rows_kernel<<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(src), ss,
+                                            static_cast<__nv_bfloat16*>(dst), ds, rows, cols);
+  else
+    copy_rows_kernel<<<blocks, 256, 0, s>>>(static_cast<const float*>(src), ss,
+                                            static_cast<float*>(dst), ds, rows, cols);
+  MLA_LAUNCH_CHECK();
+  return MLA_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// latent append: one CTA per new row; the row is built in fp32 shared memory, then stored in the
+// cache dtype with 128-bit stores when the row pitch allows it
+// ---------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(128) append_latent_kernel(
+    T* __restrict__ cache, const int64_t* __restrict__ row_idx, const float* __restrict__ c_new,
+    const float* __restrict__ kpe_new, const int32_t* __restrict__ positions, int dc, int dr,
+    uint32_t flags, float eps, float theta, int vec8, int64_t cache_rows, int* status) {
+  extern __shared__ float row[];
+  __shared__ float red[4];
+  const int k = blockIdx.x;
+  const int64_t target = row_idx[k];
+  if (target < 0 || target >= cache_rows) {   // a row outside the cache is skipped and reported
+    if (threadIdx.x == 0) atomicExch(status, (int)MLA_ERR_SHAPE);
+    return;
+  }
+  const int W = dc + dr;
+  const float* c = c_new + (int64_t)k * dc;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < dc; i += blockDim.x) {
+    const float x = c[i];
+    row[i] = x;
+    ss = fmaf(x, x, ss);
+  }
+  if (flags & MLA_APPEND_NORM) {
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    const float tot = red[0] + red[1] + red[2] + red[3];
+    const float inv = 1.f / sqrtf(tot / (float)dc + eps);
+    for (int i = threadIdx.x; i < dc; i += blockDim.x) row[i] *= inv;
+  }
+  if (dr > 0) {
+    const float* kp = kpe_new + (int64_t)k * dr;
+    if (flags & MLA_APPEND_ROPE) {
+      const double pos = (double)positions[k];
+      for (int i = threadIdx.x; i < dr / 2; i += blockDim.x) {
+        // angle in double so that positions of tens of thousands keep full fp32 accuracy
+        const double ang = pos * pow((double)theta, -2.0 * (double)i / (double)dr);
+        double sn, cs;
+        sincos(ang, &sn, &cs);
+        const double x0 = kp[2 * i], x1 = kp[2 * i + 1];
+        row[dc + 2 * i] = (float)(x0 * cs - x1 * sn);
+        row[dc + 2 * i + 1] = (float)(x0 * sn + x1 * cs);
+      }
+    } else {
+      for (int i = threadIdx.x; i < dr; i += blockDim.x) row[dc + i] = kp[i];
+    }
+  }
+  __syncthreads();
+  T* dst = cache + target * (int64_t)W;
+  if (vec8) {
+    // 8 elements per thread per store: 16 B for bf16 (two 16 B stores for fp32)
+    for (int i = threadIdx.x * 8; i < W; i += blockDim.x * 8) {
+      if constexpr (sizeof(T) == 2) {
+        uint4 v;
+        __nv_bfloat162 p0 = __floats2bfloat162_rn(row[i], row[i + 1]);
+        __nv_bfloat162 p1 = __floats2bfloat162_rn(row[i + 2], row[i + 3]);
+        __nv_bfloat162 p2 = __floats2bfloat162_rn(row[i + 4], row[i + 5]);
+        __nv_bfloat162 p3 = __floats2bfloat162_rn(row[i + 6], row[i + 7]);
+        v.x = *reinterpret_cast<uint32_t*>(&p0);
+        v.y = *reinterpret_cast<uint32_t*>(&p1);
+        v.z = *reinterpret_cast<uint32_t*>(&p2);
+        v.w = *reinterpret_cast<uint32_t*>(&p3);
+        *reinterpret_cast<uint4*>(dst + i) = v;
+      } else {
+        *reinterpret_cast<float4*>(dst + i) = make_float4(row[i], row[i + 1], row[i + 2], row[i + 3]);
+        *reinterpret_cast<float4*>(dst + i + 4) = make_float4(row[i + 4], row[i + 5], row[i + 6], row[i + 7]);
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < W; i += blockDim.x) dst[i] = from_f32<T>(row[i]);
+  }
+}
+
+int append_latent_launch(const mla_dims& d, int32_t cache_dtype, void* cache, int64_t cache_rows,
+                         const int64_t* row_idx, const float* c_new, const float* kpe_new,
+                         const int32_t* positions, int64_t n_new, uint32_t flags, float eps,
+                         float theta, cudaStream_t s) {
+  int* status = device_status_ptr();
+  if (!status) return MLA_ERR_CUDA;
+  if (n_new == 0) return MLA_OK;
+  if (n_new > 0x7fffffff) return MLA_ERR_SHAPE;
+  const int W = d.kv_lora_rank + d.rope_dim;
+  const size_t es = dtype_bytes(cache_dtype);
+  const int vec8 = (W % 8 == 0) && aligned16(cache) && ((size_t)W * es) % 16 == 0;
+  const size_t smem = (size_t)W * sizeof(float);
+  if (smem > 48 * 1024) return MLA_ERR_UNSUPPORTED;
+  if (cache_dtype == MLA_BF16)
+    append_latent_kernel<__nv_bfloat16><<<(unsigned)n_new, 128, smem, s>>>(
+        static_cast<__nv_bfloat16*>(cache), row_idx, c_new, kpe_new, positions, d.kv_lora_rank,
+        d.rope_dim, flags, eps, theta, vec8, cache_rows, status);
+  else
+    append_latent_kernel<float><<<(unsigned)n_new, 128, smem, s>>>(
+        static_cast<float*>(cache), row_idx, c_new, kpe_new, positions, d.kv_lora_rank, d.rope_dim,
+        flags, eps, theta, vec8, cache_rows, status);
+  MLA_LAUNCH_CHECK();
+  return MLA_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// split-KV absorbed decode on CUDA cores
+//   grid: x = split of the positions, y = group of HG heads, z = query row (b * n_q + j)
+//   per tile of DG_TP positions: stage the rows in shared memory (fp32), scores for every
+//   (head, position), per-head online softmax by one warp (shuffle max / sum), O update in
+//   registers (HG * d_c accumulators spread over the block)
+// ---------------------------------------------------------------------------------------------
+constexpr int DG_THREADS = 256;
+constexpr int DG_TP = 32;
+constexpr int DG_MAXE = 32;  // accumulators per thread: HG * d_c <= DG_THREADS * DG_MAXE
+
+struct DecodeGenericParams {
+  const void* q_abs; const void* cache; const int32_t* cu;
+  int n_q, H, dc, W, HG, chunk, n_splits;
+  float scale; int causal;
+  float* out_lat; float* lse;            // used when n_splits == 1
+  float* o_part; float* m_part; float* l_part;   // [split][row][H](*dc)
+  int64_t rows;
+  int64_t total_rows;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(DG_THREADS) decode_generic_kernel(DecodeGenericParams p) {
+  extern __shared__ float sm[];
+  const int W = p.W, HG = p.HG;
+  float* qs = sm;                          // [HG][W]
+  float* Ks = qs + HG * W;                 // [DG_TP][W + 1]
+  float* Ps = Ks + DG_TP * (W + 1);        // [HG][DG_TP]
+  float* ms = Ps + HG * DG_TP;             // [HG]
+  float* ls = ms + HG;                     // [HG]
+  float* cs = ls + HG;                     // [HG]
+
+  const int split = blockIdx.x;
+  const int h0 = blockIdx.y * HG;
+  const int64_t row = blockIdx.z;
+  const int b = (int)(row / p.n_q), j = (int)(row % p.n_q);
+  // sequence bounds, clamped to the cache so that a malformed cu_seqlens cannot read outside it
+  const int64_t c0 = p.cu[b], c1 = p.cu[b + 1];
+  const int64_t start = c0 < 0 ? 0 : (c0 > p.total_rows ? p.total_rows : c0);
+  const int64_t stop = c1 < start ? start : (c1 > p.total_rows ? p.total_rows : c1);
+  const int Tb = (int)(stop - start);
+  int cnt = p.causal ? (Tb - p.n_q + j + 1) : Tb;
+  cnt = max(0, min(cnt, Tb));
+  const int lo = split * p.chunk;
+  const int hi = min(lo + p.chunk, cnt);
+  const int hg = min(HG, p.H - h0);
+
+  const T* q = static_cast<const T*>(p.q_abs) + (row * p.H + h0) * (int64_t)W;
+  for (int e = threadIdx.x; e < hg * W; e += DG_THREADS) qs[e] = to_f32(q[e]);
+  for (int hh = threadIdx.x; hh < HG; hh += DG_THREADS) { ms[hh] = -INFINITY; ls[hh] = 0.f; }
+  float o[DG_MAXE];
+#pragma unroll
+  for (int i = 0; i < DG_MAXE; ++i) o[i] = 0.f;
+  const int n_el = hg * p.dc;
+  __syncthreads();
+
+  const T* cache = static_cast<const T*>(p.cache);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int t0 = lo; t0 < hi; t0 += DG_TP) {
+    const int nt = min(DG_TP, hi - t0);
+    for (int e = threadIdx.x; e < nt * W; e += DG_THREADS) {
+      const int tt = e / W, k = e - tt * W;
+      Ks[tt * (W + 1) + k] = to_f32(cache[(start + t0 + tt) * (int64_t)W + k]);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < hg * DG_TP; e += DG_THREADS) {
+      const int hh = e / DG_TP, tt = e - hh * DG_TP;
+      float s = -INFINITY;
+      if (tt < nt) {
+        const float* qa = qs + hh * W;
+        const float* ka = Ks + tt * (W + 1);
+        float acc = 0.f;
+        for (int k = 0; k < W; ++k) acc = fmaf(qa[k], ka[k], acc);
+        s = acc * p.scale;
+      }
+      Ps[e] = s;
+    }
+    __syncthreads();
+    for (int hh = warp; hh < hg; hh += DG_THREADS / 32) {
+      const float s = Ps[hh * DG_TP + lane];
+      float mt = s;
+      for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+      const float m_old = ms[hh];
+      const float m_new = fmaxf(m_old, mt);
+      const float pr = (s == -INFINITY) ? 0.f : expf(s - m_new);
+      float sum = pr;
+      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      Ps[hh * DG_TP + lane] = pr;
+      __syncwarp();
+      if (lane == 0) {
+        const float c = (m_old == -INFINITY) ? 0.f : expf(m_old - m_new);
+        ls[hh] = ls[hh] * c + sum;
+        ms[hh] = m_new;
+        cs[hh] = c;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < DG_MAXE; ++i) {
+      const int e = threadIdx.x + i * DG_THREADS;
+      if (e < n_el) {
+        const int hh = e / p.dc, d = e - hh * p.dc;
+        float acc = o[i] * cs[hh];
+        const float* pp = Ps + hh * DG_TP;
+        for (int tt = 0; tt < nt; ++tt) acc = fmaf(pp[tt], Ks[tt * (W + 1) + d], acc);
+        o[i] = acc;
+      }
+    }
+    __syncthreads();
+  }
+
+  if (p.n_splits == 1) {
+#pragma unroll
+    for (int i = 0; i < DG_MAXE; ++i) {
+      const int e = threadIdx.x + i * DG_THREADS;
+      if (e < n_el) {
+        const int hh = e / p.dc, d = e - hh * p.dc;
+        const float l = ls[hh];
+        p.out_lat[(row * p.H + h0 + hh) * (int64_t)p.dc + d] = l > 0.f ? o[i] / l : 0.f;
+      }
+    }
+    if (p.lse)
+      for (int hh = threadIdx.x; hh < hg; hh += DG_THREADS) {
+        const float l = ls[hh];
+        p.lse[row * p.H + h0 + hh] = l > 0.f ? ms[hh] + logf(l) : -INFINITY;
+      }
+  } else {
+    const int64_t base = ((int64_t)split * p.rows + row) * p.H + h0;
+#pragma unroll
+    for (int i = 0; i < DG_MAXE; ++i) {
+      const int e = threadIdx.x + i * DG_THREADS;
+      if (e < n_el) {
+        const int hh = e / p.dc, d = e - hh * p.dc;
+        p.o_part[(base + hh) * p.dc + d] = o[i];
+      }
+    }
+    for (int hh = threadIdx.x; hh < hg; hh += DG_THREADS) {
+      p.m_part[base + hh] = ms[hh];
+      p.l_part[base + hh] = ls[hh];
+    }
+  }
+}
+
+// merge of split partials: one CTA per (row, head); out = sum_s w_s O_s / sum_s w_s l_s with
+// w_s = exp(m_s - max_s m_s)
+__global__ void decode_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ m_part,
+                                      const float* __restrict__ l_part, int n_splits, int64_t rh,
+                                      int dc, float* __restrict__ out_lat, float* __restrict__ lse) {
+  const int64_t x = blockIdx.x;  // row * H + h
+  float M = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, m_part[s * rh + x]);
+  float L = 0.f;
+  for (int s = 0; s < n_splits; ++s) {
+    const float m = m_part[s * rh + x];
+    if (m != -INFINITY) L += expf(m - M) * l_part[s * rh + x];
+  }
+  for (int d = threadIdx.x; d < dc; d += blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < n_splits; ++s) {
+      const float m = m_part[s * rh + x];
+      if (m != -INFINITY) acc += expf(m - M) * o_part[(s * rh + x) * dc + d];
+    }
+    out_lat[x * dc + d] = L > 0.f ? acc / L : 0.f;
+  }
+  if (lse && threadIdx.x == 0) lse[x] = L > 0.f ? M + logf(L) : -INFINITY;
+}
+
+struct GenericPlan { int HG, chunk, n_splits; size_t smem, ws; };
+
+static GenericPlan plan_generic(const DecodeArgs& a) {
+  GenericPlan g;
+  const int W = a.dc + a.dr;
+  g.HG = std::max(1, std::min<int>(a.H, (DG_THREADS * DG_MAXE) / std::max(1, a.dc)));
+  const int64_t rows = (int64_t)a.batch * a.n_q;
+  const int64_t base = rows * ceil_div(a.H, g.HG);
+  const int64_t want = 2LL * sm_count();
+  int64_t splits = std::max<int64_t>(1, ceil_div(want, std::max<int64_t>(1, base)));
+  const int64_t max_tiles = std::max<int64_t>(1, ceil_div(a.max_seqlen, DG_TP));
+  splits = std::min(splits, max_tiles);
+  int64_t chunk = ceil_div(std::max<int64_t>(a.max_seqlen, 1), splits);
+  chunk = ceil_div(chunk, DG_TP) * DG_TP;
+  splits = std::max<int64_t>(1, ceil_div(std::max<int64_t>(a.max_seqlen, 1), chunk));
+  g.chunk = (int)chunk;
+  g.n_splits = (int)splits;
+  g.smem = sizeof(float) * ((size_t)g.HG * W + (size_t)DG_TP * (W + 1) + (size_t)g.HG * DG_TP + 3 * (size_t)g.HG);
+  g.ws = 0;
+  if (g.n_splits > 1) {
+    const size_t rh = (size_t)rows * a.H;
+    g.ws = round_up(sizeof(float) * (size_t)g.n_splits * rh * a.dc, 256) +
+           2 * round_up(sizeof(float) * (size_t)g.n_splits * rh, 256);
+  }
+  return g;
+}
+
+size_t decode_generic_workspace(const DecodeArgs& a) { return plan_generic(a).ws; }
+
+int decode_generic_launch(const DecodeArgs& a, int32_t dtype, cudaStream_t s) {
+  const GenericPlan g = plan_generic(a);
+  const int64_t rows = (int64_t)a.batch * a.n_q;
+  if (rows == 0) return MLA_OK;
+  if (g.smem > 200 * 1024) return MLA_ERR_UNSUPPORTED;
+  if (a.workspace_bytes < g.ws || (g.ws && !a.workspace)) return MLA_ERR_WORKSPACE;
+  DecodeGenericParams p;
+  p.q_abs = a.q_abs; p.cache = a.cache; p.cu = a.cu_seqlens;
+  p.n_q = a.n_q; p.H = a.H; p.dc = a.dc; p.W = a.dc + a.dr; p.HG = g.HG;
+  p.chunk = g.chunk; p.n_splits = g.n_splits; p.scale = a.scale; p.causal = a.causal ? 1 : 0;
+  p.out_lat = a.out_lat; p.lse = a.lse; p.rows = rows; p.total_rows = a.total_rows;
+  const size_t rh = (size_t)rows * a.H;
+  char* ws = static_cast<char*>(a.workspace);
+  p.o_part = reinterpret_cast<float*>(ws);
+  p.m_part = reinterpret_cast<float*>(ws + round_up(sizeof(float) * (size_t)g.n_splits * rh * a.dc, 256));
+  p.l_part = p.m_part + round_up(sizeof(float) * (size_t)g.n_splits * rh, 256) / sizeof(float);
+  dim3 grid((unsigned)g.n_splits, (unsigned)ceil_div(a.H, g.HG), (unsigned)rows);
+  if (grid.y > 65535u || grid.z > 65535u) return MLA_ERR_UNSUPPORTED;
+  if (dtype == MLA_BF16) {
+    if (cudaFuncSetAttribute(decode_generic_kernel<__nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    decode_generic_kernel<__nv_bfloat16><<<grid, DG_THREADS, g.smem, s>>>(p);
+  } else {
+    if (cudaFuncSetAttribute(decode_generic_kernel<float>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    decode_generic_kernel<float><<<grid, DG_THREADS, g.smem, s>>>(p);
+  }
+  MLA_LAUNCH_CHECK();
+  if (g.n_splits > 1) {
+    decode_combine_kernel<<<(unsigned)rh, 128, 0, s>>>(p.o_part, p.m_part, p.l_part, g.n_splits,
+                                                       (int64_t)rh, a.dc, a.out_lat, a.lse);
+    MLA_LAUNCH_CHECK();
+  }
+  return MLA_OK;
+}
+
+}  // namespace mla

@@ -1,0 +1,30 @@
+// tc.cuh -- entry points of the tensor-core (tcgen05 / TMA / TMEM) kernels for sm_100a.
+#pragma once
+
+#include "common.cuh"
+
+namespace mla {
+
+// query absorption q_abs = W_UK^T q_nope per head (bf16 in, fp32 accumulate, bf16 out)
+bool tc_absorb_supported(const mla_dims& d, int64_t n_rows);
+int tc_absorb_query(const mla_dims& d, const void* q_nope, const void* q_pe, const void* w_uk,
+                    int64_t n_rows, void* q_abs, cudaStream_t s);
+
+// fused split-KV absorbed decode
+bool tc_decode_supported(const DecodeArgs& a);
+size_t tc_decode_workspace(const DecodeArgs& a);
+int tc_decode_launch(const DecodeArgs& a, cudaStream_t s);
+
+// value + output projection
+bool tc_out_project_supported(const mla_dims& d, int64_t n_rows);
+size_t tc_out_project_extra_workspace(const mla_dims& d, int64_t n_rows);
+int tc_out_project(const mla_dims& d, const float* out_lat, const void* w_uv, const void* w_o,
+                   const void* gate, int64_t n_rows, void* y, void* workspace, size_t ws_bytes,
+                   cudaStream_t s);
+
+// dense linear Y = X W^T
+bool tc_linear_supported(int64_t m, int64_t n, int64_t k);
+int tc_linear(const void* x, const void* w, int64_t m, int64_t n, int64_t k, int sigmoid, void* y,
+              cudaStream_t s);
+
+}  // namespace mla

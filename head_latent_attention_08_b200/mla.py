@@ -1,0 +1,282 @@
+"""Thin Python binding of libmla_b200.so (ctypes). Argument marshalling only: every step runs in
+the library's CUDA kernels. Torch tensors supply device memory and the current CUDA stream.
+
+The functions carry the C names (``mla_append_latent``, ``mla_absorb_weights``,
+``mla_decode_absorbed``, ``mla_out_project``, ``mla_linear`` ...). A non-zero status raises
+:class:`MLAError`. ``decode_step`` and ``gated_mla`` chain those calls for the two workloads.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmla_b200.so")
+
+MLA_OK = 0
+MLA_F32, MLA_BF16 = 0, 1
+MLA_ABSORB_QUERY, MLA_FOLD_QK, MLA_FOLD_VO = 0, 1, 2
+MLA_APPEND_NORM, MLA_APPEND_ROPE = 1, 2
+MLA_DECODE_CAUSAL = 1
+MLA_LINEAR_SIGMOID, MLA_LINEAR_W_KN = 1, 2
+MLA_ERR_TIMEOUT = 7
+
+EXPORTED = (
+    "mla_status_string", "mla_abi_version", "mla_append_latent", "mla_absorb_weights",
+    "mla_decode_workspace_size", "mla_decode_absorbed", "mla_out_project_workspace_size",
+    "mla_out_project", "mla_linear", "mla_check_status", "mla_set_wait_limit", "mla_launch_count",
+)
+
+
+class MLAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class mla_dims(ctypes.Structure):
+    _fields_ = [("n_heads", ctypes.c_int32), ("kv_lora_rank", ctypes.c_int32),
+                ("rope_dim", ctypes.c_int32), ("qk_nope", ctypes.c_int32),
+                ("v_head", ctypes.c_int32), ("d_model", ctypes.c_int32),
+                ("kq_scale", ctypes.c_float)]
+
+
+def dims(n_heads, kv_lora_rank, rope_dim=0, qk_nope=0, v_head=0, d_model=0, kq_scale=0.0):
+    return mla_dims(n_heads, kv_lora_rank, rope_dim, qk_nope, v_head, d_model, kq_scale)
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+_P, _I32, _I64, _U32, _F, _SZ = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32,
+                                 ctypes.c_float, ctypes.c_size_t)
+_DIMS = ctypes.POINTER(mla_dims)
+_SIGS = {
+    "mla_status_string": (ctypes.c_char_p, [_I32]),
+    "mla_abi_version": (_I32, []),
+    "mla_append_latent": (_I32, [_DIMS, _I32, _P, _I64, _P, _P, _P, _P, _I64, _U32, _F, _F, _P]),
+    "mla_absorb_weights": (_I32, [_DIMS, _I32, _I32, _P, _P, _P, _I64, _P, _P]),
+    "mla_decode_workspace_size": (_I32, [_DIMS, _I32, _I32, _I32, _I64, _I64, _U32, ctypes.POINTER(_SZ)]),
+    "mla_decode_absorbed": (_I32, [_DIMS, _I32, _P, _P, _P, _I32, _I32, _I64, _I64, _U32, _P, _P, _P,
+                                   _SZ, _P]),
+    "mla_out_project_workspace_size": (_I32, [_DIMS, _I32, _I64, ctypes.POINTER(_SZ)]),
+    "mla_out_project": (_I32, [_DIMS, _I32, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
+    "mla_linear": (_I32, [_I32, _P, _P, _I64, _I64, _I64, _U32, _P, _P]),
+    "mla_check_status": (_I32, [_P, ctypes.POINTER(_I32)]),
+    "mla_set_wait_limit": (_I32, [_I64]),
+    "mla_launch_count": (_I64, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Open the library (once). Raises if it is missing: there is no fallback path."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m head_latent_attention_08_b200.build` (nvcc, sm_100a)")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return lib().mla_status_string(int(status)).decode()
+    except Exception:  # pragma: no cover - only when the library itself cannot load
+        return f"status {status}"
+
+
+def _check(status: int, where: str):
+    if status != MLA_OK:
+        raise MLAError(status, where)
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return MLA_F32
+    if t == torch.bfloat16:
+        return MLA_BF16
+    raise TypeError(f"unsupported dtype {t}")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to the library must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+# --------------------------------------------------------------------------------------------
+# the C entry points
+# --------------------------------------------------------------------------------------------
+
+def mla_append_latent(d: mla_dims, cache: torch.Tensor, row_idx: torch.Tensor, c_new: torch.Tensor,
+                      kpe_new: Optional[torch.Tensor], positions: Optional[torch.Tensor], flags: int,
+                      eps: float = 1e-6, rope_theta: float = 10000.0, stream=None) -> None:
+    assert row_idx.dtype == torch.int64 and c_new.dtype == torch.float32
+    assert kpe_new is None or kpe_new.dtype == torch.float32
+    assert positions is None or positions.dtype == torch.int32
+    n_new = row_idx.numel()
+    _check(lib().mla_append_latent(ctypes.byref(d), _dtype_code(cache.dtype), _ptr(cache), cache.shape[0],
+                                   _ptr(row_idx), _ptr(c_new), _ptr(kpe_new), _ptr(positions), n_new,
+                                   flags, eps, rope_theta, _stream(stream)), "mla_append_latent")
+
+
+def mla_absorb_weights(d: mla_dims, mode: int, x: torch.Tensor, x_pe: Optional[torch.Tensor],
+                       w: torch.Tensor, n_rows: int, out: torch.Tensor, stream=None) -> None:
+    _check(lib().mla_absorb_weights(ctypes.byref(d), _dtype_code(x.dtype), mode, _ptr(x), _ptr(x_pe),
+                                    _ptr(w), n_rows, _ptr(out), _stream(stream)), "mla_absorb_weights")
+
+
+def mla_decode_workspace_size(d: mla_dims, dtype: torch.dtype, batch: int, n_q: int, max_seqlen: int,
+                              total_rows: int, flags: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().mla_decode_workspace_size(ctypes.byref(d), _dtype_code(dtype), batch, n_q, max_seqlen,
+                                           total_rows, flags, ctypes.byref(n)),
+           "mla_decode_workspace_size")
+    return int(n.value)
+
+
+def mla_decode_absorbed(d: mla_dims, q_abs: torch.Tensor, cache: torch.Tensor, cu_seqlens: torch.Tensor,
+                        batch: int, n_q: int, max_seqlen: int, flags: int, out_lat: torch.Tensor,
+                        lse: Optional[torch.Tensor], workspace: Optional[torch.Tensor],
+                        stream=None) -> None:
+    assert cu_seqlens.dtype == torch.int32 and out_lat.dtype == torch.float32
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().mla_decode_absorbed(ctypes.byref(d), _dtype_code(q_abs.dtype), _ptr(q_abs), _ptr(cache),
+                                     _ptr(cu_seqlens), batch, n_q, max_seqlen, cache.shape[0], flags,
+                                     _ptr(out_lat), _ptr(lse), _ptr(workspace), ws_bytes,
+                                     _stream(stream)), "mla_decode_absorbed")
+
+
+def mla_out_project_workspace_size(d: mla_dims, dtype: torch.dtype, n_rows: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().mla_out_project_workspace_size(ctypes.byref(d), _dtype_code(dtype), n_rows,
+                                                ctypes.byref(n)), "mla_out_project_workspace_size")
+    return int(n.value)
+
+
+def mla_out_project(d: mla_dims, out_lat: torch.Tensor, w_uv: torch.Tensor, w_o: torch.Tensor,
+                    gate: Optional[torch.Tensor], n_rows: int, y: torch.Tensor,
+                    workspace: torch.Tensor, stream=None) -> None:
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().mla_out_project(ctypes.byref(d), _dtype_code(w_uv.dtype), _ptr(out_lat), _ptr(w_uv),
+                                 _ptr(w_o), _ptr(gate), n_rows, _ptr(y), _ptr(workspace), ws_bytes,
+                                 _stream(stream)), "mla_out_project")
+
+
+def mla_linear(x: torch.Tensor, w: torch.Tensor, m: int, n: int, k: int, flags: int, y: torch.Tensor,
+               stream=None) -> None:
+    _check(lib().mla_linear(_dtype_code(x.dtype), _ptr(x), _ptr(w), m, n, k, flags, _ptr(y),
+                            _stream(stream)), "mla_linear")
+
+
+def mla_check_status(stream=None) -> int:
+    v = ctypes.c_int32(0)
+    _check(lib().mla_check_status(_stream(stream), ctypes.byref(v)), "mla_check_status")
+    return int(v.value)
+
+
+def mla_launch_count() -> int:
+    return int(lib().mla_launch_count())
+
+
+def mla_set_wait_limit(spins: int) -> None:
+    _check(lib().mla_set_wait_limit(int(spins)), "mla_set_wait_limit")
+
+
+# --------------------------------------------------------------------------------------------
+# chained calls
+# --------------------------------------------------------------------------------------------
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A 256-byte aligned scratch buffer of at least ``nbytes`` bytes (caller-owned)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+class DecodeStep:
+    """One absorbed-decode step over resident weights and cache: append the new tokens' latents,
+    absorb the queries, attend over the latent cache, project. Buffers are allocated once here;
+    ``__call__`` only launches the library's kernels."""
+
+    def __init__(self, d: mla_dims, dtype: torch.dtype, batch: int, n_q: int, max_seqlen: int,
+                 cache: torch.Tensor, cu_seqlens: torch.Tensor, w_uk: torch.Tensor,
+                 w_uv: torch.Tensor, w_o: torch.Tensor, causal: bool = True,
+                 append_flags: int = MLA_APPEND_NORM | MLA_APPEND_ROPE):
+        dev = cache.device
+        self.d, self.dtype, self.batch, self.n_q, self.max_seqlen = d, dtype, batch, n_q, max_seqlen
+        self.cache, self.cu, self.w_uk, self.w_uv, self.w_o = cache, cu_seqlens, w_uk, w_uv, w_o
+        self.flags = MLA_DECODE_CAUSAL if causal else 0
+        self.append_flags = append_flags
+        nq = batch * n_q
+        H, W = d.n_heads, d.kv_lora_rank + d.rope_dim
+        self.q_abs = torch.empty(nq, H, W, dtype=dtype, device=dev)
+        self.out_lat = torch.empty(nq, H, d.kv_lora_rank, dtype=torch.float32, device=dev)
+        self.lse = torch.empty(nq, H, dtype=torch.float32, device=dev)
+        self.y = torch.empty(nq, d.d_model, dtype=dtype, device=dev)
+        self.ws_dec = workspace(mla_decode_workspace_size(d, dtype, batch, n_q, max_seqlen,
+                                                          cache.shape[0], self.flags), dev)
+        self.ws_out = workspace(mla_out_project_workspace_size(d, dtype, nq), dev)
+
+    def __call__(self, q_nope, q_pe, c_new, kpe_new, row_idx, positions, stream=None):
+        d = self.d
+        nq = self.batch * self.n_q
+        mla_append_latent(d, self.cache, row_idx, c_new, kpe_new, positions, self.append_flags,
+                          stream=stream)
+        mla_absorb_weights(d, MLA_ABSORB_QUERY, q_nope, q_pe if d.rope_dim else None, self.w_uk, nq,
+                           self.q_abs, stream=stream)
+        mla_decode_absorbed(d, self.q_abs, self.cache, self.cu, self.batch, self.n_q, self.max_seqlen,
+                            self.flags, self.out_lat, self.lse, self.ws_dec, stream=stream)
+        mla_out_project(d, self.out_lat, self.w_uv, self.w_o, None, nq, self.y, self.ws_out,
+                        stream=stream)
+        return self.y
+
+
+def gated_mla(x: torch.Tensor, wq: torch.Tensor, wc: torch.Tensor, wk: torch.Tensor, wv: torch.Tensor,
+              wg: torch.Tensor, wo: torch.Tensor, num_heads: int, causal: bool = True, stream=None):
+    """Gated MLA prefill through the absorbed route: Q, C and sigmoid(X Wg^T) by mla_linear, the
+    query absorbed into the latent per head (W_UK[h] = rows h*D_h.. of Wk), attention over the latent
+    C, then W_UV[h] = rows of Wv, the gate and Wo by mla_out_project. Returns
+    {"output": [B, S, D], "latent_cache": [B, S, L]}; the inputs are not modified."""
+    B, S, D = x.shape
+    L = wc.shape[0]
+    H = num_heads
+    if D % H:
+        raise ValueError("model width must be divisible by the head count")
+    Dh = D // H
+    dev, dt = x.device, x.dtype
+    x2 = x.reshape(B * S, D)
+    q = torch.empty(B * S, D, dtype=dt, device=dev)
+    c = torch.empty(B * S, L, dtype=dt, device=dev)
+    g = torch.empty(B * S, D, dtype=dt, device=dev)
+    mla_linear(x2, wq, B * S, D, D, 0, q, stream)
+    mla_linear(x2, wc, B * S, L, D, 0, c, stream)
+    mla_linear(x2, wg, B * S, D, D, MLA_LINEAR_SIGMOID, g, stream)
+    d = dims(H, L, 0, Dh, Dh, D, 1.0 / math.sqrt(Dh))
+    q_abs = torch.empty(B * S, H, L, dtype=dt, device=dev)
+    mla_absorb_weights(d, MLA_ABSORB_QUERY, q, None, wk, B * S, q_abs, stream)
+    cu = torch.arange(0, (B + 1) * S, S, dtype=torch.int32, device=dev)
+    flags = MLA_DECODE_CAUSAL if causal else 0
+    out_lat = torch.empty(B * S, H, L, dtype=torch.float32, device=dev)
+    ws = workspace(mla_decode_workspace_size(d, dt, B, S, S, B * S, flags), dev)
+    mla_decode_absorbed(d, q_abs, c, cu, B, S, S, flags, out_lat, None, ws, stream)
+    y = torch.empty(B * S, D, dtype=dt, device=dev)
+    ws2 = workspace(mla_out_project_workspace_size(d, dt, B * S), dev)
+    mla_out_project(d, out_lat, wv, wo, g, B * S, y, ws2, stream)
+    return {"output": y.reshape(B, S, D), "latent_cache": c.reshape(B, S, L)}

@@ -1,0 +1,204 @@
+/*
+ * mla.h -- C ABI of libmla_b200.so: absorbed Multi-head Latent Attention (MLA) decode on B200.
+ *
+ * The method (cited by page title and section):
+ *   [rs]  "ferrox-core 0.23.0 src/mla_absorbed.rs", module docs "What it is" and the doc comment
+ *         of causal_mla_absorbed_attention: the query is pushed into the latent
+ *         (q_abs[h] = W_UK[h]^T q_nope[h]), attention runs as multi-query attention over ONE shared
+ *         key row concat(c_t, k_pe_t) and ONE shared value c_t per position,
+ *         score = (q_abs . c + q_pe . k_pe) * kq_scale, kq_scale = 1/sqrt(qk_nope + rope_dim),
+ *         out_lat = softmax(score) . c, and v[h] = W_UV[h] out_lat[h].
+ *   [nb]  "MLA_RoPE-less.ipynb": cache update before attention, matrix absorption
+ *         (W_aQK = W_uQ W_uK^T, W_aVO = W_uV W_O), the adding trick over heads.
+ *   [lab] "Lab 01 - Ejercicio matematico de MLA" (lynx-cortex), Bloque B: the matmul identity
+ *         q^T W_UK c = (W_UK^T q)^T c.
+ *   [fm]  "preacher-1/MLA_tutorial formula.md", Part 3, inference-form equation: o_t is the
+ *         concatenation of o^(s) W_v^(s), followed by the output projection.
+ *   [gm]  "Gated MLA" (tensortonic, Kimi K3 step 2 of 11): Y = [sigmoid(X Wg^T) * O] Wo^T,
+ *         causal mask removing later positions, the Requirements (inputs are not mutated).
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are caller-owned DEVICE memory, dense, row-major, in the dtype named by the call
+ *     (MLA_F32 or MLA_BF16), except where a parameter says float / int32 / int64 explicitly.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Every call is asynchronous
+ *     with respect to the host and enqueues its kernels on that stream only.
+ *   - Inputs are never written. Outputs are written only where documented.
+ *   - Host-side validation runs before any launch; on a violation the call returns an error and
+ *     launches nothing. A failed launch returns MLA_ERR_CUDA. Nothing aborts the process.
+ *   - The library allocates no device memory. Scratch memory is the caller's `workspace`.
+ *   - bf16 values are rounded to nearest-even wherever the library stores bf16.
+ */
+#ifndef MLA_B200_H
+#define MLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point (int32_t). */
+enum {
+  MLA_OK = 0,
+  MLA_ERR_NULL = 1,        /* a required pointer is NULL                                        */
+  MLA_ERR_SHAPE = 2,       /* a size is negative, zero where it must be positive, or inconsistent */
+  MLA_ERR_DTYPE = 3,       /* unknown dtype code, or a dtype the operation does not take         */
+  MLA_ERR_ALIGN = 4,       /* a pointer is not aligned as the operation requires (16 B for bf16) */
+  MLA_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than the size query returned             */
+  MLA_ERR_CUDA = 6,        /* a CUDA runtime call or a kernel launch failed                      */
+  MLA_ERR_TIMEOUT = 7,     /* a bounded device-side wait gave up (reported by mla_check_status)  */
+  MLA_ERR_UNSUPPORTED = 8, /* a valid request this build does not implement                      */
+  MLA_ERR_MODE = 9         /* unknown mode or flag bit                                           */
+};
+
+/* Element types. All floating-point tensors of one call share the call's dtype ([gm] Constraints). */
+enum { MLA_F32 = 0, MLA_BF16 = 1 };
+
+/* Model dimensions. kq_scale == 0 selects the default 1/sqrt(qk_nope + rope_dim): the width of the
+ * UN-absorbed head, not of the latent ([rs] module docs, the kq_scale paragraph). */
+typedef struct mla_dims {
+  int32_t n_heads;      /* H                                                        */
+  int32_t kv_lora_rank; /* d_c: width of the latent c_t, also the value width        */
+  int32_t rope_dim;     /* d_r: width of the decoupled rotary key k_pe_t (may be 0)   */
+  int32_t qk_nope;      /* n: per-head width of the non-rotary query / key            */
+  int32_t v_head;       /* d_v: per-head width of the value after W_UV                */
+  int32_t d_model;      /* D: width of the layer output                               */
+  float kq_scale;       /* score scale; 0 => 1/sqrt(qk_nope + rope_dim)               */
+} mla_dims;
+
+/* modes of mla_absorb_weights */
+enum { MLA_ABSORB_QUERY = 0, MLA_FOLD_QK = 1, MLA_FOLD_VO = 2 };
+/* flags of mla_append_latent */
+enum { MLA_APPEND_NORM = 1u, MLA_APPEND_ROPE = 2u };
+/* flags of mla_decode_absorbed */
+enum { MLA_DECODE_CAUSAL = 1u };
+/* flags of mla_linear */
+enum { MLA_LINEAR_SIGMOID = 1u, MLA_LINEAR_W_KN = 2u };
+
+/* Human-readable name of a status code (static string, never NULL). */
+MLA_API const char* mla_status_string(int32_t status);
+
+/* ABI version of this header (increments on any signature change). */
+MLA_API int32_t mla_abi_version(void);
+
+/*
+ * mla_append_latent -- write new latent-cache rows ([nb] "update cache": the new latent is
+ * stacked onto the cache before attention; [rs] fn docs: a row is the normed compressed KV
+ * followed by the roped k_pe, i.e. concat(c, k_pe)).
+ *
+ *   cache      [cache_rows, d_c + d_r] in cache_dtype; only rows row_idx[k] are written.
+ *   row_idx    int64 [n_new], each in [0, cache_rows); duplicates give an unspecified winner.
+ *   c_new      float [n_new, d_c];  kpe_new float [n_new, d_r] (may be NULL when d_r == 0).
+ *   positions  int32 [n_new] rotary positions (read only with MLA_APPEND_ROPE).
+ *   flags      MLA_APPEND_NORM: c <- c / sqrt(mean(c^2) + eps) (unit weight);
+ *              MLA_APPEND_ROPE: k_pe pair (2i, 2i+1) turns by positions[k] * rope_theta^(-2i/d_r).
+ * Errors: MLA_ERR_NULL, MLA_ERR_SHAPE (d_r odd with ROPE, n_new < 0), MLA_ERR_DTYPE, MLA_ERR_MODE.
+ */
+MLA_API int32_t mla_append_latent(const mla_dims* dims, int32_t cache_dtype, void* cache, int64_t cache_rows,
+                          const int64_t* row_idx, const float* c_new, const float* kpe_new,
+                          const int32_t* positions, int64_t n_new, uint32_t flags, float eps,
+                          float rope_theta, void* stream);
+
+/*
+ * mla_absorb_weights -- per-head products of the absorbed form.
+ *
+ * MLA_ABSORB_QUERY ([rs] module docs: q_nope_absorbed[h] = wk_b[h] . q_nope[h]; [lab] Bloque B:
+ *   q^T W_UK c = (W_UK^T q)^T c):
+ *     x    = q_nope [n_rows, H, qk_nope];  x_pe = q_pe [n_rows, H, d_r] (NULL allowed if d_r == 0);
+ *     w    = W_UK   [H, qk_nope, d_c];
+ *     out  = q_abs  [n_rows, H, d_c + d_r]:  out[t,h,j] = sum_i x[t,h,i] w[h,i,j] (j < d_c),
+ *            out[t,h,d_c + r] = x_pe[t,h,r].
+ * MLA_FOLD_QK ([nb] matrix absorption, W_aQK = W_uQ W_uK^T):
+ *     x = W_uQ heads [H, n_rows, qk_nope], w = W_uK heads [H, d_c, qk_nope],
+ *     out = W_aQK [H, n_rows, d_c] = x[h] . w[h]^T.
+ * MLA_FOLD_VO ([nb] matrix absorption, W_aVO = W_uV W_O):
+ *     x = W_uV heads [H, d_c, v_head], w = W_O heads [H, v_head, d_model],
+ *     out = W_aVO [H, d_c, d_model] = x[h] . w[h]   (n_rows must equal d_c).
+ * All operands in `dtype`; accumulation in fp32; out in `dtype`.
+ */
+MLA_API int32_t mla_absorb_weights(const mla_dims* dims, int32_t dtype, int32_t mode, const void* x,
+                           const void* x_pe, const void* w, int64_t n_rows, void* out, void* stream);
+
+/*
+ * mla_decode_workspace_size -- bytes of scratch mla_decode_absorbed needs for these sizes.
+ *   batch        number of sequences B;  n_q_per_seq  query tokens per sequence (>= 1);
+ *   max_seqlen   an upper bound on every T_b (host-side planning only);
+ *   total_rows   sum of T_b (rows of the packed cache).
+ */
+MLA_API int32_t mla_decode_workspace_size(const mla_dims* dims, int32_t dtype, int32_t batch,
+                                  int32_t n_q_per_seq, int64_t max_seqlen, int64_t total_rows,
+                                  uint32_t flags, size_t* bytes);
+
+/*
+ * mla_decode_absorbed -- attention of the absorbed queries over the shared latent cache
+ * ([rs] module docs and fn: score[h][t] = (q_abs[h] . c[t] + q_pe[h] . k_pe[t]) * kq_scale,
+ * out_lat[h] = sum_t softmax(score[h])[t] c[t], returned before W_UV; [gm] causal mask).
+ *
+ *   q_abs       [B * n_q, H, d_c + d_r]; row b*n_q + j is query j of sequence b.
+ *   cache       [total_rows, d_c + d_r]; sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1.
+ *   cu_seqlens  DEVICE int32 [B + 1], non-decreasing, cu_seqlens[0] = 0, cu_seqlens[B] = total_rows.
+ *   flags       MLA_DECODE_CAUSAL: query j of sequence b (the n_q newest tokens sit at its last
+ *               n_q rows) sees positions t <= T_b - n_q + j; otherwise it sees all T_b positions.
+ *   out_lat     float [B * n_q, H, d_c]: the softmax-weighted latent (zeros when nothing is seen).
+ *   lse         float [B * n_q, H] or NULL: natural-log sum-exp of the scaled scores (-inf if empty).
+ *   workspace   caller scratch of at least mla_decode_workspace_size() bytes, 256-byte aligned.
+ * Requirements: T_b <= max_seqlen for every b (not checked on the device: the plan assumes it
+ * when it sizes the split of each sequence), T_b >= n_q when causal.
+ * bf16 calls with d_c = 512 and d_r in {0, 64} run the tensor-core (tcgen05) kernel; every other
+ * supported shape runs the CUDA-core kernel. Both accumulate in fp32.
+ */
+MLA_API int32_t mla_decode_absorbed(const mla_dims* dims, int32_t dtype, const void* q_abs, const void* cache,
+                            const int32_t* cu_seqlens, int32_t batch, int32_t n_q_per_seq,
+                            int64_t max_seqlen, int64_t total_rows, uint32_t flags, float* out_lat,
+                            float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of scratch mla_out_project needs for n_rows query rows. */
+MLA_API int32_t mla_out_project_workspace_size(const mla_dims* dims, int32_t dtype, int64_t n_rows,
+                                       size_t* bytes);
+
+/*
+ * mla_out_project -- v[t,h] = W_UV[h] out_lat[t,h] ([rs] v = wv_b . out_lat), optional channel
+ * gate ([gm]: sigmoid(X Wg^T) * O), then y[t] = W_O concat_h v[t,h] ([fm] inference form;
+ * [nb] the adding trick is the same sum over heads).
+ *
+ *   out_lat  float [n_rows, H, d_c];  w_uv [H, v_head, d_c];  w_o [d_model, H * v_head];
+ *   gate     [n_rows, H * v_head] in `dtype`, or NULL for no gate (values are used as given: pass
+ *            sigmoid(X Wg^T), e.g. from mla_linear with MLA_LINEAR_SIGMOID);
+ *   y        [n_rows, d_model] in `dtype`.
+ */
+MLA_API int32_t mla_out_project(const mla_dims* dims, int32_t dtype, const float* out_lat, const void* w_uv,
+                        const void* w_o, const void* gate, int64_t n_rows, void* y,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * mla_linear -- Y = X W^T ([gm] problem equations, PyTorch Linear convention W = [n, k]).
+ *   x [m, k], w [n, k] (or [k, n] with MLA_LINEAR_W_KN), y [m, n]; all in `dtype`, fp32 accumulate.
+ *   MLA_LINEAR_SIGMOID applies sigmoid to Y before it is stored.
+ */
+MLA_API int32_t mla_linear(int32_t dtype, const void* x, const void* w, int64_t m, int64_t n, int64_t k,
+                   uint32_t flags, void* y, void* stream);
+
+/*
+ * mla_check_status -- synchronise `stream`, then report and clear the library's device status
+ * word: MLA_OK, or MLA_ERR_TIMEOUT when a bounded device wait gave up, or MLA_ERR_SHAPE when a kernel skipped an out-of-range row index, since the last check.
+ */
+MLA_API int32_t mla_check_status(void* stream, int32_t* device_status);
+
+/* Number of kernels this library has launched in this process (all devices, all streams). */
+MLA_API int64_t mla_launch_count(void);
+
+/* Test hook: spin limit of the bounded device waits (0 restores the default). */
+MLA_API int32_t mla_set_wait_limit(int64_t spins);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_H */
