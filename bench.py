@@ -19,7 +19,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -87,64 +86,92 @@ def recorded_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while the timed region runs."""
+    """SM clock, power and clock-event (throttle) reasons of one GPU, read through NVML every
+    ~2 ms by a background thread while the timed region runs (read-only queries)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {  # NVML clocks-event reason bits
+        "sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+        self.samples = []
+        self.window = None
+        self._stop = threading.Event()
+        self.ok = False
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = None
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(self.gpu).uuid)
+            except Exception:
+                pass
+            h = None
+            if uuid:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+                except Exception:
+                    h = None
+            self.h = h if h is not None else pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+            self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
-        except (FileNotFoundError, OSError):
-            self.proc = None
+        except Exception:
+            self.ok = False
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                power = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                self.samples.append((time.time(), sm, reasons, power))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def wait_first(self, timeout_s: float = 2.0):
+        t0 = time.time()
+        while self.ok and not self.samples and time.time() - t0 < timeout_s:
+            time.sleep(0.005)
+
+    def mark(self, t0: float, t1: float):
+        self.window = (t0, t1)
 
     def __exit__(self, *exc):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        if self.ok:
             self.t.join(timeout=2)
+            try:
+                self.nv.nvmlShutdown()
+            except Exception:
+                pass
 
     def summary(self):
-        rows = []
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
-                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
-            except ValueError:
-                continue
-        if not rows:
+        if not self.ok or not self.samples:
             return None
-        load = [r for r in rows if r["power"] > 300.0] or rows
+        rows = self.samples
+        if self.window:
+            t0, t1 = self.window
+            inside = [r for r in rows if t0 <= r[0] <= t1]
+            rows = inside or [min(rows, key=lambda r: abs(r[0] - 0.5 * (t0 + t1)))]
         reasons = set()
-        for r in rows:
-            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
-                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
-                if r[key].lower() == "active":
+        for _, _, bits, _ in rows:
+            for name, bit in self.REASONS.items():
+                if bits & bit:
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": rows[0]["smax"],
-                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load)}
+        return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_median": statistics.median(r[3] for r in rows), "source": "nvml, 2 ms polling"}
 
 
 # --------------------------------------------------------------------------------------------
@@ -272,8 +299,14 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    launches0 = M.mla_launch_count()
     with ClockSampler(torch.cuda.current_device()) as clk:
+        clk.wait_first()
+        # keep the GPU busy until the sampler has seen it under load, then time
+        for _ in range(args.warmup):
+            step(q_nope, q_pe, c_new, kpe_new, row_idx, positions)
+        torch.cuda.synchronize()
+        t_wall0 = time.time()
+        launches0 = M.mla_launch_count()
         start.record(stream)
         for k in range(args.steps):
             M.mla_append_latent(d, cache, row_idx, c_new, kpe_new, positions, step.append_flags)
@@ -285,6 +318,7 @@ def run_ours(args):
             M.mla_out_project(d, step.out_lat, step.w_uv, step.w_o, None, nq, step.y, step.ws_out)
         stop.record(stream)
         torch.cuda.synchronize()
+        clk.mark(t_wall0, time.time())
     launches = M.mla_launch_count() - launches0
     if world > 1:
         dist.barrier()

@@ -18,7 +18,7 @@ namespace mla {
 // device status word (one per device that loads the library)
 static __device__ int g_device_status = 0;
 static long long g_wait_limit_host = 0;
-constexpr long long kDefaultWaitLimit = 1LL << 26;
+constexpr long long kDefaultWaitLimit = 2000000000LL;  // 2 s of the device's global timer
 
 int* device_status_ptr() {
   static int* cached[64] = {nullptr};

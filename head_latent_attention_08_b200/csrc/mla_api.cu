@@ -289,6 +289,12 @@ int32_t mla_check_status(void* stream, int32_t* device_status) {
   return MLA_OK;
 }
 
+int32_t mla_set_decode_clusters(int32_t n) {
+  if (n < 0) return MLA_ERR_SHAPE;
+  set_decode_clusters(n);
+  return MLA_OK;
+}
+
 int64_t mla_launch_count(void) { return (int64_t)launch_count(); }
 
 int32_t mla_set_wait_limit(int64_t spins) {

@@ -14,6 +14,7 @@ int tc_absorb_query(const mla_dims& d, const void* q_nope, const void* q_pe, con
 bool tc_decode_supported(const DecodeArgs& a);
 size_t tc_decode_workspace(const DecodeArgs& a);
 int tc_decode_launch(const DecodeArgs& a, cudaStream_t s);
+void set_decode_clusters(int n);   // 0 = one cluster per SM pair
 
 // value + output projection
 bool tc_out_project_supported(const mla_dims& d, int64_t n_rows);

@@ -1,0 +1,443 @@
+// tc_gemm.cu -- tensor-core GEMM for sm_100a (TMA -> shared memory -> tcgen05.mma -> TMEM) and the
+// three products of the absorbed form that run on it:
+//   * query absorption  q_abs[t,h,:d_c] = W_UK[h]^T q_nope[t,h]   (per head: M = d_c, N = tokens)
+//   * value projection  v[t,h] = gate * (W_UV[h] out_lat[t,h])      (per head: M = v_head, N = tokens)
+//   * output projection y[t] = W_O v[t]                            (M = d_model, N = tokens, split-K)
+//   * dense linear      Y = X W^T                                  (M = out features, N = tokens)
+//
+// Shape of one CTA: D[128 x BN] (fp32, TMEM) = A[128 x K] . B[BN x K]^T with A the weight tile and B
+// the token tile, both bf16 in 128-byte-swizzled shared memory, fed by TMA through a ring of stages.
+// One thread issues the TMA loads, one thread issues the MMAs (4 x K16 per 64-wide K chunk), and the
+// four warps drain TMEM in the epilogue (warp w owns accumulator rows 32w..32w+31). The result is
+// stored transposed, out[t][m]: consecutive lanes write consecutive addresses. Weights wider than one
+// wave of tiles are split along K; the fp32 partials are summed in a fixed order by a second kernel.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "sm100.cuh"
+#include "tc.cuh"
+
+namespace mla {
+
+using namespace sm100;
+
+// ---------------------------------------------------------------------------------------------
+// host: tensor maps
+// ---------------------------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      (void)cudaGetLastError();
+  });
+  return fn;
+}
+
+bool encode_tmap_bf16(CUtensorMap* map, void* base, int rank, const uint64_t* dims,
+                      const uint64_t* strides_bytes, const uint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t d[5], st[4];
+  cuuint32_t b[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    es[i] = 1;
+    if (i + 1 < rank) st[i] = strides_bytes[i];
+  }
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, base, d, st, b, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------------------------
+// the GEMM kernel
+// ---------------------------------------------------------------------------------------------
+struct TcGemmParams {
+  int M, N, K;
+  int n_tiles;       // BN-wide token tiles
+  int k_chunks;      // 64-wide K chunks per split
+  int n_splits;
+  int batch;
+  void* out; int64_t out_sb, out_st; int out_f32;
+  const __nv_bfloat16* gate; int64_t gate_sb, gate_st;
+  float* partial;    // [split][batch][N][M] when n_splits > 1
+  int sigmoid;
+  int* status;
+  unsigned long long wait_ns;
+};
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int A_BYTES = 128 * 64 * 2;
+  static constexpr int B_BYTES = BN * 64 * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int STAGES_FIT = (192 * 1024) / STAGE;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+  static constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;
+};
+
+__device__ __forceinline__ float apply_epilogue(float v, int sigmoid, const __nv_bfloat16* gate, int64_t gidx) {
+  if (sigmoid) v = 1.f / (1.f + expf(-v));
+  if (gate) v *= __bfloat162float(gate[gidx]);
+  return v;
+}
+
+template <int BN, bool A_MN>
+__global__ void __launch_bounds__(128, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
+                   TcGemmParams p) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int STAGES = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE);
+  uint64_t* empty = full + STAGES;
+  uint64_t* done = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * 128;
+  const int split = blockIdx.y / p.n_tiles, n0 = (blockIdx.y % p.n_tiles) * BN;
+  const int bz = blockIdx.z;
+  const int total_chunks = (p.K + 63) / 64;
+  const int kc0 = split * p.k_chunks;
+  const int nk = max(0, min(kc0 + p.k_chunks, total_chunks) - kc0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&ta);
+    prefetch_tmap(&tb);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+  int issued = 0;
+
+  if (warp == 0 && lane == 0) {
+    // TMA producer
+    for (int i = 0; i < nk; ++i) {
+      const int s = i % STAGES;
+      if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, p.wait_ns, p.status)) {
+        *abort_flag = 1;
+        break;
+      }
+      if (*abort_flag) break;
+      uint8_t* a_dst = smem + s * Cfg::STAGE;
+      uint8_t* b_dst = a_dst + Cfg::A_BYTES;
+      mbar_arrive_expect_tx(&full[s], Cfg::STAGE);
+      const int kx = (kc0 + i) * 64;
+      if (A_MN) {
+        tma_load_3d(a_dst, &ta, &full[s], m0, kx, bz);
+        tma_load_3d(a_dst + 8192, &ta, &full[s], m0 + 64, kx, bz);
+      } else {
+        tma_load_3d(a_dst, &ta, &full[s], kx, m0, bz);
+      }
+      tma_load_3d(b_dst, &tb, &full[s], kx, n0, bz);
+      ++issued;
+    }
+  } else if (warp == 1 && lane == 0) {
+    // MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(128, BN, A_MN, false);
+    for (int i = 0; i < nk; ++i) {
+      const int s = i % STAGES;
+      if (!mbar_wait(&full[s], (i / STAGES) & 1, p.wait_ns, p.status)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t a_base = smem_u32(smem + s * Cfg::STAGE);
+      const uint32_t b_base = a_base + Cfg::A_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = A_MN ? smem_desc_sw128(a_base + kk * 2048, 8192, 1024)
+                                 : smem_desc_sw128(a_base + kk * 32, 16, 1024);
+        const uint64_t bd = smem_desc_sw128(b_base + kk * 32, 16, 1024);
+        mma_bf16_ss(tmem_d, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(&empty[s]);
+    }
+    mma_commit(done);
+  }
+  __syncwarp();
+
+  // epilogue: 128 threads, thread = accumulator row
+  const bool ok = mbar_wait(done, 0, p.wait_ns, p.status);
+  tc_fence_after();
+  const bool write = ok && !*abort_flag;
+  const int m = m0 + warp * 32 + lane;
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    uint32_t r[32];
+    tmem_ld32(tmem_d + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, r);
+    tmem_wait_ld();
+    if (!write || m >= p.M) continue;
+#pragma unroll 4
+    for (int j = 0; j < 32; ++j) {
+      const int t = n0 + c + j;
+      if (t >= p.N) break;
+      const float acc = nk > 0 ? __uint_as_float(r[j]) : 0.f;
+      if (p.n_splits > 1) {
+        p.partial[(((int64_t)split * p.batch + bz) * p.N + t) * p.M + m] = acc;
+      } else {
+        const float v = apply_epilogue(acc, p.sigmoid, p.gate, bz * p.gate_sb + (int64_t)t * p.gate_st + m);
+        const int64_t o = bz * p.out_sb + (int64_t)t * p.out_st + m;
+        if (p.out_f32)
+          static_cast<float*>(p.out)[o] = v;
+        else
+          static_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(v);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    // do not leave TMA writes in flight behind an abandoned CTA: wait (bounded) for the loads
+    for (int i = max(0, issued - STAGES); i < issued; ++i)
+      (void)mbar_wait(&full[i % STAGES], (i / STAGES) & 1, p.wait_ns, p.status);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_d, Cfg::TMEM_COLS);
+  }
+}
+
+// fixed-order sum of split-K partials + epilogue
+__global__ void splitk_reduce_kernel(const float* __restrict__ partial, int n_splits, int batch, int N, int M,
+                                     void* out, int64_t out_sb, int64_t out_st, int out_f32,
+                                     const __nv_bfloat16* gate, int64_t gate_sb, int64_t gate_st, int sigmoid) {
+  const int64_t per = (int64_t)batch * N * M;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < per; e += (int64_t)gridDim.x * blockDim.x) {
+    float v = 0.f;
+    for (int s = 0; s < n_splits; ++s) v += partial[s * per + e];
+    const int m = (int)(e % M);
+    const int64_t bt = e / M;
+    const int t = (int)(bt % N);
+    const int bz = (int)(bt / N);
+    v = apply_epilogue(v, sigmoid, gate, bz * gate_sb + (int64_t)t * gate_st + m);
+    const int64_t o = bz * out_sb + (int64_t)t * out_st + m;
+    if (out_f32)
+      static_cast<float*>(out)[o] = v;
+    else
+      static_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(v);
+  }
+}
+
+// out_lat fp32 -> bf16 (the tensor-core operand of the value projection)
+__global__ void f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst, int64_t n4) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 v = src[i];
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 o;
+    o.x = *reinterpret_cast<uint32_t*>(&a);
+    o.y = *reinterpret_cast<uint32_t*>(&b);
+    dst[i] = o;
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// host: one GEMM
+// ---------------------------------------------------------------------------------------------
+struct GemmOperand {
+  // a 3-D bf16 tensor seen as [batch][rows][k] (K-major) or [batch][k][rows] (MN-major)
+  void* base;
+  uint64_t inner, mid, outer;            // dims from innermost
+  uint64_t stride_mid, stride_outer;     // bytes
+};
+
+struct GemmPlan {
+  int BN, n_tiles, m_tiles, splits, k_chunks;
+};
+
+static GemmPlan plan_gemm(int M, int N, int K, int batch) {
+  GemmPlan g;
+  g.BN = N <= 64 ? 64 : (N <= 128 ? 128 : 256);
+  g.n_tiles = (int)ceil_div(N, g.BN);
+  g.m_tiles = M / 128;
+  const int total_chunks = (int)ceil_div(K, 64);
+  const int64_t base = (int64_t)g.m_tiles * g.n_tiles * batch;
+  int splits = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count() / std::max<int64_t>(base, 1),
+                                                            total_chunks / 4));
+  g.k_chunks = (int)ceil_div(total_chunks, splits);
+  g.splits = (int)ceil_div(total_chunks, g.k_chunks);
+  return g;
+}
+
+static size_t gemm_partial_bytes(int M, int N, int K, int batch) {
+  GemmPlan g = plan_gemm(M, N, K, batch);
+  return g.splits > 1 ? round_up((size_t)g.splits * batch * N * M * sizeof(float), 256) : 0;
+}
+
+template <int BN, bool A_MN>
+static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmParams& p, dim3 grid,
+                         cudaStream_t s) {
+  static bool attr_set[64] = {false};
+  const int dev = current_device();
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(tc_gemm_kernel<BN, A_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<BN>::SMEM) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  tc_gemm_kernel<BN, A_MN><<<grid, 128, GemmCfg<BN>::SMEM, s>>>(ta, tb, p);
+  MLA_LAUNCH_CHECK();
+  return MLA_OK;
+}
+
+// out[bz][t][m] = epi(sum_k A[bz](m, k) B[bz](t, k)); A MN-major when a_mn
+static int tc_gemm(const GemmOperand& A, bool a_mn, const GemmOperand& Bop, int M, int N, int K, int batch,
+                   void* out, int64_t out_sb, int64_t out_st, bool out_f32, const void* gate, int64_t gate_sb,
+                   int64_t gate_st, bool sigmoid, void* partial_ws, cudaStream_t s) {
+  if (M % 128 || K % 64 || N <= 0 || batch <= 0) return MLA_ERR_UNSUPPORTED;
+  const GemmPlan g = plan_gemm(M, N, K, batch);
+  CUtensorMap ta, tb;
+  {
+    const uint64_t dims[3] = {A.inner, A.mid, A.outer};
+    const uint64_t st[2] = {A.stride_mid, A.stride_outer};
+    const uint32_t box[3] = {64, a_mn ? 64u : 128u, 1};
+    if (!encode_tmap_bf16(&ta, A.base, 3, dims, st, box)) return MLA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[3] = {Bop.inner, Bop.mid, Bop.outer};
+    const uint64_t st[2] = {Bop.stride_mid, Bop.stride_outer};
+    const uint32_t box[3] = {64, (uint32_t)g.BN, 1};
+    if (!encode_tmap_bf16(&tb, Bop.base, 3, dims, st, box)) return MLA_ERR_CUDA;
+  }
+  TcGemmParams p{};
+  p.M = M; p.N = N; p.K = K; p.n_tiles = g.n_tiles; p.k_chunks = g.k_chunks; p.n_splits = g.splits;
+  p.batch = batch; p.out = out; p.out_sb = out_sb; p.out_st = out_st; p.out_f32 = out_f32 ? 1 : 0;
+  p.gate = static_cast<const __nv_bfloat16*>(gate); p.gate_sb = gate_sb; p.gate_st = gate_st;
+  p.partial = static_cast<float*>(partial_ws); p.sigmoid = sigmoid ? 1 : 0;
+  p.status = device_status_ptr(); p.wait_ns = (unsigned long long)wait_limit();
+  if (!p.status) return MLA_ERR_CUDA;
+  if (g.splits > 1 && !partial_ws) return MLA_ERR_WORKSPACE;
+  dim3 grid((unsigned)g.m_tiles, (unsigned)(g.n_tiles * g.splits), (unsigned)batch);
+  if (grid.y > 65535u || grid.z > 65535u) return MLA_ERR_UNSUPPORTED;
+  int st;
+  if (a_mn) {
+    st = g.BN == 64 ? launch_gemm_t<64, true>(ta, tb, p, grid, s)
+                    : g.BN == 128 ? launch_gemm_t<128, true>(ta, tb, p, grid, s)
+                                  : launch_gemm_t<256, true>(ta, tb, p, grid, s);
+  } else {
+    st = g.BN == 64 ? launch_gemm_t<64, false>(ta, tb, p, grid, s)
+                    : g.BN == 128 ? launch_gemm_t<128, false>(ta, tb, p, grid, s)
+                                  : launch_gemm_t<256, false>(ta, tb, p, grid, s);
+  }
+  if (st) return st;
+  if (g.splits > 1) {
+    const int64_t per = (int64_t)batch * N * M;
+    const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(per, 256), 8 * sm_count());
+    splitk_reduce_kernel<<<blocks, 256, 0, s>>>(p.partial, g.splits, batch, N, M, out, out_sb, out_st,
+                                                p.out_f32, p.gate, gate_sb, gate_st, p.sigmoid);
+    MLA_LAUNCH_CHECK();
+  }
+  return MLA_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// the library's products on the tensor-core GEMM
+// ---------------------------------------------------------------------------------------------
+bool tc_absorb_supported(const mla_dims& d, int64_t n_rows) {
+  return d.kv_lora_rank % 128 == 0 && d.qk_nope % 64 == 0 && d.qk_nope > 0 && n_rows > 0 &&
+         n_rows < (1LL << 30) && ((int64_t)d.n_heads * d.qk_nope * 2) % 16 == 0 &&
+         ((int64_t)d.kv_lora_rank * 2) % 16 == 0 && d.rope_dim % 8 == 0;
+}
+
+int tc_absorb_query(const mla_dims& d, const void* q_nope, const void* q_pe, const void* w_uk, int64_t n_rows,
+                    void* q_abs, cudaStream_t s) {
+  const int64_t H = d.n_heads, n = d.qk_nope, dc = d.kv_lora_rank, dr = d.rope_dim, W = dc + dr;
+  // A = W_UK[h] viewed as (m = j, k = i): MN-major, tensor [H][n][dc]
+  GemmOperand A{const_cast<void*>(w_uk), (uint64_t)dc, (uint64_t)n, (uint64_t)H, (uint64_t)(dc * 2),
+                (uint64_t)(n * dc * 2)};
+  // B = q_nope[:, h, :]: tensor [rows][H][n] seen as (k = i, t, h)
+  GemmOperand B{const_cast<void*>(q_nope), (uint64_t)n, (uint64_t)n_rows, (uint64_t)H, (uint64_t)(H * n * 2),
+                (uint64_t)(n * 2)};
+  int st = tc_gemm(A, true, B, (int)dc, (int)n_rows, (int)n, (int)H, q_abs, W, H * W, false, nullptr, 0, 0,
+                   false, nullptr, s);
+  if (st) return st;
+  if (dr > 0)
+    return copy_rows_strided(q_pe, dr, static_cast<char*>(q_abs) + dc * 2, W, n_rows * H, dr, MLA_BF16, s);
+  return MLA_OK;
+}
+
+bool tc_out_project_supported(const mla_dims& d, int64_t n_rows) {
+  const int64_t H = d.n_heads, dc = d.kv_lora_rank, dv = d.v_head, D = d.d_model;
+  return dv % 128 == 0 && dc % 64 == 0 && D % 128 == 0 && (H * dv) % 64 == 0 && n_rows > 0 &&
+         n_rows < (1LL << 30) && dc % 4 == 0;
+}
+
+// scratch beyond v: out_lat in bf16, then the split-K partials of the output projection
+size_t tc_out_project_extra_workspace(const mla_dims& d, int64_t n_rows) {
+  if (!tc_out_project_supported(d, n_rows)) return 0;
+  const int64_t H = d.n_heads, dc = d.kv_lora_rank, dv = d.v_head, D = d.d_model;
+  return round_up((size_t)n_rows * H * dc * 2, 256) + gemm_partial_bytes((int)D, (int)n_rows, (int)(H * dv), 1);
+}
+
+int tc_out_project(const mla_dims& d, const float* out_lat, const void* w_uv, const void* w_o, const void* gate,
+                   int64_t n_rows, void* y, void* workspace, size_t ws_bytes, cudaStream_t s) {
+  const int64_t H = d.n_heads, dc = d.kv_lora_rank, dv = d.v_head, D = d.d_model;
+  char* ws = static_cast<char*>(workspace);
+  void* v = ws;
+  const size_t v_bytes = round_up((size_t)n_rows * H * dv * 2, 256);
+  void* lat16 = ws + v_bytes;
+  const size_t lat_bytes = round_up((size_t)n_rows * H * dc * 2, 256);
+  void* partial = ws + v_bytes + lat_bytes;
+  if (ws_bytes < v_bytes + tc_out_project_extra_workspace(d, n_rows)) return MLA_ERR_WORKSPACE;
+  {
+    const int64_t n4 = n_rows * H * dc / 4;
+    const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(n4, 256), 8 * sm_count());
+    f32_to_bf16_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(out_lat),
+                                              static_cast<uint2*>(lat16), n4);
+    MLA_LAUNCH_CHECK();
+  }
+  // v[t, h, i] = gate * sum_j W_UV[h, i, j] lat[t, h, j]: A = W_UV[h] K-major, B = lat[:, h, :]
+  GemmOperand A1{const_cast<void*>(w_uv), (uint64_t)dc, (uint64_t)dv, (uint64_t)H, (uint64_t)(dc * 2),
+                 (uint64_t)(dv * dc * 2)};
+  GemmOperand B1{lat16, (uint64_t)dc, (uint64_t)n_rows, (uint64_t)H, (uint64_t)(H * dc * 2), (uint64_t)(dc * 2)};
+  int st = tc_gemm(A1, false, B1, (int)dv, (int)n_rows, (int)dc, (int)H, v, dv, H * dv, false, gate, dv, H * dv,
+                   false, nullptr, s);
+  if (st) return st;
+  // y[t, o] = sum_k W_O[o, k] v[t, k]
+  const int64_t K = H * dv;
+  GemmOperand A2{const_cast<void*>(w_o), (uint64_t)K, (uint64_t)D, 1, (uint64_t)(K * 2), (uint64_t)(D * K * 2)};
+  GemmOperand B2{v, (uint64_t)K, (uint64_t)n_rows, 1, (uint64_t)(K * 2), (uint64_t)(n_rows * K * 2)};
+  return tc_gemm(A2, false, B2, (int)D, (int)n_rows, (int)K, 1, y, 0, D, false, nullptr, 0, 0, false, partial, s);
+}
+
+bool tc_linear_supported(int64_t m, int64_t n, int64_t k) {
+  return n % 128 == 0 && k % 64 == 0 && m > 0 && m < (1LL << 30) && n < (1LL << 30) && k < (1LL << 30) &&
+         gemm_partial_bytes((int)n, (int)m, (int)k, 1) == 0;
+}
+
+int tc_linear(const void* x, const void* w, int64_t m, int64_t n, int64_t k, int sigmoid, void* y, cudaStream_t s) {
+  // Y[t, o] = sum_k W[o, k] X[t, k]: A = W (M = n), B = X (N = m)
+  GemmOperand A{const_cast<void*>(w), (uint64_t)k, (uint64_t)n, 1, (uint64_t)(k * 2), (uint64_t)(n * k * 2)};
+  GemmOperand B{const_cast<void*>(x), (uint64_t)k, (uint64_t)m, 1, (uint64_t)(k * 2), (uint64_t)(m * k * 2)};
+  return tc_gemm(A, false, B, (int)n, (int)m, (int)k, 1, y, 0, n, false, nullptr, 0, 0, sigmoid != 0, nullptr, s);
+}
+
+}  // namespace mla

@@ -29,6 +29,7 @@ EXPORTED = (
     "mla_status_string", "mla_abi_version", "mla_append_latent", "mla_absorb_weights",
     "mla_decode_workspace_size", "mla_decode_absorbed", "mla_out_project_workspace_size",
     "mla_out_project", "mla_linear", "mla_check_status", "mla_set_wait_limit", "mla_launch_count",
+    "mla_set_decode_clusters",
 )
 
 
@@ -68,6 +69,7 @@ _SIGS = {
     "mla_check_status": (_I32, [_P, ctypes.POINTER(_I32)]),
     "mla_set_wait_limit": (_I32, [_I64]),
     "mla_launch_count": (_I64, []),
+    "mla_set_decode_clusters": (_I32, [_I32]),
 }
 
 
@@ -195,6 +197,10 @@ def mla_check_status(stream=None) -> int:
 
 def mla_launch_count() -> int:
     return int(lib().mla_launch_count())
+
+
+def mla_set_decode_clusters(n: int) -> None:
+    _check(lib().mla_set_decode_clusters(int(n)), "mla_set_decode_clusters")
 
 
 def mla_set_wait_limit(spins: int) -> None:

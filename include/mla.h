@@ -191,10 +191,15 @@ MLA_API int32_t mla_linear(int32_t dtype, const void* x, const void* w, int64_t 
  */
 MLA_API int32_t mla_check_status(void* stream, int32_t* device_status);
 
+/* Tuning hook: number of 2-CTA clusters the tensor-core decode spreads its work over (0 = one per
+ * pair of SMs, the default). Affects only the work split, never the result beyond rounding. */
+MLA_API int32_t mla_set_decode_clusters(int32_t n);
+
 /* Number of kernels this library has launched in this process (all devices, all streams). */
 MLA_API int64_t mla_launch_count(void);
 
-/* Test hook: spin limit of the bounded device waits (0 restores the default). */
+/* Test hook: time limit, in nanoseconds of the device's global timer, of every bounded device-side
+ * wait (0 restores the default of 2 s). */
 MLA_API int32_t mla_set_wait_limit(int64_t spins);
 
 #ifdef __cplusplus

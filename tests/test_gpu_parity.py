@@ -255,3 +255,36 @@ def test_gated_shape_examples_on_gpu(shape, L, H, causal):
     y_ref, c_ref = O.gated_mla(gp.x, gp.wq, gp.wc, gp.wk, gp.wv, gp.wg, gp.wo, H, causal)
     assert tuple(r["output"].shape) == shape and tuple(r["latent_cache"].shape) == (shape[0], shape[1], L)
     assert_close(host(r["output"]), y_ref, "f32", "output")
+
+
+@pytest.mark.parametrize("dtype,m,n,k,flags", [
+    ("bf16", 7, 128, 64, 0), ("bf16", 300, 256, 192, M.MLA_LINEAR_SIGMOID), ("bf16", 64, 5120, 1024, 0),
+    ("bf16", 513, 512, 2048, 0), ("f32", 5, 33, 17, M.MLA_LINEAR_SIGMOID), ("bf16", 3, 40, 24, 0)])
+def test_linear(dtype, m, n, k, flags):
+    rng = np.random.default_rng(m * 1000 + n)
+    x = I.round_to(rng.standard_normal((m, k)).astype(np.float32), dtype)
+    w = I.round_to((rng.standard_normal((n, k)) / math.sqrt(k)).astype(np.float32), dtype)
+    y = torch.empty(m, n, dtype=dev(x, dtype).dtype, device="cuda")
+    M.mla_linear(dev(x, dtype), dev(w, dtype), m, n, k, flags, y)
+    torch.cuda.synchronize()
+    ref = O.linear(x, w, sigmoid_out=bool(flags & M.MLA_LINEAR_SIGMOID))
+    assert_close(host(y), ref, dtype, "linear")
+
+
+@pytest.mark.parametrize("rows,D", [(64, 5120), (5, 256), (130, 1024)])
+def test_out_project_bf16(rows, D):
+    H, dc, dv = 128, 512, 128
+    rng = np.random.default_rng(rows + D)
+    out_lat = rng.standard_normal((rows, H, dc)).astype(np.float32)
+    w_uv = I.round_to((rng.standard_normal((H, dv, dc)) / math.sqrt(dc)).astype(np.float32), "bf16")
+    w_o = I.round_to((rng.standard_normal((D, H * dv)) / math.sqrt(H * dv)).astype(np.float32), "bf16")
+    gate = I.round_to(rng.random((rows, H * dv)).astype(np.float32), "bf16")
+    d = M.dims(H, dc, 64, 128, dv, D)
+    for g in (None, gate):
+        y = torch.empty(rows, D, dtype=torch.bfloat16, device="cuda")
+        ws = M.workspace(M.mla_out_project_workspace_size(d, torch.bfloat16, rows), "cuda")
+        M.mla_out_project(d, dev(out_lat), dev(w_uv, "bf16"), dev(w_o, "bf16"),
+                          None if g is None else dev(g, "bf16"), rows, y, ws)
+        torch.cuda.synchronize()
+        ref = O.out_project(out_lat, w_uv, w_o, g)
+        assert_close(host(y), ref, "bf16", "y")
