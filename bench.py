@@ -410,9 +410,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=WORKLOAD["batch"],
+                    help="sequences per step (default 64: the benchmark workload; smaller batches "
+                         "are for profiling captures and are not benchmark numbers)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
+    if args.batch != WORKLOAD["batch"]:
+        WORKLOAD["batch"] = args.batch
+        CONFIG["batch"] = args.batch
+        CONFIG["workload"] += f" [batch reduced to {args.batch}: profiling case, not the benchmark]"
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -40,10 +40,11 @@ namespace mla {
 using namespace sm100;
 
 constexpr int DEC_BT = 64;          // positions per tile
-constexpr int DEC_THREADS = 256;
+constexpr int DEC_THREADS = 384;   // warp 0 TMA, warp 1 MMA, warps 4-7 and 8-11 softmax
 constexpr int DEC_DC = 512;         // latent width handled by this kernel
 constexpr int DEC_HALF = 256;       // latent columns per CTA
 constexpr int DEC_ROWS = 128;       // rows per block
+constexpr int DEC_PREFETCH = 4;     // tiles brought into L2 beyond the shared-memory ring
 
 template <int DR>
 struct DecCfg {
@@ -52,13 +53,14 @@ struct DecCfg {
   static constexpr int K_BOX = DEC_BT * 128;            // 64 rows x 128 B
   static constexpr int Q_BYTES = KA_MAX * Q_BOX;
   static constexpr int STAGE_BYTES = KA_MAX * K_BOX;
-  static constexpr int STAGES = DR == 0 ? 3 : 2;
-  static constexpr int X_SLOT = DEC_ROWS * DEC_BT * 4;  // one partial S tile, fp32
+  static constexpr int STAGES = DR == 0 ? 4 : 3;
+  static constexpr int X_WG = DEC_ROWS * 32 * 2;         // one warpgroup's partial scores, fp16
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = Q_BYTES;
   static constexpr int OFF_X = OFF_K + STAGES * STAGE_BYTES;
-  static constexpr int OFF_BAR = OFF_X + 2 * X_SLOT;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int OFF_BAR = OFF_X + 2 * X_WG;
+  static constexpr int OFF_RED = OFF_BAR + 256;          // row maxima [2][2][128], row sums [2][128]
+  static constexpr int SMEM = OFF_RED + 6 * DEC_ROWS * 4 + 1024;
 };
 
 struct DecParams {
@@ -173,7 +175,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + Cfg::OFF_Q;
   uint8_t* sK = smem + Cfg::OFF_K;
-  float* sX = reinterpret_cast<float*>(smem + Cfg::OFF_X);
+  uint8_t* sX = smem + Cfg::OFF_X;
+  float* red = reinterpret_cast<float*>(smem + Cfg::OFF_RED);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint64_t* k_full = bars;
   uint64_t* k_empty = k_full + ST;
@@ -182,9 +185,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
   uint64_t* s_full = q_empty + 1;     // [2]
   uint64_t* p_full = s_full + 2;      // [2]
   uint64_t* o_done = p_full + 2;      // [1]
-  uint64_t* x_full = o_done + 1;      // [2]
-  uint64_t* x_empty = x_full + 2;     // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x_empty + 2);
+  uint64_t* x_full = o_done + 1;      // [2] per softmax warpgroup
+  uint64_t* x_empty = x_full + 2;     // [2] per softmax warpgroup
+  uint64_t* drain = x_empty + 2;      // [1] MMA drain on abort
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -203,11 +207,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
-      mbar_init(&x_full[s], 128);
-      mbar_init(&x_empty[s], 128);
+      mbar_init(&p_full[s], 2);       // one arrival per softmax warpgroup
+      mbar_init(&x_full[s], 1);       // [warpgroup]
+      mbar_init(&x_empty[s], 1);      // [warpgroup]
     }
     mbar_init(o_done, 1);
+    mbar_init(drain, 1);
+    // arm the first use of each exchange buffer: one local arrival plus the peer's 8 KB of stores
+    for (int s = 0; s < 2; ++s) mbar_arrive_expect_tx(&x_full[s], Cfg::X_WG);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tq);
@@ -255,6 +262,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           ok = false;
           break;
         }
+        if (tt == 0) {
+          // the first tiles of a segment: warm L2 for the loads that follow the shared-memory ring
+          for (int pt = ST; pt < ST + DEC_PREFETCH && pt < ntl; ++pt)
+            for (int kb = 0; kb < KA; ++kb)
+              tma_prefetch_2d(&tk, dim0 + kb * 64, (int)(sstart + (int64_t)(tile0 + pt) * DEC_BT));
+        }
+        if (tt + ST + DEC_PREFETCH < ntl) {
+          const int yp = (int)(sstart + (int64_t)(tile0 + tt + ST + DEC_PREFETCH) * DEC_BT);
+          for (int kb = 0; kb < KA; ++kb) tma_prefetch_2d(&tk, dim0 + kb * 64, yp);
+        }
         uint8_t* dst = sK + s * Cfg::STAGE_BYTES;
         mbar_arrive_expect_tx(&k_full[s], KA * Cfg::K_BOX);
         const int y = (int)(sstart + (int64_t)(tile0 + tt) * DEC_BT);
@@ -273,78 +290,129 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------- MMA issuer -------------------------------
+    // An event loop: P.C of the oldest tile whose P is ready is issued first (it frees a shared
+    // memory stage for the producer), and QK^T of the next tile as soon as its cache tile has landed
+    // and its S/P slot is free (the P.C two tiles back has been issued; MMAs run in issue order).
     constexpr uint32_t idesc_qk = idesc_bf16_f32(128, DEC_BT, false, false);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, DEC_HALF, false, true);
     const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK);
-    int64_t g = 0;
-    int seg = 0;
-    bool have_prev = false, prev_first = false;
-    int64_t prev_g = 0;
+    const int64_t n_total = u1 - u0;
+    int64_t gq = 0, gp = 0;               // next tile for QK^T, next tile for P.C
+    int64_t qseg_start = 0, qseg_end = 0; // tiles [start, end) of the segment QK^T is in
+    int segq = -1;
+    bool q_loaded = false;
+    int64_t useg = u0;
+    int kseg = u0 < u1 ? find_block(p.prefix, p.nblocks, u0) : 0;
+    uint32_t first_bits = 0;              // bit (g & 31): tile g opens its segment
+    uint32_t idle = 0;
+    uint64_t t_idle = 0;
     bool ok = true;
-    auto issue_pv = [&](int64_t pg, bool first) -> bool {
-      const int sl = (int)(pg & 1);
-      if (*abort_flag || !mbar_wait(&p_full[sl], (int)(pg >> 1) & 1, p.wait_ns, p.status)) return false;
-      tc_fence_after();
-      const int s = (int)(pg % ST);
-      const uint32_t c_base = k_base + s * Cfg::STAGE_BYTES;
-#pragma unroll
-      for (int kk = 0; kk < DEC_BT / 16; ++kk) {
-        const uint64_t bd = smem_desc_sw128(c_base + kk * 2048, Cfg::K_BOX, 1024);
-        mma_bf16_ts(tO, tS + sl * 64 + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
-      }
-      mma_commit(&k_empty[s]);
-      mma_commit(o_done);
-      return true;
-    };
-    int64_t u = u0;
-    int k = u0 < u1 ? find_block(p.prefix, p.nblocks, u0) : 0;
-    while (u < u1 && ok) {
-      const int64_t bend = p.prefix[k + 1];
-      const int64_t send = u1 < bend ? u1 : bend;
-      const int ntl = (int)(send - u);
-      if (*abort_flag || !mbar_wait(q_full, seg & 1, p.wait_ns, p.status)) { ok = false; break; }
-      tc_fence_after();
-      for (int tt = 0; tt < ntl; ++tt, ++g) {
-        const int s = (int)(g % ST);
-        const int sl = (int)(g & 1);
-        if (*abort_flag || !mbar_wait(&k_full[s], (int)(g / ST) & 1, p.wait_ns, p.status)) { ok = false; break; }
+    while (gp < n_total) {
+      if (*abort_flag) { ok = false; break; }
+      bool progressed = false;
+      if (gp < gq && mbar_test_wait(&p_full[gp & 1], (uint32_t)(gp >> 1) & 1u)) {
         tc_fence_after();
-        const uint32_t kst = k_base + s * Cfg::STAGE_BYTES;
-        for (int kb = 0; kb < KA; ++kb) {
+        const int sl = (int)(gp & 1);
+        const int s = (int)(gp % ST);
+        const bool first = (first_bits >> (gp & 31)) & 1u;
+        const uint32_t c_base = k_base + s * Cfg::STAGE_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = smem_desc_sw128(q_base + kb * Cfg::Q_BOX + kk * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(kst + kb * Cfg::K_BOX + kk * 32, 16, 1024);
-            mma_bf16_ss(tS + sl * 64, ad, bd, idesc_qk, (kb | kk) ? 1u : 0u);
-          }
+        for (int kk = 0; kk < DEC_BT / 16; ++kk) {
+          const uint64_t bd = smem_desc_sw128(c_base + kk * 2048, Cfg::K_BOX, 1024);
+          mma_bf16_ts(tO, tS + sl * 64 + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
         }
-        mma_commit(&s_full[sl]);
-        if (tt == ntl - 1) mma_commit(q_empty);
-        if (have_prev && !issue_pv(prev_g, prev_first)) { ok = false; break; }
-        have_prev = true;
-        prev_g = g;
-        prev_first = (tt == 0);
+        mma_commit(&k_empty[s]);
+        mma_commit(o_done);
+        ++gp;
+        progressed = true;
       }
-      u = send;
-      ++seg;
-      if (u < u1) k = find_block(p.prefix, p.nblocks, u);
+      if (gq < n_total && gq <= gp + 1) {
+        if (gq == qseg_end) {
+          const int64_t bend = p.prefix[kseg + 1];
+          const int64_t send = u1 < bend ? u1 : bend;
+          qseg_start = gq;
+          qseg_end = gq + (send - useg);
+          ++segq;
+          q_loaded = false;
+          useg = send;
+          if (useg < u1) kseg = find_block(p.prefix, p.nblocks, useg);
+        }
+        if (!q_loaded && mbar_test_wait(q_full, (uint32_t)segq & 1u)) {
+          tc_fence_after();
+          q_loaded = true;
+        }
+        const int s = (int)(gq % ST);
+        if (q_loaded && mbar_test_wait(&k_full[s], (uint32_t)(gq / ST) & 1u)) {
+          tc_fence_after();
+          const int sl = (int)(gq & 1);
+          const uint32_t kst = k_base + s * Cfg::STAGE_BYTES;
+          for (int kb = 0; kb < KA; ++kb) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = smem_desc_sw128(q_base + kb * Cfg::Q_BOX + kk * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(kst + kb * Cfg::K_BOX + kk * 32, 16, 1024);
+              mma_bf16_ss(tS + sl * 64, ad, bd, idesc_qk, (kb | kk) ? 1u : 0u);
+            }
+          }
+          mma_commit(&s_full[sl]);
+          if (gq + 1 == qseg_end) mma_commit(q_empty);
+          const uint32_t bit = 1u << (gq & 31);
+          first_bits = (gq == qseg_start) ? (first_bits | bit) : (first_bits & ~bit);
+          ++gq;
+          progressed = true;
+        }
+      }
+      if (progressed) {
+        idle = 0;
+      } else {
+        if (idle == 0) t_idle = globaltimer_ns();
+        if ((++idle & 63u) == 0 && globaltimer_ns() - t_idle > p.wait_ns) {
+          report_timeout(p.status);
+          ok = false;
+          break;
+        }
+      }
     }
-    if (ok && have_prev) ok = issue_pv(prev_g, prev_first);
-    if (!ok) *abort_flag = 1;
+    if (!ok) {
+      *abort_flag = 1;
+      // every MMA issued so far must finish before TMEM is released
+      mma_commit(drain);
+      (void)mbar_wait(drain, 0, drain_ns, p.status);
+    }
   } else if (warp >= 4) {
     // ---------------------- softmax, exchange and epilogue ----------------------
-    const int row = tid - 128;                         // TMEM lane = block row
-    const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
-    const uint32_t x_local = smem_u32(sX);
+    // Two warpgroups share every tile: warpgroup wg owns score columns [32 wg, 32 wg + 32) of each
+    // row (thread = row = TMEM lane), packed P columns [16 wg, 16 wg + 16) and O columns
+    // [128 wg, 128 wg + 128). They meet once per tile to agree on the row maximum.
+    const int wg = (warp - 4) >> 2;
+    const int quarter = (warp - 4) & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t bar_wg = 1 + wg;                       // named barrier of this warpgroup
+    const uint32_t x_local = smem_u32(sX + wg * Cfg::X_WG);
     const uint32_t x_remote = map_to_cta(x_local, peer);
-    const uint32_t xf_remote = map_to_cta(smem_u32(x_full), peer);
-    const uint32_t xe_remote = map_to_cta(smem_u32(x_empty), peer);
+    const uint32_t xf_remote = map_to_cta(smem_u32(&x_full[wg]), peer);
+    const uint32_t xe_remote = map_to_cta(smem_u32(&x_empty[wg]), peer);
+    const uint32_t xrow = (uint32_t)(row * 64);           // 32 fp16 per row, 4 chunks of 16 B
+    const int swz = (row >> 1) & 3;                       // chunk swizzle against bank conflicts
+    float* mx = red;                                      // [2 tiles][2 warpgroups][128]
+    float* lx = red + 4 * DEC_ROWS;                       // [2 warpgroups][128]
     int64_t g = 0, pv_waited = 0;
     int seg = 0;
     int64_t u = u0;
     int k = u0 < u1 ? find_block(p.prefix, p.nblocks, u0) : 0;
-    bool ok = true;
-    while (u < u1 && ok) {
+    // A wait that gives up sets the abort flag; from then on every wait is skipped but the loop
+    // structure is walked unchanged, so that all threads keep meeting the same named barriers and
+    // warp-collective TMEM instructions (no thread is left waiting).
+    auto wait_cta = [&](uint64_t* bar, int parity) {
+      if (*abort_flag) return;
+      if (!mbar_wait(bar, (uint32_t)parity, p.wait_ns, p.status)) *abort_flag = 1;
+    };
+    auto wait_cluster = [&](uint64_t* bar, int parity) {
+      if (*abort_flag) return;
+      if (!mbar_wait_cluster(bar, (uint32_t)parity, p.wait_ns, p.status)) *abort_flag = 1;
+    };
+    while (u < u1) {
       const int64_t bstart = p.prefix[k], bend = p.prefix[k + 1];
       const int64_t send = u1 < bend ? u1 : bend;
       const int tile0 = (int)(u - bstart), ntl = (int)(send - u);
@@ -362,117 +430,136 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           cnt = cnt < 0 ? 0 : (cnt > T ? T : cnt);
         }
       }
-      float m_ref = -INFINITY, l = 0.f;
+      float m_ref = -INFINITY, l = 0.f;     // reference maximum (log2 units), this group's sum
       for (int tt = 0; tt < ntl; ++tt, ++g) {
         const int sl = (int)(g & 1);
-        const int use = (int)(g >> 1);
-        if (*abort_flag || !mbar_wait(&s_full[sl], use & 1, p.wait_ns, p.status)) { ok = false; break; }
+        wait_cta(&s_full[sl], (int)(g >> 1) & 1);
         tc_fence_after();
-        float s[DEC_BT];
+        uint32_t h[16];   // this CTA's partial scores, rounded to fp16 pairs
         {
           uint32_t r[32];
-          tmem_ld32(tS + lane_off + sl * 64, r);
+          tmem_ld32(tS + lane_off + sl * 64 + wg * 32, r);
           tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(r[c]);
-          tmem_ld32(tS + lane_off + sl * 64 + 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) s[32 + c] = __uint_as_float(r[c]);
-        }
-        // exchange the partial scores with the peer CTA (16-byte chunks, XOR-swizzled by row)
-        if (use >= 1 && !mbar_wait_cluster(&x_empty[sl], (use - 1) & 1, p.wait_ns, p.status)) { ok = false; break; }
-        const uint32_t xrow_r = x_remote + (uint32_t)(sl * Cfg::X_SLOT + row * DEC_BT * 4);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const uint32_t chunk = (uint32_t)(c ^ (row & 7));
-          st_cluster_v4(xrow_r + chunk * 16, s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
-        }
-        mbar_arrive_remote(xf_remote + sl * 8);
-        if (!mbar_wait_cluster(&x_full[sl], use & 1, p.wait_ns, p.status)) { ok = false; break; }
-        {
-          const float4* xr = reinterpret_cast<const float4*>(sX + sl * (Cfg::X_SLOT / 4) + row * DEC_BT);
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const float4 v = xr[c ^ (row & 7)];
-            s[4 * c] += v.x;
-            s[4 * c + 1] += v.y;
-            s[4 * c + 2] += v.z;
-            s[4 * c + 3] += v.w;
+            __half2 v = __floats2half2_rn(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1]));
+            h[c] = *reinterpret_cast<uint32_t*>(&v);
           }
         }
-        mbar_arrive_remote(xe_remote + sl * 8);
-        // scale (log2 domain), mask, running maximum
-        const int t0 = (tile0 + tt) * DEC_BT;
-        float mx = -INFINITY;
+        // exchange: asynchronous stores into the peer's buffer complete its armed barrier
+        if (g >= 1) wait_cluster(&x_empty[wg], (int)((g - 1) & 1));
 #pragma unroll
-        for (int c = 0; c < DEC_BT; ++c) {
-          const float v = (t0 + c < cnt) ? s[c] * p.scale_log2 : -INFINITY;
-          s[c] = v;
-          mx = fmaxf(mx, v);
+        for (int c = 0; c < 4; ++c)
+          st_async_v4_b32(x_remote + xrow + (uint32_t)((c ^ swz) * 16), h[4 * c], h[4 * c + 1], h[4 * c + 2],
+                          h[4 * c + 3], xf_remote);
+        wait_cta(&x_full[wg], (int)(g & 1));
+        // S = fp16(own partial) + fp16(peer partial): the same sum in both CTAs of the pair
+        float s[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(sX + wg * Cfg::X_WG + xrow + (uint32_t)((c ^ swz) * 16));
+          const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h[4 * c + j]));
+            const float2 bq = __half22float2(*reinterpret_cast<const __half2*>(&pv[j]));
+            s[8 * c + 2 * j] = a.x + bq.x;
+            s[8 * c + 2 * j + 1] = a.y + bq.y;
+          }
         }
+        named_bar_sync(bar_wg, 128);          // every row has read the buffer
+        if (row == 0) {
+          mbar_arrive_expect_tx(&x_full[wg], Cfg::X_WG);   // re-arm for the next tile
+          mbar_arrive_remote(xe_remote);                   // the peer may refill it
+        }
+        // mask (only where the tile crosses a row's limit) and the raw row maximum
+        const int t0 = (tile0 + tt) * DEC_BT + wg * 32;
+        if (t0 + 32 > cnt) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (t0 + c >= cnt) s[c] = -INFINITY;
+        }
+        float m4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+        for (int c = 4; c < 32; c += 4) {
+          m4[0] = fmaxf(m4[0], s[c]);
+          m4[1] = fmaxf(m4[1], s[c + 1]);
+          m4[2] = fmaxf(m4[2], s[c + 2]);
+          m4[3] = fmaxf(m4[3], s[c + 3]);
+        }
+        float* mxs = mx + (g & 1) * 2 * DEC_ROWS;
+        mxs[wg * DEC_ROWS + row] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        named_bar_sync(3, 256);               // both warpgroups' maxima are in
+        const float mx_raw = fmaxf(mxs[row], mxs[DEC_ROWS + row]);
+        const float mx_t = mx_raw * p.scale_log2;   // the scale is positive: the order is kept
         bool need = false;
         float factor = 1.f;
-        if (mx > m_ref + 8.f) {
+        if (mx_t > m_ref + 8.f) {
           if (m_ref != -INFINITY) {
             need = true;
-            factor = ex2(m_ref - mx);
+            factor = ex2(m_ref - mx_t);
             l *= factor;
           }
-          m_ref = mx;
+          m_ref = mx_t;
         }
         const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-        float sum = 0.f;
-        uint32_t pk[32];
+        float sum0 = 0.f, sum1 = 0.f;
+        uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float p0 = ex2(s[2 * c] - mu), p1 = ex2(s[2 * c + 1] - mu);
-          sum += p0 + p1;
-          __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-          pk[c] = *reinterpret_cast<uint32_t*>(&h);
+        for (int c = 0; c < 16; ++c) {
+          const float p0 = ex2(fmaf(s[2 * c], p.scale_log2, -mu));
+          const float p1 = ex2(fmaf(s[2 * c + 1], p.scale_log2, -mu));
+          sum0 += p0;
+          sum1 += p1;
+          __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+          pk[c] = *reinterpret_cast<uint32_t*>(&hb);
         }
-        l += sum;
-        tmem_st32(tS + lane_off + sl * 64, pk);
+        l += sum0 + sum1;
+        // P overwrites columns of S: the barrier above guarantees both groups have loaded theirs
+        tmem_st16(tS + lane_off + sl * 64 + wg * 16, pk);
         tmem_wait_st();
         // the previous tile's P.C must be done before O is touched and before this P is released
         if (g > pv_waited) {
-          if (!mbar_wait(o_done, (int)((g - 1) & 1), p.wait_ns, p.status)) { ok = false; break; }
+          wait_cta(o_done, (int)((g - 1) & 1));
           pv_waited = g;
         }
         tc_fence_after();
         if (__any_sync(0xffffffffu, need)) {
 #pragma unroll 1
-          for (int cc = 0; cc < DEC_HALF; cc += 32) {
+          for (int cc = 0; cc < DEC_HALF / 2; cc += 32) {
             uint32_t r[32];
-            tmem_ld32(tO + lane_off + cc, r);
+            tmem_ld32(tO + lane_off + wg * 128 + cc, r);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * factor);
-            tmem_st32(tO + lane_off + cc, r);
+            tmem_st32(tO + lane_off + wg * 128 + cc, r);
           }
           tmem_wait_st();
         }
         tc_fence_before();
-        mbar_arrive(&p_full[sl]);
+        named_bar_sync(bar_wg, 128);
+        if (row == 0) mbar_arrive(&p_full[sl]);
       }
-      if (!ok) break;
-      // epilogue of the segment: wait for its last P.C, then read this CTA's half of O
+      // epilogue of the segment: wait for its last P.C, then read this group's quarter of O
       if (g > pv_waited) {
-        if (!mbar_wait(o_done, (int)((g - 1) & 1), p.wait_ns, p.status)) { ok = false; break; }
+        wait_cta(o_done, (int)((g - 1) & 1));
         pv_waited = g;
       }
       tc_fence_after();
+      lx[wg * DEC_ROWS + row] = l;
+      named_bar_sync(3, 256);
+      const float ltot = lx[row] + lx[DEC_ROWS + row];
       const int64_t orow = (int64_t)b * p.n_q * p.H + ri;
       const int slot = 2 * pair + (seg == 0 ? 0 : 1);
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      float* dst = complete ? p.out_lat + orow * DEC_DC + dim0
-                            : p.o_part + ((int64_t)slot * DEC_ROWS + row) * DEC_DC + dim0;
+      const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+      float* dst = complete ? p.out_lat + orow * DEC_DC + dim0 + wg * 128
+                            : p.o_part + ((int64_t)slot * DEC_ROWS + row) * DEC_DC + dim0 + wg * 128;
       const float mul = complete ? inv : 1.f;
       const bool write = complete ? valid : true;
 #pragma unroll 1
-      for (int cc = 0; cc < DEC_HALF; cc += 32) {
+      for (int cc = 0; cc < DEC_HALF / 2; cc += 32) {
         uint32_t r[32];
-        tmem_ld32(tO + lane_off + cc, r);
+        tmem_ld32(tO + lane_off + wg * 128 + cc, r);
         tmem_wait_ld();
         if (write) {
           float4* d4 = reinterpret_cast<float4*>(dst + cc);
@@ -482,12 +569,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
                                 __uint_as_float(r[4 * c + 2]) * mul, __uint_as_float(r[4 * c + 3]) * mul);
         }
       }
-      if (rank == 0) {
+      if (rank == 0 && wg == 0) {
         if (complete) {
-          if (valid && p.lse) p.lse[orow] = l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+          if (valid && p.lse) p.lse[orow] = ltot > 0.f ? (m_ref + log2f(ltot)) * 0.69314718055994531f : -INFINITY;
         } else {
           p.m_part[(int64_t)slot * DEC_ROWS + row] = m_ref;
-          p.l_part[(int64_t)slot * DEC_ROWS + row] = l;
+          p.l_part[(int64_t)slot * DEC_ROWS + row] = ltot;
         }
       }
       tc_fence_before();
@@ -495,7 +582,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       ++seg;
       if (u < u1) k = find_block(p.prefix, p.nblocks, u);
     }
-    if (!ok) *abort_flag = 1;
   }
 
   tc_fence_before();
@@ -512,6 +598,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
 // zeros / -inf for blocks with nothing to attend to
 // ---------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
+  __shared__ int slots[256];
+  __shared__ float wts[8][256];
+  __shared__ int nsl;
   const int k = blockIdx.x;
   const int64_t bstart = p.prefix[k], bend = p.prefix[k + 1];
   const int b = k / p.nbps, rb = k % p.nbps;
@@ -530,32 +619,50 @@ __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
   const int64_t U = p.prefix[p.nblocks];
   const int p0 = find_owner(U, p.G, bstart), p1 = find_owner(U, p.G, bend - 1);
   if (p0 == p1) return;   // written whole by one cluster
+  if (threadIdx.x == 0) {
+    // the partial of cluster q for this block: its first segment (slot 2q) unless the block
+    // started inside q's range (then it is q's last segment, slot 2q + 1); clusters without work
+    // are skipped
+    int n = 0;
+    for (int q = p0; q <= p1 && n < 256; ++q) {
+      const int64_t qs = range_start(U, p.G, q);
+      if (range_start(U, p.G, q + 1) == qs) continue;
+      slots[n++] = (q == p0 && bstart > qs) ? 2 * q + 1 : 2 * q;
+    }
+    nsl = n;
+  }
+  __syncthreads();
+  const int n = nsl;
   for (int r = warp; r < DEC_ROWS; r += 8) {
     const int ri = rb * DEC_ROWS + r;
     if (ri >= rows_seq) break;
     float M = -INFINITY;
-    for (int q = p0; q <= p1; ++q) {
-      const int slot = (q == p0 && bstart > range_start(U, p.G, q)) ? 2 * q + 1 : 2 * q;
-      M = fmaxf(M, p.m_part[(int64_t)slot * DEC_ROWS + r]);
-    }
+    for (int i = lane; i < n; i += 32) M = fmaxf(M, p.m_part[(int64_t)slots[i] * DEC_ROWS + r]);
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
     float L = 0.f;
-    for (int q = p0; q <= p1; ++q) {
-      const int slot = (q == p0 && bstart > range_start(U, p.G, q)) ? 2 * q + 1 : 2 * q;
-      const float m = p.m_part[(int64_t)slot * DEC_ROWS + r];
-      if (m != -INFINITY) L += ex2(m - M) * p.l_part[(int64_t)slot * DEC_ROWS + r];
+    for (int i = lane; i < n; i += 32) {
+      const float m = p.m_part[(int64_t)slots[i] * DEC_ROWS + r];
+      const float w = m == -INFINITY ? 0.f : ex2(m - M);
+      wts[warp][i] = w;
+      L += w * p.l_part[(int64_t)slots[i] * DEC_ROWS + r];
     }
-    const int64_t orow = (int64_t)b * rows_seq + ri;
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    __syncwarp();
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    for (int d = lane; d < DEC_DC; d += 32) {
-      float acc = 0.f;
-      for (int q = p0; q <= p1; ++q) {
-        const int slot = (q == p0 && bstart > range_start(U, p.G, q)) ? 2 * q + 1 : 2 * q;
-        const float m = p.m_part[(int64_t)slot * DEC_ROWS + r];
-        if (m != -INFINITY) acc += ex2(m - M) * p.o_part[((int64_t)slot * DEC_ROWS + r) * DEC_DC + d];
+    const int64_t orow = (int64_t)b * rows_seq + ri;
+    float4* dst = reinterpret_cast<float4*>(p.out_lat + orow * DEC_DC);
+    for (int d4 = lane; d4 < DEC_DC / 4; d4 += 32) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int i = 0; i < n; ++i) {
+        const float w = wts[warp][i];
+        if (w == 0.f) continue;
+        const float4 o = reinterpret_cast<const float4*>(p.o_part + ((int64_t)slots[i] * DEC_ROWS + r) * DEC_DC)[d4];
+        acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
       }
-      p.out_lat[orow * DEC_DC + d] = acc * inv;
+      dst[d4] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     }
     if (lane == 0 && p.lse) p.lse[orow] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    __syncwarp();
   }
 }
 
@@ -564,7 +671,7 @@ __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
 // ---------------------------------------------------------------------------------------------
 static int g_decode_clusters_override = 0;
 
-void set_decode_clusters(int n) { g_decode_clusters_override = n > 0 ? n : 0; }
+void set_decode_clusters(int n) { g_decode_clusters_override = n > 0 ? (n > 256 ? 256 : n) : 0; }
 
 bool tc_decode_supported(const DecodeArgs& a) {
   return a.dc == DEC_DC && (a.dr == 0 || a.dr == 64) && a.H > 0 && a.n_q > 0 && a.total_rows > 0 &&
@@ -576,12 +683,49 @@ struct TcDecodePlan {
   size_t off_prefix, off_o, off_m, off_l, total;
 };
 
+// clusters of two CTAs that can be resident at once (the kernel is persistent: more would run as a
+// second wave); computed once per device and tile variant
+static int max_active_clusters(int dr) {
+  static int cached[64][2] = {{0}};
+  const int dev = current_device();
+  const int v = dr == 0 ? 0 : 1;
+  if (dev < 0 || dev >= 64) return sm_count() / 2;
+  if (cached[dev][v] == 0) {
+    int n = 0;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
+    cfg.blockDim = dim3(DEC_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = dr == 0 ? DecCfg<0>::SMEM : DecCfg<64>::SMEM;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (dr == 0) {
+      cudaFuncSetAttribute(tc_decode_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg<0>::SMEM);
+      e = cudaOccupancyMaxActiveClusters(&n, (void*)tc_decode_kernel<0>, &cfg);
+    } else {
+      cudaFuncSetAttribute(tc_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg<64>::SMEM);
+      e = cudaOccupancyMaxActiveClusters(&n, (void*)tc_decode_kernel<64>, &cfg);
+    }
+    if (e != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();
+      n = sm_count() / 2;
+    }
+    cached[dev][v] = n;
+  }
+  return cached[dev][v];
+}
+
 static TcDecodePlan plan_tc(const DecodeArgs& a) {
   TcDecodePlan t;
   t.nbps = (int)ceil_div((int64_t)a.n_q * a.H, DEC_ROWS);
   t.nblocks = a.batch * t.nbps;
   const int64_t units_max = (int64_t)t.nblocks * std::max<int64_t>(1, ceil_div(a.max_seqlen, DEC_BT));
-  int G = sm_count() / 2;
+  int G = max_active_clusters(a.dr);
   if (g_decode_clusters_override > 0) G = g_decode_clusters_override;
   G = (int)std::max<int64_t>(1, std::min<int64_t>(G, units_max));
   t.G = G;

@@ -273,7 +273,7 @@ struct GemmPlan {
   int BN, n_tiles, m_tiles, splits, k_chunks;
 };
 
-static GemmPlan plan_gemm(int M, int N, int K, int batch) {
+static GemmPlan plan_gemm(int M, int N, int K, int batch, int max_splits) {
   GemmPlan g;
   g.BN = N <= 64 ? 64 : (N <= 128 ? 128 : 256);
   g.n_tiles = (int)ceil_div(N, g.BN);
@@ -282,13 +282,14 @@ static GemmPlan plan_gemm(int M, int N, int K, int batch) {
   const int64_t base = (int64_t)g.m_tiles * g.n_tiles * batch;
   int splits = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count() / std::max<int64_t>(base, 1),
                                                             total_chunks / 4));
+  splits = std::min(splits, std::max(1, max_splits));
   g.k_chunks = (int)ceil_div(total_chunks, splits);
   g.splits = (int)ceil_div(total_chunks, g.k_chunks);
   return g;
 }
 
 static size_t gemm_partial_bytes(int M, int N, int K, int batch) {
-  GemmPlan g = plan_gemm(M, N, K, batch);
+  GemmPlan g = plan_gemm(M, N, K, batch, 1 << 20);
   return g.splits > 1 ? round_up((size_t)g.splits * batch * N * M * sizeof(float), 256) : 0;
 }
 
@@ -313,7 +314,7 @@ static int tc_gemm(const GemmOperand& A, bool a_mn, const GemmOperand& Bop, int 
                    void* out, int64_t out_sb, int64_t out_st, bool out_f32, const void* gate, int64_t gate_sb,
                    int64_t gate_st, bool sigmoid, void* partial_ws, cudaStream_t s) {
   if (M % 128 || K % 64 || N <= 0 || batch <= 0) return MLA_ERR_UNSUPPORTED;
-  const GemmPlan g = plan_gemm(M, N, K, batch);
+  const GemmPlan g = plan_gemm(M, N, K, batch, partial_ws ? (1 << 20) : 1);
   CUtensorMap ta, tb;
   {
     const uint64_t dims[3] = {A.inner, A.mid, A.outer};
