@@ -10,24 +10,27 @@
 //  * Rows: 128 consecutive rows of q_abs form one M = 128 block (all 128 heads of one query token at
 //    DeepSeek-V2 scale; 8 tokens x 16 heads in gated prefill). Every row of a block shares the key row
 //    [c_t | k_pe_t] and the value c_t, so QK^T and P.C are dense 128-row MMAs.
-//  * TMEM cannot hold O (128 x 512 fp32 = all 512 columns) next to S, so a CLUSTER OF TWO CTAs shares
-//    one block: CTA 0 owns latent dims [0, 256), CTA 1 owns [256, 512) plus the 64 rotary dims. Each
+//  * TMEM (512 columns) cannot hold O (128 x 512 fp32) next to S, so a CLUSTER OF TWO CTAs shares a
+//    block: CTA r owns latent columns [256 r, 256 r + 256) and rotary columns [512 + 32 r, +32). Each
 //    streams only its own columns of every cache tile (each cache byte crosses HBM once), computes the
-//    partial S over its columns on tcgen05 into TMEM, and the two partials are exchanged through
-//    distributed shared memory and summed (both CTAs form bit-identical S = S0 + S1). Each CTA then
-//    runs the same fp32 online softmax and accumulates its half of O = P . C in TMEM (256 columns).
-//  * P (bf16) is written back into the TMEM columns of its own S tile and used as the A operand of
-//    the P . C MMA straight from TMEM. S is double-buffered, so QK^T of tile i+1 overlaps the softmax
-//    of tile i.
+//    partial S over them, and the two partials (rounded to fp16) are exchanged through distributed
+//    shared memory; both CTAs form the same S = fp16(S0) + fp16(S1), run the same fp32 online
+//    softmax and accumulate their half of O = P . C in TMEM (256 columns).
+//  * This CTA's 256 latent columns of the query block live in TMEM (128 columns of packed bf16) and
+//    are the A operand of QK^T straight from TMEM: shared memory is left to the cache tiles (4 stages)
+//    and its bandwidth to the B operands. P (bf16) is written over its S tile and is the A operand of
+//    P . C from TMEM. TMEM: Q 128 + O 256 + two 64-column S/P slots = 512 columns.
 //  * O is rescaled only when a row's running maximum grows by more than 2^8 (the result is exact:
 //    numerator and denominator share the stale reference maximum).
 //  * Work: the (block, 64-position tile) units of all sequences are split evenly over the clusters
-//    (persistent, one cluster per SM pair). A cluster that covers a whole block writes the normalised
-//    result; split blocks leave (O, max, sum) partials that a combine kernel merges.
-//  * Warp roles per CTA (256 threads): warp 0 lane 0 issues TMA loads, warp 1 lane 0 issues MMAs,
-//    warps 4-7 (one thread per row / TMEM lane) run the softmax, the exchange and the epilogue.
+//    (persistent). A cluster that covers a whole block writes the normalised result; split blocks
+//    leave (O, max, sum) partials that a combine kernel merges.
+//  * Warp roles per CTA (512 threads): warp 0 lane 0 issues TMA loads, warp 1 lane 0 issues MMAs
+//    (event loop), warps 12-15 load the query block into TMEM and exchange the partial scores,
+//    warps 4-11 (two warpgroups, thread = row = TMEM lane) run the softmax and the epilogue.
 //  * Every wait is bounded (global-timer limit); a wait that gives up sets the library's status word,
-//    and the CTA abandons its work, drains its own TMA loads and exits through the cluster barrier.
+//    and the CTA abandons its work, drains its own TMA loads and MMAs and exits through the cluster
+//    barrier.
 #include <math.h>
 
 #include <algorithm>
@@ -40,7 +43,7 @@ namespace mla {
 using namespace sm100;
 
 constexpr int DEC_BT = 64;          // positions per tile
-constexpr int DEC_THREADS = 384;   // warp 0 TMA, warp 1 MMA, warps 4-7 and 8-11 softmax
+constexpr int DEC_THREADS = 512;   // warp 0 TMA, warp 1 MMA, warps 4-11 softmax, warps 12-15 query + exchange
 constexpr int DEC_DC = 512;         // latent width handled by this kernel
 constexpr int DEC_HALF = 256;       // latent columns per CTA
 constexpr int DEC_ROWS = 128;       // rows per block
@@ -48,22 +51,25 @@ constexpr int DEC_PREFETCH = 4;     // tiles brought into L2 beyond the shared-m
 
 template <int DR>
 struct DecCfg {
-  static constexpr int KA_MAX = 4 + DR / 64;            // 64-wide column boxes of CTA 1
-  static constexpr int Q_BOX = 128 * 128;               // 128 rows x 128 B
-  static constexpr int K_BOX = DEC_BT * 128;            // 64 rows x 128 B
-  static constexpr int Q_BYTES = KA_MAX * Q_BOX;
-  static constexpr int STAGE_BYTES = KA_MAX * K_BOX;
-  static constexpr int STAGES = DR == 0 ? 4 : 3;
-  static constexpr int X_WG = DEC_ROWS * 32 * 2;         // one warpgroup's partial scores, fp16
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = Q_BYTES;
+  static constexpr int QR_BOX = DR ? 128 * 64 : 0;      // this CTA's 32 rotary query columns, 128 x 64 B
+  static constexpr int K_BOX = DEC_BT * 128;            // 64 positions x 64 latent columns (128 B)
+  static constexpr int KR_BOX = DR ? DEC_BT * 64 : 0;   // 64 positions x 32 rotary columns (64 B)
+  static constexpr int STAGE_BYTES = 4 * K_BOX + KR_BOX;
+  static constexpr int STAGES = 4;
+  static constexpr int X_TILE = DEC_ROWS * DEC_BT * 2;   // one tile of partial scores, fp16
+  static constexpr int OFF_QR = 0;
+  static constexpr int OFF_K = QR_BOX;
   static constexpr int OFF_X = OFF_K + STAGES * STAGE_BYTES;
-  static constexpr int OFF_BAR = OFF_X + 2 * X_WG;
+  static constexpr int OFF_XS = OFF_X + 2 * X_TILE;      // two receive slots, then the send staging
+  static constexpr int OFF_BAR = OFF_XS + X_TILE;
   static constexpr int OFF_RED = OFF_BAR + 256;          // row maxima [2][2][128], row sums [2][128]
   static constexpr int SMEM = OFF_RED + 6 * DEC_ROWS * 4 + 1024;
 };
 
 struct DecParams {
+  const __nv_bfloat16* q_abs;  // [q_rows][W]
+  int64_t q_rows;
+  int W;
   const int32_t* cu;
   int32_t batch, n_q, H, nbps, nblocks;
   int64_t total_rows;
@@ -167,27 +173,29 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecParams p, int32_t*
 // ---------------------------------------------------------------------------------------------
 template <int DR>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
-    tc_decode_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                     DecParams p) {
+    tc_decode_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tkr,
+                     const __grid_constant__ CUtensorMap tqr, DecParams p) {
   using Cfg = DecCfg<DR>;
   constexpr int ST = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem + Cfg::OFF_Q;
+  uint8_t* sQR = smem + Cfg::OFF_QR;
   uint8_t* sK = smem + Cfg::OFF_K;
   uint8_t* sX = smem + Cfg::OFF_X;
   float* red = reinterpret_cast<float*>(smem + Cfg::OFF_RED);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
-  uint64_t* k_full = bars;
-  uint64_t* k_empty = k_full + ST;
-  uint64_t* q_full = k_empty + ST;
-  uint64_t* q_empty = q_full + 1;
-  uint64_t* s_full = q_empty + 1;     // [2]
-  uint64_t* p_full = s_full + 2;      // [2]
-  uint64_t* o_done = p_full + 2;      // [1]
-  uint64_t* x_full = o_done + 1;      // [2] per softmax warpgroup
-  uint64_t* x_empty = x_full + 2;     // [2] per softmax warpgroup
-  uint64_t* drain = x_empty + 2;      // [1] MMA drain on abort
+  uint64_t* k_full = bars;              // [ST] cache tile landed
+  uint64_t* k_empty = k_full + ST;      // [ST] cache tile consumed by its P.C
+  uint64_t* qr_full = k_empty + ST;     // rotary query columns landed (TMA)
+  uint64_t* ql_full = qr_full + 1;      // latent query columns written to TMEM (query warps)
+  uint64_t* q_empty = ql_full + 1;      // last QK^T of a segment done: the query may be replaced
+  uint64_t* s_full = q_empty + 1;       // [2] partial S of a slot computed (MMA -> exchange)
+  uint64_t* s_sum = s_full + 2;         // [2] summed S written back (exchange -> softmax)
+  uint64_t* p_full = s_sum + 2;         // [2] P written (softmax -> MMA)
+  uint64_t* o_done = p_full + 2;        // [1] a P.C completed
+  uint64_t* x_full = o_done + 1;        // [2] peer's partial scores arrived (transaction count)
+  uint64_t* x_empty = x_full + 2;       // [2] peer has read this CTA's scores
+  uint64_t* drain = x_empty + 2;        // [1] MMA drain on abort
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -195,30 +203,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
   const int pair = blockIdx.x >> 1;
-  const int KA = rank == 0 ? 4 : 4 + DR / 64;
-  const int dim0 = rank == 0 ? 0 : DEC_HALF;
+  const int dim0 = rank == 0 ? 0 : DEC_HALF;           // first latent column of this CTA
+  const int rdim0 = DEC_DC + (int)rank * (DR / 2);     // first rotary column of this CTA
 
   if (tid == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
     }
-    mbar_init(q_full, 1);
+    mbar_init(qr_full, 1);
+    mbar_init(ql_full, 1);
     mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
+      mbar_init(&s_sum[s], 1);
       mbar_init(&p_full[s], 2);       // one arrival per softmax warpgroup
-      mbar_init(&x_full[s], 1);       // [warpgroup]
-      mbar_init(&x_empty[s], 1);      // [warpgroup]
+      mbar_init(&x_full[s], 1);
+      mbar_init(&x_empty[s], 1);
     }
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
-    // arm the first use of each exchange buffer: one local arrival plus the peer's 8 KB of stores
-    for (int s = 0; s < 2; ++s) mbar_arrive_expect_tx(&x_full[s], Cfg::X_WG);
+    // arm the first use of each receive slot: one local arrival plus the peer's 16 KB of stores
+    for (int s = 0; s < 2; ++s) mbar_arrive_expect_tx(&x_full[s], Cfg::X_TILE);
     *abort_flag = 0;
     fence_mbar_init();
-    prefetch_tmap(&tq);
     prefetch_tmap(&tk);
+    if (DR) {
+      prefetch_tmap(&tkr);
+      prefetch_tmap(&tqr);
+    }
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
@@ -226,14 +239,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
-  cluster_sync();           // the peer's barriers are initialised before any remote arrive
+  cluster_sync();           // the peer's barriers are initialised before any remote access
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tO = tmem;               // columns [0, 256): this CTA's half of O
-  const uint32_t tS = tmem + 256;         // columns [256, 384): two 64-column S / P tiles
+  const uint32_t tQ = tmem;               // columns [0, 128): this CTA's latent query columns, bf16 pairs
+  const uint32_t tO = tmem + 128;         // columns [128, 384): this CTA's half of O
+  const uint32_t tS = tmem + 384;         // columns [384, 512): two 64-column S / P slots
 
   const int64_t U = p.prefix[p.nblocks];
   const int64_t u0 = range_start(U, p.G, pair), u1 = range_start(U, p.G, pair + 1);
+  const int64_t n_total = u1 - u0;
   const int64_t drain_ns = p.wait_ns > 100000000ull ? p.wait_ns : 100000000ull;
 
   if (warp == 0 && lane == 0) {
@@ -251,31 +266,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       const int b = k / p.nbps, rb = k % p.nbps;
       int64_t sstart; int T;
       seq_bounds(p, b, sstart, T);
-      const int qrow = (int)((int64_t)b * p.n_q * p.H + (int64_t)rb * DEC_ROWS);
-      if (seg > 0 && (*abort_flag || !mbar_wait(q_empty, (seg - 1) & 1, p.wait_ns, p.status))) { ok = false; break; }
-      mbar_arrive_expect_tx(q_full, KA * Cfg::Q_BOX);
-      for (int kb = 0; kb < KA; ++kb) tma_load_2d(sQ + kb * Cfg::Q_BOX, &tq, q_full, dim0 + kb * 64, qrow);
-      ++q_loads;
+      if (DR) {
+        const int qrow = (int)((int64_t)b * p.n_q * p.H + (int64_t)rb * DEC_ROWS);
+        if (seg > 0 && (*abort_flag || !mbar_wait(q_empty, (seg - 1) & 1, p.wait_ns, p.status))) { ok = false; break; }
+        mbar_arrive_expect_tx(qr_full, Cfg::QR_BOX);
+        tma_load_2d(sQR, &tqr, qr_full, rdim0, qrow);
+        ++q_loads;
+      }
       for (int tt = 0; tt < ntl; ++tt, ++g) {
         const int s = (int)(g % ST);
         if (g >= ST && (*abort_flag || !mbar_wait(&k_empty[s], (int)((g / ST) - 1) & 1, p.wait_ns, p.status))) {
           ok = false;
           break;
         }
-        if (tt == 0) {
-          // the first tiles of a segment: warm L2 for the loads that follow the shared-memory ring
-          for (int pt = ST; pt < ST + DEC_PREFETCH && pt < ntl; ++pt)
-            for (int kb = 0; kb < KA; ++kb)
-              tma_prefetch_2d(&tk, dim0 + kb * 64, (int)(sstart + (int64_t)(tile0 + pt) * DEC_BT));
-        }
-        if (tt + ST + DEC_PREFETCH < ntl) {
-          const int yp = (int)(sstart + (int64_t)(tile0 + tt + ST + DEC_PREFETCH) * DEC_BT);
-          for (int kb = 0; kb < KA; ++kb) tma_prefetch_2d(&tk, dim0 + kb * 64, yp);
+        if (tt == 0 || tt + ST + DEC_PREFETCH - 1 < ntl) {
+          // warm L2 for the tiles after the shared-memory ring
+          const int first = tt == 0 ? ST : ST + DEC_PREFETCH - 1;
+          for (int pt = tt + first; pt < tt + ST + DEC_PREFETCH && pt < ntl; ++pt) {
+            const int yp = (int)(sstart + (int64_t)(tile0 + pt) * DEC_BT);
+            for (int kb = 0; kb < 4; ++kb) tma_prefetch_2d(&tk, dim0 + kb * 64, yp);
+            if (DR) tma_prefetch_2d(&tkr, rdim0, yp);
+          }
         }
         uint8_t* dst = sK + s * Cfg::STAGE_BYTES;
-        mbar_arrive_expect_tx(&k_full[s], KA * Cfg::K_BOX);
+        mbar_arrive_expect_tx(&k_full[s], Cfg::STAGE_BYTES);
         const int y = (int)(sstart + (int64_t)(tile0 + tt) * DEC_BT);
-        for (int kb = 0; kb < KA; ++kb) tma_load_2d(dst + kb * Cfg::K_BOX, &tk, &k_full[s], dim0 + kb * 64, y);
+        for (int kb = 0; kb < 4; ++kb) tma_load_2d(dst + kb * Cfg::K_BOX, &tk, &k_full[s], dim0 + kb * 64, y);
+        if (DR) tma_load_2d(dst + 4 * Cfg::K_BOX, &tkr, &k_full[s], rdim0, y);
       }
       u = send;
       ++seg;
@@ -286,21 +303,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       // drain this CTA's own loads in flight before the shared memory is released
       for (int64_t i = (g > ST ? g - ST : 0); i < g; ++i)
         (void)mbar_wait(&k_full[i % ST], (int)(i / ST) & 1, drain_ns, p.status);
-      if (q_loads > 0) (void)mbar_wait(q_full, (q_loads - 1) & 1, drain_ns, p.status);
+      if (q_loads > 0) (void)mbar_wait(qr_full, (q_loads - 1) & 1, drain_ns, p.status);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------- MMA issuer -------------------------------
     // An event loop: P.C of the oldest tile whose P is ready is issued first (it frees a shared
-    // memory stage for the producer), and QK^T of the next tile as soon as its cache tile has landed
-    // and its S/P slot is free (the P.C two tiles back has been issued; MMAs run in issue order).
+    // memory stage for the producer), and QK^T of the next tile as soon as its cache tile has landed,
+    // its query is in place and its S/P slot is free (the P.C two tiles back has been issued; MMAs
+    // run in issue order).
     constexpr uint32_t idesc_qk = idesc_bf16_f32(128, DEC_BT, false, false);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, DEC_HALF, false, true);
-    const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK);
-    const int64_t n_total = u1 - u0;
+    const uint32_t qr_base = smem_u32(sQR), k_base = smem_u32(sK);
     int64_t gq = 0, gp = 0;               // next tile for QK^T, next tile for P.C
     int64_t qseg_start = 0, qseg_end = 0; // tiles [start, end) of the segment QK^T is in
     int segq = -1;
-    bool q_loaded = false;
+    bool ql_ok = false, qr_ok = false;
     int64_t useg = u0;
     int kseg = u0 < u1 ? find_block(p.prefix, p.nblocks, u0) : 0;
     uint32_t first_bits = 0;              // bit (g & 31): tile g opens its segment
@@ -315,6 +332,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         const int sl = (int)(gp & 1);
         const int s = (int)(gp % ST);
         const bool first = (first_bits >> (gp & 31)) & 1u;
+        // B = this CTA's 256 latent columns of the tile: MN-major, 64-column boxes K_BOX apart
         const uint32_t c_base = k_base + s * Cfg::STAGE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < DEC_BT / 16; ++kk) {
@@ -333,25 +351,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           qseg_start = gq;
           qseg_end = gq + (send - useg);
           ++segq;
-          q_loaded = false;
+          ql_ok = false;
+          qr_ok = !DR;
           useg = send;
           if (useg < u1) kseg = find_block(p.prefix, p.nblocks, useg);
         }
-        if (!q_loaded && mbar_test_wait(q_full, (uint32_t)segq & 1u)) {
+        if (!ql_ok && mbar_test_wait(ql_full, (uint32_t)segq & 1u)) {
           tc_fence_after();
-          q_loaded = true;
+          ql_ok = true;
         }
+        if (!qr_ok && mbar_test_wait(qr_full, (uint32_t)segq & 1u)) qr_ok = true;
         const int s = (int)(gq % ST);
-        if (q_loaded && mbar_test_wait(&k_full[s], (uint32_t)(gq / ST) & 1u)) {
+        if (ql_ok && qr_ok && mbar_test_wait(&k_full[s], (uint32_t)(gq / ST) & 1u)) {
           tc_fence_after();
           const int sl = (int)(gq & 1);
           const uint32_t kst = k_base + s * Cfg::STAGE_BYTES;
-          for (int kb = 0; kb < KA; ++kb) {
+          for (int kb = 0; kb < 4; ++kb) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = smem_desc_sw128(q_base + kb * Cfg::Q_BOX + kk * 32, 16, 1024);
               const uint64_t bd = smem_desc_sw128(kst + kb * Cfg::K_BOX + kk * 32, 16, 1024);
-              mma_bf16_ss(tS + sl * 64, ad, bd, idesc_qk, (kb | kk) ? 1u : 0u);
+              mma_bf16_ts(tS + sl * 64, tQ + kb * 32 + kk * 8, bd, idesc_qk, (kb | kk) ? 1u : 0u);
+            }
+          }
+          if (DR) {
+            // this CTA's 32 rotary columns: rows of 64 B, 8-row groups 512 B apart
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              const uint64_t ad = smem_desc_sw64(qr_base + kk * 32, 16, 512);
+              const uint64_t bd = smem_desc_sw64(kst + 4 * Cfg::K_BOX + kk * 32, 16, 512);
+              mma_bf16_ss(tS + sl * 64, ad, bd, idesc_qk, 1u);
             }
           }
           mma_commit(&s_full[sl]);
@@ -379,8 +407,140 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       mma_commit(drain);
       (void)mbar_wait(drain, 0, drain_ns, p.status);
     }
+  } else if (warp >= 12) {
+    // ------------------------- query loads and score exchange -------------------------
+    // Thread = row = TMEM lane. At each segment: this CTA's 256 latent query columns of the block's
+    // row are read from global memory and stored into TMEM (after the previous segment's last QK^T).
+    // For each tile: load this CTA's partial scores (64 columns), round them to fp16 and send them to
+    // the peer (asynchronous stores completing the peer's armed barrier); then add the peer's fp16
+    // partials and write the summed scores back into the same TMEM slot. Both CTAs form
+    // S = fp16(S0) + fp16(S1) identically. Tile g+1 is sent before tile g is received.
+    const int quarter = warp - 12;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t x_remote = map_to_cta(smem_u32(sX), peer);
+    const uint32_t xf_remote = map_to_cta(smem_u32(x_full), peer);
+    const uint32_t xe_remote = map_to_cta(smem_u32(x_empty), peer);
+    const uint32_t xrow = (uint32_t)(row * 128);          // 64 fp16 per row: 8 chunks of 16 B
+    const int swz = row & 7;                              // chunk swizzle against bank conflicts
+    auto wait_cta = [&](uint64_t* bar, int parity) {
+      if (*abort_flag) return;
+      if (!mbar_wait(bar, (uint32_t)parity, p.wait_ns, p.status)) *abort_flag = 1;
+    };
+    // segment walker: the tile index at which the next segment starts, and its block
+    int64_t useg = u0;
+    int kseg = u0 < u1 ? find_block(p.prefix, p.nblocks, u0) : 0;
+    int64_t next_seg_tile = 0;
+    int seg_loaded = 0;
+    auto load_query = [&]() {
+      // the block of the segment starting at tile next_seg_tile
+      const int64_t bend = p.prefix[kseg + 1];
+      const int64_t send = u1 < bend ? u1 : bend;
+      const int b = kseg / p.nbps, rb = kseg % p.nbps;
+      const int64_t qr = (int64_t)b * p.n_q * p.H + (int64_t)rb * DEC_ROWS + row;
+      if (seg_loaded > 0) wait_cta(q_empty, (seg_loaded - 1) & 1);
+      tc_fence_after();
+      const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + qr * p.W + dim0);
+      const bool in = qr < p.q_rows;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {   // 4 x 32 TMEM columns = 256 bf16
+        uint32_t r[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint4 v = in ? src[cc * 8 + j] : make_uint4(0u, 0u, 0u, 0u);
+          r[4 * j] = v.x; r[4 * j + 1] = v.y; r[4 * j + 2] = v.z; r[4 * j + 3] = v.w;
+        }
+        tmem_st32(tQ + lane_off + cc * 32, r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      named_bar_sync(4, 128);
+      if (row == 0) mbar_arrive(ql_full);
+      ++seg_loaded;
+      next_seg_tile += send - useg;
+      useg = send;
+      if (useg < u1) kseg = find_block(p.prefix, p.nblocks, useg);
+    };
+    uint8_t* staging = smem + Cfg::OFF_XS;
+    uint32_t h_next[32];
+    auto send = [&](int64_t gs) {
+      const int sl = (int)(gs & 1);
+      wait_cta(&s_full[sl], (int)(gs >> 1) & 1);
+      tc_fence_after();
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r[32];
+        tmem_ld32(tS + lane_off + sl * 64 + half * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          __half2 v = __floats2half2_rn(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1]));
+          h_next[half * 16 + c] = *reinterpret_cast<uint32_t*>(&v);
+        }
+      }
+      // the previous bulk copy has finished reading the staging buffer
+      if (row == 0) bulk_wait_group_read<0>();
+      named_bar_sync(5, 128);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(staging + xrow + ((c ^ swz) * 16)) =
+            make_uint4(h_next[4 * c], h_next[4 * c + 1], h_next[4 * c + 2], h_next[4 * c + 3]);
+      fence_proxy_async_smem();             // generic writes -> visible to the bulk copy
+      named_bar_sync(5, 128);
+      const int xs = (int)(gs & 1);
+      if (row == 0) {
+        if (gs >= 2) wait_cta(&x_empty[xs], (int)((gs >> 1) - 1) & 1);
+        // one bulk copy of the whole tile into the peer's receive slot
+        bulk_copy_to_cta(x_remote + (uint32_t)(xs * Cfg::X_TILE), staging, Cfg::X_TILE, xf_remote + xs * 8);
+        bulk_commit_group();
+      }
+    };
+    if (n_total > 0) {
+      load_query();
+      send(0);
+    }
+    for (int64_t g = 0; g < n_total; ++g) {
+      const int sl = (int)(g & 1);
+      uint32_t h[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) h[c] = h_next[c];
+      if (g + 1 < n_total) {
+        if (g + 1 == next_seg_tile) load_query();
+        send(g + 1);
+      }
+      const int xs = (int)(g & 1);
+      wait_cta(&x_full[xs], (int)(g >> 1) & 1);
+      const uint8_t* xr = sX + xs * Cfg::X_TILE + xrow;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int cc = half * 4 + c;
+          const uint4 v = *reinterpret_cast<const uint4*>(xr + (cc ^ swz) * 16);
+          const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h[4 * cc + j]));
+            const float2 bq = __half22float2(*reinterpret_cast<const __half2*>(&pv[j]));
+            r[8 * c + 2 * j] = __float_as_uint(a.x + bq.x);
+            r[8 * c + 2 * j + 1] = __float_as_uint(a.y + bq.y);
+          }
+        }
+        tmem_st32(tS + lane_off + sl * 64 + half * 32, r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      named_bar_sync(5, 128);               // every row has read the slot and written its S
+      if (row == 0) {
+        mbar_arrive_expect_tx(&x_full[xs], Cfg::X_TILE);   // re-arm for its next use
+        mbar_arrive_remote(xe_remote + xs * 8);             // the peer may refill the slot
+        mbar_arrive(&s_sum[sl]);
+      }
+    }
+    if (row == 0) bulk_wait_group_read<0>();   // the staging buffer is read before the CTA exits
   } else if (warp >= 4) {
-    // ---------------------- softmax, exchange and epilogue ----------------------
+    // ---------------------------- softmax and epilogue ----------------------------
     // Two warpgroups share every tile: warpgroup wg owns score columns [32 wg, 32 wg + 32) of each
     // row (thread = row = TMEM lane), packed P columns [16 wg, 16 wg + 16) and O columns
     // [128 wg, 128 wg + 128). They meet once per tile to agree on the row maximum.
@@ -389,12 +549,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t bar_wg = 1 + wg;                       // named barrier of this warpgroup
-    const uint32_t x_local = smem_u32(sX + wg * Cfg::X_WG);
-    const uint32_t x_remote = map_to_cta(x_local, peer);
-    const uint32_t xf_remote = map_to_cta(smem_u32(&x_full[wg]), peer);
-    const uint32_t xe_remote = map_to_cta(smem_u32(&x_empty[wg]), peer);
-    const uint32_t xrow = (uint32_t)(row * 64);           // 32 fp16 per row, 4 chunks of 16 B
-    const int swz = (row >> 1) & 3;                       // chunk swizzle against bank conflicts
     float* mx = red;                                      // [2 tiles][2 warpgroups][128]
     float* lx = red + 4 * DEC_ROWS;                       // [2 warpgroups][128]
     int64_t g = 0, pv_waited = 0;
@@ -408,15 +562,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       if (*abort_flag) return;
       if (!mbar_wait(bar, (uint32_t)parity, p.wait_ns, p.status)) *abort_flag = 1;
     };
-    auto wait_cluster = [&](uint64_t* bar, int parity) {
-      if (*abort_flag) return;
-      if (!mbar_wait_cluster(bar, (uint32_t)parity, p.wait_ns, p.status)) *abort_flag = 1;
-    };
     while (u < u1) {
       const int64_t bstart = p.prefix[k], bend = p.prefix[k + 1];
-      const int64_t send = u1 < bend ? u1 : bend;
-      const int tile0 = (int)(u - bstart), ntl = (int)(send - u);
-      const bool complete = (u == bstart) && (send == bend);
+      const int64_t send_u = u1 < bend ? u1 : bend;
+      const int tile0 = (int)(u - bstart), ntl = (int)(send_u - u);
+      const bool complete = (u == bstart) && (send_u == bend);
       const int b = k / p.nbps, rb = k % p.nbps;
       int64_t sstart; int T;
       seq_bounds(p, b, sstart, T);
@@ -433,44 +583,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       float m_ref = -INFINITY, l = 0.f;     // reference maximum (log2 units), this group's sum
       for (int tt = 0; tt < ntl; ++tt, ++g) {
         const int sl = (int)(g & 1);
-        wait_cta(&s_full[sl], (int)(g >> 1) & 1);
+        wait_cta(&s_sum[sl], (int)(g >> 1) & 1);
         tc_fence_after();
-        uint32_t h[16];   // this CTA's partial scores, rounded to fp16 pairs
+        float s[32];
         {
           uint32_t r[32];
           tmem_ld32(tS + lane_off + sl * 64 + wg * 32, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            __half2 v = __floats2half2_rn(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1]));
-            h[c] = *reinterpret_cast<uint32_t*>(&v);
-          }
-        }
-        // exchange: asynchronous stores into the peer's buffer complete its armed barrier
-        if (g >= 1) wait_cluster(&x_empty[wg], (int)((g - 1) & 1));
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          st_async_v4_b32(x_remote + xrow + (uint32_t)((c ^ swz) * 16), h[4 * c], h[4 * c + 1], h[4 * c + 2],
-                          h[4 * c + 3], xf_remote);
-        wait_cta(&x_full[wg], (int)(g & 1));
-        // S = fp16(own partial) + fp16(peer partial): the same sum in both CTAs of the pair
-        float s[32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 v = *reinterpret_cast<const uint4*>(sX + wg * Cfg::X_WG + xrow + (uint32_t)((c ^ swz) * 16));
-          const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h[4 * c + j]));
-            const float2 bq = __half22float2(*reinterpret_cast<const __half2*>(&pv[j]));
-            s[8 * c + 2 * j] = a.x + bq.x;
-            s[8 * c + 2 * j + 1] = a.y + bq.y;
-          }
-        }
-        named_bar_sync(bar_wg, 128);          // every row has read the buffer
-        if (row == 0) {
-          mbar_arrive_expect_tx(&x_full[wg], Cfg::X_WG);   // re-arm for the next tile
-          mbar_arrive_remote(xe_remote);                   // the peer may refill it
+          for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(r[c]);
         }
         // mask (only where the tile crosses a row's limit) and the raw row maximum
         const int t0 = (tile0 + tt) * DEC_BT + wg * 32;
@@ -489,7 +610,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         }
         float* mxs = mx + (g & 1) * 2 * DEC_ROWS;
         mxs[wg * DEC_ROWS + row] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        named_bar_sync(3, 256);               // both warpgroups' maxima are in
+        named_bar_sync(3, 256);               // both warpgroups' maxima are in (and S is loaded)
         const float mx_raw = fmaxf(mxs[row], mxs[DEC_ROWS + row]);
         const float mx_t = mx_raw * p.scale_log2;   // the scale is positive: the order is kept
         bool need = false;
@@ -578,7 +699,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         }
       }
       tc_fence_before();
-      u = send;
+      u = send_u;
       ++seg;
       if (u < u1) k = find_block(p.prefix, p.nblocks, u);
     }
@@ -602,12 +723,13 @@ __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
   __shared__ float wts[8][256];
   __shared__ int nsl;
   const int k = blockIdx.x;
+  const int r0 = blockIdx.y * 8;     // this CTA's 8 rows of the block (one per warp)
   const int64_t bstart = p.prefix[k], bend = p.prefix[k + 1];
   const int b = k / p.nbps, rb = k % p.nbps;
   const int rows_seq = p.n_q * p.H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (bend == bstart) {
-    for (int r = warp; r < DEC_ROWS; r += 8) {
+    for (int r = r0 + warp; r < r0 + 8; r += 8) {
       const int ri = rb * DEC_ROWS + r;
       if (ri >= rows_seq) break;
       const int64_t orow = (int64_t)b * rows_seq + ri;
@@ -633,7 +755,7 @@ __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
   }
   __syncthreads();
   const int n = nsl;
-  for (int r = warp; r < DEC_ROWS; r += 8) {
+  for (int r = r0 + warp; r < r0 + 8; r += 8) {
     const int ri = rb * DEC_ROWS + r;
     if (ri >= rows_seq) break;
     float M = -INFINITY;
@@ -725,7 +847,12 @@ static TcDecodePlan plan_tc(const DecodeArgs& a) {
   t.nbps = (int)ceil_div((int64_t)a.n_q * a.H, DEC_ROWS);
   t.nblocks = a.batch * t.nbps;
   const int64_t units_max = (int64_t)t.nblocks * std::max<int64_t>(1, ceil_div(a.max_seqlen, DEC_BT));
-  int G = max_active_clusters(a.dr);
+  const int maxc = max_active_clusters(a.dr);
+  int G = maxc;
+  // Equal-length sequences with one row block each: give every block the same number of clusters
+  // (no block is split unevenly and, with one cluster per block, no partials are written at all).
+  const bool equal_blocks = a.total_rows == (int64_t)a.batch * a.max_seqlen && (!a.causal || t.nbps == 1);
+  if (equal_blocks && t.nblocks <= maxc) G = t.nblocks * (maxc / t.nblocks);
   if (g_decode_clusters_override > 0) G = g_decode_clusters_override;
   G = (int)std::max<int64_t>(1, std::min<int64_t>(G, units_max));
   t.G = G;
@@ -740,7 +867,8 @@ static TcDecodePlan plan_tc(const DecodeArgs& a) {
 size_t tc_decode_workspace(const DecodeArgs& a) { return plan_tc(a).total; }
 
 template <int DR>
-static int launch_decode_t(const CUtensorMap& tq, const CUtensorMap& tk, const DecParams& p, cudaStream_t s) {
+static int launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tkr, const CUtensorMap& tqr,
+                           const DecParams& p, cudaStream_t s) {
   static bool attr_set[64] = {false};
   const int dev = current_device();
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
@@ -749,7 +877,7 @@ static int launch_decode_t(const CUtensorMap& tq, const CUtensorMap& tk, const D
       return MLA_ERR_CUDA;
     attr_set[dev] = true;
   }
-  tc_decode_kernel<DR><<<2 * p.G, DEC_THREADS, DecCfg<DR>::SMEM, s>>>(tq, tk, p);
+  tc_decode_kernel<DR><<<2 * p.G, DEC_THREADS, DecCfg<DR>::SMEM, s>>>(tk, tkr, tqr, p);
   MLA_LAUNCH_CHECK();
   return MLA_OK;
 }
@@ -759,6 +887,9 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
   const int W = a.dc + a.dr;
   char* ws = static_cast<char*>(a.workspace);
   DecParams p{};
+  p.q_abs = static_cast<const __nv_bfloat16*>(a.q_abs);
+  p.q_rows = (int64_t)a.batch * a.n_q * a.H;
+  p.W = W;
   p.cu = a.cu_seqlens; p.batch = a.batch; p.n_q = a.n_q; p.H = a.H; p.nbps = t.nbps; p.nblocks = t.nblocks;
   p.total_rows = a.total_rows; p.causal = a.causal ? 1 : 0;
   p.scale_log2 = a.scale * 1.4426950408889634f;
@@ -773,13 +904,7 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
   if (!p.status) return MLA_ERR_CUDA;
   if (t.nblocks == 0) return MLA_OK;
 
-  CUtensorMap tq, tk;
-  {
-    const uint64_t dims[2] = {(uint64_t)W, (uint64_t)a.batch * a.n_q * a.H};
-    const uint64_t st[1] = {(uint64_t)W * 2};
-    const uint32_t box[2] = {64, DEC_ROWS};
-    if (!encode_tmap_bf16(&tq, const_cast<void*>(a.q_abs), 2, dims, st, box)) return MLA_ERR_CUDA;
-  }
+  CUtensorMap tk, tkr, tqr;
   {
     const uint64_t rows = (uint64_t)std::max<int64_t>(a.total_rows, 1);
     const uint64_t dims[2] = {(uint64_t)W, rows};
@@ -787,11 +912,29 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
     const uint32_t box[2] = {64, DEC_BT};
     if (!encode_tmap_bf16(&tk, const_cast<void*>(a.cache), 2, dims, st, box)) return MLA_ERR_CUDA;
   }
+  tkr = tk;
+  tqr = tk;
+  if (a.dr) {
+    // rotary columns: boxes of 32 columns, 64-byte swizzle
+    {
+      const uint64_t rows = (uint64_t)std::max<int64_t>(a.total_rows, 1);
+      const uint64_t dims[2] = {(uint64_t)W, rows};
+      const uint64_t st[1] = {(uint64_t)W * 2};
+      const uint32_t box[2] = {32, DEC_BT};
+      if (!encode_tmap_bf16(&tkr, const_cast<void*>(a.cache), 2, dims, st, box, 64)) return MLA_ERR_CUDA;
+    }
+    {
+      const uint64_t dims[2] = {(uint64_t)W, (uint64_t)a.batch * a.n_q * a.H};
+      const uint64_t st[1] = {(uint64_t)W * 2};
+      const uint32_t box[2] = {32, DEC_ROWS};
+      if (!encode_tmap_bf16(&tqr, const_cast<void*>(a.q_abs), 2, dims, st, box, 64)) return MLA_ERR_CUDA;
+    }
+  }
   decode_plan_kernel<<<1, 1024, 0, s>>>(p, const_cast<int32_t*>(p.prefix));
   MLA_LAUNCH_CHECK();
-  int st = a.dr == 0 ? launch_decode_t<0>(tq, tk, p, s) : launch_decode_t<64>(tq, tk, p, s);
+  int st = a.dr == 0 ? launch_decode_t<0>(tk, tkr, tqr, p, s) : launch_decode_t<64>(tk, tkr, tqr, p, s);
   if (st) return st;
-  decode_combine_tc_kernel<<<t.nblocks, 256, 0, s>>>(p);
+  decode_combine_tc_kernel<<<dim3((unsigned)t.nblocks, DEC_ROWS / 8), 256, 0, s>>>(p);
   MLA_LAUNCH_CHECK();
   return MLA_OK;
 }
