@@ -42,7 +42,23 @@ CONFIG = {
     "parallelism": "replicas (one independent decode per GPU, no collective)",
 }
 DECODE_SOURCES = ("head_latent_attention_08_b200/csrc/tc_decode.cu",
-                  "head_latent_attention_08_b200/csrc/generic.cu")
+                  "head_latent_attention_08_b200/csrc/sm100.cuh",
+                  "head_latent_attention_08_b200/csrc/common.cuh")
+
+
+def replica_seed(rank: int) -> int:
+    """Every rank decodes its own replica of the workload, drawn from its own seed."""
+    return SEED + rank
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The slowest rank sets the job's time (all ranks take part; world size 1 returns value)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def cache_bytes() -> int:
@@ -268,7 +284,7 @@ def run_ours(args):
     B, H, dc, dr, T = w["batch"], w["n_heads"], w["kv_lora_rank"], w["rope_dim"], w["seqlen"]
     p = I.decode_problem(batch=B, n_heads=H, kv_lora_rank=dc, rope_dim=dr, qk_nope=w["qk_nope"],
                          v_head=w["v_head"], d_model=w["d_model"], seqlens=[T] * B, dtype="bf16",
-                         seed=SEED + rank)
+                         seed=replica_seed(rank))
     bf = torch.bfloat16
     dev = torch.device("cuda", local)
 
@@ -322,12 +338,8 @@ def run_ours(args):
     launches = M.mla_launch_count() - launches0
     if world > 1:
         dist.barrier()
-    elapsed_ms = start.elapsed_time(stop)
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), dist if world > 1 else None, dev)
     dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
     status = M.mla_check_status()
 
     # ---- end to end through the public API with host buffers --------------------------------
@@ -358,11 +370,7 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
 
     cpu = cpu_baseline() if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
     if world > 1:

@@ -26,7 +26,7 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // ---------------------------------------------------------------------------------------------
 // Kernels with bounded waits receive the word's device address and the spin limit as parameters.
 int* device_status_ptr();        // device address of the status word on the current device
-long long wait_limit();          // spins before a bounded wait gives up
+long long wait_limit();          // nanoseconds before a bounded device wait gives up
 void set_wait_limit(long long);  // 0 restores the default
 
 __device__ __forceinline__ void report_timeout(int* status) {

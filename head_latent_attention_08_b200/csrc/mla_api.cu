@@ -297,10 +297,12 @@ int32_t mla_set_decode_clusters(int32_t n) {
 
 int64_t mla_launch_count(void) { return (int64_t)launch_count(); }
 
-int32_t mla_set_wait_limit(int64_t spins) {
-  if (spins < 0) return MLA_ERR_SHAPE;
-  set_wait_limit((long long)spins);
+int32_t mla_set_wait_limit(int64_t limit_ns) {
+  if (limit_ns < 0) return MLA_ERR_SHAPE;
+  set_wait_limit((long long)limit_ns);
   return MLA_OK;
 }
+
+int32_t mla_wait_selftest(void* stream) { return wait_selftest_launch(as_stream(stream)); }
 
 }  // extern "C"

@@ -69,9 +69,9 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns, int* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
+  for (;;) {   // each failed poll has already been suspended by the hardware: read the timer every time
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0 && globaltimer_ns() - t0 > limit_ns) {   // the timer is read every 64 polls
+    if (globaltimer_ns() - t0 > limit_ns) {
       report_timeout(status);
       return false;
     }
@@ -108,9 +108,9 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
                                                   int* status) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
+  for (;;) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((i & 63u) == 0 && globaltimer_ns() - t0 > limit_ns) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       report_timeout(status);
       return false;
     }

@@ -28,4 +28,7 @@ bool tc_linear_supported(int64_t m, int64_t n, int64_t k);
 int tc_linear(const void* x, const void* w, int64_t m, int64_t n, int64_t k, int sigmoid, void* y,
               cudaStream_t s);
 
+// one CTA waiting, through the bounded wait of the tensor-core kernels, on a barrier nothing completes
+int wait_selftest_launch(cudaStream_t s);
+
 }  // namespace mla

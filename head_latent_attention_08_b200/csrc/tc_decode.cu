@@ -60,8 +60,8 @@ struct DecCfg {
   static constexpr int OFF_QR = 0;
   static constexpr int OFF_K = QR_BOX;
   static constexpr int OFF_X = OFF_K + STAGES * STAGE_BYTES;
-  static constexpr int OFF_XS = OFF_X + 2 * X_TILE;      // two receive slots, then the send staging
-  static constexpr int OFF_BAR = OFF_XS + X_TILE;
+  static constexpr int OFF_XS = OFF_X + 2 * X_TILE;      // two receive slots, then two send stagings
+  static constexpr int OFF_BAR = OFF_XS + 2 * X_TILE;
   static constexpr int OFF_RED = OFF_BAR + 256;          // row maxima [2][2][128], row sums [2][128]
   static constexpr int SMEM = OFF_RED + 6 * DEC_ROWS * 4 + 1024;
 };
@@ -394,7 +394,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         idle = 0;
       } else {
         if (idle == 0) t_idle = globaltimer_ns();
-        if ((++idle & 63u) == 0 && globaltimer_ns() - t_idle > p.wait_ns) {
+        if ((++idle & 7u) == 0 && globaltimer_ns() - t_idle > p.wait_ns) {
           report_timeout(p.status);
           ok = false;
           break;
@@ -478,22 +478,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           h_next[half * 16 + c] = *reinterpret_cast<uint32_t*>(&v);
         }
       }
-      // the previous bulk copy has finished reading the staging buffer
-      if (row == 0) bulk_wait_group_read<0>();
+      // staging buffer xs and the peer's receive slot xs were last used by tile gs - 2: once the peer
+      // has read that tile (x_empty), its copy is complete and both may be reused
+      const int xs = (int)(gs & 1);
+      if (row == 0 && gs >= 2) wait_cta(&x_empty[xs], (int)((gs >> 1) - 1) & 1);
       named_bar_sync(5, 128);
+      uint8_t* stg = staging + xs * Cfg::X_TILE;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(staging + xrow + ((c ^ swz) * 16)) =
+        *reinterpret_cast<uint4*>(stg + xrow + ((c ^ swz) * 16)) =
             make_uint4(h_next[4 * c], h_next[4 * c + 1], h_next[4 * c + 2], h_next[4 * c + 3]);
       fence_proxy_async_smem();             // generic writes -> visible to the bulk copy
       named_bar_sync(5, 128);
-      const int xs = (int)(gs & 1);
-      if (row == 0) {
-        if (gs >= 2) wait_cta(&x_empty[xs], (int)((gs >> 1) - 1) & 1);
-        // one bulk copy of the whole tile into the peer's receive slot
-        bulk_copy_to_cta(x_remote + (uint32_t)(xs * Cfg::X_TILE), staging, Cfg::X_TILE, xf_remote + xs * 8);
-        bulk_commit_group();
-      }
+      // one bulk copy of the whole tile into the peer's receive slot, completing the peer's barrier
+      // (none once this CTA has abandoned its work: the peer's waits then run out instead)
+      if (row == 0 && !*abort_flag)
+        bulk_copy_to_cta(x_remote + (uint32_t)(xs * Cfg::X_TILE), stg, Cfg::X_TILE, xf_remote + xs * 8);
     };
     if (n_total > 0) {
       load_query();
@@ -533,12 +533,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       tc_fence_before();
       named_bar_sync(5, 128);               // every row has read the slot and written its S
       if (row == 0) {
-        mbar_arrive_expect_tx(&x_full[xs], Cfg::X_TILE);   // re-arm for its next use
-        mbar_arrive_remote(xe_remote + xs * 8);             // the peer may refill the slot
+        // Re-arm only after this thread's own wait saw the phase complete (the flag is still clear):
+        // an arrival on a phase whose arrival is already in but whose bytes are still pending would
+        // take its count below zero. After an abort neither barrier is touched again, so the peer
+        // sends nothing more into this slot.
+        if (!*abort_flag) {
+          mbar_arrive_expect_tx(&x_full[xs], Cfg::X_TILE);   // re-arm for its next use
+          mbar_arrive_remote(xe_remote + xs * 8);             // the peer may refill the slot
+        }
         mbar_arrive(&s_sum[sl]);
       }
     }
-    if (row == 0) bulk_wait_group_read<0>();   // the staging buffer is read before the CTA exits
   } else if (warp >= 4) {
     // ---------------------------- softmax and epilogue ----------------------------
     // Two warpgroups share every tile: warpgroup wg owns score columns [32 wg, 32 wg + 32) of each
@@ -706,6 +711,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
   }
 
   tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && *abort_flag) {
+    // abandoned work: let any bulk copy already issued between the pair land before either CTA
+    // leaves (in normal operation every copy has been consumed before this point)
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 1000000ull) {
+    }
+  }
   __syncthreads();
   cluster_sync();     // the peer may write into this CTA's exchange buffer until it is done
   if (warp == 0) {

@@ -186,6 +186,7 @@ __global__ void __launch_bounds__(128, 1)
 
   // epilogue: 128 threads, thread = accumulator row
   const bool ok = mbar_wait(done, 0, p.wait_ns, p.status);
+  if (!ok) *abort_flag = 1;
   tc_fence_after();
   const bool write = ok && !*abort_flag;
   const int m = m0 + warp * 32 + lane;
@@ -215,9 +216,13 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 0 && lane == 0 && *abort_flag) {
-    // do not leave TMA writes in flight behind an abandoned CTA: wait (bounded) for the loads
+    // Abandoned work: neither TMA writes nor MMAs may be left in flight behind the CTA or its tensor
+    // memory. Every load issued and the MMA issuer's final commit (made on both of its paths, before
+    // the barrier above) complete by themselves; the limit here only bounds the wait.
+    const uint64_t drain_ns = p.wait_ns > 100000000ull ? p.wait_ns : 100000000ull;
     for (int i = max(0, issued - STAGES); i < issued; ++i)
-      (void)mbar_wait(&full[i % STAGES], (i / STAGES) & 1, p.wait_ns, p.status);
+      (void)mbar_wait(&full[i % STAGES], (i / STAGES) & 1, drain_ns, p.status);
+    (void)mbar_wait(done, 0, drain_ns, p.status);
   }
   __syncthreads();
   if (warp == 0) {

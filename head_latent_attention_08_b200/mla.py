@@ -23,13 +23,13 @@ MLA_ABSORB_QUERY, MLA_FOLD_QK, MLA_FOLD_VO = 0, 1, 2
 MLA_APPEND_NORM, MLA_APPEND_ROPE = 1, 2
 MLA_DECODE_CAUSAL = 1
 MLA_LINEAR_SIGMOID, MLA_LINEAR_W_KN = 1, 2
-MLA_ERR_TIMEOUT = 7
+MLA_ERR_SHAPE, MLA_ERR_TIMEOUT = 2, 7
 
 EXPORTED = (
     "mla_status_string", "mla_abi_version", "mla_append_latent", "mla_absorb_weights",
     "mla_decode_workspace_size", "mla_decode_absorbed", "mla_out_project_workspace_size",
     "mla_out_project", "mla_linear", "mla_check_status", "mla_set_wait_limit", "mla_launch_count",
-    "mla_set_decode_clusters",
+    "mla_set_decode_clusters", "mla_wait_selftest",
 )
 
 
@@ -70,6 +70,7 @@ _SIGS = {
     "mla_set_wait_limit": (_I32, [_I64]),
     "mla_launch_count": (_I64, []),
     "mla_set_decode_clusters": (_I32, [_I32]),
+    "mla_wait_selftest": (_I32, [_P]),
 }
 
 
@@ -203,8 +204,12 @@ def mla_set_decode_clusters(n: int) -> None:
     _check(lib().mla_set_decode_clusters(int(n)), "mla_set_decode_clusters")
 
 
-def mla_set_wait_limit(spins: int) -> None:
-    _check(lib().mla_set_wait_limit(int(spins)), "mla_set_wait_limit")
+def mla_set_wait_limit(limit_ns: int) -> None:
+    _check(lib().mla_set_wait_limit(int(limit_ns)), "mla_set_wait_limit")
+
+
+def mla_wait_selftest(stream=None) -> None:
+    _check(lib().mla_wait_selftest(_stream(stream)), "mla_wait_selftest")
 
 
 # --------------------------------------------------------------------------------------------

@@ -199,8 +199,19 @@ MLA_API int32_t mla_set_decode_clusters(int32_t n);
 MLA_API int64_t mla_launch_count(void);
 
 /* Test hook: time limit, in nanoseconds of the device's global timer, of every bounded device-side
- * wait (0 restores the default of 2 s). */
-MLA_API int32_t mla_set_wait_limit(int64_t spins);
+ * wait (0 restores the default of 2 s; negative: MLA_ERR_SHAPE). Applies to kernels launched after
+ * the call. A wait that runs out sets MLA_ERR_TIMEOUT in the status word and its kernel abandons its
+ * work (outputs undefined) after its own copies and tensor-core operations in flight have ended. */
+MLA_API int32_t mla_set_wait_limit(int64_t limit_ns);
+
+/*
+ * mla_wait_selftest -- diagnostic with no counterpart in the method: launches one CTA on `stream`
+ * that allocates tensor memory, waits on an mbarrier that nothing completes (through the same
+ * bounded wait as the tensor-core kernels), gives up after the current wait limit, releases its
+ * tensor memory and returns. The status word then reads MLA_ERR_TIMEOUT (mla_check_status) and the
+ * context stays usable. Returns MLA_ERR_CUDA if the launch fails.
+ */
+MLA_API int32_t mla_wait_selftest(void* stream);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,76 @@
+"""Failure detection without a GPU fault: every device-side wait of the tensor-core kernels is bounded
+by a global-timer limit. A wait that runs out sets MLA_ERR_TIMEOUT in the status word, its kernel
+abandons its work after its own copies and MMAs in flight have ended, and the context stays usable.
+The case here waits on a barrier nothing completes, so its wait certainly runs out."""
+import numpy as np
+import pytest
+import torch
+
+from head_latent_attention_08_b200 import mla as M
+from head_latent_attention_08_b200 import inputs as I
+from oracle import mla_oracle as O
+from gpu_helpers import assert_close, dev, host, mla_dims_of
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from head_latent_attention_08_b200 import build
+    build.build()
+    M.lib()
+
+
+def _small_decode_is_correct():
+    p = I.decode_problem(batch=2, n_heads=128, kv_lora_rank=512, rope_dim=64, qk_nope=128, v_head=128,
+                         d_model=128, seqlens=[200, 65], dtype="bf16", seed=33)
+    d = mla_dims_of(p)
+    q_abs = dev(O.absorb_query(p.q_nope, p.q_pe, p.w_uk), "bf16")
+    cache = dev(p.cache, "bf16")
+    cu = torch.from_numpy(p.cu_seqlens.astype(np.int32)).cuda()
+    out = torch.empty(2, 128, 512, device="cuda")
+    ws = M.workspace(M.mla_decode_workspace_size(d, torch.bfloat16, 2, 1, 200, cache.shape[0], 1), "cuda")
+    M.mla_decode_absorbed(d, q_abs, cache, cu, 2, 1, 200, M.MLA_DECODE_CAUSAL, out, None, ws)
+    assert M.mla_check_status() == M.MLA_OK
+    ref, _ = O.decode_absorbed(O.store_as(O.absorb_query(p.q_nope, p.q_pe, p.w_uk), "bf16"), p.cache,
+                               p.cu_seqlens, 1, 512, p.kq_scale, True)
+    assert_close(host(out), ref, "bf16", "out_lat")
+
+
+def test_wait_on_a_barrier_nothing_completes_runs_out():
+    assert M.mla_check_status() == M.MLA_OK
+    limit_ns = 2_000_000
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    try:
+        M.mla_set_wait_limit(limit_ns)
+        ev0.record()
+        M.mla_wait_selftest()
+        ev1.record()
+        torch.cuda.synchronize()
+    finally:
+        M.mla_set_wait_limit(0)
+    assert M.mla_check_status() == M.MLA_ERR_TIMEOUT
+    assert M.mla_check_status() == M.MLA_OK          # reading the status clears it
+    ms = ev0.elapsed_time(ev1)
+    assert limit_ns * 1e-6 <= ms < 1000.0, ms         # it waited its limit, and no longer than bounded
+    _small_decode_is_correct()
+
+
+def test_negative_wait_limit_is_rejected():
+    with pytest.raises(M.MLAError):
+        M.mla_set_wait_limit(-1)
+
+
+def test_out_of_range_append_row_is_skipped_and_reported():
+    p = I.decode_problem(batch=1, n_heads=2, kv_lora_rank=16, rope_dim=8, qk_nope=8, v_head=8, d_model=8,
+                         seqlens=[4], dtype="f32", seed=32, with_weights=False)
+    cache = dev(p.cache)
+    before = cache.clone()
+    rows = torch.tensor([4], dtype=torch.int64, device="cuda")      # one past the end
+    M.mla_append_latent(mla_dims_of(p), cache, rows, dev(p.c_new), dev(p.kpe_new),
+                        torch.from_numpy(p.positions).cuda(), 0)
+    torch.cuda.synchronize()
+    assert M.mla_check_status() == M.MLA_ERR_SHAPE
+    assert torch.equal(cache, before)
