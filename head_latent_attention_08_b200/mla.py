@@ -29,7 +29,7 @@ EXPORTED = (
     "mla_status_string", "mla_abi_version", "mla_append_latent", "mla_absorb_weights",
     "mla_decode_workspace_size", "mla_decode_absorbed", "mla_out_project_workspace_size",
     "mla_out_project", "mla_linear", "mla_check_status", "mla_set_wait_limit", "mla_launch_count",
-    "mla_set_decode_clusters", "mla_wait_selftest",
+    "mla_set_decode_clusters", "mla_wait_selftest", "mla_decode_absorbed_noalloc",
 )
 
 
@@ -71,6 +71,8 @@ _SIGS = {
     "mla_launch_count": (_I64, []),
     "mla_set_decode_clusters": (_I32, [_I32]),
     "mla_wait_selftest": (_I32, [_P]),
+    "mla_decode_absorbed_noalloc": (_I32, [_DIMS, _I32, _P, _P, _P, _I32, _I32, _I64, _I64, _U32, _P, _P,
+                                           _P]),
 }
 
 
@@ -166,6 +168,19 @@ def mla_decode_absorbed(d: mla_dims, q_abs: torch.Tensor, cache: torch.Tensor, c
                                      _ptr(cu_seqlens), batch, n_q, max_seqlen, cache.shape[0], flags,
                                      _ptr(out_lat), _ptr(lse), _ptr(workspace), ws_bytes,
                                      _stream(stream)), "mla_decode_absorbed")
+
+
+MLA_DECODE_NOALLOC_MAX_BYTES = 40 << 20
+
+
+def mla_decode_absorbed_noalloc(d: mla_dims, q_abs: torch.Tensor, cache: torch.Tensor,
+                                cu_seqlens: torch.Tensor, batch: int, n_q: int, max_seqlen: int, flags: int,
+                                out_lat: torch.Tensor, lse: Optional[torch.Tensor], stream=None) -> None:
+    assert cu_seqlens.dtype == torch.int32 and out_lat.dtype == torch.float32
+    _check(lib().mla_decode_absorbed_noalloc(ctypes.byref(d), _dtype_code(q_abs.dtype), _ptr(q_abs),
+                                             _ptr(cache), _ptr(cu_seqlens), batch, n_q, max_seqlen,
+                                             cache.shape[0], flags, _ptr(out_lat), _ptr(lse),
+                                             _stream(stream)), "mla_decode_absorbed_noalloc")
 
 
 def mla_out_project_workspace_size(d: mla_dims, dtype: torch.dtype, n_rows: int) -> int:

@@ -213,6 +213,25 @@ MLA_API int32_t mla_set_wait_limit(int64_t limit_ns);
  */
 MLA_API int32_t mla_wait_selftest(void* stream);
 
+/*
+ * mla_decode_absorbed_noalloc -- an addition of this library with no counterpart in the method: the
+ * same decode as mla_decode_absorbed (same arguments, layouts and results), with its scratch in a
+ * fixed array of MLA_DECODE_NOALLOC_MAX_BYTES inside the library's device image instead of a
+ * caller workspace. It allocates no memory (no cudaMalloc / cudaFree, no allocating library call);
+ * the array's address is looked up once per device, with that device current.
+ *   Errors: those of mla_decode_absorbed; MLA_ERR_WORKSPACE when the problem needs more scratch than
+ *   MLA_DECODE_NOALLOC_MAX_BYTES (mla_decode_workspace_size reports the need); MLA_ERR_CUDA when the
+ *   array's address cannot be obtained.
+ *   Nothing in the scratch has to start at zero. All calls on one device share the one array: calls
+ *   whose executions overlap on the GPU (different streams without ordering between them) race on
+ *   it and give undefined results; calls ordered on one stream do not.
+ */
+#define MLA_DECODE_NOALLOC_MAX_BYTES ((size_t)40 << 20)
+MLA_API int32_t mla_decode_absorbed_noalloc(const mla_dims* dims, int32_t dtype, const void* q_abs,
+                                            const void* cache, const int32_t* cu_seqlens, int32_t batch,
+                                            int32_t n_q, int64_t max_seqlen, int64_t total_rows,
+                                            uint32_t flags, float* out_lat, float* lse, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
