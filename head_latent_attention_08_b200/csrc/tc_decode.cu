@@ -25,9 +25,12 @@
 //  * Work: the (block, 64-position tile) units of all sequences are split evenly over the clusters
 //    (persistent). A cluster that covers a whole block writes the normalised result; split blocks
 //    leave (O, max, sum) partials that a combine kernel merges.
-//  * Warp roles per CTA (512 threads): warp 0 lane 0 issues TMA loads, warp 1 lane 0 issues MMAs
-//    (event loop), warps 12-15 load the query block into TMEM and exchange the partial scores,
-//    warps 4-11 (two warpgroups, thread = row = TMEM lane) run the softmax and the epilogue.
+//  * Warp roles per CTA (384 threads): warp 0 lane 0 issues TMA loads, warp 1 lane 0 issues MMAs
+//    (event loop), warps 4-11 form two softmax warpgroups (thread = row = TMEM lane). Warpgroup wg
+//    owns score columns [32 wg, 32 wg + 32) of every tile: it rounds its partial scores to fp16,
+//    sends them to the same warpgroup of the peer CTA with one bulk copy, adds the peer's half of
+//    the same columns and runs the softmax. The two warpgroups meet once per tile for the row
+//    maximum. They also load the query block into TMEM at each segment and run the epilogue.
 //  * Every wait is bounded (global-timer limit); a wait that gives up sets the library's status word,
 //    and the CTA abandons its work, drains its own TMA loads and MMAs and exits through the cluster
 //    barrier.
@@ -43,7 +46,7 @@ namespace mla {
 using namespace sm100;
 
 constexpr int DEC_BT = 64;          // positions per tile
-constexpr int DEC_THREADS = 512;   // warp 0 TMA, warp 1 MMA, warps 4-11 softmax, warps 12-15 query + exchange
+constexpr int DEC_THREADS = 384;   // warp 0 TMA, warp 1 MMA, warps 4-11 query, exchange and softmax
 constexpr int DEC_DC = 512;         // latent width handled by this kernel
 constexpr int DEC_HALF = 256;       // latent columns per CTA
 constexpr int DEC_ROWS = 128;       // rows per block
@@ -56,11 +59,12 @@ struct DecCfg {
   static constexpr int KR_BOX = DR ? DEC_BT * 64 : 0;   // 64 positions x 32 rotary columns (64 B)
   static constexpr int STAGE_BYTES = 4 * K_BOX + KR_BOX;
   static constexpr int STAGES = 4;
-  static constexpr int X_TILE = DEC_ROWS * DEC_BT * 2;   // one tile of partial scores, fp16
+  static constexpr int X_HALF = DEC_ROWS * 32 * 2;       // one warpgroup's 32 partial-score columns, fp16
+  static constexpr int X_TILE = 2 * X_HALF;
   static constexpr int OFF_QR = 0;
   static constexpr int OFF_K = QR_BOX;
   static constexpr int OFF_X = OFF_K + STAGES * STAGE_BYTES;
-  static constexpr int OFF_XS = OFF_X + 2 * X_TILE;      // two receive slots, then two send stagings
+  static constexpr int OFF_XS = OFF_X + 2 * X_TILE;      // receive slots [2][2 wg], then send stagings [2][2 wg]
   static constexpr int OFF_BAR = OFF_XS + 2 * X_TILE;
   static constexpr int OFF_RED = OFF_BAR + 256;          // row maxima [2][2][128], row sums [2][128]
   static constexpr int SMEM = OFF_RED + 6 * DEC_ROWS * 4 + 1024;
@@ -189,13 +193,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
   uint64_t* qr_full = k_empty + ST;     // rotary query columns landed (TMA)
   uint64_t* ql_full = qr_full + 1;      // latent query columns written to TMEM (query warps)
   uint64_t* q_empty = ql_full + 1;      // last QK^T of a segment done: the query may be replaced
-  uint64_t* s_full = q_empty + 1;       // [2] partial S of a slot computed (MMA -> exchange)
-  uint64_t* s_sum = s_full + 2;         // [2] summed S written back (exchange -> softmax)
-  uint64_t* p_full = s_sum + 2;         // [2] P written (softmax -> MMA)
+  uint64_t* s_full = q_empty + 1;       // [2] partial S of a slot computed (MMA -> softmax)
+  uint64_t* p_full = s_full + 2;        // [2] P written (softmax -> MMA)
   uint64_t* o_done = p_full + 2;        // [1] a P.C completed
-  uint64_t* x_full = o_done + 1;        // [2] peer's partial scores arrived (transaction count)
-  uint64_t* x_empty = x_full + 2;       // [2] peer has read this CTA's scores
-  uint64_t* drain = x_empty + 2;        // [1] MMA drain on abort
+  uint64_t* x_full = o_done + 1;        // [2 slots][2 wg] peer's partial scores arrived (transaction count)
+  uint64_t* x_empty = x_full + 4;       // [2 slots][2 wg] peer has read this CTA's scores
+  uint64_t* drain = x_empty + 4;        // [1] MMA drain on abort
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -212,19 +215,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       mbar_init(&k_empty[s], 1);
     }
     mbar_init(qr_full, 1);
-    mbar_init(ql_full, 1);
+    mbar_init(ql_full, 2);            // one arrival per softmax warpgroup (each writes half the query)
     mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_sum[s], 1);
       mbar_init(&p_full[s], 2);       // one arrival per softmax warpgroup
+    }
+    for (int s = 0; s < 4; ++s) {
       mbar_init(&x_full[s], 1);
       mbar_init(&x_empty[s], 1);
     }
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
-    // arm the first use of each receive slot: one local arrival plus the peer's 16 KB of stores
-    for (int s = 0; s < 2; ++s) mbar_arrive_expect_tx(&x_full[s], Cfg::X_TILE);
+    // arm the first use of each receive slot: one local arrival plus the peer's 8 KB bulk copy
+    for (int s = 0; s < 4; ++s) mbar_arrive_expect_tx(&x_full[s], Cfg::X_HALF);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tk);
@@ -407,148 +411,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       mma_commit(drain);
       (void)mbar_wait(drain, 0, drain_ns, p.status);
     }
-  } else if (warp >= 12) {
-    // ------------------------- query loads and score exchange -------------------------
-    // Thread = row = TMEM lane. At each segment: this CTA's 256 latent query columns of the block's
-    // row are read from global memory and stored into TMEM (after the previous segment's last QK^T).
-    // For each tile: load this CTA's partial scores (64 columns), round them to fp16 and send them to
-    // the peer (asynchronous stores completing the peer's armed barrier); then add the peer's fp16
-    // partials and write the summed scores back into the same TMEM slot. Both CTAs form
-    // S = fp16(S0) + fp16(S1) identically. Tile g+1 is sent before tile g is received.
-    const int quarter = warp - 12;
-    const int row = quarter * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t x_remote = map_to_cta(smem_u32(sX), peer);
-    const uint32_t xf_remote = map_to_cta(smem_u32(x_full), peer);
-    const uint32_t xe_remote = map_to_cta(smem_u32(x_empty), peer);
-    const uint32_t xrow = (uint32_t)(row * 128);          // 64 fp16 per row: 8 chunks of 16 B
-    const int swz = row & 7;                              // chunk swizzle against bank conflicts
-    auto wait_cta = [&](uint64_t* bar, int parity) {
-      if (*abort_flag) return;
-      if (!mbar_wait(bar, (uint32_t)parity, p.wait_ns, p.status)) *abort_flag = 1;
-    };
-    // segment walker: the tile index at which the next segment starts, and its block
-    int64_t useg = u0;
-    int kseg = u0 < u1 ? find_block(p.prefix, p.nblocks, u0) : 0;
-    int64_t next_seg_tile = 0;
-    int seg_loaded = 0;
-    auto load_query = [&]() {
-      // the block of the segment starting at tile next_seg_tile
-      const int64_t bend = p.prefix[kseg + 1];
-      const int64_t send = u1 < bend ? u1 : bend;
-      const int b = kseg / p.nbps, rb = kseg % p.nbps;
-      const int64_t qr = (int64_t)b * p.n_q * p.H + (int64_t)rb * DEC_ROWS + row;
-      if (seg_loaded > 0) wait_cta(q_empty, (seg_loaded - 1) & 1);
-      tc_fence_after();
-      const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + qr * p.W + dim0);
-      const bool in = qr < p.q_rows;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {   // 4 x 32 TMEM columns = 256 bf16
-        uint32_t r[32];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint4 v = in ? src[cc * 8 + j] : make_uint4(0u, 0u, 0u, 0u);
-          r[4 * j] = v.x; r[4 * j + 1] = v.y; r[4 * j + 2] = v.z; r[4 * j + 3] = v.w;
-        }
-        tmem_st32(tQ + lane_off + cc * 32, r);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      named_bar_sync(4, 128);
-      if (row == 0) mbar_arrive(ql_full);
-      ++seg_loaded;
-      next_seg_tile += send - useg;
-      useg = send;
-      if (useg < u1) kseg = find_block(p.prefix, p.nblocks, useg);
-    };
-    uint8_t* staging = smem + Cfg::OFF_XS;
-    uint32_t h_next[32];
-    auto send = [&](int64_t gs) {
-      const int sl = (int)(gs & 1);
-      wait_cta(&s_full[sl], (int)(gs >> 1) & 1);
-      tc_fence_after();
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t r[32];
-        tmem_ld32(tS + lane_off + sl * 64 + half * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          __half2 v = __floats2half2_rn(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1]));
-          h_next[half * 16 + c] = *reinterpret_cast<uint32_t*>(&v);
-        }
-      }
-      // staging buffer xs and the peer's receive slot xs were last used by tile gs - 2: once the peer
-      // has read that tile (x_empty), its copy is complete and both may be reused
-      const int xs = (int)(gs & 1);
-      if (row == 0 && gs >= 2) wait_cta(&x_empty[xs], (int)((gs >> 1) - 1) & 1);
-      named_bar_sync(5, 128);
-      uint8_t* stg = staging + xs * Cfg::X_TILE;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(stg + xrow + ((c ^ swz) * 16)) =
-            make_uint4(h_next[4 * c], h_next[4 * c + 1], h_next[4 * c + 2], h_next[4 * c + 3]);
-      fence_proxy_async_smem();             // generic writes -> visible to the bulk copy
-      named_bar_sync(5, 128);
-      // one bulk copy of the whole tile into the peer's receive slot, completing the peer's barrier
-      // (none once this CTA has abandoned its work: the peer's waits then run out instead)
-      if (row == 0 && !*abort_flag)
-        bulk_copy_to_cta(x_remote + (uint32_t)(xs * Cfg::X_TILE), stg, Cfg::X_TILE, xf_remote + xs * 8);
-    };
-    if (n_total > 0) {
-      load_query();
-      send(0);
-    }
-    for (int64_t g = 0; g < n_total; ++g) {
-      const int sl = (int)(g & 1);
-      uint32_t h[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) h[c] = h_next[c];
-      if (g + 1 < n_total) {
-        if (g + 1 == next_seg_tile) load_query();
-        send(g + 1);
-      }
-      const int xs = (int)(g & 1);
-      wait_cta(&x_full[xs], (int)(g >> 1) & 1);
-      const uint8_t* xr = sX + xs * Cfg::X_TILE + xrow;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t r[32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int cc = half * 4 + c;
-          const uint4 v = *reinterpret_cast<const uint4*>(xr + (cc ^ swz) * 16);
-          const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h[4 * cc + j]));
-            const float2 bq = __half22float2(*reinterpret_cast<const __half2*>(&pv[j]));
-            r[8 * c + 2 * j] = __float_as_uint(a.x + bq.x);
-            r[8 * c + 2 * j + 1] = __float_as_uint(a.y + bq.y);
-          }
-        }
-        tmem_st32(tS + lane_off + sl * 64 + half * 32, r);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      named_bar_sync(5, 128);               // every row has read the slot and written its S
-      if (row == 0) {
-        // Re-arm only after this thread's own wait saw the phase complete (the flag is still clear):
-        // an arrival on a phase whose arrival is already in but whose bytes are still pending would
-        // take its count below zero. After an abort neither barrier is touched again, so the peer
-        // sends nothing more into this slot.
-        if (!*abort_flag) {
-          mbar_arrive_expect_tx(&x_full[xs], Cfg::X_TILE);   // re-arm for its next use
-          mbar_arrive_remote(xe_remote + xs * 8);             // the peer may refill the slot
-        }
-        mbar_arrive(&s_sum[sl]);
-      }
-    }
   } else if (warp >= 4) {
-    // ---------------------------- softmax and epilogue ----------------------------
+    // ------------------------ query, score exchange, softmax, epilogue ------------------------
     // Two warpgroups share every tile: warpgroup wg owns score columns [32 wg, 32 wg + 32) of each
     // row (thread = row = TMEM lane), packed P columns [16 wg, 16 wg + 16) and O columns
-    // [128 wg, 128 wg + 128). They meet once per tile to agree on the row maximum.
+    // [128 wg, 128 wg + 128). Per tile it rounds its partial scores to fp16, sends them to the same
+    // warpgroup of the peer CTA (one 8 KB bulk copy into the peer's receive slot, completing the
+    // peer's barrier), and adds the peer's fp16 partials of the same columns: both CTAs form
+    // S = fp16(S0) + fp16(S1) identically. The warpgroups meet once per tile on the row maximum.
     const int wg = (warp - 4) >> 2;
     const int quarter = (warp - 4) & 3;
     const int row = quarter * 32 + lane;
@@ -556,17 +426,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     const uint32_t bar_wg = 1 + wg;                       // named barrier of this warpgroup
     float* mx = red;                                      // [2 tiles][2 warpgroups][128]
     float* lx = red + 4 * DEC_ROWS;                       // [2 warpgroups][128]
+    uint8_t* staging = smem + Cfg::OFF_XS;
+    const uint32_t x_remote = map_to_cta(smem_u32(sX), peer);
+    const uint32_t xf_remote = map_to_cta(smem_u32(x_full), peer);
+    const uint32_t xe_remote = map_to_cta(smem_u32(x_empty), peer);
+    const uint32_t xrow = (uint32_t)(row * 64);           // 32 fp16 per row: 4 chunks of 16 B
+    const int swz = (row >> 1) & 3;                       // chunk swizzle against bank conflicts
     int64_t g = 0, pv_waited = 0;
     int seg = 0;
     int64_t u = u0;
     int k = u0 < u1 ? find_block(p.prefix, p.nblocks, u0) : 0;
     // A wait that gives up sets the abort flag; from then on every wait is skipped but the loop
     // structure is walked unchanged, so that all threads keep meeting the same named barriers and
-    // warp-collective TMEM instructions (no thread is left waiting).
+    // warp-collective TMEM instructions (no thread is left waiting). No bulk copy is issued and no
+    // barrier with a transaction count is re-armed after an abort.
     auto wait_cta = [&](uint64_t* bar, int parity) {
       if (*abort_flag) return;
       if (!mbar_wait(bar, (uint32_t)parity, p.wait_ns, p.status)) *abort_flag = 1;
     };
+    // this warpgroup's 128 of the CTA's 256 latent query columns of block kq, into TMEM, once the
+    // previous segment's last QK^T has read the query
+    auto load_query = [&](int kq, int segment) {
+      const int b = kq / p.nbps, rb = kq % p.nbps;
+      const int64_t qr = (int64_t)b * p.n_q * p.H + (int64_t)rb * DEC_ROWS + row;
+      if (segment > 0) wait_cta(q_empty, (segment - 1) & 1);
+      tc_fence_after();
+      const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + qr * p.W + dim0 + wg * 128);
+      const bool in = qr < p.q_rows;
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {   // 2 x 32 TMEM columns = 128 bf16
+        uint32_t r[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint4 v = in ? src[cc * 8 + j] : make_uint4(0u, 0u, 0u, 0u);
+          r[4 * j] = v.x; r[4 * j + 1] = v.y; r[4 * j + 2] = v.z; r[4 * j + 3] = v.w;
+        }
+        tmem_st32(tQ + lane_off + wg * 64 + cc * 32, r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      named_bar_sync(bar_wg, 128);
+      if (row == 0) mbar_arrive(ql_full);
+    };
+    if (u0 < u1) load_query(k, 0);
     while (u < u1) {
       const int64_t bstart = p.prefix[k], bend = p.prefix[k + 1];
       const int64_t send_u = u1 < bend ? u1 : bend;
@@ -588,15 +490,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       float m_ref = -INFINITY, l = 0.f;     // reference maximum (log2 units), this group's sum
       for (int tt = 0; tt < ntl; ++tt, ++g) {
         const int sl = (int)(g & 1);
-        wait_cta(&s_sum[sl], (int)(g >> 1) & 1);
+        const int xi = sl * 2 + wg;           // this warpgroup's exchange slot
+        wait_cta(&s_full[sl], (int)(g >> 1) & 1);
         tc_fence_after();
-        float s[32];
+        uint32_t own[16];                     // this CTA's partial scores, fp16 pairs
         {
           uint32_t r[32];
           tmem_ld32(tS + lane_off + sl * 64 + wg * 32, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(r[c]);
+          for (int c = 0; c < 16; ++c) {
+            __half2 v = __floats2half2_rn(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1]));
+            own[c] = *reinterpret_cast<uint32_t*>(&v);
+          }
+        }
+        // send: staging slot xi and the peer's receive slot xi were last used by tile g - 2; once the
+        // peer has read that tile (x_empty) the copy from it is complete and both may be reused
+        if (g >= 2) wait_cta(&x_empty[xi], (int)((g >> 1) - 1) & 1);
+        uint8_t* stg = staging + xi * Cfg::X_HALF;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(stg + xrow + ((c ^ swz) * 16)) =
+              make_uint4(own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3]);
+        fence_proxy_async_smem();             // generic writes -> visible to the bulk copy
+        named_bar_sync(bar_wg, 128);
+        if (row == 0 && !*abort_flag)
+          bulk_copy_to_cta(x_remote + (uint32_t)(xi * Cfg::X_HALF), stg, Cfg::X_HALF, xf_remote + xi * 8);
+        // receive the peer's partials of the same columns and form S
+        wait_cta(&x_full[xi], (int)(g >> 1) & 1);
+        float s[32];
+        {
+          const uint8_t* xr = sX + xi * Cfg::X_HALF + xrow;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(xr + ((c ^ swz) * 16));
+            const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&own[4 * c + j]));
+              const float2 bq = __half22float2(*reinterpret_cast<const __half2*>(&pv[j]));
+              s[8 * c + 2 * j] = a.x + bq.x;
+              s[8 * c + 2 * j + 1] = a.y + bq.y;
+            }
+          }
         }
         // mask (only where the tile crosses a row's limit) and the raw row maximum
         const int t0 = (tile0 + tt) * DEC_BT + wg * 32;
@@ -615,7 +551,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         }
         float* mxs = mx + (g & 1) * 2 * DEC_ROWS;
         mxs[wg * DEC_ROWS + row] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        named_bar_sync(3, 256);               // both warpgroups' maxima are in (and S is loaded)
+        named_bar_sync(3, 256);               // both maxima are in; S and the receive slot are read
+        if (row == 0 && !*abort_flag) {
+          // this thread's own wait saw the slot's phase complete (the flag is still clear), so the
+          // re-arm cannot meet a phase with bytes outstanding; the peer may then refill the slot
+          mbar_arrive_expect_tx(&x_full[xi], Cfg::X_HALF);
+          mbar_arrive_remote(xe_remote + xi * 8);
+        }
         const float mx_raw = fmaxf(mxs[row], mxs[DEC_ROWS + row]);
         const float mx_t = mx_raw * p.scale_log2;   // the scale is positive: the order is kept
         bool need = false;
@@ -666,6 +608,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         named_bar_sync(bar_wg, 128);
         if (row == 0) mbar_arrive(&p_full[sl]);
       }
+      // the next segment's query can go in now (its QK^T overlaps this epilogue)
+      const int k_next = send_u < u1 ? find_block(p.prefix, p.nblocks, send_u) : k;
+      if (send_u < u1) load_query(k_next, seg + 1);
       // epilogue of the segment: wait for its last P.C, then read this group's quarter of O
       if (g > pv_waited) {
         wait_cta(o_done, (int)((g - 1) & 1));
@@ -706,7 +651,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       tc_fence_before();
       u = send_u;
       ++seg;
-      if (u < u1) k = find_block(p.prefix, p.nblocks, u);
+      k = k_next;
     }
   }
 
