@@ -25,12 +25,13 @@
 //  * Work: the (block, 64-position tile) units of all sequences are split evenly over the clusters
 //    (persistent). A cluster that covers a whole block writes the normalised result; split blocks
 //    leave (O, max, sum) partials that a combine kernel merges.
-//  * Warp roles per CTA (384 threads): warp 0 lane 0 issues TMA loads, warp 1 lane 0 issues MMAs
-//    (event loop), warps 4-11 form two softmax warpgroups (thread = row = TMEM lane). Warpgroup wg
-//    owns score columns [32 wg, 32 wg + 32) of every tile: it rounds its partial scores to fp16,
-//    sends them to the same warpgroup of the peer CTA with one bulk copy, adds the peer's half of
-//    the same columns and runs the softmax. The two warpgroups meet once per tile for the row
-//    maximum. They also load the query block into TMEM at each segment and run the epilogue.
+//  * Warp roles per CTA (512 threads): warp 0 lane 0 issues TMA loads, warp 1 lane 0 issues MMAs
+//    (event loop), warps 12-15 send the partial scores (rounded to fp16; each warp copies its 32
+//    rows of each softmax warpgroup's half to the peer and never waits on the peer), warps 4-11 form
+//    two softmax warpgroups (thread = row = TMEM lane): warpgroup wg loads half the query block into
+//    TMEM at each segment, adds its own and the peer's fp16 partials of score columns
+//    [32 wg, 32 wg + 32), meets the other warpgroup once per tile for the row maximum, writes P and
+//    runs the epilogue.
 //  * Every wait is bounded (global-timer limit); a wait that gives up sets the library's status word,
 //    and the CTA abandons its work, drains its own TMA loads and MMAs and exits through the cluster
 //    barrier.
@@ -46,7 +47,7 @@ namespace mla {
 using namespace sm100;
 
 constexpr int DEC_BT = 64;          // positions per tile
-constexpr int DEC_THREADS = 384;   // warp 0 TMA, warp 1 MMA, warps 4-11 query, exchange and softmax
+constexpr int DEC_THREADS = 512;   // warp 0 TMA, warp 1 MMA, warps 4-11 softmax, warps 12-15 query + sender
 constexpr int DEC_DC = 512;         // latent width handled by this kernel
 constexpr int DEC_HALF = 256;       // latent columns per CTA
 constexpr int DEC_ROWS = 128;       // rows per block
@@ -59,12 +60,11 @@ struct DecCfg {
   static constexpr int KR_BOX = DR ? DEC_BT * 64 : 0;   // 64 positions x 32 rotary columns (64 B)
   static constexpr int STAGE_BYTES = 4 * K_BOX + KR_BOX;
   static constexpr int STAGES = 4;
-  static constexpr int X_HALF = DEC_ROWS * 32 * 2;       // one warpgroup's 32 partial-score columns, fp16
-  static constexpr int X_TILE = 2 * X_HALF;
+  static constexpr int X_TILE = DEC_ROWS * DEC_BT * 2;   // one tile of partial scores, fp16, rows of 128 B
   static constexpr int OFF_QR = 0;
   static constexpr int OFF_K = QR_BOX;
   static constexpr int OFF_X = OFF_K + STAGES * STAGE_BYTES;
-  static constexpr int OFF_XS = OFF_X + 2 * X_TILE;      // receive slots [2][2 wg], then send stagings [2][2 wg]
+  static constexpr int OFF_XS = OFF_X + 2 * X_TILE;      // two receive slots, then two send stagings
   static constexpr int OFF_BAR = OFF_XS + 2 * X_TILE;
   static constexpr int OFF_RED = OFF_BAR + 256;          // row maxima [2][2][128], row sums [2][128]
   static constexpr int SMEM = OFF_RED + 6 * DEC_ROWS * 4 + 1024;
@@ -193,12 +193,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
   uint64_t* qr_full = k_empty + ST;     // rotary query columns landed (TMA)
   uint64_t* ql_full = qr_full + 1;      // latent query columns written to TMEM (query warps)
   uint64_t* q_empty = ql_full + 1;      // last QK^T of a segment done: the query may be replaced
-  uint64_t* s_full = q_empty + 1;       // [2] partial S of a slot computed (MMA -> softmax)
-  uint64_t* p_full = s_full + 2;        // [2] P written (softmax -> MMA)
+  uint64_t* s_full = q_empty + 1;       // [2] partial S of a slot computed (MMA -> sender)
+  uint64_t* own_ready = s_full + 2;     // [2] own fp16 partials staged, S read (sender -> softmax)
+  uint64_t* p_full = own_ready + 2;     // [2] P written (softmax -> MMA)
   uint64_t* o_done = p_full + 2;        // [1] a P.C completed
-  uint64_t* x_full = o_done + 1;        // [2 slots][2 wg] peer's partial scores arrived (transaction count)
-  uint64_t* x_empty = x_full + 4;       // [2 slots][2 wg] peer has read this CTA's scores
-  uint64_t* drain = x_empty + 4;        // [1] MMA drain on abort
+  uint64_t* x_full = o_done + 1;        // [2] peer's partial scores arrived (transaction count)
+  uint64_t* x_empty = x_full + 2;       // [2] both softmaxes have read this CTA's scores
+  uint64_t* drain = x_empty + 2;        // [1] MMA drain on abort
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -215,20 +216,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       mbar_init(&k_empty[s], 1);
     }
     mbar_init(qr_full, 1);
-    mbar_init(ql_full, 2);            // one arrival per softmax warpgroup (each writes half the query)
+    mbar_init(ql_full, 8);            // one arrival per softmax warp (each writes its rows' half)
     mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 2);       // one arrival per softmax warpgroup
+      mbar_init(&own_ready[s], 4);    // one arrival per sender warp
+      mbar_init(&p_full[s], 8);       // one arrival per softmax warp
     }
-    for (int s = 0; s < 4; ++s) {
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&x_full[s], 1);
-      mbar_init(&x_empty[s], 1);
+      mbar_init(&x_empty[s], 2);      // the peer's softmax (remote) and this CTA's (local)
     }
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
-    // arm the first use of each receive slot: one local arrival plus the peer's 8 KB bulk copy
-    for (int s = 0; s < 4; ++s) mbar_arrive_expect_tx(&x_full[s], Cfg::X_HALF);
+    // arm the first use of each receive slot: one local arrival plus the peer's four 4 KB bulk copies
+    for (int s = 0; s < 2; ++s) mbar_arrive_expect_tx(&x_full[s], Cfg::X_TILE);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tk);
@@ -277,17 +279,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         tma_load_2d(sQR, &tqr, qr_full, rdim0, qrow);
         ++q_loads;
       }
+      int pf_next = 0;                      // next tile of this segment to warm in L2
       for (int tt = 0; tt < ntl; ++tt, ++g) {
         const int s = (int)(g % ST);
         if (g >= ST && (*abort_flag || !mbar_wait(&k_empty[s], (int)((g / ST) - 1) & 1, p.wait_ns, p.status))) {
           ok = false;
           break;
         }
-        if (tt == 0 || tt + ST + DEC_PREFETCH - 1 < ntl) {
-          // warm L2 for the tiles after the shared-memory ring
-          const int first = tt == 0 ? ST : ST + DEC_PREFETCH - 1;
-          for (int pt = tt + first; pt < tt + ST + DEC_PREFETCH && pt < ntl; ++pt) {
-            const int yp = (int)(sstart + (int64_t)(tile0 + pt) * DEC_BT);
+        // the first query block is read by the softmax warps at the same time: hold the rest of the
+        // ring until it is in, so that it does not queue behind four tiles of every CTA
+        if (g == 1 && (*abort_flag || !mbar_wait(ql_full, 0, p.wait_ns, p.status))) {
+          ok = false;
+          break;
+        }
+        if (g >= ST) {
+          // warm L2 for up to DEC_PREFETCH tiles beyond the shared-memory ring, at most two per step:
+          // while the ring first fills, nothing is prefetched, so that the first tiles of all CTAs do
+          // not queue behind a burst of prefetches
+          if (pf_next < tt + ST) pf_next = tt + ST;
+          const int pf_end = min(ntl, tt + ST + DEC_PREFETCH);
+          for (int n = 0; n < 2 && pf_next < pf_end; ++n, ++pf_next) {
+            const int yp = (int)(sstart + (int64_t)(tile0 + pf_next) * DEC_BT);
             for (int kb = 0; kb < 4; ++kb) tma_prefetch_2d(&tk, dim0 + kb * 64, yp);
             if (DR) tma_prefetch_2d(&tkr, rdim0, yp);
           }
@@ -315,9 +327,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     // memory stage for the producer), and QK^T of the next tile as soon as its cache tile has landed,
     // its query is in place and its S/P slot is free (the P.C two tiles back has been issued; MMAs
     // run in issue order).
+    // One thread issues every MMA, and its scalar work sits between consecutive MMAs: descriptors are
+    // built once for stage 0 and advanced by constant offsets (the 14-bit start-address field holds
+    // shared addresses >> 4 below 256 KB, so the additions never carry into the other fields).
     constexpr uint32_t idesc_qk = idesc_bf16_f32(128, DEC_BT, false, false);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, DEC_HALF, false, true);
+    constexpr uint64_t kStage = (uint64_t)(Cfg::STAGE_BYTES >> 4);
     const uint32_t qr_base = smem_u32(sQR), k_base = smem_u32(sK);
+    const uint64_t kd0 = smem_desc_sw128(k_base, 16, 1024);                  // cache tile, K-major (B of QK^T)
+    const uint64_t cd0 = smem_desc_sw128(k_base, Cfg::K_BOX, 1024);          // cache tile, MN-major (B of P.C)
+    const uint64_t rd0 = smem_desc_sw64(k_base + 4 * Cfg::K_BOX, 16, 512);   // rotary columns of the tile
+    const uint64_t qd0 = smem_desc_sw64(qr_base, 16, 512);                   // rotary query columns
     int64_t gq = 0, gp = 0;               // next tile for QK^T, next tile for P.C
     int64_t qseg_start = 0, qseg_end = 0; // tiles [start, end) of the segment QK^T is in
     int segq = -1;
@@ -337,12 +357,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         const int s = (int)(gp % ST);
         const bool first = (first_bits >> (gp & 31)) & 1u;
         // B = this CTA's 256 latent columns of the tile: MN-major, 64-column boxes K_BOX apart
-        const uint32_t c_base = k_base + s * Cfg::STAGE_BYTES;
+        const uint64_t cd = cd0 + (uint64_t)s * kStage;
+        const uint32_t ta = tS + sl * 64;
 #pragma unroll
-        for (int kk = 0; kk < DEC_BT / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(c_base + kk * 2048, Cfg::K_BOX, 1024);
-          mma_bf16_ts(tO, tS + sl * 64 + kk * 8, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
-        }
+        for (int kk = 0; kk < DEC_BT / 16; ++kk)
+          mma_bf16_ts(tO, ta + kk * 8, cd + (uint64_t)(kk * (2048 >> 4)), idesc_pv, (first && kk == 0) ? 0u : 1u);
         mma_commit(&k_empty[s]);
         mma_commit(o_done);
         ++gp;
@@ -369,22 +388,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         if (ql_ok && qr_ok && mbar_test_wait(&k_full[s], (uint32_t)(gq / ST) & 1u)) {
           tc_fence_after();
           const int sl = (int)(gq & 1);
-          const uint32_t kst = k_base + s * Cfg::STAGE_BYTES;
+          const uint32_t td = tS + sl * 64;
+          const uint64_t kd = kd0 + (uint64_t)s * kStage;
+#pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t bd = smem_desc_sw128(kst + kb * Cfg::K_BOX + kk * 32, 16, 1024);
-              mma_bf16_ts(tS + sl * 64, tQ + kb * 32 + kk * 8, bd, idesc_qk, (kb | kk) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ts(td, tQ + kb * 32 + kk * 8, kd + (uint64_t)((kb * Cfg::K_BOX + kk * 32) >> 4), idesc_qk,
+                          (kb | kk) ? 1u : 0u);
           }
           if (DR) {
             // this CTA's 32 rotary columns: rows of 64 B, 8-row groups 512 B apart
+            const uint64_t rd = rd0 + (uint64_t)s * kStage;
 #pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-              const uint64_t ad = smem_desc_sw64(qr_base + kk * 32, 16, 512);
-              const uint64_t bd = smem_desc_sw64(kst + 4 * Cfg::K_BOX + kk * 32, 16, 512);
-              mma_bf16_ss(tS + sl * 64, ad, bd, idesc_qk, 1u);
-            }
+            for (int kk = 0; kk < 2; ++kk) mma_bf16_ss(td, qd0 + (uint64_t)(kk * 2), rd + (uint64_t)(kk * 2), idesc_qk, 1u);
           }
           mma_commit(&s_full[sl]);
           if (gq + 1 == qseg_end) mma_commit(q_empty);
@@ -411,62 +428,121 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       mma_commit(drain);
       (void)mbar_wait(drain, 0, drain_ns, p.status);
     }
+  } else if (warp >= 12) {
+    // -------------------------------- score sender --------------------------------
+    // Thread = row = TMEM lane, and each warp handles its 32 rows on its own. For each tile: load this
+    // CTA's partial scores (64 columns), round them to fp16 into the staging slots of the two softmax
+    // warpgroups (the softmax reads its own partials there) and send the warp's rows of each half to
+    // the same slot of the peer with one 2 KB bulk copy per half. The sender never waits for the
+    // peer's scores, so the peer receives tile g as soon as this CTA's QK^T of tile g is done.
+    // One copy per warp carries its rows of both halves (4 KB).
+    const int quarter = warp - 12;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t x_remote = map_to_cta(smem_u32(sX), peer);
+    const uint32_t xf_remote = map_to_cta(smem_u32(x_full), peer);
+    const uint32_t xrow = (uint32_t)(row * 128);          // 64 fp16 per row: 8 chunks of 16 B
+    const uint32_t xwarp = (uint32_t)(quarter * 32 * 128);// this warp's 32 rows: 4 KB of each slot
+    const int swz = row & 7;                              // chunk swizzle against bank conflicts
+    uint8_t* staging = smem + Cfg::OFF_XS;
+    auto wait_cta = [&](uint64_t* bar, int parity) {
+      if (*abort_flag) return;
+      if (!mbar_wait(bar, (uint32_t)parity, p.wait_ns, p.status)) *abort_flag = 1;
+    };
+    for (int64_t g = 0; g < n_total; ++g) {
+      const int sl = (int)(g & 1);
+      wait_cta(&s_full[sl], (int)(g >> 1) & 1);
+      tc_fence_after();
+      uint32_t h[32];                       // fp16 pairs: [0, 16) for warpgroup 0, [16, 32) for 1
+      {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(tS + lane_off + sl * 64, r0);
+        tmem_ld32(tS + lane_off + sl * 64 + 32, r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          __half2 v0 = __floats2half2_rn(__uint_as_float(r0[2 * c]), __uint_as_float(r0[2 * c + 1]));
+          __half2 v1 = __floats2half2_rn(__uint_as_float(r1[2 * c]), __uint_as_float(r1[2 * c + 1]));
+          h[c] = *reinterpret_cast<uint32_t*>(&v0);
+          h[16 + c] = *reinterpret_cast<uint32_t*>(&v1);
+        }
+      }
+      // staging slot sl and the peer's receive slot sl were last used by tile g - 2: both this CTA's
+      // softmax and the peer's have read that tile once x_empty completes (2 arrivals)
+      if (g >= 2) wait_cta(&x_empty[sl], (int)((g >> 1) - 1) & 1);
+      {
+        uint8_t* stg = staging + sl * Cfg::X_TILE + xrow;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(stg + ((c ^ swz) * 16)) =
+              make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
+      }
+      fence_proxy_async_smem();             // generic writes -> visible to the bulk copies
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (!*abort_flag) {
+          const uint32_t off = (uint32_t)(sl * Cfg::X_TILE) + xwarp;
+          bulk_copy_to_cta(x_remote + off, staging + off, 32 * 128, xf_remote + sl * 8);
+        }
+        mbar_arrive(&own_ready[sl]);        // this warp's partials staged and read: P may overwrite
+      }
+    }
   } else if (warp >= 4) {
-    // ------------------------ query, score exchange, softmax, epilogue ------------------------
+    // ---------------------------- softmax and epilogue ----------------------------
     // Two warpgroups share every tile: warpgroup wg owns score columns [32 wg, 32 wg + 32) of each
     // row (thread = row = TMEM lane), packed P columns [16 wg, 16 wg + 16) and O columns
-    // [128 wg, 128 wg + 128). Per tile it rounds its partial scores to fp16, sends them to the same
-    // warpgroup of the peer CTA (one 8 KB bulk copy into the peer's receive slot, completing the
-    // peer's barrier), and adds the peer's fp16 partials of the same columns: both CTAs form
-    // S = fp16(S0) + fp16(S1) identically. The warpgroups meet once per tile on the row maximum.
+    // [128 wg, 128 wg + 128). S = fp16(own partial) + fp16(peer's partial), both read from shared
+    // memory (the sender's staging slot and the peer's copy), identically in both CTAs. The
+    // warpgroups meet once per tile on the row maximum.
     const int wg = (warp - 4) >> 2;
     const int quarter = (warp - 4) & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t bar_wg = 1 + wg;                       // named barrier of this warpgroup
     float* mx = red;                                      // [2 tiles][2 warpgroups][128]
     float* lx = red + 4 * DEC_ROWS;                       // [2 warpgroups][128]
-    uint8_t* staging = smem + Cfg::OFF_XS;
-    const uint32_t x_remote = map_to_cta(smem_u32(sX), peer);
-    const uint32_t xf_remote = map_to_cta(smem_u32(x_full), peer);
+    const uint8_t* staging = smem + Cfg::OFF_XS;
     const uint32_t xe_remote = map_to_cta(smem_u32(x_empty), peer);
-    const uint32_t xrow = (uint32_t)(row * 64);           // 32 fp16 per row: 4 chunks of 16 B
-    const int swz = (row >> 1) & 3;                       // chunk swizzle against bank conflicts
+    const uint32_t xrow = (uint32_t)(row * 128);
+    const int swz = row & 7;
     int64_t g = 0, pv_waited = 0;
     int seg = 0;
     int64_t u = u0;
     int k = u0 < u1 ? find_block(p.prefix, p.nblocks, u0) : 0;
     // A wait that gives up sets the abort flag; from then on every wait is skipped but the loop
     // structure is walked unchanged, so that all threads keep meeting the same named barriers and
-    // warp-collective TMEM instructions (no thread is left waiting). No bulk copy is issued and no
-    // barrier with a transaction count is re-armed after an abort.
+    // warp-collective TMEM instructions (no thread is left waiting). No barrier with a transaction
+    // count is re-armed and no slot is released to the peer after an abort.
     auto wait_cta = [&](uint64_t* bar, int parity) {
       if (*abort_flag) return;
       if (!mbar_wait(bar, (uint32_t)parity, p.wait_ns, p.status)) *abort_flag = 1;
     };
-    // this warpgroup's 128 of the CTA's 256 latent query columns of block kq, into TMEM, once the
-    // previous segment's last QK^T has read the query
+    // this warpgroup's 128 of the CTA's 256 latent query columns of block kq, into TMEM (one batch of
+    // loads per thread), once the previous segment's last QK^T has read the query
     auto load_query = [&](int kq, int segment) {
-      const int b = kq / p.nbps, rb = kq % p.nbps;
-      const int64_t qr = (int64_t)b * p.n_q * p.H + (int64_t)rb * DEC_ROWS + row;
+      const int bq = kq / p.nbps, rbq = kq % p.nbps;
+      const int64_t qr = (int64_t)bq * p.n_q * p.H + (int64_t)rbq * DEC_ROWS + row;
       if (segment > 0) wait_cta(q_empty, (segment - 1) & 1);
       tc_fence_after();
       const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + qr * p.W + dim0 + wg * 128);
       const bool in = qr < p.q_rows;
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {   // 2 x 32 TMEM columns = 128 bf16
+      uint4 v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = in ? src[j] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {      // 2 x 32 TMEM columns = 128 bf16
         uint32_t r[32];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const uint4 v = in ? src[cc * 8 + j] : make_uint4(0u, 0u, 0u, 0u);
-          r[4 * j] = v.x; r[4 * j + 1] = v.y; r[4 * j + 2] = v.z; r[4 * j + 3] = v.w;
+          r[4 * j] = v[cc * 8 + j].x; r[4 * j + 1] = v[cc * 8 + j].y;
+          r[4 * j + 2] = v[cc * 8 + j].z; r[4 * j + 3] = v[cc * 8 + j].w;
         }
         tmem_st32(tQ + lane_off + wg * 64 + cc * 32, r);
       }
       tmem_wait_st();
       tc_fence_before();
-      named_bar_sync(bar_wg, 128);
-      if (row == 0) mbar_arrive(ql_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ql_full);
     };
     if (u0 < u1) load_query(k, 0);
     while (u < u1) {
@@ -490,47 +566,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       float m_ref = -INFINITY, l = 0.f;     // reference maximum (log2 units), this group's sum
       for (int tt = 0; tt < ntl; ++tt, ++g) {
         const int sl = (int)(g & 1);
-        const int xi = sl * 2 + wg;           // this warpgroup's exchange slot
-        wait_cta(&s_full[sl], (int)(g >> 1) & 1);
-        tc_fence_after();
-        uint32_t own[16];                     // this CTA's partial scores, fp16 pairs
-        {
-          uint32_t r[32];
-          tmem_ld32(tS + lane_off + sl * 64 + wg * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            __half2 v = __floats2half2_rn(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1]));
-            own[c] = *reinterpret_cast<uint32_t*>(&v);
-          }
-        }
-        // send: staging slot xi and the peer's receive slot xi were last used by tile g - 2; once the
-        // peer has read that tile (x_empty) the copy from it is complete and both may be reused
-        if (g >= 2) wait_cta(&x_empty[xi], (int)((g >> 1) - 1) & 1);
-        uint8_t* stg = staging + xi * Cfg::X_HALF;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(stg + xrow + ((c ^ swz) * 16)) =
-              make_uint4(own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3]);
-        fence_proxy_async_smem();             // generic writes -> visible to the bulk copy
-        named_bar_sync(bar_wg, 128);
-        if (row == 0 && !*abort_flag)
-          bulk_copy_to_cta(x_remote + (uint32_t)(xi * Cfg::X_HALF), stg, Cfg::X_HALF, xf_remote + xi * 8);
-        // receive the peer's partials of the same columns and form S
-        wait_cta(&x_full[xi], (int)(g >> 1) & 1);
+        const int xi = sl;                    // the tile's exchange slot (this warpgroup reads its half)
         float s[32];
+        wait_cta(&own_ready[sl], (int)(g >> 1) & 1);
+        tc_fence_after();
+        uint4 own[4];
         {
-          const uint8_t* xr = sX + xi * Cfg::X_HALF + xrow;
+          const uint8_t* xo = staging + xi * Cfg::X_TILE + xrow;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) own[c] = *reinterpret_cast<const uint4*>(xo + (((4 * wg + c) ^ swz) * 16));
+        }
+        wait_cta(&x_full[xi], (int)(g >> 1) & 1);
+        {
+          const uint8_t* xr = sX + xi * Cfg::X_TILE + xrow;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const uint4 v = *reinterpret_cast<const uint4*>(xr + ((c ^ swz) * 16));
+            const uint4 v = *reinterpret_cast<const uint4*>(xr + (((4 * wg + c) ^ swz) * 16));
             const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
+            const uint32_t ov[4] = {own[c].x, own[c].y, own[c].z, own[c].w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&own[4 * c + j]));
-              const float2 bq = __half22float2(*reinterpret_cast<const __half2*>(&pv[j]));
-              s[8 * c + 2 * j] = a.x + bq.x;
-              s[8 * c + 2 * j + 1] = a.y + bq.y;
+              // the sum of the two fp16 partials, in fp16 (commutative: the same in both CTAs), then
+              // widened once
+              const __half2 sh = __hadd2(*reinterpret_cast<const __half2*>(&ov[j]),
+                                         *reinterpret_cast<const __half2*>(&pv[j]));
+              const float2 f = __half22float2(sh);
+              s[8 * c + 2 * j] = f.x;
+              s[8 * c + 2 * j + 1] = f.y;
             }
           }
         }
@@ -551,12 +613,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         }
         float* mxs = mx + (g & 1) * 2 * DEC_ROWS;
         mxs[wg * DEC_ROWS + row] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        named_bar_sync(3, 256);               // both maxima are in; S and the receive slot are read
-        if (row == 0 && !*abort_flag) {
-          // this thread's own wait saw the slot's phase complete (the flag is still clear), so the
-          // re-arm cannot meet a phase with bytes outstanding; the peer may then refill the slot
-          mbar_arrive_expect_tx(&x_full[xi], Cfg::X_HALF);
+        named_bar_sync(3, 256);               // both maxima are in; the slots of this tile are read
+        if (wg == 0 && row == 0 && !*abort_flag) {
+          // both warpgroups have read both slots (the barrier above); this thread's own wait saw the
+          // receive slot's phase complete (the flag is still clear), so the re-arm cannot meet a phase
+          // with bytes outstanding. Then release the slot to the peer's sender and the staging slot to
+          // this CTA's sender.
+          mbar_arrive_expect_tx(&x_full[xi], Cfg::X_TILE);
           mbar_arrive_remote(xe_remote + xi * 8);
+          mbar_arrive(&x_empty[xi]);
         }
         const float mx_raw = fmaxf(mxs[row], mxs[DEC_ROWS + row]);
         const float mx_t = mx_raw * p.scale_log2;   // the scale is positive: the order is kept
@@ -571,28 +636,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           m_ref = mx_t;
         }
         const float mu = m_ref == -INFINITY ? 0.f : m_ref;
+        // P in bf16 by truncation (the top half of each fp32: one byte permute per pair instead of a
+        // conversion), and the row sum of the same truncated values, so that numerator and
+        // denominator of the normalisation share the rounding
         float sum0 = 0.f, sum1 = 0.f;
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float p0 = ex2(fmaf(s[2 * c], p.scale_log2, -mu));
-          const float p1 = ex2(fmaf(s[2 * c + 1], p.scale_log2, -mu));
-          sum0 += p0;
-          sum1 += p1;
-          __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
-          pk[c] = *reinterpret_cast<uint32_t*>(&hb);
+          const uint32_t b0 = __float_as_uint(ex2(fmaf(s[2 * c], p.scale_log2, -mu))) & 0xFFFF0000u;
+          const uint32_t b1 = __float_as_uint(ex2(fmaf(s[2 * c + 1], p.scale_log2, -mu))) & 0xFFFF0000u;
+          sum0 += __uint_as_float(b0);
+          sum1 += __uint_as_float(b1);
+          pk[c] = __byte_perm(b0, b1, 0x7632);
         }
         l += sum0 + sum1;
-        // P overwrites columns of S: the barrier above guarantees both groups have loaded theirs
+        // P overwrites the S slot: the sender has read it (own_ready)
         tmem_st16(tS + lane_off + sl * 64 + wg * 16, pk);
         tmem_wait_st();
-        // the previous tile's P.C must be done before O is touched and before this P is released
-        if (g > pv_waited) {
+        // O may be touched only once every earlier P.C is done: needed when a row of this warp rescales,
+        // and at the last tile of a segment (so that the epilogue's wait is one phase away). Here P.C of
+        // tile g - 2 is complete (QK^T of tile g reused its slot) and P.C of tile g is not issued yet, so
+        // o_done is at most one phase behind and the parity names P.C of tile g - 1 unambiguously.
+        const bool rescale = __any_sync(0xffffffffu, need);
+        if ((rescale || tt + 1 == ntl) && g > pv_waited) {
           wait_cta(o_done, (int)((g - 1) & 1));
           pv_waited = g;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, need)) {
+        if (rescale) {
 #pragma unroll 1
           for (int cc = 0; cc < DEC_HALF / 2; cc += 32) {
             uint32_t r[32];
@@ -605,8 +676,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           tmem_wait_st();
         }
         tc_fence_before();
-        named_bar_sync(bar_wg, 128);
-        if (row == 0) mbar_arrive(&p_full[sl]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[sl]);   // this warp's rows of P are in (and O rescaled)
       }
       // the next segment's query can go in now (its QK^T overlaps this epilogue)
       const int k_next = send_u < u1 ? find_block(p.prefix, p.nblocks, send_u) : k;
