@@ -751,14 +751,13 @@ __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
   __shared__ int slots[256];
   __shared__ float wts[8][256];
   __shared__ int nsl;
-  const int k = blockIdx.x;
-  const int r0 = blockIdx.y * 8;     // this CTA's 8 rows of the block (one per warp)
+  const int k = blockIdx.x;         // one CTA per block: warp w merges rows w, w + 8, ...
   const int64_t bstart = p.prefix[k], bend = p.prefix[k + 1];
   const int b = k / p.nbps, rb = k % p.nbps;
   const int rows_seq = p.n_q * p.H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (bend == bstart) {
-    for (int r = r0 + warp; r < r0 + 8; r += 8) {
+    for (int r = warp; r < DEC_ROWS; r += 8) {
       const int ri = rb * DEC_ROWS + r;
       if (ri >= rows_seq) break;
       const int64_t orow = (int64_t)b * rows_seq + ri;
@@ -784,7 +783,7 @@ __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
   }
   __syncthreads();
   const int n = nsl;
-  for (int r = r0 + warp; r < r0 + 8; r += 8) {
+  for (int r = warp; r < DEC_ROWS; r += 8) {
     const int ri = rb * DEC_ROWS + r;
     if (ri >= rows_seq) break;
     float M = -INFINITY;
@@ -963,7 +962,7 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
   MLA_LAUNCH_CHECK();
   int st = a.dr == 0 ? launch_decode_t<0>(tk, tkr, tqr, p, s) : launch_decode_t<64>(tk, tkr, tqr, p, s);
   if (st) return st;
-  decode_combine_tc_kernel<<<dim3((unsigned)t.nblocks, DEC_ROWS / 8), 256, 0, s>>>(p);
+  decode_combine_tc_kernel<<<(unsigned)t.nblocks, 256, 0, s>>>(p);
   MLA_LAUNCH_CHECK();
   return MLA_OK;
 }

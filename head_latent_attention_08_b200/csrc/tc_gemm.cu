@@ -73,6 +73,10 @@ struct TcGemmParams {
   const __nv_bfloat16* gate; int64_t gate_sb, gate_st;
   float* partial;    // [split][batch][N][M] when n_splits > 1
   int sigmoid;
+  int stages;        // depth of the shared-memory ring (<= GemmCfg::STAGES; sized to the K chunks)
+  // optional tail: out[bz][t][tail_off + c] = tail[bz * tail_sb + t * tail_st + c], c < tail_cols
+  // (copied by the m-tile-0, split-0 CTA of each token tile; bf16 output only, 16-byte rows)
+  const __nv_bfloat16* tail; int64_t tail_sb, tail_st, tail_off; int tail_cols;
   int* status;
   unsigned long long wait_ns;
 };
@@ -99,7 +103,7 @@ __global__ void __launch_bounds__(128, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
                    TcGemmParams p) {
   using Cfg = GemmCfg<BN>;
-  constexpr int STAGES = Cfg::STAGES;
+  const int STAGES = p.stages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE);
@@ -138,10 +142,10 @@ __global__ void __launch_bounds__(128, 1)
   int issued = 0;
 
   if (warp == 0 && lane == 0) {
-    // TMA producer
+    // TMA producer (stage s of round ph: the previous round's MMAs must have released it)
+    int s = 0, ph = 0;
     for (int i = 0; i < nk; ++i) {
-      const int s = i % STAGES;
-      if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, p.wait_ns, p.status)) {
+      if (i >= STAGES && !mbar_wait(&empty[s], (uint32_t)(ph ^ 1), p.wait_ns, p.status)) {
         *abort_flag = 1;
         break;
       }
@@ -158,13 +162,14 @@ __global__ void __launch_bounds__(128, 1)
       }
       tma_load_3d(b_dst, &tb, &full[s], kx, n0, bz);
       ++issued;
+      if (++s == STAGES) { s = 0; ph ^= 1; }
     }
   } else if (warp == 1 && lane == 0) {
     // MMA issuer
     constexpr uint32_t idesc = idesc_bf16_f32(128, BN, A_MN, false);
+    int s = 0, ph = 0;
     for (int i = 0; i < nk; ++i) {
-      const int s = i % STAGES;
-      if (!mbar_wait(&full[s], (i / STAGES) & 1, p.wait_ns, p.status)) {
+      if (!mbar_wait(&full[s], (uint32_t)ph, p.wait_ns, p.status)) {
         *abort_flag = 1;
         break;
       }
@@ -179,38 +184,75 @@ __global__ void __launch_bounds__(128, 1)
         mma_bf16_ss(tmem_d, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
       }
       mma_commit(&empty[s]);
+      if (++s == STAGES) { s = 0; ph ^= 1; }
     }
     mma_commit(done);
   }
   __syncwarp();
 
-  // epilogue: 128 threads, thread = accumulator row
+  // epilogue: thread = accumulator row m. The tile goes out through shared memory (the ring is idle
+  // once `done` has completed: every load has landed and every MMA has read it), 32 tokens at a time:
+  // thread m writes its 32 values to column m of a [32][128] fp32 tile, then the block writes whole
+  // 16-byte runs of 4 consecutive outputs of each token row (out[t][m] is contiguous along m).
   const bool ok = mbar_wait(done, 0, p.wait_ns, p.status);
   if (!ok) *abort_flag = 1;
   tc_fence_after();
   const bool write = ok && !*abort_flag;
-  const int m = m0 + warp * 32 + lane;
+  float* tile = reinterpret_cast<float*>(smem);          // [32][128]
 #pragma unroll 1
   for (int c = 0; c < BN; c += 32) {
     uint32_t r[32];
     tmem_ld32(tmem_d + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, r);
     tmem_wait_ld();
-    if (!write || m >= p.M) continue;
-#pragma unroll 4
-    for (int j = 0; j < 32; ++j) {
-      const int t = n0 + c + j;
-      if (t >= p.N) break;
-      const float acc = nk > 0 ? __uint_as_float(r[j]) : 0.f;
-      if (p.n_splits > 1) {
-        p.partial[(((int64_t)split * p.batch + bz) * p.N + t) * p.M + m] = acc;
-      } else {
-        const float v = apply_epilogue(acc, p.sigmoid, p.gate, bz * p.gate_sb + (int64_t)t * p.gate_st + m);
+    __syncthreads();                                      // the previous chunk's tile has been read
+    if (write) {                                          // (an abandoned CTA may still have loads landing)
+#pragma unroll
+      for (int j = 0; j < 32; ++j) tile[j * 128 + threadIdx.x] = nk > 0 ? __uint_as_float(r[j]) : 0.f;
+    }
+    __syncthreads();
+    if (write) {
+#pragma unroll 2
+      for (int q = threadIdx.x; q < 32 * 32; q += 128) {
+        const int tl = q >> 5, mq = (q & 31) * 4;
+        const int t = n0 + c + tl, m = m0 + mq;
+        if (t >= p.N || m >= p.M) continue;
+        float4 v = *reinterpret_cast<const float4*>(tile + tl * 128 + mq);
+        if (p.n_splits > 1) {
+          *reinterpret_cast<float4*>(p.partial + (((int64_t)split * p.batch + bz) * p.N + t) * p.M + m) = v;
+          continue;
+        }
+        if (p.sigmoid) {
+          v.x = 1.f / (1.f + expf(-v.x)); v.y = 1.f / (1.f + expf(-v.y));
+          v.z = 1.f / (1.f + expf(-v.z)); v.w = 1.f / (1.f + expf(-v.w));
+        }
+        if (p.gate) {
+          const uint2 gv = *reinterpret_cast<const uint2*>(p.gate + bz * p.gate_sb + (int64_t)t * p.gate_st + m);
+          const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv.x));
+          const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv.y));
+          v.x *= g0.x; v.y *= g0.y; v.z *= g1.x; v.w *= g1.y;
+        }
         const int64_t o = bz * p.out_sb + (int64_t)t * p.out_st + m;
-        if (p.out_f32)
-          static_cast<float*>(p.out)[o] = v;
-        else
-          static_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(v);
+        if (p.out_f32) {
+          *reinterpret_cast<float4*>(static_cast<float*>(p.out) + o) = v;
+        } else {
+          __nv_bfloat162 b0 = __floats2bfloat162_rn(v.x, v.y), b1 = __floats2bfloat162_rn(v.z, v.w);
+          uint2 w;
+          w.x = *reinterpret_cast<uint32_t*>(&b0);
+          w.y = *reinterpret_cast<uint32_t*>(&b1);
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + o) = w;
+        }
       }
+    }
+  }
+  if (p.tail && write && blockIdx.x == 0 && split == 0) {
+    // the tail columns of this CTA's tokens (16-byte chunks; the host checks the alignment)
+    const int cpr = p.tail_cols / 8;
+    for (int idx = threadIdx.x; idx < BN * cpr; idx += 128) {
+      const int t = n0 + idx / cpr, q = idx % cpr;
+      if (t >= p.N) break;
+      const uint4 v = reinterpret_cast<const uint4*>(p.tail + bz * p.tail_sb + (int64_t)t * p.tail_st)[q];
+      reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + bz * p.out_sb + (int64_t)t * p.out_st +
+                               p.tail_off)[q] = v;
     }
   }
   tc_fence_before();
@@ -300,7 +342,7 @@ static size_t gemm_partial_bytes(int M, int N, int K, int batch) {
 }
 
 template <int BN, bool A_MN>
-static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmParams& p, dim3 grid,
+static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, TcGemmParams p, dim3 grid,
                          cudaStream_t s) {
   static bool attr_set[64] = {false};
   const int dev = current_device();
@@ -310,16 +352,30 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const TcG
       return MLA_ERR_CUDA;
     attr_set[dev] = true;
   }
-  tc_gemm_kernel<BN, A_MN><<<grid, 128, GemmCfg<BN>::SMEM, s>>>(ta, tb, p);
+  // a ring no deeper than the K chunks of one CTA: short-K products then fit several CTAs per SM
+  p.stages = std::max(1, std::min(GemmCfg<BN>::STAGES, p.k_chunks));
+  const int smem = p.stages * GemmCfg<BN>::STAGE + 1024 + 256;
+  tc_gemm_kernel<BN, A_MN><<<grid, 128, smem, s>>>(ta, tb, p);
   MLA_LAUNCH_CHECK();
   return MLA_OK;
 }
 
 // out[bz][t][m] = epi(sum_k A[bz](m, k) B[bz](t, k)); A MN-major when a_mn
+struct GemmTail {
+  const void* src = nullptr;
+  int64_t sb = 0, st = 0, off = 0;
+  int cols = 0;
+};
+
 static int tc_gemm(const GemmOperand& A, bool a_mn, const GemmOperand& Bop, int M, int N, int K, int batch,
                    void* out, int64_t out_sb, int64_t out_st, bool out_f32, const void* gate, int64_t gate_sb,
-                   int64_t gate_st, bool sigmoid, void* partial_ws, cudaStream_t s) {
+                   int64_t gate_st, bool sigmoid, void* partial_ws, cudaStream_t s,
+                   const GemmTail& tail = GemmTail()) {
   if (M % 128 || K % 64 || N <= 0 || batch <= 0) return MLA_ERR_UNSUPPORTED;
+  // the epilogue writes runs of 4 consecutive outputs (8 or 16 bytes) and reads 4 gate values
+  if (out_sb % 4 || out_st % 4 || (reinterpret_cast<uintptr_t>(out) & 15) ||
+      (gate && (gate_sb % 4 || gate_st % 4 || (reinterpret_cast<uintptr_t>(gate) & 7))))
+    return MLA_ERR_UNSUPPORTED;
   const GemmPlan g = plan_gemm(M, N, K, batch, partial_ws ? (1 << 20) : 1);
   CUtensorMap ta, tb;
   {
@@ -339,6 +395,13 @@ static int tc_gemm(const GemmOperand& A, bool a_mn, const GemmOperand& Bop, int 
   p.batch = batch; p.out = out; p.out_sb = out_sb; p.out_st = out_st; p.out_f32 = out_f32 ? 1 : 0;
   p.gate = static_cast<const __nv_bfloat16*>(gate); p.gate_sb = gate_sb; p.gate_st = gate_st;
   p.partial = static_cast<float*>(partial_ws); p.sigmoid = sigmoid ? 1 : 0;
+  if (tail.src && tail.cols > 0) {
+    if (out_f32 || tail.cols % 8 || tail.sb % 8 || tail.st % 8 || tail.off % 8 || out_sb % 8 || out_st % 8 ||
+        (reinterpret_cast<uintptr_t>(tail.src) & 15) || (reinterpret_cast<uintptr_t>(out) & 15))
+      return MLA_ERR_UNSUPPORTED;
+    p.tail = static_cast<const __nv_bfloat16*>(tail.src);
+    p.tail_sb = tail.sb; p.tail_st = tail.st; p.tail_off = tail.off; p.tail_cols = tail.cols;
+  }
   p.status = device_status_ptr(); p.wait_ns = (unsigned long long)wait_limit();
   if (!p.status) return MLA_ERR_CUDA;
   if (g.splits > 1 && !partial_ws) return MLA_ERR_WORKSPACE;
@@ -383,12 +446,13 @@ int tc_absorb_query(const mla_dims& d, const void* q_nope, const void* q_pe, con
   // B = q_nope[:, h, :]: tensor [rows][H][n] seen as (k = i, t, h)
   GemmOperand B{const_cast<void*>(q_nope), (uint64_t)n, (uint64_t)n_rows, (uint64_t)H, (uint64_t)(H * n * 2),
                 (uint64_t)(n * 2)};
-  int st = tc_gemm(A, true, B, (int)dc, (int)n_rows, (int)n, (int)H, q_abs, W, H * W, false, nullptr, 0, 0,
-                   false, nullptr, s);
-  if (st) return st;
-  if (dr > 0)
-    return copy_rows_strided(q_pe, dr, static_cast<char*>(q_abs) + dc * 2, W, n_rows * H, dr, MLA_BF16, s);
-  return MLA_OK;
+  // the rotary tail q_abs[t, h, d_c:] = q_pe[t, h] is copied by the same kernel
+  GemmTail tail;
+  if (dr > 0) {
+    tail.src = q_pe; tail.sb = dr; tail.st = H * dr; tail.off = dc; tail.cols = (int)dr;
+  }
+  return tc_gemm(A, true, B, (int)dc, (int)n_rows, (int)n, (int)H, q_abs, W, H * W, false, nullptr, 0, 0,
+                 false, nullptr, s, tail);
 }
 
 bool tc_out_project_supported(const mla_dims& d, int64_t n_rows) {
