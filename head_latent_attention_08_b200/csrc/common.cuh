@@ -47,6 +47,42 @@ int current_device();
 void count_launch();      // one more kernel launched by this library (see mla_launch_count)
 long long launch_count();
 
+// Programmatic dependent launch. The hot-path kernels are launched with launch_pdl: such a kernel may
+// begin (prologue: barriers, tensor memory, descriptor prefetch) while the previous kernel of the
+// stream is still running. Every CTA calls griddep_wait() before it touches memory that earlier work
+// in the stream writes or reads; it returns once the previous kernel has completed and its writes are
+// visible (a no-op without a programmatic dependency). Because every such kernel waits in every CTA,
+// completion stays ordered through the whole chain. griddep_launch_dependents() lets the next kernel
+// start launching once every CTA of this grid has called it or exited (all CTAs are then resident,
+// so the early start cannot take SMs that this grid still needs).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+void count_launch();
+
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  count_launch();
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
+
 // after every kernel launch: count it and turn a launch error into MLA_ERR_CUDA
 #define MLA_LAUNCH_CHECK()                                   \
   do {                                                       \

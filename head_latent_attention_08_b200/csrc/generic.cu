@@ -186,9 +186,11 @@ template <typename T>
 __global__ void __launch_bounds__(128) append_latent_kernel(
     T* __restrict__ cache, const int64_t* __restrict__ row_idx, const float* __restrict__ c_new,
     const float* __restrict__ kpe_new, const int32_t* __restrict__ positions, int dc, int dr,
-    uint32_t flags, float eps, float theta, int vec8, int64_t cache_rows, int* status) {
+    uint32_t flags, float eps, double log2_theta, int vec8, int64_t cache_rows, int* status) {
   extern __shared__ float row[];
   __shared__ float red[4];
+  griddep_wait();
+  griddep_launch_dependents();
   const int k = blockIdx.x;
   const int64_t target = row_idx[k];
   if (target < 0 || target >= cache_rows) {   // a row outside the cache is skipped and reported
@@ -216,13 +218,16 @@ __global__ void __launch_bounds__(128) append_latent_kernel(
     if (flags & MLA_APPEND_ROPE) {
       const double pos = (double)positions[k];
       for (int i = threadIdx.x; i < dr / 2; i += blockDim.x) {
-        // angle in double so that positions of tens of thousands keep full fp32 accuracy
-        const double ang = pos * pow((double)theta, -2.0 * (double)i / (double)dr);
-        double sn, cs;
-        sincos(ang, &sn, &cs);
-        const double x0 = kp[2 * i], x1 = kp[2 * i + 1];
-        row[dc + 2 * i] = (float)(x0 * cs - x1 * sn);
-        row[dc + 2 * i + 1] = (float)(x0 * sn + x1 * cs);
+        // angle pos * theta^(-2i/d_r) in double, reduced to [-pi, pi] in double, so that the fp32
+        // sine and cosine of the remainder keep full accuracy at positions of tens of thousands
+        const double two_pi = 6.283185307179586476925286766559;
+        const double ang = pos * exp2(-2.0 * (double)i / (double)dr * log2_theta);
+        const double turns = rint(ang * (1.0 / two_pi));
+        float sn, cs;
+        sincosf((float)fma(-turns, two_pi, ang), &sn, &cs);
+        const float x0 = kp[2 * i], x1 = kp[2 * i + 1];
+        row[dc + 2 * i] = fmaf(x0, cs, -x1 * sn);
+        row[dc + 2 * i + 1] = fmaf(x0, sn, x1 * cs);
       }
     } else {
       for (int i = threadIdx.x; i < dr; i += blockDim.x) row[dc + i] = kp[i];
@@ -268,13 +273,13 @@ int append_latent_launch(const mla_dims& d, int32_t cache_dtype, void* cache, in
   const size_t smem = (size_t)W * sizeof(float);
   if (smem > 48 * 1024) return MLA_ERR_UNSUPPORTED;
   if (cache_dtype == MLA_BF16)
-    append_latent_kernel<__nv_bfloat16><<<(unsigned)n_new, 128, smem, s>>>(
-        static_cast<__nv_bfloat16*>(cache), row_idx, c_new, kpe_new, positions, d.kv_lora_rank,
-        d.rope_dim, flags, eps, theta, vec8, cache_rows, status);
+    return launch_pdl(append_latent_kernel<__nv_bfloat16>, dim3((unsigned)n_new), dim3(128), smem, s,
+                      static_cast<__nv_bfloat16*>(cache), row_idx, c_new, kpe_new, positions, d.kv_lora_rank,
+                      d.rope_dim, flags, eps, log2((double)theta), vec8, cache_rows, status);
   else
     append_latent_kernel<float><<<(unsigned)n_new, 128, smem, s>>>(
         static_cast<float*>(cache), row_idx, c_new, kpe_new, positions, d.kv_lora_rank, d.rope_dim,
-        flags, eps, theta, vec8, cache_rows, status);
+        flags, eps, log2((double)theta), vec8, cache_rows, status);
   MLA_LAUNCH_CHECK();
   return MLA_OK;
 }

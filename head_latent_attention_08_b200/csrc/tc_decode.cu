@@ -145,6 +145,8 @@ __device__ __forceinline__ int find_owner(int64_t U, int G, int64_t u) {
 // ---------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) decode_plan_kernel(DecParams p, int32_t* prefix) {
   __shared__ int64_t sums[1024];
+  griddep_wait();                // cu_seqlens and the workspace may be in use by earlier work
+  griddep_launch_dependents();
   const int n = p.nblocks;
   const int per = (n + 1023) / 1024;
   const int k0 = threadIdx.x * per, k1 = min(n, k0 + per);
@@ -247,6 +249,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
   __syncthreads();
   cluster_sync();           // the peer's barriers are initialised before any remote access
   tc_fence_after();
+  griddep_wait();           // the plan, the query block and the cache come from earlier kernels
+  griddep_launch_dependents();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tQ = tmem;               // columns [0, 128): this CTA's latent query columns, bf16 pairs
   const uint32_t tO = tmem + 128;         // columns [128, 384): this CTA's half of O
@@ -751,6 +755,8 @@ __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
   __shared__ int slots[256];
   __shared__ float wts[8][256];
   __shared__ int nsl;
+  griddep_wait();
+  griddep_launch_dependents();
   const int k = blockIdx.x;         // one CTA per block: warp w merges rows w, w + 8, ...
   const int64_t bstart = p.prefix[k], bend = p.prefix[k + 1];
   const int b = k / p.nbps, rb = k % p.nbps;
@@ -905,9 +911,8 @@ static int launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tkr, const 
       return MLA_ERR_CUDA;
     attr_set[dev] = true;
   }
-  tc_decode_kernel<DR><<<2 * p.G, DEC_THREADS, DecCfg<DR>::SMEM, s>>>(tk, tkr, tqr, p);
-  MLA_LAUNCH_CHECK();
-  return MLA_OK;
+  return launch_pdl(tc_decode_kernel<DR>, dim3(2 * p.G), dim3(DEC_THREADS), (size_t)DecCfg<DR>::SMEM, s, tk, tkr,
+                    tqr, p);
 }
 
 int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
@@ -958,13 +963,11 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
       if (!encode_tmap_bf16(&tqr, const_cast<void*>(a.q_abs), 2, dims, st, box, 64)) return MLA_ERR_CUDA;
     }
   }
-  decode_plan_kernel<<<1, 1024, 0, s>>>(p, const_cast<int32_t*>(p.prefix));
-  MLA_LAUNCH_CHECK();
+  int st0 = launch_pdl(decode_plan_kernel, dim3(1), dim3(1024), 0, s, p, const_cast<int32_t*>(p.prefix));
+  if (st0) return st0;
   int st = a.dr == 0 ? launch_decode_t<0>(tk, tkr, tqr, p, s) : launch_decode_t<64>(tk, tkr, tqr, p, s);
   if (st) return st;
-  decode_combine_tc_kernel<<<(unsigned)t.nblocks, 256, 0, s>>>(p);
-  MLA_LAUNCH_CHECK();
-  return MLA_OK;
+  return launch_pdl(decode_combine_tc_kernel, dim3((unsigned)t.nblocks), dim3(256), 0, s, p);
 }
 
 }  // namespace mla

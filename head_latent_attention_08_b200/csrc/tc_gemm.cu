@@ -138,6 +138,8 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();                // the operands may come from the previous kernel of the stream
+  griddep_launch_dependents();
   const uint32_t tmem_d = *tmem_slot;
   int issued = 0;
 
@@ -277,6 +279,8 @@ __global__ void __launch_bounds__(128, 1)
 __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int n_splits, int batch, int N, int M,
                                      void* out, int64_t out_sb, int64_t out_st, int out_f32,
                                      const __nv_bfloat16* gate, int64_t gate_sb, int64_t gate_st, int sigmoid) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t per = (int64_t)batch * N * M;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < per; e += (int64_t)gridDim.x * blockDim.x) {
     float v = 0.f;
@@ -296,6 +300,8 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int n_sp
 
 // out_lat fp32 -> bf16 (the tensor-core operand of the value projection)
 __global__ void f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst, int64_t n4) {
+  griddep_wait();
+  griddep_launch_dependents();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
     const float4 v = src[i];
     __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
@@ -355,9 +361,7 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, TcGemmPar
   // a ring no deeper than the K chunks of one CTA: short-K products then fit several CTAs per SM
   p.stages = std::max(1, std::min(GemmCfg<BN>::STAGES, p.k_chunks));
   const int smem = p.stages * GemmCfg<BN>::STAGE + 1024 + 256;
-  tc_gemm_kernel<BN, A_MN><<<grid, 128, smem, s>>>(ta, tb, p);
-  MLA_LAUNCH_CHECK();
-  return MLA_OK;
+  return launch_pdl(tc_gemm_kernel<BN, A_MN>, grid, dim3(128), (size_t)smem, s, ta, tb, p);
 }
 
 // out[bz][t][m] = epi(sum_k A[bz](m, k) B[bz](t, k)); A MN-major when a_mn
@@ -421,9 +425,10 @@ static int tc_gemm(const GemmOperand& A, bool a_mn, const GemmOperand& Bop, int 
   if (g.splits > 1) {
     const int64_t per = (int64_t)batch * N * M;
     const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(per, 256), 8 * sm_count());
-    splitk_reduce_kernel<<<blocks, 256, 0, s>>>(p.partial, g.splits, batch, N, M, out, out_sb, out_st,
-                                                p.out_f32, p.gate, gate_sb, gate_st, p.sigmoid);
-    MLA_LAUNCH_CHECK();
+    st = launch_pdl(splitk_reduce_kernel, dim3(blocks), dim3(256), 0, s, (const float*)p.partial, g.splits, batch,
+                    N, M, out, (int64_t)out_sb, (int64_t)out_st, p.out_f32, p.gate, (int64_t)gate_sb,
+                    (int64_t)gate_st, p.sigmoid);
+    if (st) return st;
   }
   return MLA_OK;
 }
@@ -481,9 +486,9 @@ int tc_out_project(const mla_dims& d, const float* out_lat, const void* w_uv, co
   {
     const int64_t n4 = n_rows * H * dc / 4;
     const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(n4, 256), 8 * sm_count());
-    f32_to_bf16_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(out_lat),
-                                              static_cast<uint2*>(lat16), n4);
-    MLA_LAUNCH_CHECK();
+    const int st0 = launch_pdl(f32_to_bf16_kernel, dim3(blocks), dim3(256), 0, s,
+                               reinterpret_cast<const float4*>(out_lat), static_cast<uint2*>(lat16), n4);
+    if (st0) return st0;
   }
   // v[t, h, i] = gate * sum_j W_UV[h, i, j] lat[t, h, j]: A = W_UV[h] K-major, B = lat[:, h, :]
   GemmOperand A1{const_cast<void*>(w_uv), (uint64_t)dc, (uint64_t)dv, (uint64_t)H, (uint64_t)(dc * 2),
