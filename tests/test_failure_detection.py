@@ -1,7 +1,8 @@
 """Failure detection without a GPU fault: every device-side wait of the tensor-core kernels is bounded
 by a global-timer limit. A wait that runs out sets MLA_ERR_TIMEOUT in the status word, its kernel
 abandons its work after its own copies and MMAs in flight have ended, and the context stays usable.
-The case here waits on a barrier nothing completes, so its wait certainly runs out."""
+The deterministic case waits on a barrier nothing completes; the decode case cuts the limit to 1 ns,
+so whichever of its waits is not already satisfied gives up, and the next call must be correct."""
 import numpy as np
 import pytest
 import torch
@@ -61,6 +62,35 @@ def test_wait_on_a_barrier_nothing_completes_runs_out():
 def test_negative_wait_limit_is_rejected():
     with pytest.raises(M.MLAError):
         M.mla_set_wait_limit(-1)
+
+
+def test_decode_with_a_tiny_wait_limit_abandons_cleanly():
+    p = I.decode_problem(batch=4, n_heads=128, kv_lora_rank=512, rope_dim=64, qk_nope=128, v_head=128,
+                         d_model=128, seqlens=[300, 65, 1000, 7], dtype="bf16", seed=31)
+    d = mla_dims_of(p)
+    q_abs = dev(O.absorb_query(p.q_nope, p.q_pe, p.w_uk), "bf16")
+    cache = dev(p.cache, "bf16")
+    cu = torch.from_numpy(p.cu_seqlens.astype(np.int32)).cuda()
+    out = torch.empty(4, 128, 512, device="cuda")
+    ws = M.workspace(M.mla_decode_workspace_size(d, torch.bfloat16, 4, 1, 1000, cache.shape[0], 1), "cuda")
+    assert M.mla_check_status() == M.MLA_OK
+    try:
+        M.mla_set_wait_limit(1)
+        M.mla_decode_absorbed(d, q_abs, cache, cu, 4, 1, 1000, M.MLA_DECODE_CAUSAL, out, None, ws)
+        torch.cuda.synchronize()
+        # every wait that was not satisfied at its first poll gives up; the status says whether any did
+        status = M.mla_check_status()
+    finally:
+        M.mla_set_wait_limit(0)
+    assert status in (M.MLA_OK, M.MLA_ERR_TIMEOUT)
+    print(f"decode with a 1 ns wait limit: status {status}")
+    # the status word was cleared by the read, the context is usable and the result correct again
+    M.mla_decode_absorbed(d, q_abs, cache, cu, 4, 1, 1000, M.MLA_DECODE_CAUSAL, out, None, ws)
+    torch.cuda.synchronize()
+    assert M.mla_check_status() == M.MLA_OK
+    ref, _ = O.decode_absorbed(O.store_as(O.absorb_query(p.q_nope, p.q_pe, p.w_uk), "bf16"), p.cache,
+                               p.cu_seqlens, 1, 512, p.kq_scale, True)
+    assert_close(host(out), ref, "bf16", "out_lat after recovery")
 
 
 def test_out_of_range_append_row_is_skipped_and_reported():
