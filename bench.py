@@ -17,6 +17,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import sys
@@ -411,6 +412,127 @@ def run_ours(args):
     return 0
 
 
+def run_rows(args):
+    """Each step of the path on its own (the hot-path rows), timed with CUDA events around the C-ABI
+    call, the L2 flushed between repetitions, against its roofline time max(bytes / HBM, FLOPs /
+    tensor peak). One JSON line per row. Inputs are seeded and drawn on the device with the
+    workloads' shapes and distributions; parity lives in the tests."""
+    import torch
+    from head_latent_attention_08_b200 import build, mla as M
+    from head_latent_attention_08_b200 import inputs as I
+    build.build()
+    M.lib()
+    dev = torch.device("cuda")
+    bf, f32 = torch.bfloat16, torch.float32
+    hbm, tflops, src = peaks()
+    sustained = float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops_sustained"]) \
+        if src == "measured" else 1400.0
+    gen = torch.Generator(device=dev).manual_seed(SEED)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    clk = ClockSampler(torch.cuda.current_device()).__enter__()
+
+    def rnd(*shape, scale=1.0, dtype=bf):
+        return (torch.randn(*shape, device=dev, generator=gen) * scale).to(dtype)
+
+    def timed(fn, reps=20):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(); fn(); b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    def report(row, config, ms, nbytes, flops, note=""):
+        t_mem, t_flop = nbytes / (hbm * 1e9), flops / (tflops * 1e12)
+        bound = "hbm" if t_mem >= t_flop else "tensor"
+        roof_ms = 1e3 * max(t_mem, t_flop)
+        line = {"row": row, "config": config, "ms": ms, "bound": bound, "roofline_ms": roof_ms,
+                "frac": roof_ms / ms, "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
+                "tensor_tflops": flops / (ms * 1e-3) / 1e12 if flops else 0.0,
+                "peaks": {"hbm_gbs": hbm, "bf16_tflops": tflops, "bf16_tflops_sustained": sustained,
+                          "source": src},
+                "frac_of_sustained_tensor": (flops / (sustained * 1e12)) * 1e3 / ms if flops else None}
+        if note:
+            line["note"] = note
+        print(json.dumps(line), flush=True)
+
+    # ---- C3: B64 H128 d_c512 d_r64 T4096, one query token per sequence --------------------------
+    B, H, dc, dr, n, dv, D, T = 64, 128, 512, 64, 128, 128, 5120, 4096
+    d = M.dims(H, dc, dr, n, dv, D)
+    cache = rnd(B * T, dc + dr)
+    cu = torch.arange(0, (B + 1) * T, T, dtype=torch.int32, device=dev)
+    w_uk, w_uv, w_o = rnd(H, n, dc, scale=n ** -0.5), rnd(H, dv, dc, scale=dc ** -0.5), rnd(D, H * dv, scale=(H * dv) ** -0.5)
+    step = M.DecodeStep(d, bf, B, 1, T, cache, cu, w_uk, w_uv, w_o)
+    q_nope, q_pe = rnd(B, H, n), rnd(B, H, dr)
+    c_new, kpe_new = rnd(B, dc, dtype=f32), rnd(B, dr, dtype=f32)
+    row_idx = torch.arange(B, device=dev, dtype=torch.int64) * T + T - 1
+    positions = torch.full((B,), T - 1, dtype=torch.int32, device=dev)
+    c3 = "C3 B64 H128 d_c512 d_r64 T4096 bf16"
+    ms = timed(lambda: M.mla_append_latent(d, cache, row_idx, c_new, kpe_new, positions, step.append_flags))
+    report("a1 latent append (RMSNorm + RoPE)", c3, ms, B * (dc + dr) * (4 + 2), 0,
+           "64 rows: launch- and latency-bound, the roofline time is a few ns")
+    ms = timed(lambda: M.mla_absorb_weights(d, M.MLA_ABSORB_QUERY, q_nope, q_pe, w_uk, B, step.q_abs))
+    report("a2 query absorption", c3, ms, 2 * (H * n * dc + B * H * (n + dr) + B * H * (dc + dr)),
+           2 * B * H * n * dc)
+    ms = timed(lambda: M.mla_decode_absorbed(d, step.q_abs, cache, cu, B, 1, T, step.flags, step.out_lat,
+                                             step.lse, step.ws_dec))
+    report("a3+a4 split-KV decode + combine", c3, ms, B * T * (dc + dr) * 2, B * H * T * (2 * (dc + dr) + 2 * dc))
+    ms = timed(lambda: M.mla_out_project(d, step.out_lat, w_uv, w_o, None, B, step.y, step.ws_out))
+    report("a5 value + output projection", c3, ms, 4 * B * H * dc + 2 * (H * dv * dc + D * H * dv + B * D),
+           2 * B * H * dv * dc + 2 * B * D * H * dv)
+    ms = timed(lambda: step(q_nope, q_pe, c_new, kpe_new, row_idx, positions))
+    report("a1..a5 whole decode step", c3, ms,
+           B * T * (dc + dr) * 2 + 2 * (H * n * dc + H * dv * dc + D * H * dv),
+           B * H * T * (2 * (dc + dr) + 2 * dc) + 2 * B * H * (n * dc + dv * dc) + 2 * B * D * H * dv)
+    del cache, step, w_o
+    torch.cuda.empty_cache()
+    # ---- C4: B16, T ~ U[1024, 32768], n_q 1 and 4 (causal) -----------------------------------------
+    Bs = 16
+    lens = I.ragged_seqlens(Bs, 1024, 32768, seed=I.CONFIG_SEEDS[4])
+    cu4 = torch.from_numpy(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)).to(dev)
+    rows_total, tmax = int(lens.sum()), int(lens.max())
+    cache4 = rnd(rows_total, dc + dr)
+    for nq in (1, 4):
+        q4 = rnd(Bs * nq, H, dc + dr)
+        out4 = torch.empty(Bs * nq, H, dc, device=dev)
+        lse4 = torch.empty(Bs * nq, H, device=dev)
+        ws4 = M.workspace(M.mla_decode_workspace_size(d, bf, Bs, nq, tmax, rows_total, M.MLA_DECODE_CAUSAL), dev)
+        ms = timed(lambda: M.mla_decode_absorbed(d, q4, cache4, cu4, Bs, nq, tmax, M.MLA_DECODE_CAUSAL, out4,
+                                                 lse4, ws4))
+        seen = sum(int(t) - nq + 1 + j for t in lens for j in range(nq))
+        report("a3+a4 split-KV decode + combine", f"C4 B16 T~U[1024,32768] (sum {rows_total}) n_q {nq} causal",
+               ms, rows_total * (dc + dr) * 2, H * seen * (2 * (dc + dr) + 2 * dc))
+    del cache4
+    torch.cuda.empty_cache()
+    # ---- C5: gated prefill B4 S2048 D2048 H16 L512 (causal): the decode with n_q = S and the linears --
+    B5, S5, D5, H5, L5 = 4, 2048, 2048, 16, 512
+    d5 = M.dims(H5, L5, 0, D5 // H5, D5 // H5, D5, 1.0 / math.sqrt(D5 // H5))
+    c5 = "C5 gated prefill B4 S2048 D2048 H16 L512 causal bf16"
+    x = rnd(B5 * S5, D5)
+    wq = rnd(D5, D5, scale=D5 ** -0.5)
+    yq = torch.empty(B5 * S5, D5, dtype=bf, device=dev)
+    ms = timed(lambda: M.mla_linear(x, wq, B5 * S5, D5, D5, 0, yq))
+    report("a6 dense linear (Q = X Wq^T)", c5, ms, 2 * (B5 * S5 * D5 * 2 + D5 * D5), 2 * B5 * S5 * D5 * D5)
+    q5 = rnd(B5 * S5, H5, L5)
+    cache5 = rnd(B5 * S5, L5)
+    cu5 = torch.arange(0, (B5 + 1) * S5, S5, dtype=torch.int32, device=dev)
+    out5 = torch.empty(B5 * S5, H5, L5, device=dev)
+    ws5 = M.workspace(M.mla_decode_workspace_size(d5, bf, B5, S5, S5, B5 * S5, M.MLA_DECODE_CAUSAL), dev)
+    ms = timed(lambda: M.mla_decode_absorbed(d5, q5, cache5, cu5, B5, S5, S5, M.MLA_DECODE_CAUSAL, out5, None,
+                                             ws5))
+    seen5 = B5 * H5 * S5 * (S5 + 1) // 2
+    report("a3+a4 split-KV decode + combine", c5 + " (n_q = S, rows = (token, head))", ms,
+           B5 * S5 * L5 * 2 + B5 * S5 * H5 * L5 * (2 + 4), seen5 * (2 * L5 + 2 * L5))
+    clk.__exit__(None, None, None)
+    print(json.dumps({"clocks": clk.summary(), "device_status": M.mla_check_status()}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -418,6 +540,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rows", action="store_true",
+                    help="time each step of the path on its own against its roofline (one JSON line "
+                         "per row) instead of the benchmark line")
     ap.add_argument("--batch", type=int, default=WORKLOAD["batch"],
                     help="sequences per step (default 64: the benchmark workload; smaller batches "
                          "are for profiling captures and are not benchmark numbers)")
@@ -430,6 +555,8 @@ def main():
         CONFIG["workload"] += f" [batch reduced to {args.batch}: profiling case, not the benchmark]"
     if args.impl == "reference":
         return run_reference(args)
+    if args.rows:
+        return run_rows(args)
     return run_ours(args)
 
 

@@ -748,7 +748,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------------------------
-// combine: one CTA per block; merges the partials of blocks split across clusters and writes
+// combine: 16 CTAs per block (8 rows each); merges the partials of blocks split across clusters and writes
 // zeros / -inf for blocks with nothing to attend to
 // ---------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
@@ -757,13 +757,14 @@ __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
   __shared__ int nsl;
   griddep_wait();
   griddep_launch_dependents();
-  const int k = blockIdx.x;         // one CTA per block: warp w merges rows w, w + 8, ...
+  const int k = blockIdx.x;
+  const int r0 = blockIdx.y * 8;     // this CTA's 8 rows of the block (one per warp)
   const int64_t bstart = p.prefix[k], bend = p.prefix[k + 1];
   const int b = k / p.nbps, rb = k % p.nbps;
   const int rows_seq = p.n_q * p.H;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (bend == bstart) {
-    for (int r = warp; r < DEC_ROWS; r += 8) {
+    for (int r = r0 + warp; r < r0 + 8; r += 8) {
       const int ri = rb * DEC_ROWS + r;
       if (ri >= rows_seq) break;
       const int64_t orow = (int64_t)b * rows_seq + ri;
@@ -789,7 +790,7 @@ __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
   }
   __syncthreads();
   const int n = nsl;
-  for (int r = warp; r < DEC_ROWS; r += 8) {
+  for (int r = r0 + warp; r < r0 + 8; r += 8) {
     const int ri = rb * DEC_ROWS + r;
     if (ri >= rows_seq) break;
     float M = -INFINITY;
@@ -967,7 +968,8 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
   if (st0) return st0;
   int st = a.dr == 0 ? launch_decode_t<0>(tk, tkr, tqr, p, s) : launch_decode_t<64>(tk, tkr, tqr, p, s);
   if (st) return st;
-  return launch_pdl(decode_combine_tc_kernel, dim3((unsigned)t.nblocks), dim3(256), 0, s, p);
+  // 16 CTAs per block (8 rows each): a split block's merge reads 2-3 partial slots of 256 KB
+  return launch_pdl(decode_combine_tc_kernel, dim3((unsigned)t.nblocks, DEC_ROWS / 8), dim3(256), 0, s, p);
 }
 
 }  // namespace mla
