@@ -260,18 +260,82 @@ class DecodeStep:
                                                           cache.shape[0], self.flags), dev)
         self.ws_out = workspace(mla_out_project_workspace_size(d, dtype, nq), dev)
 
-    def __call__(self, q_nope, q_pe, c_new, kpe_new, row_idx, positions, stream=None):
+    def __call__(self, q_nope, q_pe, c_new, kpe_new, row_idx, positions, stream=None, y=None):
         d = self.d
         nq = self.batch * self.n_q
+        y = self.y if y is None else y
         mla_append_latent(d, self.cache, row_idx, c_new, kpe_new, positions, self.append_flags,
                           stream=stream)
         mla_absorb_weights(d, MLA_ABSORB_QUERY, q_nope, q_pe if d.rope_dim else None, self.w_uk, nq,
                            self.q_abs, stream=stream)
         mla_decode_absorbed(d, self.q_abs, self.cache, self.cu, self.batch, self.n_q, self.max_seqlen,
                             self.flags, self.out_lat, self.lse, self.ws_dec, stream=stream)
-        mla_out_project(d, self.out_lat, self.w_uv, self.w_o, None, nq, self.y, self.ws_out,
+        mla_out_project(d, self.out_lat, self.w_uv, self.w_o, None, nq, y, self.ws_out,
                         stream=stream)
-        return self.y
+        return y
+
+
+class HostStream:
+    """Decode steps fed from pinned host memory, with the transfers overlapped with the compute.
+    While step k runs on the compute stream, step k+1's inputs travel host -> device on one side
+    stream and step k-1's output travels device -> host on another. Two sets of device buffers
+    alternate, and events order every reuse: a buffer set takes new inputs once the step that read
+    it is done, and its output buffer is written again once its previous output has reached the
+    host. ``submit`` enqueues one step and returns at once; ``wait(stream)`` makes ``stream`` wait
+    for every submitted step's output to be in host memory."""
+
+    def __init__(self, step: DecodeStep, stream=None):
+        self.step = step
+        dev = step.cache.device
+        self.compute = stream if stream is not None else torch.cuda.current_stream(dev)
+        self.h2d = torch.cuda.Stream(device=dev)
+        self.d2h = torch.cuda.Stream(device=dev)
+        d, nq = step.d, step.batch * step.n_q
+
+        def buffers():
+            return dict(q_nope=torch.empty(nq, d.n_heads, d.qk_nope, dtype=step.dtype, device=dev),
+                        q_pe=torch.empty(nq, d.n_heads, d.rope_dim, dtype=step.dtype, device=dev),
+                        c_new=torch.empty(nq, d.kv_lora_rank, dtype=torch.float32, device=dev),
+                        kpe_new=torch.empty(nq, d.rope_dim, dtype=torch.float32, device=dev),
+                        y=torch.empty_like(step.y))
+
+        self.buf = [buffers(), buffers()]
+        self.inputs_in = [torch.cuda.Event() for _ in range(2)]
+        self.step_done = [torch.cuda.Event() for _ in range(2)]
+        self.output_out = [torch.cuda.Event() for _ in range(2)]
+        self.used = [False, False]
+        self.k = 0
+
+    def submit(self, h_q_nope, h_q_pe, h_c_new, h_kpe, row_idx, positions, h_y):
+        i = self.k & 1
+        b = self.buf[i]
+        with torch.cuda.stream(self.h2d):
+            if self.used[i]:
+                self.h2d.wait_event(self.step_done[i])
+            b["q_nope"].copy_(h_q_nope, non_blocking=True)
+            b["q_pe"].copy_(h_q_pe, non_blocking=True)
+            b["c_new"].copy_(h_c_new, non_blocking=True)
+            b["kpe_new"].copy_(h_kpe, non_blocking=True)
+            self.inputs_in[i].record(self.h2d)
+        self.compute.wait_event(self.inputs_in[i])
+        if self.used[i]:
+            self.compute.wait_event(self.output_out[i])
+        with torch.cuda.stream(self.compute):
+            self.step(b["q_nope"], b["q_pe"], b["c_new"], b["kpe_new"], row_idx, positions,
+                      stream=self.compute, y=b["y"])
+            self.step_done[i].record(self.compute)
+        with torch.cuda.stream(self.d2h):
+            self.d2h.wait_event(self.step_done[i])
+            h_y.copy_(b["y"], non_blocking=True)
+            self.output_out[i].record(self.d2h)
+        self.used[i] = True
+        self.k += 1
+
+    def wait(self, stream=None):
+        s = stream if stream is not None else self.compute
+        for i in range(2):
+            if self.used[i]:
+                s.wait_event(self.output_out[i])
 
 
 def gated_mla(x: torch.Tensor, wq: torch.Tensor, wc: torch.Tensor, wk: torch.Tensor, wv: torch.Tensor,
