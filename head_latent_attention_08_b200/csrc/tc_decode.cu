@@ -330,7 +330,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     // An event loop: P.C of the oldest tile whose P is ready is issued first (it frees a shared
     // memory stage for the producer), and QK^T of the next tile as soon as its cache tile has landed,
     // its query is in place and its S/P slot is free (the P.C two tiles back has been issued; MMAs
-    // run in issue order).
+    // run in issue order). A ready P waits while a QK^T is being issued: putting its P.C between the
+    // QK^T's MMAs measured slower, since the scores, not P.C, are on the per-tile critical path.
     // One thread issues every MMA, and its scalar work sits between consecutive MMAs: descriptors are
     // built once for stage 0 and advanced by constant offsets (the 14-bit start-address field holds
     // shared addresses >> 4 below 256 KB, so the additions never carry into the other fields).
@@ -352,25 +353,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     uint32_t idle = 0;
     uint64_t t_idle = 0;
     bool ok = true;
+    // issue P.C of tile gp if its P is in (gq_lim: tiles whose QK^T has been issued)
+    auto try_pv = [&](int64_t gq_lim) -> bool {
+      if (gp >= gq_lim || !mbar_test_wait(&p_full[gp & 1], (uint32_t)(gp >> 1) & 1u)) return false;
+      tc_fence_after();
+      const int sl = (int)(gp & 1);
+      const int s = (int)(gp % ST);
+      const bool first = (first_bits >> (gp & 31)) & 1u;
+      // B = this CTA's 256 latent columns of the tile: MN-major, 64-column boxes K_BOX apart
+      const uint64_t cd = cd0 + (uint64_t)s * kStage;
+      const uint32_t ta = tS + sl * 64;
+#pragma unroll
+      for (int kk = 0; kk < DEC_BT / 16; ++kk)
+        mma_bf16_ts(tO, ta + kk * 8, cd + (uint64_t)(kk * (2048 >> 4)), idesc_pv, (first && kk == 0) ? 0u : 1u);
+      mma_commit(&k_empty[s]);
+      mma_commit(o_done);
+      ++gp;
+      return true;
+    };
     while (gp < n_total) {
       if (*abort_flag) { ok = false; break; }
-      bool progressed = false;
-      if (gp < gq && mbar_test_wait(&p_full[gp & 1], (uint32_t)(gp >> 1) & 1u)) {
-        tc_fence_after();
-        const int sl = (int)(gp & 1);
-        const int s = (int)(gp % ST);
-        const bool first = (first_bits >> (gp & 31)) & 1u;
-        // B = this CTA's 256 latent columns of the tile: MN-major, 64-column boxes K_BOX apart
-        const uint64_t cd = cd0 + (uint64_t)s * kStage;
-        const uint32_t ta = tS + sl * 64;
-#pragma unroll
-        for (int kk = 0; kk < DEC_BT / 16; ++kk)
-          mma_bf16_ts(tO, ta + kk * 8, cd + (uint64_t)(kk * (2048 >> 4)), idesc_pv, (first && kk == 0) ? 0u : 1u);
-        mma_commit(&k_empty[s]);
-        mma_commit(o_done);
-        ++gp;
-        progressed = true;
-      }
+      bool progressed = try_pv(gq);
       if (gq < n_total && gq <= gp + 1) {
         if (gq == qseg_end) {
           const int64_t bend = p.prefix[kseg + 1];
@@ -394,6 +397,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           const int sl = (int)(gq & 1);
           const uint32_t td = tS + sl * 64;
           const uint64_t kd = kd0 + (uint64_t)s * kStage;
+          // the first tile of a segment opens its P.C with accumulate = 0
+          const uint32_t bit = 1u << (gq & 31);
+          first_bits = (gq == qseg_start) ? (first_bits | bit) : (first_bits & ~bit);
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
 #pragma unroll
@@ -409,8 +415,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           }
           mma_commit(&s_full[sl]);
           if (gq + 1 == qseg_end) mma_commit(q_empty);
-          const uint32_t bit = 1u << (gq & 31);
-          first_bits = (gq == qseg_start) ? (first_bits | bit) : (first_bits & ~bit);
           ++gq;
           progressed = true;
         }
@@ -521,27 +525,65 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       if (*abort_flag) return;
       if (!mbar_wait(bar, (uint32_t)parity, p.wait_ns, p.status)) *abort_flag = 1;
     };
-    // this warpgroup's 128 of the CTA's 256 latent query columns of block kq, into TMEM (one batch of
-    // loads per thread), once the previous segment's last QK^T has read the query
+    // this warpgroup's 128 of the CTA's 256 latent query columns of block kq, into TMEM, once the
+    // previous segment's last QK^T has read the query. Thread = row = TMEM lane, so a plain load gives
+    // each thread its own row and every load instruction touches 32 rows. The first query of the CTA
+    // (all CTAs load theirs at once) goes through this warp's 4 KB of the send-staging slots instead,
+    // which nothing else touches before this CTA's first QK^T: coalesced loads (4 rows x 128 B per
+    // instruction), then each thread reads its row back. Chunks are stored swizzled (chunk ^ row % 8),
+    // so both the stores and the row reads are free of bank conflicts.
+    uint8_t* wscratch_q = smem + Cfg::OFF_XS + (warp - 4) * 4096;
     auto load_query = [&](int kq, int segment) {
       const int bq = kq / p.nbps, rbq = kq % p.nbps;
-      const int64_t qr = (int64_t)bq * p.n_q * p.H + (int64_t)rbq * DEC_ROWS + row;
+      const int64_t qr0 = (int64_t)bq * p.n_q * p.H + (int64_t)rbq * DEC_ROWS + quarter * 32;   // warp's first row
       if (segment > 0) wait_cta(q_empty, (segment - 1) & 1);
       tc_fence_after();
-      const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + qr * p.W + dim0 + wg * 128);
-      const bool in = qr < p.q_rows;
-      uint4 v[16];
+      if (segment == 0) {
+        uint4 v[16];
+        const int chunk = lane & 7;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] = in ? src[j] : make_uint4(0u, 0u, 0u, 0u);
+        for (int h = 0; h < 2; ++h) {
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {      // 2 x 32 TMEM columns = 128 bf16
-        uint32_t r[32];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          r[4 * j] = v[cc * 8 + j].x; r[4 * j + 1] = v[cc * 8 + j].y;
-          r[4 * j + 2] = v[cc * 8 + j].z; r[4 * j + 3] = v[cc * 8 + j].w;
+          for (int j = 0; j < 8; ++j) {
+            const int64_t qr = qr0 + 4 * j + (lane >> 3);
+            const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + qr * p.W + dim0 + wg * 128 + h * 64) + chunk;
+            v[h * 8 + j] = qr < p.q_rows ? *src : make_uint4(0u, 0u, 0u, 0u);
+          }
         }
-        tmem_st32(tQ + lane_off + wg * 64 + cc * 32, r);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int rr = 4 * j + (lane >> 3);
+            *reinterpret_cast<uint4*>(wscratch_q + rr * 128 + ((chunk ^ (rr & 7)) * 16)) = v[h * 8 + j];
+          }
+          __syncwarp();
+          uint32_t r[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 w = *reinterpret_cast<const uint4*>(wscratch_q + lane * 128 + ((c ^ (lane & 7)) * 16));
+            r[4 * c] = w.x; r[4 * c + 1] = w.y; r[4 * c + 2] = w.z; r[4 * c + 3] = w.w;
+          }
+          __syncwarp();
+          tmem_st32(tQ + lane_off + wg * 64 + h * 32, r);
+        }
+      } else {
+        const int64_t qr = qr0 + lane;
+        const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + qr * p.W + dim0 + wg * 128);
+        const bool in = qr < p.q_rows;
+        uint4 v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = in ? src[j] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {      // 2 x 32 TMEM columns = 128 bf16
+          uint32_t r[32];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            r[4 * j] = v[cc * 8 + j].x; r[4 * j + 1] = v[cc * 8 + j].y;
+            r[4 * j + 2] = v[cc * 8 + j].z; r[4 * j + 3] = v[cc * 8 + j].w;
+          }
+          tmem_st32(tQ + lane_off + wg * 64 + cc * 32, r);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -702,17 +744,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
                             : p.o_part + ((int64_t)slot * DEC_ROWS + row) * DEC_DC + dim0 + wg * 128;
       const float mul = complete ? inv : 1.f;
       const bool write = complete ? valid : true;
+      if (send_u >= u1 && !*abort_flag) {
+        // the CTA's last segment: every tile of the peer has landed and been read, so the receive
+        // slots are free. Each warp turns its 32 rows x 32 columns of O around in its 4 KB of them
+        // (swizzled as for the query) and stores 4 rows x 128 B per instruction.
+        uint8_t* wscratch = smem + Cfg::OFF_X + (warp - 4) * 4096;
+        const int chunk = lane & 7;
 #pragma unroll 1
-      for (int cc = 0; cc < DEC_HALF / 2; cc += 32) {
-        uint32_t r[32];
-        tmem_ld32(tO + lane_off + wg * 128 + cc, r);
-        tmem_wait_ld();
-        if (write) {
-          float4* d4 = reinterpret_cast<float4*>(dst + cc);
+        for (int cc = 0; cc < DEC_HALF / 2; cc += 32) {
+          uint32_t r[32];
+          tmem_ld32(tO + lane_off + wg * 128 + cc, r);
+          tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            d4[c] = make_float4(__uint_as_float(r[4 * c]) * mul, __uint_as_float(r[4 * c + 1]) * mul,
-                                __uint_as_float(r[4 * c + 2]) * mul, __uint_as_float(r[4 * c + 3]) * mul);
+            *reinterpret_cast<float4*>(wscratch + lane * 128 + ((c ^ (lane & 7)) * 16)) =
+                make_float4(__uint_as_float(r[4 * c]) * mul, __uint_as_float(r[4 * c + 1]) * mul,
+                            __uint_as_float(r[4 * c + 2]) * mul, __uint_as_float(r[4 * c + 3]) * mul);
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int rr = 4 * j + (lane >> 3);            // row within the warp's 32
+            const int rw = quarter * 32 + rr;              // row within the block
+            const float4 w = *reinterpret_cast<const float4*>(wscratch + rr * 128 + ((chunk ^ (rr & 7)) * 16));
+            float* d;
+            bool ok_row;
+            if (complete) {
+              ok_row = rb * DEC_ROWS + rw < p.n_q * p.H;
+              d = p.out_lat + ((int64_t)b * p.n_q * p.H + rb * DEC_ROWS + rw) * DEC_DC;
+            } else {
+              ok_row = true;
+              d = p.o_part + ((int64_t)slot * DEC_ROWS + rw) * DEC_DC;
+            }
+            if (ok_row) *reinterpret_cast<float4*>(d + dim0 + wg * 128 + cc + chunk * 4) = w;
+          }
+          __syncwarp();
+        }
+      } else {
+#pragma unroll 1
+        for (int cc = 0; cc < DEC_HALF / 2; cc += 32) {
+          uint32_t r[32];
+          tmem_ld32(tO + lane_off + wg * 128 + cc, r);
+          tmem_wait_ld();
+          if (write) {
+            float4* d4 = reinterpret_cast<float4*>(dst + cc);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              d4[c] = make_float4(__uint_as_float(r[4 * c]) * mul, __uint_as_float(r[4 * c + 1]) * mul,
+                                  __uint_as_float(r[4 * c + 2]) * mul, __uint_as_float(r[4 * c + 3]) * mul);
+          }
         }
       }
       if (rank == 0 && wg == 0) {
