@@ -16,10 +16,11 @@
 //    partial S over them, and the two partials (rounded to fp16) are exchanged through distributed
 //    shared memory; both CTAs form the same S = fp16(S0) + fp16(S1), run the same fp32 online
 //    softmax and accumulate their half of O = P . C in TMEM (256 columns).
-//  * This CTA's 256 latent columns of the query block live in TMEM (128 columns of packed bf16) and
-//    are the A operand of QK^T straight from TMEM: shared memory is left to the cache tiles (4 stages)
-//    and its bandwidth to the B operands. P (bf16) is written over its S tile and is the A operand of
-//    P . C from TMEM. TMEM: Q 128 + O 256 + two 64-column S/P slots = 512 columns.
+//  * The first 128 of this CTA's 256 latent query columns live in TMEM (64 columns of packed bf16,
+//    the A operand of QK^T straight from TMEM), the other 128 and the rotary columns in shared memory
+//    (brought by TMA). P (bf16) is written over its S tile and is the A operand of P . C from TMEM.
+//    TMEM: Q 64 + O 256 + three 64-column S/P slots = 512 columns, so three tiles are between QK^T
+//    and P.C at once; shared memory holds three cache stages.
 //  * O is rescaled only when a row's running maximum grows by more than 2^8 (the result is exact:
 //    numerator and denominator share the stale reference maximum).
 //  * Work: the (block, 64-position tile) units of all sequences are split evenly over the clusters
@@ -52,20 +53,24 @@ constexpr int DEC_DC = 512;         // latent width handled by this kernel
 constexpr int DEC_HALF = 256;       // latent columns per CTA
 constexpr int DEC_ROWS = 128;       // rows per block
 constexpr int DEC_PREFETCH = 4;     // tiles brought into L2 beyond the shared-memory ring
+constexpr int DEC_SLOTS = 3;        // S/P slots in TMEM: tiles between QK^T and P.C at once
+constexpr int DEC_XSLOTS = 1;       // score-exchange slots (receive + send staging) in shared memory
 
 template <int DR>
 struct DecCfg {
+  static constexpr int QL_BOX = DEC_ROWS * 128;         // 128 rows x 64 latent query columns (128 B)
   static constexpr int QR_BOX = DR ? 128 * 64 : 0;      // this CTA's 32 rotary query columns, 128 x 64 B
   static constexpr int K_BOX = DEC_BT * 128;            // 64 positions x 64 latent columns (128 B)
   static constexpr int KR_BOX = DR ? DEC_BT * 64 : 0;   // 64 positions x 32 rotary columns (64 B)
   static constexpr int STAGE_BYTES = 4 * K_BOX + KR_BOX;
   static constexpr int STAGES = 4;
   static constexpr int X_TILE = DEC_ROWS * DEC_BT * 2;   // one tile of partial scores, fp16, rows of 128 B
-  static constexpr int OFF_QR = 0;
-  static constexpr int OFF_K = QR_BOX;
+  static constexpr int OFF_QL = 0;                       // latent query columns [128, 256) of this CTA
+  static constexpr int OFF_QR = 2 * QL_BOX;
+  static constexpr int OFF_K = OFF_QR + QR_BOX;
   static constexpr int OFF_X = OFF_K + STAGES * STAGE_BYTES;
-  static constexpr int OFF_XS = OFF_X + 2 * X_TILE;      // two receive slots, then two send stagings
-  static constexpr int OFF_BAR = OFF_XS + 2 * X_TILE;
+  static constexpr int OFF_XS = OFF_X + DEC_XSLOTS * X_TILE;   // receive slots, then send stagings
+  static constexpr int OFF_BAR = OFF_XS + DEC_XSLOTS * X_TILE;
   static constexpr int OFF_RED = OFF_BAR + 256;          // row maxima [2][2][128], row sums [2][128]
   static constexpr int SMEM = OFF_RED + 6 * DEC_ROWS * 4 + 1024;
 };
@@ -180,11 +185,15 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecParams p, int32_t*
 template <int DR>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tkr,
-                     const __grid_constant__ CUtensorMap tqr, DecParams p) {
+                     const __grid_constant__ CUtensorMap tqr, const __grid_constant__ CUtensorMap tql,
+                     DecParams p) {
   using Cfg = DecCfg<DR>;
   constexpr int ST = Cfg::STAGES;
+  constexpr int NS = DEC_SLOTS;
+  constexpr int XS = DEC_XSLOTS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQL = smem + Cfg::OFF_QL;
   uint8_t* sQR = smem + Cfg::OFF_QR;
   uint8_t* sK = smem + Cfg::OFF_K;
   uint8_t* sX = smem + Cfg::OFF_X;
@@ -192,17 +201,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint64_t* k_full = bars;              // [ST] cache tile landed
   uint64_t* k_empty = k_full + ST;      // [ST] cache tile consumed by its P.C
-  uint64_t* qr_full = k_empty + ST;     // rotary query columns landed (TMA)
-  uint64_t* ql_full = qr_full + 1;      // latent query columns written to TMEM (query warps)
+  uint64_t* qr_full = k_empty + ST;     // query columns in shared memory landed (TMA)
+  uint64_t* ql_full = qr_full + 1;      // latent query columns written to TMEM (softmax warps)
   uint64_t* q_empty = ql_full + 1;      // last QK^T of a segment done: the query may be replaced
-  uint64_t* s_full = q_empty + 1;       // [2] partial S of a slot computed (MMA -> sender)
-  uint64_t* own_ready = s_full + 2;     // [2] own fp16 partials staged, S read (sender -> softmax)
-  uint64_t* p_full = own_ready + 2;     // [2] P written (softmax -> MMA)
-  uint64_t* o_done = p_full + 2;        // [1] a P.C completed
-  uint64_t* x_full = o_done + 1;        // [2] peer's partial scores arrived (transaction count)
-  uint64_t* x_empty = x_full + 2;       // [2] both softmaxes have read this CTA's scores
-  uint64_t* drain = x_empty + 2;        // [1] MMA drain on abort
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* s_full = q_empty + 1;       // [NS] partial S of a slot computed (MMA -> sender)
+  uint64_t* own_ready = s_full + NS;    // [NS] own fp16 partials staged, S read (sender -> softmax)
+  uint64_t* p_full = own_ready + NS;    // [NS] P written (softmax -> MMA)
+  uint64_t* o_done = p_full + NS;       // [NS] the P.C of a tile of this slot completed
+  uint64_t* x_full = o_done + NS;       // [XS] peer's partial scores arrived (transaction count)
+  uint64_t* x_empty = x_full + XS;      // [XS] both softmaxes have read this CTA's scores
+  uint64_t* drain = x_empty + XS;       // [2] MMA drain on abort, one per issuing thread
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -220,22 +229,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     mbar_init(qr_full, 1);
     mbar_init(ql_full, 8);            // one arrival per softmax warp (each writes its rows' half)
     mbar_init(q_empty, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&own_ready[s], 4);    // one arrival per sender warp
       mbar_init(&p_full[s], 8);       // one arrival per softmax warp
+      mbar_init(&o_done[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < XS; ++s) {
       mbar_init(&x_full[s], 1);
       mbar_init(&x_empty[s], 2);      // the peer's softmax (remote) and this CTA's (local)
     }
-    mbar_init(o_done, 1);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     // arm the first use of each receive slot: one local arrival plus the peer's four 4 KB bulk copies
-    for (int s = 0; s < 2; ++s) mbar_arrive_expect_tx(&x_full[s], Cfg::X_TILE);
+    for (int s = 0; s < XS; ++s) mbar_arrive_expect_tx(&x_full[s], Cfg::X_TILE);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tk);
+    prefetch_tmap(&tql);
     if (DR) {
       prefetch_tmap(&tkr);
       prefetch_tmap(&tqr);
@@ -252,9 +263,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
   griddep_wait();           // the plan, the query block and the cache come from earlier kernels
   griddep_launch_dependents();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tQ = tmem;               // columns [0, 128): this CTA's latent query columns, bf16 pairs
-  const uint32_t tO = tmem + 128;         // columns [128, 384): this CTA's half of O
-  const uint32_t tS = tmem + 384;         // columns [384, 512): two 64-column S / P slots
+  const uint32_t tQ = tmem;               // columns [0, 64): this CTA's latent query columns [0, 128), bf16 pairs
+  const uint32_t tO = tmem + 64;          // columns [64, 320): this CTA's half of O
+  const uint32_t tS = tmem + 320;         // columns [320, 512): three 64-column S / P slots
 
   const int64_t U = p.prefix[p.nblocks];
   const int64_t u0 = range_start(U, p.G, pair), u1 = range_start(U, p.G, pair + 1);
@@ -276,11 +287,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       const int b = k / p.nbps, rb = k % p.nbps;
       int64_t sstart; int T;
       seq_bounds(p, b, sstart, T);
-      if (DR) {
+      {
+        // the query columns that QK^T reads from shared memory: latent [128, 256) of this CTA and
+        // its rotary columns, once the previous segment's last QK^T is done
         const int qrow = (int)((int64_t)b * p.n_q * p.H + (int64_t)rb * DEC_ROWS);
         if (seg > 0 && (*abort_flag || !mbar_wait(q_empty, (seg - 1) & 1, p.wait_ns, p.status))) { ok = false; break; }
-        mbar_arrive_expect_tx(qr_full, Cfg::QR_BOX);
-        tma_load_2d(sQR, &tqr, qr_full, rdim0, qrow);
+        mbar_arrive_expect_tx(qr_full, 2 * Cfg::QL_BOX + Cfg::QR_BOX);
+        for (int kb = 0; kb < 2; ++kb) tma_load_2d(sQL + kb * Cfg::QL_BOX, &tql, qr_full, dim0 + 128 + kb * 64, qrow);
+        if (DR) tma_load_2d(sQR, &tqr, qr_full, rdim0, qrow);
         ++q_loads;
       }
       int pf_next = 0;                      // next tile of this segment to warm in L2
@@ -325,116 +339,106 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         (void)mbar_wait(&k_full[i % ST], (int)(i / ST) & 1, drain_ns, p.status);
       if (q_loads > 0) (void)mbar_wait(qr_full, (q_loads - 1) & 1, drain_ns, p.status);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ------------------------------- MMA issuer -------------------------------
-    // An event loop: P.C of the oldest tile whose P is ready is issued first (it frees a shared
-    // memory stage for the producer), and QK^T of the next tile as soon as its cache tile has landed,
-    // its query is in place and its S/P slot is free (the P.C two tiles back has been issued; MMAs
-    // run in issue order). A ready P waits while a QK^T is being issued: putting its P.C between the
-    // QK^T's MMAs measured slower, since the scores, not P.C, are on the per-tile critical path.
-    // One thread issues every MMA, and its scalar work sits between consecutive MMAs: descriptors are
-    // built once for stage 0 and advanced by constant offsets (the 14-bit start-address field holds
-    // shared addresses >> 4 below 256 KB, so the additions never carry into the other fields).
+  } else if ((warp == 1 || warp == 2) && lane == 0) {
+    // ------------------------------- MMA issuers -------------------------------
+    // Two threads issue the MMAs (one thread alone issues about one MMA per 50-90 cycles, and QK^T is
+    // 18 MMAs): warp 1 issues QK^T of every tile, warp 2 P.C of every tile. Tile g's QK^T writes the
+    // S/P slot that P.C of tile g - NS read, so it waits for that P.C to complete (its o_done phase).
+    // P.C of tile g reads the cache stage that QK^T of tile g read as well; QK^T completed before the
+    // softmax could write P (s_full), so the stage's release after P.C covers both readers. Only
+    // warp 2 accumulates into O, in issue order.
+    // Each thread's scalar work sits between consecutive MMAs: descriptors are built once for stage 0
+    // and advanced by constant offsets (the 14-bit start-address field holds shared addresses >> 4
+    // below 256 KB, so the additions never carry into the other fields).
+    const bool qk_issuer = warp == 1;
     constexpr uint32_t idesc_qk = idesc_bf16_f32(128, DEC_BT, false, false);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, DEC_HALF, false, true);
     constexpr uint64_t kStage = (uint64_t)(Cfg::STAGE_BYTES >> 4);
     const uint32_t qr_base = smem_u32(sQR), k_base = smem_u32(sK);
+    const uint64_t qld0 = smem_desc_sw128(smem_u32(sQL), 16, 1024);          // latent query [128, 256), K-major (A)
     const uint64_t kd0 = smem_desc_sw128(k_base, 16, 1024);                  // cache tile, K-major (B of QK^T)
     const uint64_t cd0 = smem_desc_sw128(k_base, Cfg::K_BOX, 1024);          // cache tile, MN-major (B of P.C)
     const uint64_t rd0 = smem_desc_sw64(k_base + 4 * Cfg::K_BOX, 16, 512);   // rotary columns of the tile
     const uint64_t qd0 = smem_desc_sw64(qr_base, 16, 512);                   // rotary query columns
-    int64_t gq = 0, gp = 0;               // next tile for QK^T, next tile for P.C
-    int64_t qseg_start = 0, qseg_end = 0; // tiles [start, end) of the segment QK^T is in
-    int segq = -1;
-    bool ql_ok = false, qr_ok = false;
-    int64_t useg = u0;
+    auto wait_mma = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return !*abort_flag && mbar_wait(bar, parity, p.wait_ns, p.status);
+    };
+    // segments in tile order: [seg_start, seg_end) is the segment holding tile g
+    int64_t useg = u0, seg_start = 0, seg_end = 0;
     int kseg = u0 < u1 ? find_block(p.prefix, p.nblocks, u0) : 0;
-    uint32_t first_bits = 0;              // bit (g & 31): tile g opens its segment
-    uint32_t idle = 0;
-    uint64_t t_idle = 0;
-    bool ok = true;
-    // issue P.C of tile gp if its P is in (gq_lim: tiles whose QK^T has been issued)
-    auto try_pv = [&](int64_t gq_lim) -> bool {
-      if (gp >= gq_lim || !mbar_test_wait(&p_full[gp & 1], (uint32_t)(gp >> 1) & 1u)) return false;
-      tc_fence_after();
-      const int sl = (int)(gp & 1);
-      const int s = (int)(gp % ST);
-      const bool first = (first_bits >> (gp & 31)) & 1u;
-      // B = this CTA's 256 latent columns of the tile: MN-major, 64-column boxes K_BOX apart
-      const uint64_t cd = cd0 + (uint64_t)s * kStage;
-      const uint32_t ta = tS + sl * 64;
-#pragma unroll
-      for (int kk = 0; kk < DEC_BT / 16; ++kk)
-        mma_bf16_ts(tO, ta + kk * 8, cd + (uint64_t)(kk * (2048 >> 4)), idesc_pv, (first && kk == 0) ? 0u : 1u);
-      mma_commit(&k_empty[s]);
-      mma_commit(o_done);
-      ++gp;
+    int segi = -1;
+    auto advance_segment = [&](int64_t g) {
+      if (g < seg_end) return false;
+      const int64_t bend = p.prefix[kseg + 1];
+      const int64_t send = u1 < bend ? u1 : bend;
+      seg_start = g;
+      seg_end = g + (send - useg);
+      ++segi;
+      useg = send;
+      if (useg < u1) kseg = find_block(p.prefix, p.nblocks, useg);
       return true;
     };
-    while (gp < n_total) {
-      if (*abort_flag) { ok = false; break; }
-      bool progressed = try_pv(gq);
-      if (gq < n_total && gq <= gp + 1) {
-        if (gq == qseg_end) {
-          const int64_t bend = p.prefix[kseg + 1];
-          const int64_t send = u1 < bend ? u1 : bend;
-          qseg_start = gq;
-          qseg_end = gq + (send - useg);
-          ++segq;
-          ql_ok = false;
-          qr_ok = !DR;
-          useg = send;
-          if (useg < u1) kseg = find_block(p.prefix, p.nblocks, useg);
+    bool ok = true;
+    if (qk_issuer) {
+      for (int64_t g = 0; g < n_total; ++g) {
+        if (advance_segment(g)) {
+          // this segment's query: TMEM half (softmax warps) and shared-memory half (TMA)
+          if (!wait_mma(ql_full, (uint32_t)segi & 1u) || !wait_mma(qr_full, (uint32_t)segi & 1u)) { ok = false; break; }
         }
-        if (!ql_ok && mbar_test_wait(ql_full, (uint32_t)segq & 1u)) {
-          tc_fence_after();
-          ql_ok = true;
+        const int s = (int)(g % ST);
+        const int sl = (int)(g % NS);
+        if (!wait_mma(&k_full[s], (uint32_t)(g / ST) & 1u)) { ok = false; break; }
+        if (g >= NS && !wait_mma(&o_done[sl], (uint32_t)((g / NS) - 1) & 1u)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t td = tS + sl * 64;
+        const uint64_t kd = kd0 + (uint64_t)s * kStage;
+        // latent columns [0, 128) of this CTA: the query from TMEM; [128, 256): from shared memory
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ts(td, tQ + kb * 32 + kk * 8, kd + (uint64_t)((kb * Cfg::K_BOX + kk * 32) >> 4), idesc_qk,
+                        (kb | kk) ? 1u : 0u);
         }
-        if (!qr_ok && mbar_test_wait(qr_full, (uint32_t)segq & 1u)) qr_ok = true;
-        const int s = (int)(gq % ST);
-        if (ql_ok && qr_ok && mbar_test_wait(&k_full[s], (uint32_t)(gq / ST) & 1u)) {
-          tc_fence_after();
-          const int sl = (int)(gq & 1);
-          const uint32_t td = tS + sl * 64;
-          const uint64_t kd = kd0 + (uint64_t)s * kStage;
-          // the first tile of a segment opens its P.C with accumulate = 0
-          const uint32_t bit = 1u << (gq & 31);
-          first_bits = (gq == qseg_start) ? (first_bits | bit) : (first_bits & ~bit);
 #pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
+        for (int kb = 2; kb < 4; ++kb) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ts(td, tQ + kb * 32 + kk * 8, kd + (uint64_t)((kb * Cfg::K_BOX + kk * 32) >> 4), idesc_qk,
-                          (kb | kk) ? 1u : 0u);
-          }
-          if (DR) {
-            // this CTA's 32 rotary columns: rows of 64 B, 8-row groups 512 B apart
-            const uint64_t rd = rd0 + (uint64_t)s * kStage;
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk) mma_bf16_ss(td, qd0 + (uint64_t)(kk * 2), rd + (uint64_t)(kk * 2), idesc_qk, 1u);
-          }
-          mma_commit(&s_full[sl]);
-          if (gq + 1 == qseg_end) mma_commit(q_empty);
-          ++gq;
-          progressed = true;
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(td, qld0 + (uint64_t)(((kb - 2) * Cfg::QL_BOX + kk * 32) >> 4),
+                        kd + (uint64_t)((kb * Cfg::K_BOX + kk * 32) >> 4), idesc_qk, 1u);
         }
+        if (DR) {
+          // this CTA's 32 rotary columns: rows of 64 B, 8-row groups 512 B apart
+          const uint64_t rd = rd0 + (uint64_t)s * kStage;
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) mma_bf16_ss(td, qd0 + (uint64_t)(kk * 2), rd + (uint64_t)(kk * 2), idesc_qk, 1u);
+        }
+        mma_commit(&s_full[sl]);
+        if (g + 1 == seg_end) mma_commit(q_empty);
       }
-      if (progressed) {
-        idle = 0;
-      } else {
-        if (idle == 0) t_idle = globaltimer_ns();
-        if ((++idle & 7u) == 0 && globaltimer_ns() - t_idle > p.wait_ns) {
-          report_timeout(p.status);
-          ok = false;
-          break;
-        }
+    } else {
+      for (int64_t g = 0; g < n_total; ++g) {
+        const bool first = advance_segment(g);   // the first tile of a segment opens O (accumulate = 0)
+        const int s = (int)(g % ST);
+        const int sl = (int)(g % NS);
+        if (!wait_mma(&p_full[sl], (uint32_t)(g / NS) & 1u)) { ok = false; break; }
+        tc_fence_after();
+        // B = this CTA's 256 latent columns of the tile: MN-major, 64-column boxes K_BOX apart
+        const uint64_t cd = cd0 + (uint64_t)s * kStage;
+        const uint32_t ta = tS + sl * 64;
+#pragma unroll
+        for (int kk = 0; kk < DEC_BT / 16; ++kk)
+          mma_bf16_ts(tO, ta + kk * 8, cd + (uint64_t)(kk * (2048 >> 4)), idesc_pv, (first && kk == 0) ? 0u : 1u);
+        mma_commit(&k_empty[s]);
+        mma_commit(&o_done[sl]);
       }
     }
-    if (!ok) {
+    if (!ok || *abort_flag) {
       *abort_flag = 1;
-      // every MMA issued so far must finish before TMEM is released
-      mma_commit(drain);
-      (void)mbar_wait(drain, 0, drain_ns, p.status);
+      // every MMA this thread issued must finish before TMEM is released
+      uint64_t* d = &drain[qk_issuer ? 0 : 1];
+      mma_commit(d);
+      (void)mbar_wait(d, 0, drain_ns, p.status);
     }
   } else if (warp >= 12) {
     // -------------------------------- score sender --------------------------------
@@ -458,8 +462,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       if (!mbar_wait(bar, (uint32_t)parity, p.wait_ns, p.status)) *abort_flag = 1;
     };
     for (int64_t g = 0; g < n_total; ++g) {
-      const int sl = (int)(g & 1);
-      wait_cta(&s_full[sl], (int)(g >> 1) & 1);
+      const int sl = (int)(g % NS);         // S slot
+      const int xs = (int)(g % XS);         // exchange slot
+      wait_cta(&s_full[sl], (int)(g / NS) & 1);
       tc_fence_after();
       uint32_t h[32];                       // fp16 pairs: [0, 16) for warpgroup 0, [16, 32) for 1
       {
@@ -475,11 +480,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           h[16 + c] = *reinterpret_cast<uint32_t*>(&v1);
         }
       }
-      // staging slot sl and the peer's receive slot sl were last used by tile g - 2: both this CTA's
+      // staging slot xs and the peer's receive slot xs were last used by tile g - XS: both this CTA's
       // softmax and the peer's have read that tile once x_empty completes (2 arrivals)
-      if (g >= 2) wait_cta(&x_empty[sl], (int)((g >> 1) - 1) & 1);
+      if (g >= XS) wait_cta(&x_empty[xs], (int)((g / XS) - 1) & 1);
       {
-        uint8_t* stg = staging + sl * Cfg::X_TILE + xrow;
+        uint8_t* stg = staging + xs * Cfg::X_TILE + xrow;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
           *reinterpret_cast<uint4*>(stg + ((c ^ swz) * 16)) =
@@ -490,8 +495,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       __syncwarp();
       if (lane == 0) {
         if (!*abort_flag) {
-          const uint32_t off = (uint32_t)(sl * Cfg::X_TILE) + xwarp;
-          bulk_copy_to_cta(x_remote + off, staging + off, 32 * 128, xf_remote + sl * 8);
+          const uint32_t off = (uint32_t)(xs * Cfg::X_TILE) + xwarp;
+          bulk_copy_to_cta(x_remote + off, staging + off, 32 * 128, xf_remote + xs * 8);
         }
         mbar_arrive(&own_ready[sl]);        // this warp's partials staged and read: P may overwrite
       }
@@ -525,66 +530,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       if (*abort_flag) return;
       if (!mbar_wait(bar, (uint32_t)parity, p.wait_ns, p.status)) *abort_flag = 1;
     };
-    // this warpgroup's 128 of the CTA's 256 latent query columns of block kq, into TMEM, once the
-    // previous segment's last QK^T has read the query. Thread = row = TMEM lane, so a plain load gives
-    // each thread its own row and every load instruction touches 32 rows. The first query of the CTA
-    // (all CTAs load theirs at once) goes through this warp's 4 KB of the send-staging slots instead,
-    // which nothing else touches before this CTA's first QK^T: coalesced loads (4 rows x 128 B per
-    // instruction), then each thread reads its row back. Chunks are stored swizzled (chunk ^ row % 8),
-    // so both the stores and the row reads are free of bank conflicts.
-    uint8_t* wscratch_q = smem + Cfg::OFF_XS + (warp - 4) * 4096;
+    // this warpgroup's 64 of the CTA's first 128 latent query columns of block kq, into TMEM (the other
+    // 128 come to shared memory by TMA), once the previous segment's last QK^T has read the query.
+    // Thread = row = TMEM lane, so a plain load gives each thread its own row and every load
+    // instruction touches 32 rows. The first query of the CTA (all CTAs load theirs at once) goes
+    // through this warp's 4 KB of cache stage 1 instead, which the producer fills only once this query
+    // is in (ql_full): coalesced loads (4 rows x 128 B per instruction), then each thread reads its row
+    // back. Chunks are stored swizzled (chunk ^ row % 8), so both the stores and the row reads are free
+    // of bank conflicts.
+    uint8_t* wscratch_q = sK + Cfg::STAGE_BYTES + (warp - 4) * 4096;
     auto load_query = [&](int kq, int segment) {
       const int bq = kq / p.nbps, rbq = kq % p.nbps;
       const int64_t qr0 = (int64_t)bq * p.n_q * p.H + (int64_t)rbq * DEC_ROWS + quarter * 32;   // warp's first row
+      const int col0 = dim0 + wg * 64;
       if (segment > 0) wait_cta(q_empty, (segment - 1) & 1);
       tc_fence_after();
+      uint32_t r[32];
       if (segment == 0) {
-        uint4 v[16];
+        uint4 v[8];
         const int chunk = lane & 7;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int64_t qr = qr0 + 4 * j + (lane >> 3);
-            const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + qr * p.W + dim0 + wg * 128 + h * 64) + chunk;
-            v[h * 8 + j] = qr < p.q_rows ? *src : make_uint4(0u, 0u, 0u, 0u);
-          }
+        for (int j = 0; j < 8; ++j) {
+          const int64_t qr = qr0 + 4 * j + (lane >> 3);
+          const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + qr * p.W + col0) + chunk;
+          v[j] = qr < p.q_rows ? *src : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int rr = 4 * j + (lane >> 3);
-            *reinterpret_cast<uint4*>(wscratch_q + rr * 128 + ((chunk ^ (rr & 7)) * 16)) = v[h * 8 + j];
-          }
-          __syncwarp();
-          uint32_t r[32];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 w = *reinterpret_cast<const uint4*>(wscratch_q + lane * 128 + ((c ^ (lane & 7)) * 16));
-            r[4 * c] = w.x; r[4 * c + 1] = w.y; r[4 * c + 2] = w.z; r[4 * c + 3] = w.w;
-          }
-          __syncwarp();
-          tmem_st32(tQ + lane_off + wg * 64 + h * 32, r);
+        for (int j = 0; j < 8; ++j) {
+          const int rr = 4 * j + (lane >> 3);
+          *reinterpret_cast<uint4*>(wscratch_q + rr * 128 + ((chunk ^ (rr & 7)) * 16)) = v[j];
         }
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 w = *reinterpret_cast<const uint4*>(wscratch_q + lane * 128 + ((c ^ (lane & 7)) * 16));
+          r[4 * c] = w.x; r[4 * c + 1] = w.y; r[4 * c + 2] = w.z; r[4 * c + 3] = w.w;
+        }
+        fence_proxy_async_smem();           // these generic accesses come before the stage's TMA fill
+        __syncwarp();
       } else {
         const int64_t qr = qr0 + lane;
-        const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + qr * p.W + dim0 + wg * 128);
+        const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + qr * p.W + col0);
         const bool in = qr < p.q_rows;
-        uint4 v[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = in ? src[j] : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {      // 2 x 32 TMEM columns = 128 bf16
-          uint32_t r[32];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            r[4 * j] = v[cc * 8 + j].x; r[4 * j + 1] = v[cc * 8 + j].y;
-            r[4 * j + 2] = v[cc * 8 + j].z; r[4 * j + 3] = v[cc * 8 + j].w;
-          }
-          tmem_st32(tQ + lane_off + wg * 64 + cc * 32, r);
+        for (int j = 0; j < 8; ++j) {
+          const uint4 w = in ? src[j] : make_uint4(0u, 0u, 0u, 0u);
+          r[4 * j] = w.x; r[4 * j + 1] = w.y; r[4 * j + 2] = w.z; r[4 * j + 3] = w.w;
         }
       }
+      tmem_st32(tQ + lane_off + wg * 32, r);   // 32 TMEM columns = 64 bf16
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -611,10 +605,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       }
       float m_ref = -INFINITY, l = 0.f;     // reference maximum (log2 units), this group's sum
       for (int tt = 0; tt < ntl; ++tt, ++g) {
-        const int sl = (int)(g & 1);
-        const int xi = sl;                    // the tile's exchange slot (this warpgroup reads its half)
+        const int sl = (int)(g % NS);         // the tile's S / P slot
+        const int xi = (int)(g % XS);         // the tile's exchange slot (this warpgroup reads its half)
         float s[32];
-        wait_cta(&own_ready[sl], (int)(g >> 1) & 1);
+        wait_cta(&own_ready[sl], (int)(g / NS) & 1);
         tc_fence_after();
         uint4 own[4];
         {
@@ -622,7 +616,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
 #pragma unroll
           for (int c = 0; c < 4; ++c) own[c] = *reinterpret_cast<const uint4*>(xo + (((4 * wg + c) ^ swz) * 16));
         }
-        wait_cta(&x_full[xi], (int)(g >> 1) & 1);
+        wait_cta(&x_full[xi], (int)(g / XS) & 1);
         {
           const uint8_t* xr = sX + xi * Cfg::X_TILE + xrow;
 #pragma unroll
@@ -700,12 +694,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         tmem_st16(tS + lane_off + sl * 64 + wg * 16, pk);
         tmem_wait_st();
         // O may be touched only once every earlier P.C is done: needed when a row of this warp rescales,
-        // and at the last tile of a segment (so that the epilogue's wait is one phase away). Here P.C of
-        // tile g - 2 is complete (QK^T of tile g reused its slot) and P.C of tile g is not issued yet, so
-        // o_done is at most one phase behind and the parity names P.C of tile g - 1 unambiguously.
+        // and at the last tile of a segment. P.C of tile g - 1 commits to its slot's o_done barrier, whose
+        // previous phase (P.C of tile g - 1 - NS) completed before QK^T of tile g - 1 could use the slot;
+        // its completion implies every earlier P.C's (one issuing thread, in-order pipe).
         const bool rescale = __any_sync(0xffffffffu, need);
         if ((rescale || tt + 1 == ntl) && g > pv_waited) {
-          wait_cta(o_done, (int)((g - 1) & 1));
+          wait_cta(&o_done[(g - 1) % NS], (int)(((g - 1) / NS) & 1));
           pv_waited = g;
         }
         tc_fence_after();
@@ -730,7 +724,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       if (send_u < u1) load_query(k_next, seg + 1);
       // epilogue of the segment: wait for its last P.C, then read this group's quarter of O
       if (g > pv_waited) {
-        wait_cta(o_done, (int)((g - 1) & 1));
+        wait_cta(&o_done[(g - 1) % NS], (int)(((g - 1) / NS) & 1));
         pv_waited = g;
       }
       tc_fence_after();
@@ -745,10 +739,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       const float mul = complete ? inv : 1.f;
       const bool write = complete ? valid : true;
       if (send_u >= u1 && !*abort_flag) {
-        // the CTA's last segment: every tile of the peer has landed and been read, so the receive
-        // slots are free. Each warp turns its 32 rows x 32 columns of O around in its 4 KB of them
-        // (swizzled as for the query) and stores 4 rows x 128 B per instruction.
-        uint8_t* wscratch = smem + Cfg::OFF_X + (warp - 4) * 4096;
+        // the CTA's last segment: every tile has been loaded and every MMA is done (the last P.C
+        // above), so the cache stages are free. Each warp turns its 32 rows x 32 columns of O around
+        // in its 4 KB of stage 0 (swizzled as for the query) and stores 4 rows x 128 B per instruction.
+        uint8_t* wscratch = sK + (warp - 4) * 4096;
         const int chunk = lane & 7;
 #pragma unroll 1
         for (int cc = 0; cc < DEC_HALF / 2; cc += 32) {
@@ -982,7 +976,7 @@ size_t tc_decode_workspace(const DecodeArgs& a) { return plan_tc(a).total; }
 
 template <int DR>
 static int launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tkr, const CUtensorMap& tqr,
-                           const DecParams& p, cudaStream_t s) {
+                           const CUtensorMap& tql, const DecParams& p, cudaStream_t s) {
   static bool attr_set[64] = {false};
   const int dev = current_device();
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
@@ -992,7 +986,7 @@ static int launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tkr, const 
     attr_set[dev] = true;
   }
   return launch_pdl(tc_decode_kernel<DR>, dim3(2 * p.G), dim3(DEC_THREADS), (size_t)DecCfg<DR>::SMEM, s, tk, tkr,
-                    tqr, p);
+                    tqr, tql, p);
 }
 
 int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
@@ -1017,13 +1011,20 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
   if (!p.status) return MLA_ERR_CUDA;
   if (t.nblocks == 0) return MLA_OK;
 
-  CUtensorMap tk, tkr, tqr;
+  CUtensorMap tk, tkr, tqr, tql;
   {
     const uint64_t rows = (uint64_t)std::max<int64_t>(a.total_rows, 1);
     const uint64_t dims[2] = {(uint64_t)W, rows};
     const uint64_t st[1] = {(uint64_t)W * 2};
     const uint32_t box[2] = {64, DEC_BT};
     if (!encode_tmap_bf16(&tk, const_cast<void*>(a.cache), 2, dims, st, box)) return MLA_ERR_CUDA;
+  }
+  {
+    // latent query columns: boxes of 64 columns x 128 rows, 128-byte swizzle (the A operand layout)
+    const uint64_t dims[2] = {(uint64_t)W, (uint64_t)a.batch * a.n_q * a.H};
+    const uint64_t st[1] = {(uint64_t)W * 2};
+    const uint32_t box[2] = {64, DEC_ROWS};
+    if (!encode_tmap_bf16(&tql, const_cast<void*>(a.q_abs), 2, dims, st, box)) return MLA_ERR_CUDA;
   }
   tkr = tk;
   tqr = tk;
@@ -1045,7 +1046,7 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
   }
   int st0 = launch_pdl(decode_plan_kernel, dim3(1), dim3(1024), 0, s, p, const_cast<int32_t*>(p.prefix));
   if (st0) return st0;
-  int st = a.dr == 0 ? launch_decode_t<0>(tk, tkr, tqr, p, s) : launch_decode_t<64>(tk, tkr, tqr, p, s);
+  int st = a.dr == 0 ? launch_decode_t<0>(tk, tkr, tqr, tql, p, s) : launch_decode_t<64>(tk, tkr, tqr, tql, p, s);
   if (st) return st;
   // 16 CTAs per block (8 rows each): a split block's merge reads 2-3 partial slots of 256 KB
   return launch_pdl(decode_combine_tc_kernel, dim3((unsigned)t.nblocks, DEC_ROWS / 8), dim3(256), 0, s, p);
