@@ -429,7 +429,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < DEC_BT / 16; ++kk)
           mma_bf16_ts(tO, ta + kk * 8, cd + (uint64_t)(kk * (2048 >> 4)), idesc_pv, (first && kk == 0) ? 0u : 1u);
-        mma_commit(&k_empty[s]);
+        // the stage of a segment's last tile is released by the softmax warps after the epilogue,
+        // which turns O around in it
+        if (g + 1 != seg_end) mma_commit(&k_empty[s]);
         mma_commit(&o_done[sl]);
       }
     }
@@ -532,50 +534,65 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     };
     // this warpgroup's 64 of the CTA's first 128 latent query columns of block kq, into TMEM (the other
     // 128 come to shared memory by TMA), once the previous segment's last QK^T has read the query.
-    // Thread = row = TMEM lane, so a plain load gives each thread its own row and every load
-    // instruction touches 32 rows. The first query of the CTA (all CTAs load theirs at once) goes
-    // through this warp's 4 KB of cache stage 1 instead, which the producer fills only once this query
-    // is in (ql_full): coalesced loads (4 rows x 128 B per instruction), then each thread reads its row
-    // back. Chunks are stored swizzled (chunk ^ row % 8), so both the stores and the row reads are free
-    // of bank conflicts.
-    uint8_t* wscratch_q = sK + Cfg::STAGE_BYTES + (warp - 4) * 4096;
-    auto load_query = [&](int kq, int segment) {
+    // Thread = row = TMEM lane, but a load with one row per thread touches 32 rows per instruction, so
+    // the rows are loaded 4 x 128 B per instruction and turned around in shared memory, swizzled
+    // (chunk ^ row % 8: both the stores and the row reads are free of bank conflicts):
+    //  * the first query of the CTA in this warp's 4 KB of cache stage 1, which the producer fills
+    //    only once this query is in (ql_full);
+    //  * a later one in this warp's 2 KB of the send-staging slot, in two rounds of 16 rows, once the
+    //    exchange of the previous segment's last tile is complete (x_empty: the peer has read the
+    //    copy, so no bulk copy still reads the slot; the sender writes it again only after the next
+    //    QK^T, which needs this query).
+    auto load_query = [&](int kq, int segment, int64_t g_prev) {
       const int bq = kq / p.nbps, rbq = kq % p.nbps;
       const int64_t qr0 = (int64_t)bq * p.n_q * p.H + (int64_t)rbq * DEC_ROWS + quarter * 32;   // warp's first row
       const int col0 = dim0 + wg * 64;
       if (segment > 0) wait_cta(q_empty, (segment - 1) & 1);
       tc_fence_after();
+      uint4 v[8];
+      const int chunk = lane & 7;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int64_t qr = qr0 + 4 * j + (lane >> 3);
+        const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + qr * p.W + col0) + chunk;
+        v[j] = qr < p.q_rows ? *src : make_uint4(0u, 0u, 0u, 0u);
+      }
       uint32_t r[32];
       if (segment == 0) {
-        uint4 v[8];
-        const int chunk = lane & 7;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int64_t qr = qr0 + 4 * j + (lane >> 3);
-          const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + qr * p.W + col0) + chunk;
-          v[j] = qr < p.q_rows ? *src : make_uint4(0u, 0u, 0u, 0u);
-        }
+        uint8_t* scr = sK + Cfg::STAGE_BYTES + (warp - 4) * 4096;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int rr = 4 * j + (lane >> 3);
-          *reinterpret_cast<uint4*>(wscratch_q + rr * 128 + ((chunk ^ (rr & 7)) * 16)) = v[j];
+          *reinterpret_cast<uint4*>(scr + rr * 128 + ((chunk ^ (rr & 7)) * 16)) = v[j];
         }
         __syncwarp();
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const uint4 w = *reinterpret_cast<const uint4*>(wscratch_q + lane * 128 + ((c ^ (lane & 7)) * 16));
+          const uint4 w = *reinterpret_cast<const uint4*>(scr + lane * 128 + ((c ^ (lane & 7)) * 16));
           r[4 * c] = w.x; r[4 * c + 1] = w.y; r[4 * c + 2] = w.z; r[4 * c + 3] = w.w;
         }
         fence_proxy_async_smem();           // these generic accesses come before the stage's TMA fill
         __syncwarp();
       } else {
-        const int64_t qr = qr0 + lane;
-        const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + qr * p.W + col0);
-        const bool in = qr < p.q_rows;
+        wait_cta(&x_empty[g_prev % XS], (int)((g_prev / XS) & 1));
+        uint8_t* scr = smem + Cfg::OFF_XS + (warp - 4) * 2048;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint4 w = in ? src[j] : make_uint4(0u, 0u, 0u, 0u);
-          r[4 * j] = w.x; r[4 * j + 1] = w.y; r[4 * j + 2] = w.z; r[4 * j + 3] = w.w;
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int j = 4 * h; j < 4 * h + 4; ++j) {
+            const int rr = 4 * j + (lane >> 3) - 16 * h;
+            *reinterpret_cast<uint4*>(scr + rr * 128 + ((chunk ^ (rr & 7)) * 16)) = v[j];
+          }
+          __syncwarp();
+          if ((lane >> 4) == h) {
+            const int rr = lane - 16 * h;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const uint4 w = *reinterpret_cast<const uint4*>(scr + rr * 128 + ((c ^ (rr & 7)) * 16));
+              r[4 * c] = w.x; r[4 * c + 1] = w.y; r[4 * c + 2] = w.z; r[4 * c + 3] = w.w;
+            }
+          }
+          __syncwarp();
         }
       }
       tmem_st32(tQ + lane_off + wg * 32, r);   // 32 TMEM columns = 64 bf16
@@ -584,7 +601,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(ql_full);
     };
-    if (u0 < u1) load_query(k, 0);
+    if (u0 < u1) load_query(k, 0, 0);
     while (u < u1) {
       const int64_t bstart = p.prefix[k], bend = p.prefix[k + 1];
       const int64_t send_u = u1 < bend ? u1 : bend;
@@ -721,7 +738,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       }
       // the next segment's query can go in now (its QK^T overlaps this epilogue)
       const int k_next = send_u < u1 ? find_block(p.prefix, p.nblocks, send_u) : k;
-      if (send_u < u1) load_query(k_next, seg + 1);
+      if (send_u < u1) load_query(k_next, seg + 1, g - 1);
       // epilogue of the segment: wait for its last P.C, then read this group's quarter of O
       if (g > pv_waited) {
         wait_cta(&o_done[(g - 1) % NS], (int)(((g - 1) / NS) & 1));
@@ -738,11 +755,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
                             : p.o_part + ((int64_t)slot * DEC_ROWS + row) * DEC_DC + dim0 + wg * 128;
       const float mul = complete ? inv : 1.f;
       const bool write = complete ? valid : true;
-      if (send_u >= u1 && !*abort_flag) {
-        // the CTA's last segment: every tile has been loaded and every MMA is done (the last P.C
-        // above), so the cache stages are free. Each warp turns its 32 rows x 32 columns of O around
-        // in its 4 KB of stage 0 (swizzled as for the query) and stores 4 rows x 128 B per instruction.
-        uint8_t* wscratch = sK + (warp - 4) * 4096;
+      const int s_last = (int)((g - 1) % ST);   // cache stage of the segment's last tile, held for us
+      if (!*abort_flag) {
+        // The segment's last P.C is done (above), and the P.C issuer left that tile's cache stage to
+        // this epilogue. Each warp turns its 32 rows x 32 columns of O around in its 4 KB of the stage
+        // (swizzled as for the query) and stores 4 rows x 128 B per instruction.
+        uint8_t* wscratch = sK + s_last * Cfg::STAGE_BYTES + (warp - 4) * 4096;
         const int chunk = lane & 7;
 #pragma unroll 1
         for (int cc = 0; cc < DEC_HALF / 2; cc += 32) {
@@ -788,6 +806,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           }
         }
       }
+      // hand the stage back to the producer: the generic accesses above come before its TMA fill
+      fence_proxy_async_smem();
+      named_bar_sync(3, 256);
+      if (wg == 0 && row == 0) mbar_arrive(&k_empty[s_last]);
       if (rank == 0 && wg == 0) {
         if (complete) {
           if (valid && p.lse) p.lse[orow] = ltot > 0.f ? (m_ref + log2f(ltot)) * 0.69314718055994531f : -INFINITY;
