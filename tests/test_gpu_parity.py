@@ -132,8 +132,7 @@ SMALL = [
 ]
 
 
-@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}-H{c[1]}-dc{c[2]}-dr{c[3]}-T{c[7]}-nq{c[8]}-c{int(c[9])}")
-def test_decode_small(case):
+def _check_decode_case(case):
     dtype, H, dc, dr, n, dv, D, seqlens, n_q, causal = case
     p = I.decode_problem(batch=len(seqlens), n_heads=H, kv_lora_rank=dc, rope_dim=dr, qk_nope=n,
                          v_head=dv, d_model=D, seqlens=seqlens, n_q=n_q, dtype=dtype, seed=23)
@@ -146,6 +145,24 @@ def test_decode_small(case):
         assert_close(out_lat[rows], ref_lat, dtype, f"out_lat b={b}")
         assert_close(y[rows], ref_y, dtype, f"y b={b}")
         np.testing.assert_allclose(lse[rows], ref_lse, rtol=0, atol=TOL[dtype] * 10)
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}-H{c[1]}-dc{c[2]}-dr{c[3]}-T{c[7]}-nq{c[8]}-c{int(c[9])}")
+def test_decode_small(case):
+    _check_decode_case(case)
+
+
+@pytest.mark.parametrize("clusters", [1, 2, 3])
+@pytest.mark.parametrize("case", [SMALL[3], SMALL[6]], ids=["dr64-ragged-nq1", "dr0-causal-nq100"])
+def test_decode_many_segments_per_cluster(case, clusters):
+    """One to three clusters for all the work: every CTA pair crosses many blocks (whole blocks and
+    split ones), so each block boundary's query hand-over, epilogue and cache-stage release runs
+    many times per CTA, next to the combine of split blocks."""
+    M.mla_set_decode_clusters(clusters)
+    try:
+        _check_decode_case(case)
+    finally:
+        M.mla_set_decode_clusters(0)
 
 
 def test_decode_empty_and_zero_length_sequences():
