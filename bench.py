@@ -16,6 +16,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -90,12 +91,20 @@ def sustained_tflops() -> float:
     return 1400.0
 
 
+def _code_only(text: str) -> str:
+    """The source without comments, blank lines or trailing spaces: edits to comments do not change
+    the kernel the counters were taken on."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def source_hash() -> str:
     h = hashlib.sha256()
     for rel in DECODE_SOURCES:
         p = os.path.join(ROOT, rel)
         if os.path.exists(p):
-            h.update(open(p, "rb").read())
+            h.update(_code_only(open(p, encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

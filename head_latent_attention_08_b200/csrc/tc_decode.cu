@@ -20,17 +20,18 @@
 //    the A operand of QK^T straight from TMEM), the other 128 and the rotary columns in shared memory
 //    (brought by TMA). P (bf16) is written over its S tile and is the A operand of P . C from TMEM.
 //    TMEM: Q 64 + O 256 + three 64-column S/P slots = 512 columns, so three tiles are between QK^T
-//    and P.C at once; shared memory holds three cache stages.
+//    and P.C at once. Shared memory: the query half, four cache stages and one receive and one
+//    send-staging slot for the fp16 scores.
 //  * O is rescaled only when a row's running maximum grows by more than 2^8 (the result is exact:
 //    numerator and denominator share the stale reference maximum).
 //  * Work: the (block, 64-position tile) units of all sequences are split evenly over the clusters
 //    (persistent). A cluster that covers a whole block writes the normalised result; split blocks
 //    leave (O, max, sum) partials that a combine kernel merges.
-//  * Warp roles per CTA (512 threads): warp 0 lane 0 issues TMA loads, warp 1 lane 0 issues MMAs
-//    (event loop), warps 12-15 send the partial scores (rounded to fp16; each warp copies its 32
-//    rows of each softmax warpgroup's half to the peer and never waits on the peer), warps 4-11 form
-//    two softmax warpgroups (thread = row = TMEM lane): warpgroup wg loads half the query block into
-//    TMEM at each segment, adds its own and the peer's fp16 partials of score columns
+//  * Warp roles per CTA (512 threads): warp 0 lane 0 issues TMA loads, warp 1 lane 0 every QK^T and
+//    warp 2 lane 0 every P.C, warps 12-15 send the partial scores (rounded to fp16; each warp copies
+//    its 32 rows to the peer with one bulk copy and never waits on the peer), warps 4-11 form two
+//    softmax warpgroups (thread = row = TMEM lane): warpgroup wg loads its 64 of the query's TMEM
+//    columns at each segment, adds its own and the peer's fp16 partials of score columns
 //    [32 wg, 32 wg + 32), meets the other warpgroup once per tile for the row maximum, writes P and
 //    runs the epilogue.
 //  * Every wait is bounded (global-timer limit); a wait that gives up sets the library's status word,
@@ -445,11 +446,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
   } else if (warp >= 12) {
     // -------------------------------- score sender --------------------------------
     // Thread = row = TMEM lane, and each warp handles its 32 rows on its own. For each tile: load this
-    // CTA's partial scores (64 columns), round them to fp16 into the staging slots of the two softmax
-    // warpgroups (the softmax reads its own partials there) and send the warp's rows of each half to
-    // the same slot of the peer with one 2 KB bulk copy per half. The sender never waits for the
-    // peer's scores, so the peer receives tile g as soon as this CTA's QK^T of tile g is done.
-    // One copy per warp carries its rows of both halves (4 KB).
+    // CTA's partial scores (64 columns), round them to fp16 into the staging slot (the softmax reads
+    // its own partials there) and send the warp's 32 rows (4 KB, both warpgroups' halves) to the
+    // same slot of the peer with one bulk copy. The sender never waits for the peer's scores, so the
+    // peer receives tile g as soon as this CTA's QK^T of tile g is done.
     const int quarter = warp - 12;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;

@@ -31,3 +31,31 @@ def test_bench_refuses_short_warmup():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--warmup", "2"],
                        capture_output=True, text=True, timeout=120, cwd=ROOT)
     assert r.returncode != 0
+
+
+def _bench_module():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    return b
+
+
+def test_traffic_record_keyed_on_code_not_comments(tmp_path, monkeypatch):
+    """The ncu traffic record is tied to the decode sources' code: a comment edit keeps it, a code edit
+    turns the bench's traffic figure to null."""
+    b = _bench_module()
+    src = "// header\nint f(int x) {  // trailing\n  /* block\n comment */ return x + 1;\n}\n\n"
+    assert b._code_only(src) == b._code_only(src.replace("trailing", "other words") + "// more\n")
+    assert b._code_only(src) != b._code_only(src.replace("x + 1", "x + 2"))
+    (tmp_path / "k.cu").write_text(src)
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(b, "ROOT", str(tmp_path))
+    monkeypatch.setattr(b, "DECODE_SOURCES", ("k.cu",))
+    rec = {"source_hash": b.source_hash(), "dram_bytes_per_launch": 123}
+    (tmp_path / "profiles" / "decode_c3_traffic.json").write_text(json.dumps(rec))
+    assert b.recorded_traffic() == 123
+    (tmp_path / "k.cu").write_text(src + "// a note\n")
+    assert b.recorded_traffic() == 123
+    (tmp_path / "k.cu").write_text(src.replace("x + 1", "x - 1"))
+    assert b.recorded_traffic() is None
