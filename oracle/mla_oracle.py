@@ -32,7 +32,12 @@ Pins (what fixes each function independently of this file; see tests/test_oracle
   the rows); the [rs] test's wrong-scale check; invariances (score shift, permutation).
 * append_latent: exact row placement; RMS of a normed row is 1; RoPE keeps pair norms and
   composes as a rotation by the position difference.
-* fold_qk / fold_vo / notebook_forward: the printed notebook shapes; absorbed == unabsorbed.
+* fold_qk / fold_vo / notebook_forward: the printed notebook shapes; absorbed == unabsorbed;
+  the linear form against the notebook's cell restated with torch matmuls; the softmax form
+  against torch scaled_dot_product_attention (its default scale, 1/sqrt(head width)) on
+  explicit per-head Q, K, V, at the notebook's sizes and at sizes where d_2 != d_h.
+* rope_interleaved: relativity and composition, and hand-computed angles (tests/golden/
+  rope_frequencies.json: pair i of a d-wide row at position p turns by p * theta^(-2i/d)).
 * gated_mla: the worked example (output 1.0, latent_cache 2.0) and the shape examples; causal
   first query equals the first value row; gated_mla_absorbed equals gated_mla.
 * kv_values_per_token_*: the worked table of [lab] Bloque A, filled by hand in the tests.
@@ -288,6 +293,27 @@ def notebook_split_heads(w_uq, w_uk, w_uv, w_o, h: int):
     return split(w_uq), split(w_uk), split(w_uv), _f64(w_o).reshape(h, d_h, -1)
 
 
+def notebook_kq_scale(d_h: int) -> float:
+    """Score scale of the notebook's softmax form: 1/sqrt(d_h), d_h = d_3 / h the width of one
+    un-absorbed head ([rs] kq_scale paragraph: the scale of the naive head width, kept after the
+    absorption widens the dot product)."""
+    return 1.0 / math.sqrt(d_h)
+
+
+def notebook_attention_weights(s: np.ndarray, scale: float, form: str) -> np.ndarray:
+    """Attention weights of the notebook step over the last axis of the raw scores ``s``.
+
+    ``form='linear'``: the notebook literally, attn = C_Q C_KV^T with no softmax and no scale.
+    ``form='softmax'``: softmax of the scaled scores (scale inside the exponent, row max
+    subtracted first, [rs] fn body).
+    """
+    if form == "linear":
+        return s
+    m = np.max(s * scale, axis=-1, keepdims=True)
+    e = np.exp(s * scale - m)
+    return e / np.sum(e, axis=-1, keepdims=True)
+
+
 def notebook_forward(x, w_dq, w_dkv, w_uq, w_uk, w_uv, w_o, c_kv, h: int, *,
                      form: str = "softmax", route: str = "absorbed"):
     """One decode step of the notebook's RoPE-less MLA (row-vector convention, y = x W).
@@ -309,14 +335,10 @@ def notebook_forward(x, w_dq, w_dkv, w_uq, w_uk, w_uv, w_o, c_kv, h: int, *,
     new_cv = x @ _f64(w_dkv)
     ckv = np.vstack((_f64(c_kv), new_cv))
     cq_lat = x @ _f64(w_dq)                                  # [1, d_2]
-    scale = 1.0 / math.sqrt(d_h)
+    scale = notebook_kq_scale(d_h)
 
     def weights(s):
-        if form == "linear":
-            return s
-        m = np.max(s * scale, axis=-1, keepdims=True)
-        e = np.exp(s * scale - m)
-        return e / np.sum(e, axis=-1, keepdims=True)
+        return notebook_attention_weights(s, scale, form)
 
     if route == "absorbed":
         c_q = cq_lat @ w_aqk                                 # [h, 1, d_2]

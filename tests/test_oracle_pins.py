@@ -125,6 +125,95 @@ def test_notebook_linear_form_literal_with_torch():
     assert rel_err(r, out.numpy()) < 1e-12
 
 
+def sdpa_notebook_softmax(p):
+    """The notebook step with the method's softmax, built from explicit per-head Q, K, V with torch
+    (row-vector convention) and attended by scaled_dot_product_attention at its default scale,
+    1/sqrt(q.shape[-1]) = 1/sqrt(d_h); heads are summed after W_O[h] ([nb] adding trick)."""
+    h, d_2, d_3 = p.h, p.w_uq.shape[0], p.w_uq.shape[1]
+    d_h = d_3 // h
+    X = t64(p.x)
+    ckv = torch.cat([t64(p.c_kv), X @ t64(p.w_dkv)])
+    out = torch.zeros(1, p.w_o.shape[1], dtype=torch.float64)
+    for k in range(h):
+        cols = slice(k * d_h, (k + 1) * d_h)
+        q = X @ t64(p.w_dq) @ t64(p.w_uq)[:, cols]                # [1, d_h]
+        K = ckv @ t64(p.w_uk)[:, cols]                            # [T, d_h]
+        V = ckv @ t64(p.w_uv)[:, cols]
+        o = F.scaled_dot_product_attention(q[None], K[None], V[None])[0]
+        out += o @ t64(p.w_o)[cols, :]
+    return out.numpy()
+
+
+NOTEBOOK_SIZES = [dict(), dict(d_1=30, d_2=12, d_3=24, h=3, existing=4, seed=77)]
+
+
+def _notebook_softmax_pin_passes():
+    for kw in NOTEBOOK_SIZES:
+        p = I.notebook_problem(**kw)
+        ref = sdpa_notebook_softmax(p)
+        for route in ("absorbed", "unabsorbed"):
+            r = O.notebook_forward(p.x, p.w_dq, p.w_dkv, p.w_uq, p.w_uk, p.w_uv, p.w_o, p.c_kv, p.h,
+                                   form="softmax", route=route)["output"]
+            if not rel_err(r, ref) < 1e-12:
+                return False
+    return True
+
+
+def test_notebook_softmax_form_matches_torch_sdpa():
+    # the second size has d_2 = 12 != d_h = 8, so a scale taken from the latent width would differ
+    assert _notebook_softmax_pin_passes()
+
+
+def test_planted_notebook_scale_from_latent_width(monkeypatch):
+    # 1/sqrt(d_2) instead of 1/sqrt(d_h): identical at the notebook's own sizes (d_2 = d_h = 20),
+    # caught at the second size
+    monkeypatch.setattr(O, "notebook_kq_scale", lambda d_h: 1.0 / math.sqrt(12.0 if d_h == 8 else d_h))
+    assert not _notebook_softmax_pin_passes()
+
+
+def test_planted_notebook_scale_after_softmax(monkeypatch):
+    def bad(s, scale, form):
+        e = np.exp(s - np.max(s, axis=-1, keepdims=True))
+        return scale * e / np.sum(e, axis=-1, keepdims=True)
+    monkeypatch.setattr(O, "notebook_attention_weights", bad)
+    assert not _notebook_softmax_pin_passes()
+
+
+def _rope_golden_passes(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "rope_frequencies.json")))
+    for case in g["cases"]:
+        d = case["d"]
+        for i, ang in case["angles"].items():
+            i = int(i)
+            e = np.zeros((1, d))
+            e[0, 2 * i] = 1.0                      # unit vector on the first entry of pair i
+            r = O.rope_interleaved(e, [case["position"]], case["theta"])[0]
+            want = np.zeros(d)
+            want[2 * i], want[2 * i + 1] = math.cos(ang), math.sin(ang)
+            if not np.allclose(r, want, rtol=0, atol=1e-12):
+                return False
+    return True
+
+
+def test_rope_frequencies_golden(golden_dir):
+    assert _rope_golden_passes(golden_dir)
+
+
+def test_planted_rope_frequency_exponent(monkeypatch, golden_dir):
+    # theta^(-i/d) instead of theta^(-2i/d): relativity, composition and "pair 0 turns by p" all
+    # still hold, the hand-computed angles do not
+    def bad(x, positions, theta=10000.0):
+        x = np.asarray(x, dtype=np.float64)
+        d = x.shape[-1]
+        ang = np.asarray(positions, np.float64).reshape(-1, 1) * theta ** (-np.arange(d // 2) / d)
+        out = np.empty_like(x)
+        out[..., 0::2] = x[..., 0::2] * np.cos(ang) - x[..., 1::2] * np.sin(ang)
+        out[..., 1::2] = x[..., 0::2] * np.sin(ang) + x[..., 1::2] * np.cos(ang)
+        return out
+    monkeypatch.setattr(O, "rope_interleaved", bad)
+    assert not _rope_golden_passes(golden_dir)
+
+
 def test_gated_worked_example(golden_dir):
     g = json.load(open(os.path.join(golden_dir, "gated_examples.json")))["worked_example"]
     for fn in (O.gated_mla, O.gated_mla_absorbed):
