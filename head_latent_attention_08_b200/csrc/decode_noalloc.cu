@@ -45,6 +45,15 @@ extern "C" int32_t mla_decode_absorbed_noalloc(const mla_dims* dims, int32_t dty
   int32_t st = mla_decode_workspace_size(dims, dtype, batch, n_q, max_seqlen, total_rows, flags, &need);
   if (st != MLA_OK) return st;
   if (need > kScratchBytes) return MLA_ERR_WORKSPACE;
+  // the scratch address is the current device's: a stream of another device would hand its kernels
+  // an address that is not theirs, so such a call is refused before any launch
+  int cur = -1, sdev = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess ||
+      cudaStreamGetDevice(reinterpret_cast<cudaStream_t>(stream), &sdev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  if (sdev != cur) return MLA_ERR_CUDA;
   void* scratch = scratch_on_current_device();
   if (!scratch) return MLA_ERR_CUDA;
   return mla_decode_absorbed(dims, dtype, q_abs, cache, cu_seqlens, batch, n_q, max_seqlen, total_rows, flags,

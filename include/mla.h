@@ -224,7 +224,8 @@ MLA_API int32_t mla_wait_selftest(void* stream);
  * the array's address is looked up once per device, with that device current.
  *   Errors: those of mla_decode_absorbed; MLA_ERR_WORKSPACE when the problem needs more scratch than
  *   MLA_DECODE_NOALLOC_MAX_BYTES (mla_decode_workspace_size reports the need); MLA_ERR_CUDA when the
- *   array's address cannot be obtained.
+ *   array's address cannot be obtained, or when `stream` belongs to a device other than the current
+ *   one (the array is looked up on the current device; no launch happens then).
  *   Nothing in the scratch has to start at zero. All calls on one device share the one array: calls
  *   whose executions overlap on the GPU (different streams without ordering between them) race on
  *   it and give undefined results; calls ordered on one stream do not.

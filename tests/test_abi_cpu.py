@@ -104,3 +104,23 @@ def test_binding_raises_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(M, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         M.lib()
+
+
+def test_library_sources_allocate_no_device_memory():
+    """The library allocates nothing: no CUDA allocation or free call and no torch allocator anywhere in
+    its sources (the no-alloc decode and the workspace decode share every kernel and host helper).
+    Comments are ignored; a pair of allocate and free calls inside a call would not show in a
+    free-memory check, so this scan is the primary check."""
+    import glob
+    import re
+    csrc = os.path.join(ROOT, "head_latent_attention_08_b200", "csrc")
+    banned = re.compile(r"\b(cudaMalloc\w*|cudaFree\w*|cuMemAlloc\w*|cuMemFree\w*|cudaHostAlloc|"
+                        r"cudaMallocHost|malloc|calloc|realloc|torch|c10|at::)\b")
+    hits = []
+    for path in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
+        code = re.sub(r"/\*.*?\*/", "", open(path, encoding="utf-8").read(), flags=re.S)
+        for n, line in enumerate(code.splitlines(), 1):
+            line = re.sub(r"//.*$", "", line)
+            if banned.search(line):
+                hits.append(f"{os.path.basename(path)}:{n}: {line.strip()}")
+    assert not hits, "\n".join(hits)
