@@ -104,6 +104,19 @@ __device__ __forceinline__ void bulk_copy_to_cta(uint32_t dst_cluster_addr, cons
 __device__ __forceinline__ void mbar_arrive_remote_release(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
+// asynchronous store of 16 bytes into another CTA's shared memory of the cluster; completes 16 bytes of
+// transactions on that CTA's mbarrier (which must sit in the same CTA as the destination)
+__device__ __forceinline__ void st_async_v4(uint32_t dst_cluster_addr, uint4 v, uint32_t dst_cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   dst_cluster_addr),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(dst_cluster_bar)
+               : "memory");
+}
+__device__ __forceinline__ void st_async_b32(uint32_t dst_cluster_addr, uint32_t v, uint32_t dst_cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(dst_cluster_addr),
+               "r"(v), "r"(dst_cluster_bar)
+               : "memory");
+}
 // bulk-copy groups of the issuing thread
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // every committed bulk copy of this thread has finished reading its source

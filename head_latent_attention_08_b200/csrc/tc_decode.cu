@@ -29,15 +29,19 @@
 //  * Work: the (block, 128-position tile) units of all sequences are split evenly over the clusters
 //    (persistent). A cluster that covers a whole block writes the normalised result; split blocks
 //    leave (O, max, sum) partials that a combine kernel merges.
-//  * Warp roles (384 threads). Score CTA: warp 0 lane 0 TMA, warp 1 lane 0 QK^T, warps 4-11 softmax
-//    (warp w: rows 32 (w & 3) .., positions [64 h, 64 h + 64) of each tile, h = (w - 4) >> 2), which
-//    also load each block's latent query into TMEM. Value CTA: warp 0 lane 0 TMA, warp 1 lane 0 P.C,
-//    warp 2 lane 0 hands P slots back, warps 4-11 rescale and write O (warp w: rows 32 (w & 3) ..,
-//    O columns [256 h, 256 h + 256)).
+//  * Loads: one thread keeps about one TMA instruction in flight, so several threads issue them (three
+//    in the score CTA, two in the value CTA), and the value CTA fetches 64 positions x 256 columns per
+//    instruction (a 3-D box over 64-column groups). The score CTA also warms L2 a few tiles ahead.
+//  * Warp roles (384 threads). Score CTA: warps 0, 2, 3 lane 0 TMA, warp 1 lane 0 QK^T, warps 4-11
+//    softmax (warp w: rows 32 (w & 3) .., positions [64 h, 64 h + 64) of each tile, h = (w - 4) >> 2),
+//    which also move each block's latent query into TMEM. Value CTA: warps 0 and 3 lane 0 TMA, warp 1
+//    lane 0 P.C, warp 2 lane 0 hands P slots back, warps 4-11 rescale and write O (warp w: rows
+//    32 (w & 3) .., O columns [256 h, 256 h + 256)).
 //  * Every wait is bounded (global-timer limit); a wait that gives up sets the library's status word,
 //    and the CTA abandons its work: it issues nothing more, drains its own TMA loads, MMAs and bulk
 //    copies and leaves through the cluster barrier.
 #include <math.h>
+#include <stddef.h>
 
 #include <algorithm>
 
@@ -48,12 +52,16 @@ namespace mla {
 
 using namespace sm100;
 
-constexpr int DEC_BT = 128;        // positions per score tile
-constexpr int DEC_HT = 64;         // positions per P hand-over (half a tile)
-constexpr int DEC_THREADS = 384;
+constexpr int DEC_BT = 256;        // positions per score tile (the N of each QK^T MMA)
+constexpr int DEC_HT = 64;         // positions per P hand-over
+constexpr int DEC_QT = DEC_BT / DEC_HT;   // hand-overs per tile
+constexpr int DEC_THREADS = 640;   // 4 control warps + 16 softmax (score CTA) or rescale/epilogue (value CTA)
+constexpr int DEC_SW = 16;         // softmax / epilogue warps
 constexpr int DEC_DC = 512;        // latent width handled by this kernel
 constexpr int DEC_ROWS = 128;      // rows per block
-constexpr int DEC_NPH = 3;         // P half-tile slots in the value CTA
+constexpr int DEC_NPH = 4;         // P hand-over slots in the value CTA
+constexpr int DEC_PF = 2;          // cache tiles warmed in L2 ahead of the tile QK^T works on
+constexpr int DEC_NPROD = 3;       // TMA-issuing threads of the score CTA
 constexpr float DEC_MOVE = 8.f;    // the reference maximum moves when a row maximum exceeds it by 2^8
 constexpr int DEC_SMEM_LIMIT = 232448;   // dynamic shared memory per CTA (227 KB)
 constexpr int DEC_BAR_BYTES = 1024;
@@ -65,28 +73,30 @@ template <int DR>
 struct DecCfg {
   static constexpr int DATA_LIMIT = DEC_SMEM_LIMIT - 1024 - DEC_BAR_BYTES;   // 1 KB for alignment
   static constexpr int NB = 8 + (DR ? 1 : 0);              // 64-column boxes of a cache row
-  static constexpr int BOX = DEC_BT * 128;                 // 128 positions x 64 columns bf16: 16 KB
+  static constexpr int BOX = DEC_BT * 128;                 // 256 positions x 64 columns bf16: 32 KB
   // score CTA
   static constexpr int S_OFF_QR = 0;                       // rotary query [128 rows x 64 columns]
   static constexpr int S_QR = DR ? DEC_ROWS * 128 : 0;
-  static constexpr int S_OFF_PS = S_OFF_QR + S_QR;         // P staging: 8 warps x 4 KB (32 rows x 128 B)
-  static constexpr int S_OFF_SIDE = S_OFF_PS + 8 * 4096;   // side staging: 8 warps x 512 B
-  static constexpr int S_OFF_RED = S_OFF_SIDE + 8 * 512;   // row maxima [2][2][128], row sums [128]
-  static constexpr int S_OFF_K = dec_round1024(S_OFF_RED + 5 * DEC_ROWS * 4);
-  static constexpr int NK = (DATA_LIMIT - S_OFF_K) / BOX;  // cache boxes in flight
+  static constexpr int S_OFF_RED = S_OFF_QR + S_QR;        // row maxima [2][4][128], row sums [4][128]
+  static constexpr int S_OFF_K = dec_round1024(S_OFF_RED + 12 * DEC_ROWS * 4);
+  static constexpr int SUPER = 3 * BOX;                    // ring slot: three boxes (12 MMAs per wait)
+  static constexpr int NK = (DATA_LIMIT - S_OFF_K) / SUPER;  // ring slots
   // value CTA
-  static constexpr int PH = DEC_ROWS * 128;                // P of a half tile: 128 rows x 64 positions bf16
-  static constexpr int SIDE = 4 * 512;                     // side data of a half tile: 4 quarters x 512 B
+  static constexpr int PH = DEC_ROWS * 128;                // P of a hand-over: 128 rows x 64 positions bf16
+  static constexpr int SIDE = 4 * 512;                     // side data of a hand-over: 4 quarters x 512 B
   static constexpr int PSLOT = PH + SIDE;                  // 18 KB (a multiple of 1024)
+  static constexpr int SIDE_TX = 4 + 3 * 32 * 4;           // side bytes a warp stores: flag, alpha, m, l
+  static constexpr int PSLOT_TX = PH + 4 * SIDE_TX;        // bytes that land in a P slot per hand-over
   static constexpr int V_OFF_P = 0;
   static constexpr int V_OFF_V = dec_round1024(DEC_NPH * PSLOT);
   static constexpr int UNIT = DEC_HT * 512;                // 64 positions x 256 latent columns bf16: 32 KB
-  static constexpr int NV = (DATA_LIMIT - V_OFF_V) / UNIT; // value units in flight
-  static constexpr int OFF_BAR = dec_max(S_OFF_K + NK * BOX, V_OFF_V + NV * UNIT);
+  static constexpr int VUNIT = 2 * UNIT;                   // one hand-over's 64 positions x 512 columns
+  static constexpr int NV = (DATA_LIMIT - V_OFF_V) / VUNIT;  // value slots
+  static constexpr int OFF_BAR = dec_max(S_OFF_K + NK * SUPER, V_OFF_V + NV * VUNIT);
   static constexpr int SMEM = OFF_BAR + DEC_BAR_BYTES + 1024;
   static_assert(PSLOT % 1024 == 0, "P slots must keep the 1024-byte swizzle alignment");
-  static_assert(NK >= NB, "a whole tile of cache boxes must fit in the ring");
-  static_assert(NV >= 2, "the value ring needs two units");
+  static_assert(NK >= 2, "a block's query takes two ring slots");
+  static_assert(NV >= 2, "the value ring needs two slots");
   static_assert(SMEM <= DEC_SMEM_LIMIT, "shared memory budget");
 };
 
@@ -106,7 +116,7 @@ struct DecBars {
   // score CTA
   uint64_t k_full[NK], k_empty[NK];
   uint64_t qr_full, q_tm, q_empty;
-  uint64_t s_full[2], s_empty[2];
+  uint64_t s_full, s_empty;       // the S slot: computed (QK^T commit) / read out (softmax warps)
   uint64_t p_empty[DEC_NPH];      // arrived by the value CTA: a P slot may be written again
   // value CTA
   uint64_t v_full[NV], v_empty[NV];
@@ -122,6 +132,7 @@ struct DecBars {
 
 struct DecParams {
   const __nv_bfloat16* q_abs;  // [q_rows][W]
+  const __nv_bfloat16* cache;  // [total_rows][W]
   int64_t q_rows;
   int W;
   const int32_t* cu;
@@ -268,7 +279,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecParams p, int32_t*
 template <int DR>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
-                     const __grid_constant__ CUtensorMap tqr, DecParams p) {
+                     const __grid_constant__ CUtensorMap tq, DecParams p) {
   using Cfg = DecCfg<DR>;
   constexpr int NK = Cfg::NK;
   constexpr int NV = Cfg::NV;
@@ -289,32 +300,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
   if (tid == 0) {
     if (scorer) {
       for (int s = 0; s < NK; ++s) {
-        mbar_init(&bars->k_full[s], 1);
+        mbar_init(&bars->k_full[s], DEC_NPROD);   // every producer arrives once per slot use
         mbar_init(&bars->k_empty[s], 1);
       }
       mbar_init(&bars->qr_full, 1);
-      mbar_init(&bars->q_tm, 8);          // one arrival per softmax warp (each writes its share of Q)
+      mbar_init(&bars->q_tm, DEC_SW);     // one arrival per softmax warp (each writes its share of Q)
       mbar_init(&bars->q_empty, 1);
-      for (int s = 0; s < 2; ++s) {
-        mbar_init(&bars->s_full[s], 1);
-        mbar_init(&bars->s_empty[s], 8);  // every softmax warp has read its part of the slot
-      }
+      mbar_init(&bars->s_full, 1);
+      mbar_init(&bars->s_empty, DEC_SW);  // every softmax warp has read its part of the slot
       for (int s = 0; s < NPH; ++s) mbar_init(&bars->p_empty[s], 1);
     } else {
       for (int s = 0; s < NV; ++s) {
-        mbar_init(&bars->v_full[s], 1);
+        mbar_init(&bars->v_full[s], 2);           // both producers arrive once per slot use
         mbar_init(&bars->v_empty[s], 1);
       }
       for (int s = 0; s < NPH; ++s) {
         mbar_init(&bars->p_full[s], 1);
-        mbar_init(&bars->pfree[s], 9);    // the P.C commit and the 8 rescale / epilogue warps
+        mbar_init(&bars->pfree[s], DEC_SW + 1);   // the P.C commit and the rescale / epilogue warps
       }
       mbar_init(&bars->o_fix, 1);
-      mbar_init(&bars->fix_done, 8);
+      mbar_init(&bars->fix_done, DEC_SW);
       mbar_init(&bars->o_fin, 1);
-      mbar_init(&bars->o_free, 8);
+      mbar_init(&bars->o_free, DEC_SW);
       // arm the first use of every P slot: one local arrival plus the score CTA's copies
-      for (int s = 0; s < NPH; ++s) mbar_arrive_expect_tx(&bars->p_full[s], Cfg::PSLOT);
+      for (int s = 0; s < NPH; ++s) mbar_arrive_expect_tx(&bars->p_full[s], Cfg::PSLOT_TX);
     }
     mbar_init(&bars->drain[0], 1);
     mbar_init(&bars->drain[1], 1);
@@ -322,7 +331,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     fence_mbar_init();
     if (scorer) {
       prefetch_tmap(&tk);
-      if (DR) prefetch_tmap(&tqr);
+      prefetch_tmap(&tq);
     } else {
       prefetch_tmap(&tv);
     }
@@ -355,53 +364,82 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     // score CTA
     // =========================================================================================
     const uint32_t tQ = tmem;            // columns [0, 256): latent query, bf16 pairs
-    const uint32_t tS = tmem + 256;      // columns [256, 512): two 128-column S slots
+    const uint32_t tS = tmem + 256;      // columns [256, 512): the 256-position S slot
     uint8_t* sQR = smem + Cfg::S_OFF_QR;
     uint8_t* sK = smem + Cfg::S_OFF_K;
-    if (warp == 0 && lane == 0) {
-      // ------------------------------- TMA producer -------------------------------
+    if ((warp == 0 || warp == 2 || warp == 3) && lane == 0) {
+      // ------------------------------- TMA producers -------------------------------
+      // One thread keeps about one TMA instruction in flight at a time, so three threads (warps 0, 2
+      // and 3) fill the ring together: a ring slot holds three 32 KB boxes, box b of every slot use is
+      // loaded by producer b, and each producer arrives once per use (with its bytes, or without a box).
+      // Every block segment takes two uses for its latent query (boxes of 128 columns, two 128-row TMA
+      // loads each: three in the first use, the last one in the second), then three uses per
+      // 256-position tile: 64-column groups {0, 1, 2}, {3, 4, 5} and {6, 7, 8 (rotary)}.
+      const int pid = warp == 0 ? 0 : warp - 1;
       DecWalk w;
       w.begin(p, u0, u1);
       DecSeg sg;
-      int64_t n = 0;          // boxes issued
+      int64_t n = 0;          // ring slot uses walked
       int segi = 0, qr_loads = 0;
       bool ok = true;
+      auto take_slot = [&](int64_t use) -> int {
+        const int s = (int)(use % NK);
+        if (use >= NK && !wait_bar(&bars->k_empty[s], (uint32_t)((use / NK) - 1) & 1u)) return -1;
+        return s;
+      };
       while (ok && w.next(p, sg)) {
         const int qrow = (int)((int64_t)sg.b * p.n_q * p.H + (int64_t)sg.rb * DEC_ROWS);
+        if (DR && pid == 0) {
+          // the rotary query of this segment, once the previous segment's last QK^T has read the old one
+          if (segi > 0 && !wait_bar(&bars->q_empty, (uint32_t)(segi - 1) & 1u)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars->qr_full, DEC_ROWS * 128);
+          tma_load_2d(sQR, &tq, &bars->qr_full, DEC_DC, qrow);
+          ++qr_loads;
+        }
+        for (int qu = 0; qu < 2 && ok; ++qu, ++n) {
+          const int s = take_slot(n);
+          if (s < 0) { ok = false; break; }
+          if (qu == 0 || pid == 0) {
+            const int qb = qu == 0 ? pid : 3;       // 128-column query box
+            uint8_t* dst = sK + s * Cfg::SUPER + (qu == 0 ? pid : 0) * Cfg::BOX;
+            mbar_arrive_expect_tx(&bars->k_full[s], Cfg::BOX);
+            tma_load_2d(dst, &tq, &bars->k_full[s], 128 * qb, qrow);
+            tma_load_2d(dst + Cfg::BOX / 2, &tq, &bars->k_full[s], 128 * qb + 64, qrow);
+          } else {
+            mbar_arrive(&bars->k_full[s]);
+          }
+        }
         for (int tt = 0; tt < sg.ntl && ok; ++tt) {
           const int y = (int)(sg.sstart + (int64_t)(sg.tile0 + tt) * DEC_BT);
-          for (int j = 0; j < NB; ++j, ++n) {
-            const int s = (int)(n % NK);
-            if (n >= NK && !wait_bar(&bars->k_empty[s], (uint32_t)((n / NK) - 1) & 1u)) { ok = false; break; }
-            mbar_arrive_expect_tx(&bars->k_full[s], Cfg::BOX);
-            tma_load_2d(sK + s * Cfg::BOX, &tk, &bars->k_full[s], 64 * j, y);
-          }
-          if (!ok) break;
-          if (DR && tt == 0) {
-            // the rotary query of this segment, once the previous segment's last QK^T has read the old one
-            if (segi > 0 && !wait_bar(&bars->q_empty, (uint32_t)(segi - 1) & 1u)) { ok = false; break; }
-            mbar_arrive_expect_tx(&bars->qr_full, DEC_ROWS * 128);
-            tma_load_2d(sQR, &tqr, &bars->qr_full, DEC_DC, qrow);
-            ++qr_loads;
+          for (int part = 0; part < 3; ++part, ++n) {
+            const int s = take_slot(n);
+            if (s < 0) { ok = false; break; }
+            const int j = 3 * part + pid;           // 64-column group of the cache row
+            if (j < NB) {
+              mbar_arrive_expect_tx(&bars->k_full[s], Cfg::BOX);
+              tma_load_2d(sK + s * Cfg::SUPER + pid * Cfg::BOX, &tk, &bars->k_full[s], 64 * j, y);
+            } else {
+              mbar_arrive(&bars->k_full[s]);
+            }
           }
         }
         ++segi;
       }
       if (*abort_flag) {
-        // drain this CTA's own loads in flight before the shared memory is released
+        // drain the loads in flight before the shared memory is released
         for (int64_t i = (n > NK ? n - NK : 0); i < n; ++i)
           (void)mbar_wait(&bars->k_full[i % NK], (uint32_t)(i / NK) & 1u, drain_ns, p.status);
         if (qr_loads > 0) (void)mbar_wait(&bars->qr_full, (uint32_t)(qr_loads - 1) & 1u, drain_ns, p.status);
       }
     } else if (warp == 1 && lane == 0) {
       // ------------------------------- QK^T issuer -------------------------------
-      // S[slot] = Q K^T over the tile's 128 positions: latent boxes from the TMEM query (A) and the
-      // cache box (B, K-major), the rotary box from the shared-memory query. Each cache box is released
-      // by a commit as soon as its four MMAs complete.
+      // S = Q K^T over the tile's 256 positions: latent groups from the TMEM query (A) and the cache
+      // boxes (B, K-major), the rotary group from the shared-memory query. A ring slot (three groups,
+      // twelve MMAs) is released by one commit as soon as its MMAs complete; the next tile's QK^T waits
+      // only for the softmax warps to have read the S slot out.
       constexpr uint32_t idesc = idesc_bf16_f32(128, DEC_BT, false, false);
       const uint64_t kd0 = smem_desc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t qd0 = smem_desc_sw128(smem_u32(sQR), 16, 1024);
-      constexpr uint64_t kBox = (uint64_t)(Cfg::BOX >> 4);
       DecWalk w;
       w.begin(p, u0, u1);
       DecSeg sg;
@@ -409,31 +447,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       int segi = 0;
       bool ok = true;
       while (ok && w.next(p, sg)) {
+        n += 2;               // the segment's query uses (read by the softmax warps)
         if (!wait_bar(&bars->q_tm, (uint32_t)segi & 1u)) { ok = false; break; }
         if (DR && !wait_bar(&bars->qr_full, (uint32_t)segi & 1u)) { ok = false; break; }
         for (int tt = 0; tt < sg.ntl; ++tt, ++g) {
-          const int sl = (int)(g & 1);
-          if (g >= 2 && !wait_bar(&bars->s_empty[sl], (uint32_t)((g >> 1) - 1) & 1u)) { ok = false; break; }
+          if (g >= 1 && !wait_bar(&bars->s_empty, (uint32_t)(g - 1) & 1u)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t td = tS + sl * DEC_BT;
-          for (int j = 0; j < NB; ++j, ++n) {
+          for (int part = 0; part < 3; ++part, ++n) {
             const int s = (int)(n % NK);
             if (!wait_bar(&bars->k_full[s], (uint32_t)(n / NK) & 1u)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t kd = kd0 + (uint64_t)s * kBox;
-            if (j < 8) {
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ts(td, tQ + j * 32 + kk * 8, kd + (uint64_t)(kk * 2), idesc, (j | kk) ? 1u : 0u);
-            } else {
+            for (int b = 0; b < 3; ++b) {
+              const int j = 3 * part + b;
+              if (j >= NB) break;
+              const uint64_t kd = kd0 + (uint64_t)((s * Cfg::SUPER + b * Cfg::BOX) >> 4);
+              if (j < 8) {
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ss(td, qd0 + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2), idesc, 1u);
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_bf16_ts(tS, tQ + j * 32 + kk * 8, kd + (uint64_t)(kk * 2), idesc, (j | kk) ? 1u : 0u);
+              } else {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_bf16_ss(tS, qd0 + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2), idesc, 1u);
+              }
             }
             mma_commit(&bars->k_empty[s]);
           }
           if (!ok) break;
-          mma_commit(&bars->s_full[sl]);
+          mma_commit(&bars->s_full);
           if (tt + 1 == sg.ntl) mma_commit(&bars->q_empty);
         }
         ++segi;
@@ -446,77 +488,65 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       }
     } else if (warp >= 4) {
       // -------------------------------- softmax --------------------------------
-      const int w8 = warp - 4, q = w8 & 3, hh = w8 >> 2;
+      // warp (q, cg): rows 32 q .. 32 q + 31 (TMEM lanes), positions [64 cg, 64 cg + 64) of each tile;
+      // it also moves query columns [128 cg, 128 cg + 128) of each block into TMEM.
+      // Its P (32 rows x 64 positions, bf16) and side data go straight into the value CTA's P slot of
+      // hand-over 4 g + cg with asynchronous remote stores that count on that slot's barrier.
+      const int w16 = warp - 4, q = warp & 3, cg = w16 >> 2;
       const int row = q * 32 + lane;
       const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-      uint8_t* stg = smem + Cfg::S_OFF_PS + hh * 16384 + q * 4096;   // this warp's 32 rows of P
-      DecSide* side = reinterpret_cast<DecSide*>(smem + Cfg::S_OFF_SIDE + w8 * 512);
-      float* red = reinterpret_cast<float*>(smem + Cfg::S_OFF_RED);  // [2 tiles][2 halves][128], then sums
+      float* red = reinterpret_cast<float*>(smem + Cfg::S_OFF_RED);   // maxima [2][4][128], sums [4][128]
       const uint32_t p_remote = map_to_cta(smem_u32(smem + Cfg::V_OFF_P), 1);
       const uint32_t pf_remote = map_to_cta(smem_u32(&bars->p_full[0]), 1);
-      bool copies = false;    // this lane has bulk copies whose source reads may be pending
       DecWalk w;
       w.begin(p, u0, u1);
       DecSeg sg;
       int64_t g = 0;
       int segi = 0;
       while (w.next(p, sg)) {
-        // ---- the block's latent query into TMEM: rows 32 q .., latent columns [256 hh, 256 hh + 256)
-        if (segi > 0) (void)wait_bar(&bars->q_empty, (uint32_t)(segi - 1) & 1u);
-        tc_fence_after();
-        if (lane == 0 && copies) bulk_wait_read_all();   // the staging area is free again
-        __syncwarp();
+        // ---- the block's latent query into TMEM: rows 32 q .., latent columns [128 cg, 128 cg + 128),
+        // from the segment's query uses (box cg: two 128-row x 64-column TMA boxes, swizzled), once the
+        // previous segment's last QK^T has read the old query
         {
-          const int64_t qr0 = (int64_t)sg.b * p.n_q * p.H + (int64_t)sg.rb * DEC_ROWS + q * 32;
-          const int chunk = lane & 7;
+          const int64_t use0 = 2 * (int64_t)segi + 3 * g;          // the segment's first query use
+          const int64_t use = use0 + (cg < 3 ? 0 : 1);
+          const int slot = (int)(use % NK);
+          (void)wait_bar(&bars->k_full[slot], (uint32_t)(use / NK) & 1u);
+          if (segi > 0) (void)wait_bar(&bars->q_empty, (uint32_t)(segi - 1) & 1u);
+          tc_fence_after();
 #pragma unroll 1
-          for (int r4 = 0; r4 < 4; r4 += 2) {
-            uint4 v[2][8];
+          for (int bx = 0; bx < 2; ++bx) {
+            const uint8_t* src = sK + slot * Cfg::SUPER + (cg < 3 ? cg : 0) * Cfg::BOX + bx * (Cfg::BOX / 2) + row * 128;
+            uint32_t r[32];
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int col0 = hh * 256 + (r4 + h2) * 64;
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const int64_t qr = qr0 + 4 * j + (lane >> 3);
-                const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + qr * p.W + col0) + chunk;
-                v[h2][j] = qr < p.q_rows ? *src : make_uint4(0u, 0u, 0u, 0u);
-              }
+            for (int c = 0; c < 8; ++c) {
+              const uint4 x = *reinterpret_cast<const uint4*>(src + ((c ^ (row & 7)) * 16));
+              r[4 * c] = x.x; r[4 * c + 1] = x.y; r[4 * c + 2] = x.z; r[4 * c + 3] = x.w;
             }
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const int rr = 4 * j + (lane >> 3);
-                *reinterpret_cast<uint4*>(stg + rr * 128 + ((chunk ^ (rr & 7)) * 16)) = v[h2][j];
-              }
-              __syncwarp();
-              uint32_t r[32];
-#pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                const uint4 x = *reinterpret_cast<const uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) * 16));
-                r[4 * c] = x.x; r[4 * c + 1] = x.y; r[4 * c + 2] = x.z; r[4 * c + 3] = x.w;
-              }
-              __syncwarp();
-              tmem_st32(tQ + lane_off + hh * 128 + (r4 + h2) * 32, r);
-            }
+            tmem_st32(tQ + lane_off + cg * 64 + bx * 32, r);
           }
           tmem_wait_st();
           tc_fence_before();
+          fence_proxy_async_smem();     // these generic reads come before the slots' next TMA fills
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->q_tm);
+          named_bar_sync(5, 32 * DEC_SW);   // every softmax warp has read its slot: the slots go back
+          if (w16 == 0 && lane == 0 && !*abort_flag) {
+            mbar_arrive(&bars->k_empty[use0 % NK]);
+            mbar_arrive(&bars->k_empty[(use0 + 1) % NK]);
+          }
         }
         const int cnt = row_count(sg.T, p.n_q, p.H, sg.rb * DEC_ROWS + row, p.causal);
         float m_ref = -INFINITY, l = 0.f;
         for (int tt = 0; tt < sg.ntl; ++tt, ++g) {
-          const int sl = (int)(g & 1);
           const bool last = tt + 1 == sg.ntl;
           float s[64];
-          (void)wait_bar(&bars->s_full[sl], (uint32_t)(g >> 1) & 1u);
+          (void)wait_bar(&bars->s_full, (uint32_t)g & 1u);
           tc_fence_after();
           {
             uint32_t r0[32], r1[32];
-            tmem_ld32(tS + lane_off + sl * DEC_BT + hh * 64, r0);
-            tmem_ld32(tS + lane_off + sl * DEC_BT + hh * 64 + 32, r1);
+            tmem_ld32(tS + lane_off + cg * 64, r0);
+            tmem_ld32(tS + lane_off + cg * 64 + 32, r1);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
@@ -526,9 +556,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0 && !*abort_flag) mbar_arrive(&bars->s_empty[sl]);
+          if (lane == 0 && !*abort_flag) mbar_arrive(&bars->s_empty);
           // mask (only where the tile crosses the row's limit) and the raw row maximum
-          const int t0 = (sg.tile0 + tt) * DEC_BT + hh * 64;
+          const int t0 = (sg.tile0 + tt) * DEC_BT + cg * 64;
           if (t0 + 64 > cnt) {
 #pragma unroll
             for (int c = 0; c < 64; ++c)
@@ -542,10 +572,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
             m4[2] = fmaxf(m4[2], s[c + 2]);
             m4[3] = fmaxf(m4[3], s[c + 3]);
           }
-          float* mx = red + (g & 1) * 2 * DEC_ROWS;
-          mx[hh * DEC_ROWS + row] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-          named_bar_sync(1 + q, 64);          // the two warps of these rows
-          const float mx_t = fmaxf(mx[row], mx[DEC_ROWS + row]) * p.scale_log2;   // the scale is positive
+          float* mx = red + (g & 1) * 4 * DEC_ROWS;
+          mx[cg * DEC_ROWS + row] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          named_bar_sync(1 + q, 128);         // the four warps of these rows
+          const float mx_t = fmaxf(fmaxf(mx[row], mx[DEC_ROWS + row]), fmaxf(mx[2 * DEC_ROWS + row], mx[3 * DEC_ROWS + row])) *
+                             p.scale_log2;    // the scale is positive: the order is kept
           float alpha = 1.f;
           bool moved = false;
           if (mx_t > m_ref + DEC_MOVE) {
@@ -557,56 +588,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
             m_ref = mx_t;
           }
           const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-          // P in bf16 (round to nearest even), and the row sum of the same rounded values, so that
-          // numerator and denominator of the normalisation share the rounding
-          uint32_t pk[32];
-          float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(ex2(fmaf(s[2 * c], p.scale_log2, -mu)),
-                                                            ex2(fmaf(s[2 * c + 1], p.scale_log2, -mu)));
-            pk[c] = *reinterpret_cast<const uint32_t*>(&b2);
-            sum0 += __uint_as_float(pk[c] << 16);
-            sum1 += __uint_as_float(pk[c] & 0xFFFF0000u);
-          }
-          l += sum0 + sum1;
-          if (last) {
-            // the block's row sum is the sum of both halves: the second warp of the pair sends it
-            float* ls = red + 4 * DEC_ROWS;
-            if (hh == 0) ls[row] = l;
-            named_bar_sync(1 + q, 64);
-            if (hh == 1) l += ls[row];
-          }
-          const int flag = (hh == 0) ? (__any_sync(0xffffffffu, moved) ? 1 : 0) : 0;
-          // the P slot of this half tile must have been handed back by the value CTA
-          const int64_t i = 2 * g + hh;
+          // the P slot of this hand-over must have been handed back by the value CTA
+          const int64_t i = (int64_t)DEC_QT * g + cg;
           const int hs = (int)(i % NPH);
           if (i >= NPH) (void)wait_bar(&bars->p_empty[hs], (uint32_t)((i / NPH) - 1) & 1u);
-          if (lane == 0 && copies) bulk_wait_read_all();  // the previous copies have read the staging area
-          __syncwarp();
+          const bool send = !*abort_flag;
+          const uint32_t dst = p_remote + (uint32_t)(hs * Cfg::PSLOT);
+          const uint32_t bar = pf_remote + (uint32_t)(hs * 8);
+          const uint32_t prow = dst + (uint32_t)(row * 128);
+          // P in bf16 (round to nearest even), 8 positions (16 bytes, one swizzled chunk of the row) at a
+          // time, and the row sum of the same rounded values, so that numerator and denominator share
+          // the rounding
+          float sum = 0.f;
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) * 16)) =
-                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-          if (lane == 0) side->flag = flag;
-          side->alpha[lane] = hh == 0 ? alpha : 1.f;
-          side->m[lane] = m_ref;
-          side->l[lane] = l;
-          fence_proxy_async_smem();           // generic writes -> visible to the bulk copies
-          __syncwarp();
-          if (lane == 0 && !*abort_flag) {
-            const uint32_t dst = p_remote + (uint32_t)(hs * Cfg::PSLOT);
-            const uint32_t bar = pf_remote + (uint32_t)(hs * 8);
-            bulk_copy_to_cta(dst + q * 4096, stg, 4096, bar);
-            bulk_copy_to_cta(dst + Cfg::PH + q * 512, side, 512, bar);
-            bulk_commit_group();
-            copies = true;
+          for (int c = 0; c < 8; ++c) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(ex2(fmaf(s[8 * c + 2 * e], p.scale_log2, -mu)),
+                                                              ex2(fmaf(s[8 * c + 2 * e + 1], p.scale_log2, -mu)));
+              pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+              sum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
+            }
+            if (send) st_async_v4(prow + (uint32_t)((c ^ (lane & 7)) * 16), make_uint4(pk[0], pk[1], pk[2], pk[3]), bar);
+          }
+          l += sum;
+          float lsend = l;
+          if (last) {
+            // the block's row sum is the sum of the four warps' sums: the last warp of the row sends it
+            float* ls = red + 8 * DEC_ROWS;
+            ls[cg * DEC_ROWS + row] = l;
+            named_bar_sync(1 + q, 128);
+            if (cg == DEC_QT - 1)
+              lsend = (ls[row] + ls[DEC_ROWS + row]) + (ls[2 * DEC_ROWS + row] + ls[3 * DEC_ROWS + row]);
+          }
+          const int flag = (cg == 0) ? (__any_sync(0xffffffffu, moved) ? 1 : 0) : 0;
+          if (send) {
+            const uint32_t sd = dst + (uint32_t)(Cfg::PH + q * 512);
+            if (lane == 0) st_async_b32(sd + offsetof(DecSide, flag), (uint32_t)flag, bar);
+            st_async_b32(sd + offsetof(DecSide, alpha) + 4 * lane, __float_as_uint(cg == 0 ? alpha : 1.f), bar);
+            st_async_b32(sd + offsetof(DecSide, m) + 4 * lane, __float_as_uint(m_ref), bar);
+            st_async_b32(sd + offsetof(DecSide, l) + 4 * lane, __float_as_uint(lsend), bar);
           }
         }
         ++segi;
       }
-      if (lane == 0 && copies) bulk_wait_all();   // every copy into the peer has landed
-      __syncwarp();
     }
   } else {
     // =========================================================================================
@@ -615,27 +641,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     const uint32_t tO = tmem;   // all 512 columns
     uint8_t* sP = smem + Cfg::V_OFF_P;
     uint8_t* sV = smem + Cfg::V_OFF_V;
-    if (warp == 0 && lane == 0) {
-      // ------------------------------- TMA producer -------------------------------
-      // per half tile (64 positions): two units of 256 latent columns, each four 64-column boxes
+    if ((warp == 0 || warp == 3) && lane == 0) {
+      // ------------------------------- TMA producers -------------------------------
+      // per hand-over (64 positions): one value slot of 512 latent columns, loaded as two TMA
+      // instructions of four 64-column groups each (a 3-D box: columns within a group, positions,
+      // groups), one by each producer (warps 0 and 3: two instructions in flight)
+      const int pid = warp == 0 ? 0 : 1;
       DecWalk w;
       w.begin(p, u0, u1);
       DecSeg sg;
-      int64_t n = 0;
+      int64_t n = 0;          // hand-overs walked
       bool ok = true;
       while (ok && w.next(p, sg)) {
         for (int tt = 0; tt < sg.ntl && ok; ++tt) {
-          for (int hh = 0; hh < 2 && ok; ++hh) {
-            const int y = (int)(sg.sstart + (int64_t)(sg.tile0 + tt) * DEC_BT + hh * DEC_HT);
-            for (int nh = 0; nh < 2; ++nh, ++n) {
-              const int s = (int)(n % NV);
-              if (n >= NV && !wait_bar(&bars->v_empty[s], (uint32_t)((n / NV) - 1) & 1u)) { ok = false; break; }
-              mbar_arrive_expect_tx(&bars->v_full[s], Cfg::UNIT);
-              uint8_t* dst = sV + s * Cfg::UNIT;
-#pragma unroll
-              for (int bx = 0; bx < 4; ++bx)
-                tma_load_2d(dst + bx * (DEC_HT * 128), &tv, &bars->v_full[s], nh * 256 + bx * 64, y);
-            }
+          for (int cg = 0; cg < DEC_QT; ++cg, ++n) {
+            const int y = (int)(sg.sstart + (int64_t)(sg.tile0 + tt) * DEC_BT + cg * DEC_HT);
+            const int s = (int)(n % NV);
+            if (n >= NV && !wait_bar(&bars->v_empty[s], (uint32_t)((n / NV) - 1) & 1u)) { ok = false; break; }
+            mbar_arrive_expect_tx(&bars->v_full[s], Cfg::UNIT);
+            tma_load_3d(sV + s * Cfg::VUNIT + pid * Cfg::UNIT, &tv, &bars->v_full[s], 0, y, 4 * pid);
           }
         }
       }
@@ -645,22 +669,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       }
     } else if (warp == 1 && lane == 0) {
       // ------------------------------- P.C issuer -------------------------------
-      // O[:, 256 nh + ...] += P (128 x 64, K-major, from the P slot) . C (64 x 256, MN-major, the unit)
+      // O[:, 256 nh + ...] += P (128 x 64, K-major, from the P slot) . C (64 x 256, MN-major, from the
+      // hand-over's value slot)
       constexpr uint32_t idesc = idesc_bf16_f32(128, 256, false, true);
       const uint64_t pd0 = smem_desc_sw128(smem_u32(sP), 16, 1024);
       const uint64_t vd0 = smem_desc_sw128(smem_u32(sV), DEC_HT * 128, 1024);
       DecWalk w;
       w.begin(p, u0, u1);
       DecSeg sg;
-      int64_t n = 0, i = 0;
+      int64_t i = 0;
       int segi = 0, fixes = 0;
       bool ok = true;
       while (ok && w.next(p, sg)) {
         for (int tt = 0; tt < sg.ntl && ok; ++tt) {
-          for (int hh = 0; hh < 2; ++hh, ++i) {
+          for (int cg = 0; cg < DEC_QT; ++cg, ++i) {
             const int hs = (int)(i % NPH);
             if (!wait_bar(&bars->p_full[hs], (uint32_t)(i / NPH) & 1u)) { ok = false; break; }
-            const bool first = tt == 0 && hh == 0;
+            const bool first = tt == 0 && cg == 0;
             // the previous segment's epilogue must have read O before this segment overwrites it
             if (first && segi > 0 && !wait_bar(&bars->o_free, (uint32_t)(segi - 1) & 1u)) { ok = false; break; }
             const DecSide* sd = reinterpret_cast<const DecSide*>(sP + hs * Cfg::PSLOT + Cfg::PH);
@@ -671,22 +696,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
               if (!wait_bar(&bars->fix_done, (uint32_t)fixes & 1u)) { ok = false; break; }
               ++fixes;
             }
+            const int s = (int)(i % NV);
+            if (!wait_bar(&bars->v_full[s], (uint32_t)(i / NV) & 1u)) { ok = false; break; }
             tc_fence_after();
+            fence_proxy_async_smem();   // P was stored by the peer's threads: order it before the MMAs read it
             const uint64_t pd = pd0 + (uint64_t)((hs * Cfg::PSLOT) >> 4);
-            for (int nh = 0; nh < 2; ++nh, ++n) {
-              const int s = (int)(n % NV);
-              if (!wait_bar(&bars->v_full[s], (uint32_t)(n / NV) & 1u)) { ok = false; break; }
-              tc_fence_after();
-              const uint64_t vd = vd0 + (uint64_t)((s * Cfg::UNIT) >> 4);
+#pragma unroll
+            for (int nh = 0; nh < 2; ++nh) {
+              const uint64_t vd = vd0 + (uint64_t)((s * Cfg::VUNIT + nh * Cfg::UNIT) >> 4);
 #pragma unroll
               for (int kk = 0; kk < DEC_HT / 16; ++kk)
                 mma_bf16_ss(tO + nh * 256, pd + (uint64_t)(kk * 2), vd + (uint64_t)(kk * (2048 >> 4)), idesc,
                             (first && kk == 0) ? 0u : 1u);
-              mma_commit(&bars->v_empty[s]);
             }
-            if (!ok) break;
+            // one commit per hand-over: the P slot and the value slot are both released from it
             mma_commit(&bars->pfree[hs]);
-            if (tt + 1 == sg.ntl && hh == 1) mma_commit(&bars->o_fin);
+            if (tt + 1 == sg.ntl && cg == DEC_QT - 1) mma_commit(&bars->o_fin);
           }
         }
         ++segi;
@@ -698,28 +723,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       }
     } else if (warp == 2 && lane == 0) {
       // ------------------------------- slot hand-back -------------------------------
-      // once P.C has read a P slot and the rescale / epilogue warps have read its side data: re-arm
-      // the slot's landing barrier for its next use, then tell the score CTA it may write the slot
+      // once P.C of a hand-over has completed and the rescale / epilogue warps have read its side data:
+      // release its value slot to the producers, re-arm the P slot's landing barrier for its next use,
+      // then tell the score CTA it may write the P slot
       const uint32_t pe_remote = map_to_cta(smem_u32(&bars->p_empty[0]), 0);
       DecWalk w;
       w.begin(p, u0, u1);
       DecSeg sg;
       int64_t total = 0;
-      while (w.next(p, sg)) total += 2 * (int64_t)sg.ntl;
-      for (int64_t i = 0; i < total; ++i) {
+      while (w.next(p, sg)) total += (int64_t)DEC_QT * sg.ntl;
+      int64_t i = 0;
+      for (; i < total; ++i) {
         const int hs = (int)(i % NPH);
         if (!wait_bar(&bars->pfree[hs], (uint32_t)(i / NPH) & 1u)) break;
+        mbar_arrive(&bars->v_empty[i % NV]);
         if (i + NPH < total) {
-          mbar_arrive_expect_tx(&bars->p_full[hs], Cfg::PSLOT);
+          mbar_arrive_expect_tx(&bars->p_full[hs], Cfg::PSLOT_TX);
           mbar_arrive_remote_release(pe_remote + (uint32_t)(hs * 8));
         }
       }
+      if (*abort_flag) {
+        // abandoned work: the score CTA may still have remote stores in flight into the slots that are
+        // armed; wait (bounded) for each armed hand-over to land before this CTA may leave
+        for (int64_t u = i; u < total && u < i + NPH; ++u)
+          (void)mbar_wait(&bars->p_full[u % NPH], (uint32_t)(u / NPH) & 1u, drain_ns, p.status);
+      }
     } else if (warp >= 4) {
       // ------------------------------- rescale and epilogue -------------------------------
-      const int w8 = warp - 4, q = w8 & 3, hc = w8 >> 2;
+      // warp (q, cv): rows 32 q .. 32 q + 31, O columns [128 cv, 128 cv + 128)
+      const int w16 = warp - 4, q = warp & 3, cv = w16 >> 2;
       const int row = q * 32 + lane;
       const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-      const uint32_t tcol = tO + lane_off + hc * 256;
+      const uint32_t tcol = tO + lane_off + cv * 128;
       DecWalk w;
       w.begin(p, u0, u1);
       DecSeg sg;
@@ -727,11 +762,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       int segi = 0, fixes = 0;
       while (w.next(p, sg)) {
         for (int tt = 0; tt < sg.ntl; ++tt) {
-          for (int hh = 0; hh < 2; ++hh, ++i) {
+          for (int cg = 0; cg < DEC_QT; ++cg, ++i) {
             const int hs = (int)(i % NPH);
             (void)wait_bar(&bars->p_full[hs], (uint32_t)(i / NPH) & 1u);
-            uint8_t* slot = sP + hs * Cfg::PSLOT;
-            const DecSide* sd = reinterpret_cast<const DecSide*>(slot + Cfg::PH);
+            const DecSide* sd = reinterpret_cast<const DecSide*>(sP + hs * Cfg::PSLOT + Cfg::PH);
             const int any = sd[0].flag | sd[1].flag | sd[2].flag | sd[3].flag;
             if (any) {
               const bool ok = wait_bar(&bars->o_fix, (uint32_t)fixes & 1u);
@@ -740,7 +774,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
               if (ok && sd[q].flag) {
                 const float alpha = sd[q].alpha[lane];
 #pragma unroll 1
-                for (int cc = 0; cc < 256; cc += 32) {
+                for (int cc = 0; cc < 128; cc += 32) {
                   uint32_t r[32];
                   tmem_ld32(tcol + cc, r);
                   tmem_wait_ld();
@@ -754,7 +788,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
               __syncwarp();
               if (lane == 0 && !*abort_flag) mbar_arrive(&bars->fix_done);
             }
-            if (tt + 1 == sg.ntl && hh == 1) {
+            if (tt + 1 == sg.ntl && cg == DEC_QT - 1) {
               // ---- epilogue of the segment: O / l (whole block) or the partial (O, m, l)
               const float m_ref = sd[q].m[lane];
               const float ltot = sd[q].l[lane];
@@ -766,44 +800,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
               const int slotp = 2 * pair + (segi == 0 ? 0 : 1);
               const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
               const float mul = sg.complete ? inv : 1.f;
-              // this slot stays with this CTA until the epilogue is done: each warp turns its rows
-              // around in 2 KB of it (32 rows x 16 columns, fp32) for stores of 64 B per row
-              uint8_t* wst = slot + w8 * 2048;
+              float* dst = sg.complete ? p.out_lat + orow * DEC_DC : p.o_part + ((int64_t)slotp * DEC_ROWS + row) * DEC_DC;
+              const bool write = ok && (sg.complete ? ri < rows_seq : true);
 #pragma unroll 1
-              for (int cc = 0; cc < 256; cc += 16) {
+              for (int cc = 0; cc < 128; cc += 16) {
                 uint32_t r[16];
                 tmem_ld16(tcol + cc, r);
                 tmem_wait_ld();
-                if (ok) {
+                if (write) {
+                  float4* d4 = reinterpret_cast<float4*>(dst + cv * 128 + cc);
 #pragma unroll
                   for (int c = 0; c < 4; ++c)
-                    *reinterpret_cast<float4*>(wst + lane * 64 + ((c ^ ((lane >> 1) & 3)) * 16)) =
-                        make_float4(__uint_as_float(r[4 * c]) * mul, __uint_as_float(r[4 * c + 1]) * mul,
-                                    __uint_as_float(r[4 * c + 2]) * mul, __uint_as_float(r[4 * c + 3]) * mul);
+                    d4[c] = make_float4(__uint_as_float(r[4 * c]) * mul, __uint_as_float(r[4 * c + 1]) * mul,
+                                        __uint_as_float(r[4 * c + 2]) * mul, __uint_as_float(r[4 * c + 3]) * mul);
                 }
-                __syncwarp();
-                if (ok) {
-#pragma unroll
-                  for (int j = 0; j < 4; ++j) {
-                    const int rr = 8 * j + (lane >> 2);       // row within the warp's 32
-                    const int c = lane & 3;
-                    const float4 v = *reinterpret_cast<const float4*>(wst + rr * 64 + ((c ^ ((rr >> 1) & 3)) * 16));
-                    const int rw = q * 32 + rr;               // row within the block
-                    float* d;
-                    bool write;
-                    if (sg.complete) {
-                      write = sg.rb * DEC_ROWS + rw < rows_seq;
-                      d = p.out_lat + ((int64_t)sg.b * rows_seq + sg.rb * DEC_ROWS + rw) * DEC_DC;
-                    } else {
-                      write = true;
-                      d = p.o_part + ((int64_t)slotp * DEC_ROWS + rw) * DEC_DC;
-                    }
-                    if (write) *reinterpret_cast<float4*>(d + hc * 256 + cc + 4 * c) = v;
-                  }
-                }
-                __syncwarp();
               }
-              if (ok && hc == 0) {
+              if (ok && cv == 0) {
                 if (sg.complete) {
                   if (ri < rows_seq && p.lse)
                     p.lse[orow] = ltot > 0.f ? (m_ref + log2f(ltot)) * 0.69314718055994531f : -INFINITY;
@@ -812,7 +824,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
                   p.l_part[(int64_t)slotp * DEC_ROWS + row] = ltot;
                 }
               }
-              fence_proxy_async_smem();     // the slot's generic accesses come before the next copies into it
               tc_fence_before();
               __syncwarp();
               if (lane == 0 && !*abort_flag) mbar_arrive(&bars->o_free);
@@ -828,7 +839,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  cluster_sync();     // the score CTA's copies into the value CTA have landed (each issuer waited)
+  cluster_sync();     // the score CTA stores nothing into the value CTA after this point
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -992,7 +1003,7 @@ static TcDecodePlan plan_tc(const DecodeArgs& a) {
 size_t tc_decode_workspace(const DecodeArgs& a) { return plan_tc(a).total; }
 
 template <int DR>
-static int launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tqr,
+static int launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                            const DecParams& p, cudaStream_t s) {
   static bool attr_set[64] = {false};
   const int dev = current_device();
@@ -1003,7 +1014,7 @@ static int launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tv, const C
     attr_set[dev] = true;
   }
   return launch_pdl(tc_decode_kernel<DR>, dim3(2 * p.G), dim3(DEC_THREADS), (size_t)DecCfg<DR>::SMEM, s, tk, tv,
-                    tqr, p);
+                    tq, p);
 }
 
 int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
@@ -1012,6 +1023,7 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
   char* ws = static_cast<char*>(a.workspace);
   DecParams p{};
   p.q_abs = static_cast<const __nv_bfloat16*>(a.q_abs);
+  p.cache = static_cast<const __nv_bfloat16*>(a.cache);
   p.q_rows = (int64_t)a.batch * a.n_q * a.H;
   p.W = W;
   p.cu = a.cu_seqlens; p.batch = a.batch; p.n_q = a.n_q; p.H = a.H; p.nbps = t.nbps; p.nblocks = t.nblocks;
@@ -1028,9 +1040,9 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
   if (!p.status) return MLA_ERR_CUDA;
   if (t.nblocks == 0) return MLA_OK;
 
-  // the cache: 128-position boxes of 64 columns for the score CTA, 64-position boxes for the value CTA;
-  // the rotary query: 128 rows x 64 columns. All 128-byte swizzled (the MMA operand layout).
-  CUtensorMap tk, tv, tqr;
+  // the cache: 128-position boxes of 64 columns for the score CTA, 64-position x 256-column boxes for
+  // the value CTA; the query: 128 rows x 64 columns. All 128-byte swizzled (the MMA operand layout).
+  CUtensorMap tk, tv, tq;
   const uint64_t rows = (uint64_t)std::max<int64_t>(a.total_rows, 1);
   {
     const uint64_t dims[2] = {(uint64_t)W, rows};
@@ -1039,21 +1051,22 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
     if (!encode_tmap_bf16(&tk, const_cast<void*>(a.cache), 2, dims, st, box)) return MLA_ERR_CUDA;
   }
   {
-    const uint64_t dims[2] = {(uint64_t)W, rows};
-    const uint64_t st[1] = {(uint64_t)W * 2};
-    const uint32_t box[2] = {64, DEC_HT};
-    if (!encode_tmap_bf16(&tv, const_cast<void*>(a.cache), 2, dims, st, box)) return MLA_ERR_CUDA;
+    // positions step by a row, groups by 64 columns: one box is 64 positions x 256 columns, laid out
+    // as four 64-column groups of [64 positions x 128 B] (the MN-major B operand of P.C)
+    const uint64_t dims[3] = {64, rows, (uint64_t)(W / 64)};
+    const uint64_t st[2] = {(uint64_t)W * 2, 128};
+    const uint32_t box[3] = {64, DEC_HT, 4};
+    if (!encode_tmap_bf16(&tv, const_cast<void*>(a.cache), 3, dims, st, box)) return MLA_ERR_CUDA;
   }
-  tqr = tk;
-  if (a.dr) {
+  {
     const uint64_t dims[2] = {(uint64_t)W, (uint64_t)a.batch * a.n_q * a.H};
     const uint64_t st[1] = {(uint64_t)W * 2};
     const uint32_t box[2] = {64, DEC_ROWS};
-    if (!encode_tmap_bf16(&tqr, const_cast<void*>(a.q_abs), 2, dims, st, box)) return MLA_ERR_CUDA;
+    if (!encode_tmap_bf16(&tq, const_cast<void*>(a.q_abs), 2, dims, st, box)) return MLA_ERR_CUDA;
   }
   int st0 = launch_pdl(decode_plan_kernel, dim3(1), dim3(1024), 0, s, p, const_cast<int32_t*>(p.prefix));
   if (st0) return st0;
-  int st = a.dr == 0 ? launch_decode_t<0>(tk, tv, tqr, p, s) : launch_decode_t<64>(tk, tv, tqr, p, s);
+  int st = a.dr == 0 ? launch_decode_t<0>(tk, tv, tq, p, s) : launch_decode_t<64>(tk, tv, tq, p, s);
   if (st) return st;
   // 16 CTAs per block (8 rows each): a split block's merge reads 2-3 partial slots of 256 KB
   return launch_pdl(decode_combine_tc_kernel, dim3((unsigned)t.nblocks, DEC_ROWS / 8), dim3(256), 0, s, p);

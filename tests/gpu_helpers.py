@@ -34,6 +34,28 @@ def assert_close(gpu, ref, dtype, what=""):
     return e
 
 
+# lse is a log-sum-exp in nats: besides the rule above (relative to max|lse_ref|), its absolute error
+# is bounded by the arithmetic. On the bf16 path P is rounded to bf16 (relative error below 2^-9 per
+# term, numerator and row sum share it), so the row sum is off by less than 2^-8 relative: 4e-3 nats;
+# 1e-2 leaves room for the fp32 score accumulation. The fp32 path has no such rounding.
+LSE_ATOL = {"f32": 1e-4, "bf16": 1e-2}
+
+
+def assert_lse_close(gpu, ref, dtype, what="lse", atol=None):
+    gpu, ref = np.asarray(gpu, np.float64), np.asarray(ref, np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    empty = np.isneginf(ref)
+    assert np.array_equal(np.isneginf(gpu), empty), f"{what}: -inf rows differ"
+    if np.all(empty):
+        return 0.0
+    d = float(np.max(np.abs(gpu[~empty] - ref[~empty])))
+    scale = float(np.max(np.abs(ref[~empty])))
+    assert d <= TOL[dtype] * scale, f"{what}: max|gpu-ref| = {d:.3e} > {TOL[dtype]} * {scale:.3e}"
+    a = LSE_ATOL[dtype] if atol is None else atol
+    assert d <= a, f"{what}: max|gpu-ref| = {d:.3e} nats > {a}"
+    return d
+
+
 def mla_dims_of(p: I.DecodeProblem):
     return M.dims(p.n_heads, p.kv_lora_rank, p.rope_dim, p.qk_nope, p.v_head, p.d_model)
 

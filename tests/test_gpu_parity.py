@@ -12,7 +12,8 @@ import torch
 from head_latent_attention_08_b200 import mla as M
 from head_latent_attention_08_b200 import inputs as I
 from oracle import mla_oracle as O
-from gpu_helpers import (GpuDecode, TOL, assert_close, dev, host, mla_dims_of, oracle_seq, rel_err)
+from gpu_helpers import (GpuDecode, TOL, assert_close, assert_lse_close, dev, host, mla_dims_of, oracle_seq,
+                         rel_err)
 
 pytestmark = pytest.mark.gpu
 
@@ -144,7 +145,7 @@ def _check_decode_case(case):
         rows = slice(b * n_q, (b + 1) * n_q)
         assert_close(out_lat[rows], ref_lat, dtype, f"out_lat b={b}")
         assert_close(y[rows], ref_y, dtype, f"y b={b}")
-        np.testing.assert_allclose(lse[rows], ref_lse, rtol=0, atol=TOL[dtype] * 10)
+        assert_lse_close(lse[rows], ref_lse, dtype, f"lse b={b}")
 
 
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}-H{c[1]}-dc{c[2]}-dr{c[3]}-T{c[7]}-nq{c[8]}-c{int(c[9])}")

@@ -91,7 +91,7 @@ def test_repeated_calls_take_no_device_memory():
 
 
 def test_problem_beyond_the_fixed_scratch_is_rejected():
-    c = _case("bf16", [4096, 4096, 4096, 4096], 44)
+    c = _case("bf16", [4096] * 16, 44)
     p = c["p"]
     M.mla_set_decode_clusters(200)    # 400 partial slots of 256 KiB: more than the fixed array holds
     try:
