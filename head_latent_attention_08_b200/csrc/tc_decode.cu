@@ -59,7 +59,7 @@ constexpr int DEC_THREADS = 640;   // 4 control warps + 16 softmax (score CTA) o
 constexpr int DEC_SW = 16;         // softmax / epilogue warps
 constexpr int DEC_DC = 512;        // latent width handled by this kernel
 constexpr int DEC_ROWS = 128;      // rows per block
-constexpr int DEC_NPH = 4;         // P hand-over slots in the value CTA
+constexpr int DEC_NPH = 6;         // P hand-over slots in the value CTA
 constexpr int DEC_PF = 2;          // cache tiles warmed in L2 ahead of the tile QK^T works on
 constexpr int DEC_NPROD = 3;       // TMA-issuing threads of the score CTA
 constexpr float DEC_MOVE = 8.f;    // the reference maximum moves when a row maximum exceeds it by 2^8
@@ -90,9 +90,8 @@ struct DecCfg {
   static constexpr int V_OFF_P = 0;
   static constexpr int V_OFF_V = dec_round1024(DEC_NPH * PSLOT);
   static constexpr int UNIT = DEC_HT * 512;                // 64 positions x 256 latent columns bf16: 32 KB
-  static constexpr int VUNIT = 2 * UNIT;                   // one hand-over's 64 positions x 512 columns
-  static constexpr int NV = (DATA_LIMIT - V_OFF_V) / VUNIT;  // value slots
-  static constexpr int OFF_BAR = dec_max(S_OFF_K + NK * SUPER, V_OFF_V + NV * VUNIT);
+  static constexpr int NV = (DATA_LIMIT - V_OFF_V) / UNIT;  // value slots (256 latent columns each)
+  static constexpr int OFF_BAR = dec_max(S_OFF_K + NK * SUPER, V_OFF_V + NV * UNIT);
   static constexpr int SMEM = OFF_BAR + DEC_BAR_BYTES + 1024;
   static_assert(PSLOT % 1024 == 0, "P slots must keep the 1024-byte swizzle alignment");
   static_assert(NK >= 2, "a block's query takes two ring slots");
@@ -311,7 +310,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       for (int s = 0; s < NPH; ++s) mbar_init(&bars->p_empty[s], 1);
     } else {
       for (int s = 0; s < NV; ++s) {
-        mbar_init(&bars->v_full[s], 2);           // both producers arrive once per slot use
+        mbar_init(&bars->v_full[s], 1);
         mbar_init(&bars->v_empty[s], 1);
       }
       for (int s = 0; s < NPH; ++s) {
@@ -643,34 +642,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     uint8_t* sV = smem + Cfg::V_OFF_V;
     if ((warp == 0 || warp == 3) && lane == 0) {
       // ------------------------------- TMA producers -------------------------------
-      // per hand-over (64 positions): one value slot of 512 latent columns, loaded as two TMA
-      // instructions of four 64-column groups each (a 3-D box: columns within a group, positions,
-      // groups), one by each producer (warps 0 and 3: two instructions in flight)
+      // per hand-over (64 positions): two value slot uses of 256 latent columns, each one TMA
+      // instruction of four 64-column groups (a 3-D box: columns within a group, positions, groups);
+      // use m is issued by producer m % 2 (warps 0 and 3: two instructions in flight)
       const int pid = warp == 0 ? 0 : 1;
       DecWalk w;
       w.begin(p, u0, u1);
       DecSeg sg;
-      int64_t n = 0;          // hand-overs walked
+      int64_t n = 0;          // value slot uses walked
       bool ok = true;
       while (ok && w.next(p, sg)) {
         for (int tt = 0; tt < sg.ntl && ok; ++tt) {
-          for (int cg = 0; cg < DEC_QT; ++cg, ++n) {
+          for (int cg = 0; cg < DEC_QT && ok; ++cg) {
             const int y = (int)(sg.sstart + (int64_t)(sg.tile0 + tt) * DEC_BT + cg * DEC_HT);
-            const int s = (int)(n % NV);
-            if (n >= NV && !wait_bar(&bars->v_empty[s], (uint32_t)((n / NV) - 1) & 1u)) { ok = false; break; }
-            mbar_arrive_expect_tx(&bars->v_full[s], Cfg::UNIT);
-            tma_load_3d(sV + s * Cfg::VUNIT + pid * Cfg::UNIT, &tv, &bars->v_full[s], 0, y, 4 * pid);
+            for (int nh = 0; nh < 2; ++nh, ++n) {
+              if ((n & 1) != pid) continue;
+              const int s = (int)(n % NV);
+              if (n >= NV && !wait_bar(&bars->v_empty[s], (uint32_t)((n / NV) - 1) & 1u)) { ok = false; break; }
+              mbar_arrive_expect_tx(&bars->v_full[s], Cfg::UNIT);
+              tma_load_3d(sV + s * Cfg::UNIT, &tv, &bars->v_full[s], 0, y, 4 * nh);
+            }
           }
         }
       }
       if (*abort_flag) {
         for (int64_t i = (n > NV ? n - NV : 0); i < n; ++i)
-          (void)mbar_wait(&bars->v_full[i % NV], (uint32_t)(i / NV) & 1u, drain_ns, p.status);
+          if ((i & 1) == pid) (void)mbar_wait(&bars->v_full[i % NV], (uint32_t)(i / NV) & 1u, drain_ns, p.status);
       }
     } else if (warp == 1 && lane == 0) {
       // ------------------------------- P.C issuer -------------------------------
-      // O[:, 256 nh + ...] += P (128 x 64, K-major, from the P slot) . C (64 x 256, MN-major, from the
-      // hand-over's value slot)
+      // O[:, 256 nh + ...] += P (128 x 64, K-major, from the P slot) . C (64 x 256, MN-major, from a
+      // value slot); each value slot is released by its own commit
       constexpr uint32_t idesc = idesc_bf16_f32(128, 256, false, true);
       const uint64_t pd0 = smem_desc_sw128(smem_u32(sP), 16, 1024);
       const uint64_t vd0 = smem_desc_sw128(smem_u32(sV), DEC_HT * 128, 1024);
@@ -696,20 +698,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
               if (!wait_bar(&bars->fix_done, (uint32_t)fixes & 1u)) { ok = false; break; }
               ++fixes;
             }
-            const int s = (int)(i % NV);
-            if (!wait_bar(&bars->v_full[s], (uint32_t)(i / NV) & 1u)) { ok = false; break; }
             tc_fence_after();
             fence_proxy_async_smem();   // P was stored by the peer's threads: order it before the MMAs read it
             const uint64_t pd = pd0 + (uint64_t)((hs * Cfg::PSLOT) >> 4);
-#pragma unroll
             for (int nh = 0; nh < 2; ++nh) {
-              const uint64_t vd = vd0 + (uint64_t)((s * Cfg::VUNIT + nh * Cfg::UNIT) >> 4);
+              const int64_t vu = 2 * i + nh;
+              const int s = (int)(vu % NV);
+              if (!wait_bar(&bars->v_full[s], (uint32_t)(vu / NV) & 1u)) { ok = false; break; }
+              tc_fence_after();
+              const uint64_t vd = vd0 + (uint64_t)((s * Cfg::UNIT) >> 4);
 #pragma unroll
               for (int kk = 0; kk < DEC_HT / 16; ++kk)
                 mma_bf16_ss(tO + nh * 256, pd + (uint64_t)(kk * 2), vd + (uint64_t)(kk * (2048 >> 4)), idesc,
                             (first && kk == 0) ? 0u : 1u);
+              mma_commit(&bars->v_empty[s]);
             }
-            // one commit per hand-over: the P slot and the value slot are both released from it
+            if (!ok) break;
             mma_commit(&bars->pfree[hs]);
             if (tt + 1 == sg.ntl && cg == DEC_QT - 1) mma_commit(&bars->o_fin);
           }
@@ -724,8 +728,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     } else if (warp == 2 && lane == 0) {
       // ------------------------------- slot hand-back -------------------------------
       // once P.C of a hand-over has completed and the rescale / epilogue warps have read its side data:
-      // release its value slot to the producers, re-arm the P slot's landing barrier for its next use,
-      // then tell the score CTA it may write the P slot
+      // re-arm the P slot's landing barrier for its next use, then tell the score CTA it may write it
       const uint32_t pe_remote = map_to_cta(smem_u32(&bars->p_empty[0]), 0);
       DecWalk w;
       w.begin(p, u0, u1);
@@ -736,7 +739,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       for (; i < total; ++i) {
         const int hs = (int)(i % NPH);
         if (!wait_bar(&bars->pfree[hs], (uint32_t)(i / NPH) & 1u)) break;
-        mbar_arrive(&bars->v_empty[i % NV]);
         if (i + NPH < total) {
           mbar_arrive_expect_tx(&bars->p_full[hs], Cfg::PSLOT_TX);
           mbar_arrive_remote_release(pe_remote + (uint32_t)(hs * 8));
