@@ -182,6 +182,11 @@ class ClockSampler:
     def mark(self, t0: float, t1: float):
         self.window = (t0, t1)
 
+    def mark_extra(self, t0: float, t1: float):
+        """A second sampled window (the same steps repeated, untimed) whose samples count with the
+        timed region's: the timed region alone lasts a few milliseconds, a few NVML samples."""
+        self.extra = (t0, t1)
+
     def __exit__(self, *exc):
         self._stop.set()
         if self.ok:
@@ -195,18 +200,25 @@ class ClockSampler:
         if not self.ok or not self.samples:
             return None
         rows = self.samples
+        timed = extra = []
         if self.window:
             t0, t1 = self.window
-            inside = [r for r in rows if t0 <= r[0] <= t1]
-            rows = inside or [min(rows, key=lambda r: abs(r[0] - 0.5 * (t0 + t1)))]
+            timed = [r for r in rows if t0 <= r[0] <= t1]
+        if getattr(self, "extra", None):
+            e0, e1 = self.extra
+            extra = [r for r in rows if e0 <= r[0] <= e1]
+        if self.window:
+            rows = (timed + extra) or [min(rows, key=lambda r: abs(r[0] - 0.5 * (t0 + t1)))]
         reasons = set()
         for _, _, bits, _ in rows:
             for name, bit in self.REASONS.items():
                 if bits & bit:
                     reasons.add(name)
         return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(reasons), "samples": len(rows),
-                "power_w_median": statistics.median(r[3] for r in rows), "source": "nvml, 2 ms polling"}
+                "reasons": sorted(reasons), "samples": len(rows), "samples_in_timed_region": len(timed),
+                "samples_in_clock_window": len(extra),
+                "power_w_median": statistics.median(r[3] for r in rows),
+                "source": "nvml, 2 ms polling, over the timed region and an untimed window of the same steps"}
 
 
 # --------------------------------------------------------------------------------------------
@@ -390,6 +402,14 @@ def run_ours(args):
         stop.record(stream)
         torch.cuda.synchronize()
         clk.mark(t_wall0, time.time())
+        # clock window: the same steps again for about 0.3 s, untimed, so that the clock record holds
+        # enough samples (the timed region itself lasts a few milliseconds)
+        t_x0 = time.time()
+        while time.time() - t_x0 < 0.3:
+            for _ in range(20):
+                step(q_nope, q_pe, c_new, kpe_new, row_idx, positions)
+            torch.cuda.synchronize()
+        clk.mark_extra(t_x0, time.time())
     launches = M.mla_launch_count() - launches0
     if world > 1:
         dist.barrier()
@@ -461,6 +481,9 @@ def run_ours(args):
             "device_status": status,
         }
         line["roofline"]["frac_of_roofline_time"] = line["roofline"]["roofline_time_ms"] / line["roofline"]["decode_ms"]
+        if line["clocks"]:
+            # step time scaled by the sampled SM clock: comparable across boxes whose clocks differ
+            line["clocks"]["ms_per_step_x_sm_mhz"] = line["ms_per_step"] * line["clocks"]["sm_mhz"]
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
