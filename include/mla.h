@@ -152,10 +152,11 @@ MLA_API int32_t mla_decode_workspace_size(const mla_dims* dims, int32_t dtype, i
  * Requirements: T_b <= max_seqlen for every b (not checked on the device: the plan assumes it
  * when it sizes the split of each sequence), T_b >= n_q when causal.
  * bf16 calls with d_c = 512 and d_r in {0, 64} run the tensor-core (tcgen05) kernel; every other
- * supported shape runs the CUDA-core kernel. Both accumulate in fp32. The tensor-core kernel splits
- * the d_c + d_r columns over a pair of CTAs, whose partial scores are rounded to fp16 and added in
- * fp16. A raw score (q_abs . k before kq_scale) must therefore stay below 65504 in magnitude. The
- * softmax weights enter the P . C product as bf16 (truncated), and the row sums use the same values.
+ * supported shape runs the CUDA-core kernel. Both accumulate in fp32. In the tensor-core kernel the
+ * scores are fp32 from the MMA to the exponential (no range limit below fp32's); the softmax weights
+ * enter the P . C product as bf16 (round to nearest even), and the row sums add the same values.
+ * Cache rows read past the end of a sequence are multiplied by zero weights: they must hold finite
+ * values (rows of other sequences, or rows the caller keeps finite).
  */
 MLA_API int32_t mla_decode_absorbed(const mla_dims* dims, int32_t dtype, const void* q_abs, const void* cache,
                             const int32_t* cu_seqlens, int32_t batch, int32_t n_q_per_seq,
