@@ -85,8 +85,12 @@ struct DecCfg {
   static constexpr int PH = DEC_ROWS * 128;                // P of a hand-over: 128 rows x 64 positions bf16
   static constexpr int SIDE = 4 * 512;                     // side data of a hand-over: 4 quarters x 512 B
   static constexpr int PSLOT = PH + SIDE;                  // 18 KB (a multiple of 1024)
-  static constexpr int SIDE_TX = 4 + 3 * 32 * 4;           // side bytes a warp stores: flag, alpha, m, l
-  static constexpr int PSLOT_TX = PH + 4 * SIDE_TX;        // bytes that land in a P slot per hand-over
+  // bytes that land in a P slot for hand-over cg of a tile: P, then per warp a 16-byte header (the
+  // flag), the row factors on the tile's first hand-over and the row maxima and sums on its last
+  // (read at the last tile of a block segment)
+  static __host__ __device__ constexpr uint32_t slot_tx(int cg) {
+    return (uint32_t)(PH + 4 * (16 + (cg == 0 ? 128 : 0) + (cg == DEC_QT - 1 ? 256 : 0)));
+  }
   static constexpr int V_OFF_P = 0;
   static constexpr int V_OFF_V = dec_round1024(DEC_NPH * PSLOT);
   static constexpr int UNIT = DEC_HT * 512;                // 64 positions x 256 latent columns bf16: 32 KB
@@ -317,12 +321,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         mbar_init(&bars->p_full[s], 1);
         mbar_init(&bars->pfree[s], DEC_SW + 1);   // the P.C commit and the rescale / epilogue warps
       }
+      // arm the first use of every P slot (hand-over s): one local arrival plus the score CTA's stores
+      for (int s = 0; s < NPH; ++s) mbar_arrive_expect_tx(&bars->p_full[s], Cfg::slot_tx(s % DEC_QT));
       mbar_init(&bars->o_fix, 1);
       mbar_init(&bars->fix_done, DEC_SW);
       mbar_init(&bars->o_fin, 1);
       mbar_init(&bars->o_free, DEC_SW);
-      // arm the first use of every P slot: one local arrival plus the score CTA's copies
-      for (int s = 0; s < NPH; ++s) mbar_arrive_expect_tx(&bars->p_full[s], Cfg::PSLOT_TX);
+
     }
     mbar_init(&bars->drain[0], 1);
     mbar_init(&bars->drain[1], 1);
@@ -622,12 +627,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
               lsend = (ls[row] + ls[DEC_ROWS + row]) + (ls[2 * DEC_ROWS + row] + ls[3 * DEC_ROWS + row]);
           }
           const int flag = (cg == 0) ? (__any_sync(0xffffffffu, moved) ? 1 : 0) : 0;
-          if (send) {
-            const uint32_t sd = dst + (uint32_t)(Cfg::PH + q * 512);
-            if (lane == 0) st_async_b32(sd + offsetof(DecSide, flag), (uint32_t)flag, bar);
-            st_async_b32(sd + offsetof(DecSide, alpha) + 4 * lane, __float_as_uint(cg == 0 ? alpha : 1.f), bar);
-            st_async_b32(sd + offsetof(DecSide, m) + 4 * lane, __float_as_uint(m_ref), bar);
-            st_async_b32(sd + offsetof(DecSide, l) + 4 * lane, __float_as_uint(lsend), bar);
+          // side data in 16-byte stores: the flag on every hand-over, the row factors on the tile's
+          // first, the maxima and sums on its last (the value CTA reads them at a segment's end)
+          const uint32_t sd = dst + (uint32_t)(Cfg::PH + q * 512);
+          const int src4 = (4 * lane) & 31;     // lanes 0..7 gather rows 4 lane .. 4 lane + 3
+          if (send && lane == 0) st_async_v4(sd + offsetof(DecSide, flag), make_uint4((uint32_t)flag, 0u, 0u, 0u), bar);
+          if (cg == 0) {
+            uint4 v;
+            v.x = __float_as_uint(__shfl_sync(0xffffffffu, alpha, src4));
+            v.y = __float_as_uint(__shfl_sync(0xffffffffu, alpha, src4 + 1));
+            v.z = __float_as_uint(__shfl_sync(0xffffffffu, alpha, src4 + 2));
+            v.w = __float_as_uint(__shfl_sync(0xffffffffu, alpha, src4 + 3));
+            if (send && lane < 8) st_async_v4(sd + offsetof(DecSide, alpha) + 16 * lane, v, bar);
+          }
+          if (cg == DEC_QT - 1) {
+            uint4 vm, vl;
+            vm.x = __float_as_uint(__shfl_sync(0xffffffffu, m_ref, src4));
+            vm.y = __float_as_uint(__shfl_sync(0xffffffffu, m_ref, src4 + 1));
+            vm.z = __float_as_uint(__shfl_sync(0xffffffffu, m_ref, src4 + 2));
+            vm.w = __float_as_uint(__shfl_sync(0xffffffffu, m_ref, src4 + 3));
+            vl.x = __float_as_uint(__shfl_sync(0xffffffffu, lsend, src4));
+            vl.y = __float_as_uint(__shfl_sync(0xffffffffu, lsend, src4 + 1));
+            vl.z = __float_as_uint(__shfl_sync(0xffffffffu, lsend, src4 + 2));
+            vl.w = __float_as_uint(__shfl_sync(0xffffffffu, lsend, src4 + 3));
+            if (send && lane < 8) {
+              st_async_v4(sd + offsetof(DecSide, m) + 16 * lane, vm, bar);
+              st_async_v4(sd + offsetof(DecSide, l) + 16 * lane, vl, bar);
+            }
           }
         }
         ++segi;
@@ -740,7 +766,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         const int hs = (int)(i % NPH);
         if (!wait_bar(&bars->pfree[hs], (uint32_t)(i / NPH) & 1u)) break;
         if (i + NPH < total) {
-          mbar_arrive_expect_tx(&bars->p_full[hs], Cfg::PSLOT_TX);
+          mbar_arrive_expect_tx(&bars->p_full[hs], Cfg::slot_tx((int)((i + NPH) % DEC_QT)));
           mbar_arrive_remote_release(pe_remote + (uint32_t)(hs * 8));
         }
       }
