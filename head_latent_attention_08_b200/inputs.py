@@ -28,10 +28,12 @@ import torch
 __all__ = [
     "DecodeProblem",
     "GatedProblem",
+    "ProjectionWeights",
     "NotebookProblem",
     "round_to",
     "decode_problem",
     "gated_problem",
+    "projection_weights",
     "notebook_problem",
     "ragged_seqlens",
     "CONFIG_SEEDS",
@@ -142,6 +144,36 @@ def decode_problem(*, batch: int, n_heads: int, kv_lora_rank: int, rope_dim: int
     positions = np.concatenate([np.arange(seqlens[b] - n_q, seqlens[b]) for b in range(batch)]).astype(np.int32)
     return DecodeProblem(dtype, H, dc, dr, n, dv, D, n_q, seqlens, cu, q_nope, q_pe, w_uk, w_uv, w_o,
                          cache, c_new, kpe_new, row_idx, positions)
+
+
+@dataclasses.dataclass
+class ProjectionWeights:
+    """Hidden states and the input-projection weights of one decode step, PyTorch Linear
+    convention (weight = [out, in]):
+
+      x [N, d_model]; w_cq [q_rank, d_model] (the query down-projection);
+      w_qc [H * qk_nope, q_rank] and w_qr [H * rope_dim, q_rank] (head h owns rows h*qk_nope.. and
+      h*rope_dim..); w_dkv [d_c + rope_dim, d_model]: the latent rows first, then the rotary-key rows.
+    """
+
+    x: np.ndarray
+    w_cq: np.ndarray
+    w_qc: np.ndarray
+    w_qr: np.ndarray
+    w_dkv: np.ndarray
+
+
+def projection_weights(*, n_tokens: int, d_model: int, q_rank: int, n_heads: int, qk_nope: int,
+                       rope_dim: int, kv_lora_rank: int, dtype: str = "f32",
+                       seed: int = 7) -> ProjectionWeights:
+    rng = np.random.default_rng(seed)
+    H, D = n_heads, d_model
+    x = round_to(_normal(rng, (n_tokens, D)), dtype)
+    w_cq = round_to(_normal(rng, (q_rank, D), 1.0 / np.sqrt(D)), dtype)
+    w_qc = round_to(_normal(rng, (H * qk_nope, q_rank), 1.0 / np.sqrt(q_rank)), dtype)
+    w_qr = round_to(_normal(rng, (H * rope_dim, q_rank), 1.0 / np.sqrt(q_rank)), dtype)
+    w_dkv = round_to(_normal(rng, (kv_lora_rank + rope_dim, D), 1.0 / np.sqrt(D)), dtype)
+    return ProjectionWeights(x, w_cq, w_qc, w_qr, w_dkv)
 
 
 @dataclasses.dataclass

@@ -42,6 +42,10 @@ Pins (what fixes each function independently of this file; see tests/test_oracle
   first query equals the first value row; gated_mla_absorbed equals gated_mla.
 * kv_values_per_token_*: the worked table of [lab] Bloque A, filled by hand in the tests.
 * out_project / linear: equal to torch.nn.functional.linear in float64.
+* project_inputs: with absorb_query and the append's rotation, its scores equal those of [fm]
+  Part 3's training-form equation (per-head keys c_i W_kc^(s) and x_i W_kr R_i, rotations built
+  as explicit block-diagonal matrices in torch), at sizes where d = d_c' = d_c so that feeding the
+  wrong latent to a weight still runs.
 No function here is "parity unpinned".
 """
 from __future__ import annotations
@@ -276,6 +280,38 @@ def linear(x: np.ndarray, w: np.ndarray, *, sigmoid_out: bool = False) -> np.nda
     """Y = X W^T (PyTorch Linear convention, W = [out, in]).   [gm] problem equations."""
     y = _f64(x) @ _f64(w).T
     return sigmoid(y) if sigmoid_out else y
+
+
+# --------------------------------------------------------------------------------------------
+# input projections: the low-rank query chain and the KV down-projection
+# --------------------------------------------------------------------------------------------
+
+def project_inputs(x, w_cq, w_qc, w_qr, w_c, w_kr, positions, theta: float = 10000.0):
+    """The parts of [fm] Part 3's inference-form equation computed from the hidden states x_i.
+
+    In the page's row-vector notation (x [N, d]; W'_c [d, d_c']; W_qc [H, d_c', d_k];
+    W_qr [H, d_c', d_r]; W_c [d, d_c]; W_kr [d, d_r]):
+
+      c'_i        = x_i W'_c                      (the query latent, d_c' = 1536 on the page)
+      q_nope[i,s] = c'_i W_qc^(s)                 (absorbed afterwards by W_kc^(s)^T: absorb_query)
+      q_pe[i,s]   = c'_i W_qr^(s) R_i             (rotated at the token's position)
+      c_i         = x_i W_c                       (the latent, i.e. the cached key and value)
+      k_r[i]      = x_i W_kr                      (one rotary key shared by all heads, made from
+                                                   x_i and not from c_i: the page's note on the
+                                                   second term of k says so)
+
+    Returns (q_nope [N, H, d_k], q_pe [N, H, d_r], c [N, d_c], k_r [N, d_r]). k_r is returned
+    before its rotation R_i and c before any normalisation: both belong to the cache append
+    (append_latent), which writes the row concat(c_i, k_r[i] R_i).
+    """
+    x = _f64(x)
+    c_q = x @ _f64(w_cq)
+    q_nope = np.einsum("nq,hqk->nhk", c_q, _f64(w_qc))
+    q_r = np.einsum("nq,hqr->hnr", c_q, _f64(w_qr))          # heads first: one rotation per token
+    q_pe = rope_interleaved(q_r, positions, theta).transpose(1, 0, 2)
+    c = x @ _f64(w_c)
+    k_r = x @ _f64(w_kr)
+    return q_nope, q_pe, c, k_r
 
 
 # --------------------------------------------------------------------------------------------

@@ -545,3 +545,135 @@ def test_planted_softmax_missing_normalisation(monkeypatch):
         return e @ values, (m + np.log(np.sum(e, -1, keepdims=True)))[..., 0]
     monkeypatch.setattr(O, "softmax_attend", bad)
     assert not _decode_pins_pass()
+
+
+# ------------------------------------------------------------------------------------------
+# input projections: the inference form ("formula.md", Part 3) against its training form
+# ------------------------------------------------------------------------------------------
+
+# the first size has d = d_c' = d_c, so a latent handed to the wrong weight still runs (and must be
+# caught by value, not by a shape error); the second has every width different
+PROJ_SIZES = [
+    dict(N=5, d=16, dcq=16, dc=16, H=3, dk=8, dr=6, positions=[3, 17, 0, 250, 9], seed=31),
+    dict(N=4, d=20, dcq=12, dc=10, H=2, dk=6, dr=4, positions=[1, 2, 40, 7], seed=32),
+]
+
+
+def rotation_matrix(p, d, theta=10000.0):
+    """R_p as an explicit d x d block-diagonal matrix acting on row vectors (x R_p): the pair
+    (2i, 2i+1) turns by p * theta^(-2i/d), the angles fixed by tests/golden/rope_frequencies.json."""
+    R = torch.zeros(d, d, dtype=torch.float64)
+    for i in range(d // 2):
+        a = p * theta ** (-2.0 * i / d)
+        R[2 * i, 2 * i], R[2 * i, 2 * i + 1] = math.cos(a), math.sin(a)
+        R[2 * i + 1, 2 * i], R[2 * i + 1, 2 * i + 1] = -math.sin(a), math.cos(a)
+    return R
+
+
+def projection_case(sz):
+    rng = np.random.default_rng(sz["seed"])
+    N, d, dcq, dc, H, dk, dr = (sz[k] for k in ("N", "d", "dcq", "dc", "H", "dk", "dr"))
+    return dict(x=rng.standard_normal((N, d)), w_cq=rng.standard_normal((d, dcq)),
+                w_qc=rng.standard_normal((H, dcq, dk)), w_qr=rng.standard_normal((H, dcq, dr)),
+                w_c=rng.standard_normal((d, dc)), w_kr=rng.standard_normal((d, dr)),
+                w_kc=rng.standard_normal((H, dc, dk)), positions=np.asarray(sz["positions"]))
+
+
+def training_form_scores(c):
+    """Scores q_t^(s) . k_i^(s) of the training-form equation, head by head, in torch:
+    q^(s) = [c' W_qc^(s), c' W_qr^(s) R_t], k^(s) = [c W_kc^(s), x W_kr R_i], c' = x W'_c, c = x W_c."""
+    X = t64(c["x"])
+    cq, lat = X @ t64(c["w_cq"]), X @ t64(c["w_c"])
+    pos = [int(p) for p in c["positions"]]
+    dr = c["w_kr"].shape[1]
+    k_rot = torch.stack([X[i] @ t64(c["w_kr"]) @ rotation_matrix(p, dr) for i, p in enumerate(pos)])
+    out = []
+    for s in range(c["w_qc"].shape[0]):
+        q_n = cq @ t64(c["w_qc"][s])
+        q_r = torch.stack([cq[t] @ t64(c["w_qr"][s]) @ rotation_matrix(p, dr) for t, p in enumerate(pos)])
+        out.append(q_n @ (lat @ t64(c["w_kc"][s])).T + q_r @ k_rot.T)
+    return torch.stack(out).numpy()                       # [H, N (query), N (key)]
+
+
+def inference_form_scores(c):
+    """The same scores through the oracle: project_inputs, the append (rotation of k_r), then the
+    absorbed query q_abs[t, s] = [q_nope W_kc^(s)^T, q_pe] against the cache row [c, k_r R]."""
+    q_nope, q_pe, lat, k_r = O.project_inputs(c["x"], c["w_cq"], c["w_qc"], c["w_qr"], c["w_c"],
+                                              c["w_kr"], c["positions"])
+    N = lat.shape[0]
+    rows = O.append_latent(np.zeros((N, lat.shape[1] + k_r.shape[1])), np.arange(N), lat, k_r,
+                           c["positions"], norm=False, rope=True, dtype="f64")
+    q_abs = O.absorb_query(q_nope, q_pe, np.transpose(c["w_kc"], (0, 2, 1)))
+    return np.einsum("ths,is->hti", q_abs, rows)
+
+
+def _projection_pin_passes():
+    for sz in PROJ_SIZES:
+        c = projection_case(sz)
+        want = training_form_scores(c)
+        got = inference_form_scores(c)
+        if not np.allclose(got, want, rtol=1e-11, atol=1e-11 * np.max(np.abs(want))):
+            return False
+    return True
+
+
+def test_project_inputs_matches_training_form():
+    assert _projection_pin_passes()
+
+
+def _plant_projection(monkeypatch, fn):
+    monkeypatch.setattr(O, "project_inputs", fn)
+
+
+def test_planted_rotary_key_from_latent(monkeypatch):
+    # k_r = c W_kr instead of x W_kr (runs at the first size, where d_c = d)
+    orig = O.project_inputs
+
+    def bad(x, w_cq, w_qc, w_qr, w_c, w_kr, positions, theta=10000.0):
+        q_nope, q_pe, lat, _ = orig(x, w_cq, w_qc, w_qr, w_c, w_kr, positions, theta)
+        return q_nope, q_pe, lat, lat @ np.asarray(w_kr)
+    _plant_projection(monkeypatch, bad)
+    assert not _projection_pin_passes()
+
+
+def test_planted_latent_from_query_latent(monkeypatch):
+    # c = c' W_c instead of x W_c (runs at the first size, where d_c' = d)
+    orig = O.project_inputs
+
+    def bad(x, w_cq, w_qc, w_qr, w_c, w_kr, positions, theta=10000.0):
+        q_nope, q_pe, _, k_r = orig(x, w_cq, w_qc, w_qr, w_c, w_kr, positions, theta)
+        return q_nope, q_pe, (np.asarray(x) @ np.asarray(w_cq)) @ np.asarray(w_c), k_r
+    _plant_projection(monkeypatch, bad)
+    assert not _projection_pin_passes()
+
+
+def test_planted_query_from_hidden_state(monkeypatch):
+    # q_nope = x W_qc, skipping the query latent (runs at the first size, where d = d_c')
+    orig = O.project_inputs
+
+    def bad(x, w_cq, w_qc, w_qr, w_c, w_kr, positions, theta=10000.0):
+        _, q_pe, lat, k_r = orig(x, w_cq, w_qc, w_qr, w_c, w_kr, positions, theta)
+        return np.einsum("nq,hqk->nhk", np.asarray(x), np.asarray(w_qc)), q_pe, lat, k_r
+    _plant_projection(monkeypatch, bad)
+    assert not _projection_pin_passes()
+
+
+def test_planted_unrotated_query(monkeypatch):
+    orig = O.project_inputs
+
+    def bad(x, w_cq, w_qc, w_qr, w_c, w_kr, positions, theta=10000.0):
+        q_nope, _, lat, k_r = orig(x, w_cq, w_qc, w_qr, w_c, w_kr, positions, theta)
+        c_q = np.asarray(x) @ np.asarray(w_cq)
+        return q_nope, np.einsum("nq,hqr->nhr", c_q, np.asarray(w_qr)), lat, k_r
+    _plant_projection(monkeypatch, bad)
+    assert not _projection_pin_passes()
+
+
+def test_planted_query_rotated_one_position_late(monkeypatch):
+    orig = O.project_inputs
+
+    def bad(x, w_cq, w_qc, w_qr, w_c, w_kr, positions, theta=10000.0):
+        return orig(x, w_cq, w_qc, w_qr, w_c, w_kr, np.asarray(positions) + 1, theta)[:2] + \
+            orig(x, w_cq, w_qc, w_qr, w_c, w_kr, positions, theta)[2:]
+    _plant_projection(monkeypatch, bad)
+    assert not _projection_pin_passes()
