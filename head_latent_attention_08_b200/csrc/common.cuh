@@ -118,6 +118,17 @@ int append_latent_launch(const mla_dims& d, int32_t cache_dtype, void* cache, in
                          const int32_t* positions, int64_t n_new, uint32_t flags, float eps,
                          float theta, cudaStream_t stream);
 
+// the same with row strides (in floats) of c_new and kpe_new
+int append_latent_strided(const mla_dims& d, int32_t cache_dtype, void* cache, int64_t cache_rows,
+                          const int64_t* row_idx, const float* c_new, int64_t c_stride, const float* kpe_new,
+                          int64_t kpe_stride, const int32_t* positions, int64_t n_new, uint32_t flags,
+                          float eps, float theta, cudaStream_t stream);
+
+// out[t, h, :] = R_{positions[t]} src[t, h, :] (rotate) or src[t, h, :]: src fp32 [n_rows, H, dr],
+// out in dtype
+int rope_rows_launch(int32_t dtype, const float* src, void* out, const int32_t* positions, int64_t n_rows, int H,
+                     int dr, bool rotate, float theta, cudaStream_t stream);
+
 struct DecodeArgs {
   const void* q_abs; const void* cache; const int32_t* cu_seqlens;
   int32_t batch, n_q, H, dc, dr; int64_t max_seqlen, total_rows;

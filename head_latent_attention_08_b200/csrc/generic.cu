@@ -182,10 +182,21 @@ int copy_rows_strided(const void* src, int64_t ss, void* dst, int64_t ds, int64_
 // latent append: one CTA per new row; the row is built in fp32 shared memory, then stored in the
 // cache dtype with 128-bit stores when the row pitch allows it
 // ---------------------------------------------------------------------------------------------
+// sine and cosine of the RoPE angle of pair i of a dr-wide rotary part at position pos:
+// pos * theta^(-2i/d_r), computed and reduced to [-pi, pi] in double, so that the fp32 sine and cosine
+// of the remainder keep full accuracy at positions of tens of thousands
+__device__ __forceinline__ void rope_sincos(int32_t pos, int i, int dr, double log2_theta, float* sn, float* cs) {
+  const double two_pi = 6.283185307179586476925286766559;
+  const double ang = (double)pos * exp2(-2.0 * (double)i / (double)dr * log2_theta);
+  const double turns = rint(ang * (1.0 / two_pi));
+  sincosf((float)fma(-turns, two_pi, ang), sn, cs);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(128) append_latent_kernel(
     T* __restrict__ cache, const int64_t* __restrict__ row_idx, const float* __restrict__ c_new,
-    const float* __restrict__ kpe_new, const int32_t* __restrict__ positions, int dc, int dr,
+    int64_t c_stride, const float* __restrict__ kpe_new, int64_t kpe_stride,
+    const int32_t* __restrict__ positions, int dc, int dr,
     uint32_t flags, float eps, double log2_theta, int vec8, int64_t cache_rows, int* status) {
   extern __shared__ float row[];
   __shared__ float red[4];
@@ -198,7 +209,7 @@ __global__ void __launch_bounds__(128) append_latent_kernel(
     return;
   }
   const int W = dc + dr;
-  const float* c = c_new + (int64_t)k * dc;
+  const float* c = c_new + (int64_t)k * c_stride;
   float ss = 0.f;
   for (int i = threadIdx.x; i < dc; i += blockDim.x) {
     const float x = c[i];
@@ -214,17 +225,12 @@ __global__ void __launch_bounds__(128) append_latent_kernel(
     for (int i = threadIdx.x; i < dc; i += blockDim.x) row[i] *= inv;
   }
   if (dr > 0) {
-    const float* kp = kpe_new + (int64_t)k * dr;
+    const float* kp = kpe_new + (int64_t)k * kpe_stride;
     if (flags & MLA_APPEND_ROPE) {
-      const double pos = (double)positions[k];
+      const int32_t pos = positions[k];
       for (int i = threadIdx.x; i < dr / 2; i += blockDim.x) {
-        // angle pos * theta^(-2i/d_r) in double, reduced to [-pi, pi] in double, so that the fp32
-        // sine and cosine of the remainder keep full accuracy at positions of tens of thousands
-        const double two_pi = 6.283185307179586476925286766559;
-        const double ang = pos * exp2(-2.0 * (double)i / (double)dr * log2_theta);
-        const double turns = rint(ang * (1.0 / two_pi));
         float sn, cs;
-        sincosf((float)fma(-turns, two_pi, ang), &sn, &cs);
+        rope_sincos(pos, i, dr, log2_theta, &sn, &cs);
         const float x0 = kp[2 * i], x1 = kp[2 * i + 1];
         row[dc + 2 * i] = fmaf(x0, cs, -x1 * sn);
         row[dc + 2 * i + 1] = fmaf(x0, sn, x1 * cs);
@@ -263,6 +269,14 @@ int append_latent_launch(const mla_dims& d, int32_t cache_dtype, void* cache, in
                          const int64_t* row_idx, const float* c_new, const float* kpe_new,
                          const int32_t* positions, int64_t n_new, uint32_t flags, float eps,
                          float theta, cudaStream_t s) {
+  return append_latent_strided(d, cache_dtype, cache, cache_rows, row_idx, c_new, d.kv_lora_rank, kpe_new,
+                               d.rope_dim, positions, n_new, flags, eps, theta, s);
+}
+
+int append_latent_strided(const mla_dims& d, int32_t cache_dtype, void* cache, int64_t cache_rows,
+                          const int64_t* row_idx, const float* c_new, int64_t c_stride, const float* kpe_new,
+                          int64_t kpe_stride, const int32_t* positions, int64_t n_new, uint32_t flags,
+                          float eps, float theta, cudaStream_t s) {
   int* status = device_status_ptr();
   if (!status) return MLA_ERR_CUDA;
   if (n_new == 0) return MLA_OK;
@@ -274,14 +288,65 @@ int append_latent_launch(const mla_dims& d, int32_t cache_dtype, void* cache, in
   if (smem > 48 * 1024) return MLA_ERR_UNSUPPORTED;
   if (cache_dtype == MLA_BF16)
     return launch_pdl(append_latent_kernel<__nv_bfloat16>, dim3((unsigned)n_new), dim3(128), smem, s,
-                      static_cast<__nv_bfloat16*>(cache), row_idx, c_new, kpe_new, positions, d.kv_lora_rank,
-                      d.rope_dim, flags, eps, log2((double)theta), vec8, cache_rows, status);
+                      static_cast<__nv_bfloat16*>(cache), row_idx, c_new, c_stride, kpe_new, kpe_stride,
+                      positions, d.kv_lora_rank, d.rope_dim, flags, eps, log2((double)theta), vec8, cache_rows,
+                      status);
   else
     append_latent_kernel<float><<<(unsigned)n_new, 128, smem, s>>>(
-        static_cast<float*>(cache), row_idx, c_new, kpe_new, positions, d.kv_lora_rank, d.rope_dim,
-        flags, eps, log2((double)theta), vec8, cache_rows, status);
+        static_cast<float*>(cache), row_idx, c_new, c_stride, kpe_new, kpe_stride, positions, d.kv_lora_rank,
+        d.rope_dim, flags, eps, log2((double)theta), vec8, cache_rows, status);
   MLA_LAUNCH_CHECK();
   return MLA_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// rotary part of the queries: out[t, h, :] = R_{pos_t} src[t, h, :] (or a plain copy), fp32 in, the
+// storage dtype out. One CTA per token: the d_r/2 angles once into shared memory, then every head.
+// ---------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(128) rope_rows_kernel(const float* __restrict__ src, T* __restrict__ out,
+                                                        const int32_t* __restrict__ positions, int H, int dr,
+                                                        int rotate, double log2_theta) {
+  extern __shared__ float2 sc[];   // (sin, cos) of pair i
+  griddep_wait();
+  griddep_launch_dependents();
+  const int t = blockIdx.x, half = dr / 2;
+  if (rotate) {
+    const int32_t pos = positions[t];
+    for (int i = threadIdx.x; i < half; i += blockDim.x) {
+      float sn, cs;
+      rope_sincos(pos, i, dr, log2_theta, &sn, &cs);
+      sc[i] = make_float2(sn, cs);
+    }
+    __syncthreads();
+  }
+  const float2* row = reinterpret_cast<const float2*>(src + (int64_t)t * H * dr);
+  T* o = out + (int64_t)t * H * dr;
+  for (int e = threadIdx.x; e < H * half; e += blockDim.x) {
+    const float2 v = row[e];
+    float r0 = v.x, r1 = v.y;
+    if (rotate) {
+      const float2 a = sc[e % half];
+      r0 = fmaf(v.x, a.y, -v.y * a.x);
+      r1 = fmaf(v.x, a.x, v.y * a.y);
+    }
+    o[2 * e] = from_f32<T>(r0);
+    o[2 * e + 1] = from_f32<T>(r1);
+  }
+}
+
+int rope_rows_launch(int32_t dtype, const float* src, void* out, const int32_t* positions, int64_t n_rows, int H,
+                     int dr, bool rotate, float theta, cudaStream_t s) {
+  if (n_rows <= 0 || dr <= 0) return MLA_OK;
+  if (n_rows > 0x7fffffff || dr % 2) return MLA_ERR_SHAPE;
+  const size_t smem = (size_t)(dr / 2) * sizeof(float2);
+  if (smem > 48 * 1024) return MLA_ERR_UNSUPPORTED;
+  const double l2t = log2((double)theta);
+  if (dtype == MLA_BF16)
+    return launch_pdl(rope_rows_kernel<__nv_bfloat16>, dim3((unsigned)n_rows), dim3(128), smem, s, src,
+                      static_cast<__nv_bfloat16*>(out), positions, H, dr, rotate ? 1 : 0, l2t);
+  return launch_pdl(rope_rows_kernel<float>, dim3((unsigned)n_rows), dim3(128), smem, s, src,
+                    static_cast<float*>(out), positions, H, dr, rotate ? 1 : 0, l2t);
 }
 
 // ---------------------------------------------------------------------------------------------

@@ -62,7 +62,7 @@ const char* mla_status_string(int32_t s) {
   }
 }
 
-int32_t mla_abi_version(void) { return 1; }
+int32_t mla_abi_version(void) { return 2; }
 
 int32_t mla_append_latent(const mla_dims* dims, int32_t cache_dtype, void* cache, int64_t cache_rows,
                           const int64_t* row_idx, const float* c_new, const float* kpe_new,
@@ -275,6 +275,221 @@ int32_t mla_linear(int32_t dtype, const void* x, const void* w, int64_t m, int64
   g.C = y; g.sc_b = 0; g.sc_m = n; g.sc_n = 1;
   g.M = m; g.N = n; g.K = k; g.batch = 1; g.sigmoid = sig;
   return gemm_generic(g, dtype, dtype, dtype, dtype, s);
+}
+
+// ---------------------------------------------------------------------------------------------
+// input projections fused with the append
+// ---------------------------------------------------------------------------------------------
+static int check_project_sizes(const mla_dims* dims, int32_t dtype, int32_t q_rank, int64_t n_rows) {
+  int st = check_dims(dims);
+  if (st) return st;
+  if (!dtype_ok(dtype)) return MLA_ERR_DTYPE;
+  if (q_rank <= 0 || n_rows < 0 || dims->qk_nope <= 0 || dims->d_model <= 0) return MLA_ERR_SHAPE;
+  if (n_rows > 0x7fffffffLL) return MLA_ERR_SHAPE;
+  return MLA_OK;
+}
+
+struct ProjectLayout {
+  size_t c_q, q_r, kv, partial, total;   // byte offsets in the workspace
+};
+
+static ProjectLayout project_layout(const mla_dims* d, int32_t dtype, int64_t q_rank, int64_t n_rows) {
+  ProjectLayout L{};
+  const size_t es = dtype_bytes(dtype);
+  L.c_q = 0;
+  L.q_r = L.c_q + round_up((size_t)n_rows * q_rank * es, 256);
+  L.kv = L.q_r + round_up((size_t)n_rows * d->n_heads * d->rope_dim * sizeof(float), 256);
+  L.partial = L.kv + round_up((size_t)n_rows * (d->kv_lora_rank + d->rope_dim) * sizeof(float), 256);
+  L.total = L.partial;
+  if (dtype == MLA_BF16 && tc_project_supported(*d, q_rank, n_rows))
+    L.total += tc_project_partial_bytes(*d, q_rank, n_rows);
+  return L;
+}
+
+static int project_generic(const mla_dims* d, int32_t dtype, int64_t q_rank, const void* x, const void* w_cq,
+                           const void* w_qc, const void* w_qr, const void* w_dkv, int64_t n_rows, void* c_q,
+                           void* q_nope, float* q_r, float* kv, cudaStream_t s) {
+  const int64_t H = d->n_heads, n = d->qk_nope, dr = d->rope_dim, W = d->kv_lora_rank + dr, D = d->d_model;
+  // out[t, o] = sum_k in[t, k] w[o, k]
+  auto linear = [&](const void* in, int32_t in_dt, int64_t k, const void* w, int64_t rows, void* out,
+                    int32_t out_dt) {
+    GemmArgs g{};
+    g.A = in;  g.sa_b = 0; g.sa_m = k; g.sa_k = 1;
+    g.B = w;   g.sb_b = 0; g.sb_n = k; g.sb_k = 1;
+    g.C = out; g.sc_b = 0; g.sc_m = rows; g.sc_n = 1;
+    g.M = n_rows; g.N = rows; g.K = k; g.batch = 1;
+    return gemm_generic(g, in_dt, dtype, out_dt, dtype, s);
+  };
+  int st = linear(x, dtype, D, w_dkv, W, kv, MLA_F32);
+  if (st) return st;
+  if ((st = linear(x, dtype, D, w_cq, q_rank, c_q, dtype))) return st;
+  if ((st = linear(c_q, dtype, q_rank, w_qc, H * n, q_nope, dtype))) return st;
+  if (dr > 0) st = linear(c_q, dtype, q_rank, w_qr, H * dr, q_r, MLA_F32);
+  return st;
+}
+
+int32_t mla_project_workspace_size(const mla_dims* dims, int32_t dtype, int32_t q_rank, int64_t n_rows,
+                                   size_t* bytes) {
+  if (!bytes) return MLA_ERR_NULL;
+  int st = check_project_sizes(dims, dtype, q_rank, n_rows);
+  if (st) return st;
+  *bytes = project_layout(dims, dtype, q_rank, n_rows).total;
+  return MLA_OK;
+}
+
+int32_t mla_project_inputs(const mla_dims* dims, int32_t dtype, int32_t q_rank, const void* x, const void* w_cq,
+                           const void* w_qc, const void* w_qr, const void* w_dkv, int64_t n_rows,
+                           const int32_t* positions, void* q_nope, void* q_pe, void* cache, int64_t cache_rows,
+                           const int64_t* row_idx, uint32_t flags, float eps, float rope_theta, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  int st = check_project_sizes(dims, dtype, q_rank, n_rows);
+  if (st) return st;
+  if (flags & ~(uint32_t)(MLA_APPEND_NORM | MLA_APPEND_ROPE)) return MLA_ERR_MODE;
+  if (cache_rows < 0) return MLA_ERR_SHAPE;
+  if (n_rows == 0) return MLA_OK;
+  const int64_t dr = dims->rope_dim;
+  if (!x || !w_cq || !w_qc || !w_dkv || !q_nope || !cache || !row_idx) return MLA_ERR_NULL;
+  if (dr > 0 && (!w_qr || !q_pe)) return MLA_ERR_NULL;
+  if ((flags & MLA_APPEND_ROPE) && dr > 0) {
+    if (!positions) return MLA_ERR_NULL;
+    if (dr % 2) return MLA_ERR_SHAPE;
+    if (!(rope_theta > 0.f)) return MLA_ERR_SHAPE;
+  }
+  if ((flags & MLA_APPEND_NORM) && !(eps >= 0.f)) return MLA_ERR_SHAPE;
+  if ((st = check_align(dtype, {x, w_cq, w_qc, w_qr, w_dkv, q_nope, q_pe, cache}))) return st;
+  const ProjectLayout L = project_layout(dims, dtype, q_rank, n_rows);
+  if (!workspace || workspace_bytes < L.total) return MLA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return MLA_ERR_ALIGN;
+  char* ws = static_cast<char*>(workspace);
+  void* c_q = ws + L.c_q;
+  float* q_r = reinterpret_cast<float*>(ws + L.q_r);
+  float* kv = reinterpret_cast<float*>(ws + L.kv);
+  cudaStream_t s = as_stream(stream);
+  if (dtype == MLA_BF16 && tc_project_supported(*dims, q_rank, n_rows))
+    st = tc_project(*dims, q_rank, x, w_cq, w_qc, w_qr, w_dkv, n_rows, c_q, q_nope, q_r, kv, ws + L.partial, s);
+  else
+    st = project_generic(dims, dtype, q_rank, x, w_cq, w_qc, w_qr, w_dkv, n_rows, c_q, q_nope, q_r, kv, s);
+  if (st) return st;
+  const bool rotate = (flags & MLA_APPEND_ROPE) != 0;
+  if (dr > 0 && (st = rope_rows_launch(dtype, q_r, q_pe, positions, n_rows, dims->n_heads, (int)dr, rotate,
+                                       rope_theta, s)))
+    return st;
+  const int64_t W = dims->kv_lora_rank + dr;
+  return append_latent_strided(*dims, dtype, cache, cache_rows, row_idx, kv, W, kv + dims->kv_lora_rank, W,
+                               positions, n_rows, flags, eps, rope_theta, s);
+}
+
+// ---------------------------------------------------------------------------------------------
+// one decode step: project -> append -> absorb -> decode -> value/output projection
+// ---------------------------------------------------------------------------------------------
+struct StepLayout {
+  // byte offsets in the workspace
+  size_t x_in, y_out, cu, rows, pos;     // staging of the host buffers (MLA_IO_HOST)
+  size_t q_nope, q_pe, q_abs, out_lat;   // the step's intermediates
+  size_t scratch;                        // shared by the projection, the decode and the output projection
+  size_t total;
+  size_t proj_bytes, dec_bytes, out_bytes;
+};
+
+static int step_layout(const mla_dims* d, int32_t dtype, int32_t q_rank, int32_t batch, int64_t max_seqlen,
+                       int64_t total_rows, StepLayout* L) {
+  const size_t es = dtype_bytes(dtype);
+  const size_t n = (size_t)batch, H = d->n_heads, dc = d->kv_lora_rank, dr = d->rope_dim;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t at = o; o += round_up(bytes, 256); return at; };
+  L->x_in = take(n * d->d_model * es);
+  L->y_out = take(n * d->d_model * es);
+  L->cu = take((n + 1) * sizeof(int32_t));
+  L->rows = take(n * sizeof(int64_t));
+  L->pos = take(n * sizeof(int32_t));
+  L->q_nope = take(n * H * d->qk_nope * es);
+  L->q_pe = take(n * H * dr * es);
+  L->q_abs = take(n * H * (dc + dr) * es);
+  L->out_lat = take(n * H * dc * sizeof(float));
+  L->scratch = o;
+  int st = mla_project_workspace_size(d, dtype, q_rank, batch, &L->proj_bytes);
+  if (st) return st;
+  if ((st = mla_decode_workspace_size(d, dtype, batch, 1, max_seqlen, total_rows, MLA_DECODE_CAUSAL,
+                                      &L->dec_bytes)))
+    return st;
+  if ((st = mla_out_project_workspace_size(d, dtype, batch, &L->out_bytes))) return st;
+  L->total = o + round_up(std::max(L->proj_bytes, std::max(L->dec_bytes, L->out_bytes)), 256);
+  return MLA_OK;
+}
+
+int32_t mla_decode_step_workspace_size(const mla_dims* dims, int32_t dtype, int32_t q_rank, int32_t batch,
+                                       int64_t max_seqlen, int64_t total_rows, size_t* bytes) {
+  if (!bytes) return MLA_ERR_NULL;
+  int st = check_project_sizes(dims, dtype, q_rank, batch);
+  if (st) return st;
+  if ((st = check_decode_sizes(dims, dtype, batch, 1, max_seqlen, total_rows, MLA_DECODE_CAUSAL))) return st;
+  StepLayout L{};
+  if ((st = step_layout(dims, dtype, q_rank, batch, max_seqlen, total_rows, &L))) return st;
+  *bytes = L.total;
+  return MLA_OK;
+}
+
+int32_t mla_decode_step(const mla_dims* dims, int32_t dtype, int32_t q_rank, const mla_step_weights* w,
+                        const void* x, void* cache, const int32_t* cu_seqlens, int32_t batch, int64_t max_seqlen,
+                        int64_t total_rows, const int64_t* row_idx, const int32_t* positions,
+                        uint32_t append_flags, float eps, float rope_theta, void* y, int32_t io, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  int st = check_project_sizes(dims, dtype, q_rank, batch);
+  if (st) return st;
+  if ((st = check_decode_sizes(dims, dtype, batch, 1, max_seqlen, total_rows, MLA_DECODE_CAUSAL))) return st;
+  if (io != MLA_IO_DEVICE && io != MLA_IO_HOST) return MLA_ERR_MODE;
+  if (batch == 0) return MLA_OK;
+  if (!w || !x || !cache || !cu_seqlens || !row_idx || !y) return MLA_ERR_NULL;
+  if (!w->w_cq || !w->w_qc || !w->w_dkv || !w->w_uk || !w->w_uv || !w->w_o) return MLA_ERR_NULL;
+  if (dims->rope_dim > 0 && !w->w_qr) return MLA_ERR_NULL;
+  if (dims->v_head <= 0) return MLA_ERR_SHAPE;
+  StepLayout L{};
+  if ((st = step_layout(dims, dtype, q_rank, batch, max_seqlen, total_rows, &L))) return st;
+  if (!workspace || workspace_bytes < L.total) return MLA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return MLA_ERR_ALIGN;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t s = as_stream(stream);
+  const size_t es = dtype_bytes(dtype);
+  const size_t x_bytes = (size_t)batch * dims->d_model * es;
+  if (io == MLA_IO_HOST) {
+    // the step's inputs into the staging area; with pinned host memory these copies (and the output's)
+    // are asynchronous and the call returns once everything is enqueued on `stream`
+    const bool need_pos = (append_flags & MLA_APPEND_ROPE) && dims->rope_dim > 0;
+    if (need_pos && !positions) return MLA_ERR_NULL;
+    if (cudaMemcpyAsync(ws + L.x_in, x, x_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(ws + L.cu, cu_seqlens, (size_t)(batch + 1) * sizeof(int32_t), cudaMemcpyHostToDevice,
+                        s) != cudaSuccess ||
+        cudaMemcpyAsync(ws + L.rows, row_idx, (size_t)batch * sizeof(int64_t), cudaMemcpyHostToDevice, s) !=
+            cudaSuccess ||
+        (need_pos && cudaMemcpyAsync(ws + L.pos, positions, (size_t)batch * sizeof(int32_t),
+                                     cudaMemcpyHostToDevice, s) != cudaSuccess))
+      return MLA_ERR_CUDA;
+    x = ws + L.x_in;
+    cu_seqlens = reinterpret_cast<const int32_t*>(ws + L.cu);
+    row_idx = reinterpret_cast<const int64_t*>(ws + L.rows);
+    if (need_pos) positions = reinterpret_cast<const int32_t*>(ws + L.pos);
+  }
+  void* q_nope = ws + L.q_nope;
+  void* q_pe = ws + L.q_pe;
+  void* q_abs = ws + L.q_abs;
+  float* out_lat = reinterpret_cast<float*>(ws + L.out_lat);
+  void* scratch = ws + L.scratch;
+  void* y_dev = io == MLA_IO_HOST ? static_cast<void*>(ws + L.y_out) : y;
+  if ((st = mla_project_inputs(dims, dtype, q_rank, x, w->w_cq, w->w_qc, w->w_qr, w->w_dkv, batch, positions,
+                               q_nope, q_pe, cache, total_rows, row_idx, append_flags, eps, rope_theta, scratch,
+                               L.proj_bytes, stream)))
+    return st;
+  if ((st = mla_absorb_weights(dims, dtype, MLA_ABSORB_QUERY, q_nope, q_pe, w->w_uk, batch, q_abs, stream)))
+    return st;
+  if ((st = mla_decode_absorbed(dims, dtype, q_abs, cache, cu_seqlens, batch, 1, max_seqlen, total_rows,
+                                MLA_DECODE_CAUSAL, out_lat, nullptr, scratch, L.dec_bytes, stream)))
+    return st;
+  if ((st = mla_out_project(dims, dtype, out_lat, w->w_uv, w->w_o, nullptr, batch, y_dev, scratch, L.out_bytes,
+                            stream)))
+    return st;
+  if (io == MLA_IO_HOST && cudaMemcpyAsync(y, y_dev, x_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  return MLA_OK;
 }
 
 int32_t mla_check_status(void* stream, int32_t* device_status) {

@@ -23,6 +23,14 @@ int tc_out_project(const mla_dims& d, const float* out_lat, const void* w_uv, co
                    const void* gate, int64_t n_rows, void* y, void* workspace, size_t ws_bytes,
                    cudaStream_t s);
 
+// input projections of new tokens (bf16 in, fp32 accumulate): c_q = x W_cq^T and q_nope = c_q W_qc^T
+// in bf16, q_r = c_q W_qr^T and kv = x W_dkv^T in fp32; partial = split-K scratch of
+// tc_project_partial_bytes() bytes
+bool tc_project_supported(const mla_dims& d, int64_t q_rank, int64_t n_rows);
+size_t tc_project_partial_bytes(const mla_dims& d, int64_t q_rank, int64_t n_rows);
+int tc_project(const mla_dims& d, int64_t q_rank, const void* x, const void* w_cq, const void* w_qc,
+               const void* w_qr, const void* w_dkv, int64_t n_rows, void* c_q, void* q_nope, float* q_r,
+               float* kv, void* partial, cudaStream_t s);
 // dense linear Y = X W^T
 bool tc_linear_supported(int64_t m, int64_t n, int64_t k);
 int tc_linear(const void* x, const void* w, int64_t m, int64_t n, int64_t k, int sigmoid, void* y,

@@ -331,7 +331,7 @@ static GemmPlan plan_gemm(int M, int N, int K, int batch, int max_splits) {
   GemmPlan g;
   g.BN = N <= 64 ? 64 : (N <= 128 ? 128 : 256);
   g.n_tiles = (int)ceil_div(N, g.BN);
-  g.m_tiles = M / 128;
+  g.m_tiles = (int)ceil_div(M, 128);
   const int total_chunks = (int)ceil_div(K, 64);
   const int64_t base = (int64_t)g.m_tiles * g.n_tiles * batch;
   int splits = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count() / std::max<int64_t>(base, 1),
@@ -375,7 +375,9 @@ static int tc_gemm(const GemmOperand& A, bool a_mn, const GemmOperand& Bop, int 
                    void* out, int64_t out_sb, int64_t out_st, bool out_f32, const void* gate, int64_t gate_sb,
                    int64_t gate_st, bool sigmoid, void* partial_ws, cudaStream_t s,
                    const GemmTail& tail = GemmTail()) {
-  if (M % 128 || K % 64 || N <= 0 || batch <= 0) return MLA_ERR_UNSUPPORTED;
+  // a K-major A may end inside its last 128-row tile (the TMA zero-fills the rows past M and the
+  // epilogue skips them); an MN-major A loads its rows as 64-wide boxes and takes whole tiles only
+  if (M <= 0 || M % 4 || (a_mn && M % 128) || K % 64 || N <= 0 || batch <= 0) return MLA_ERR_UNSUPPORTED;
   // the epilogue writes runs of 4 consecutive outputs (8 or 16 bytes) and reads 4 gate values
   if (out_sb % 4 || out_st % 4 || (reinterpret_cast<uintptr_t>(out) & 15) ||
       (gate && (gate_sb % 4 || gate_st % 4 || (reinterpret_cast<uintptr_t>(gate) & 7))))
@@ -502,6 +504,65 @@ int tc_out_project(const mla_dims& d, const float* out_lat, const void* w_uv, co
   GemmOperand A2{const_cast<void*>(w_o), (uint64_t)K, (uint64_t)D, 1, (uint64_t)(K * 2), (uint64_t)(D * K * 2)};
   GemmOperand B2{v, (uint64_t)K, (uint64_t)n_rows, 1, (uint64_t)(K * 2), (uint64_t)(n_rows * K * 2)};
   return tc_gemm(A2, false, B2, (int)D, (int)n_rows, (int)K, 1, y, 0, D, false, nullptr, 0, 0, false, partial, s);
+}
+
+// ---------------------------------------------------------------------------------------------
+// input projections: c' = x W_cq^T (bf16 scratch), q_nope = c' W_qc^T (bf16), q_r = c' W_qr^T (fp32),
+// kv = x W_dkv^T (fp32). A = the weight (K-major, M = its output rows), B = the activations.
+// ---------------------------------------------------------------------------------------------
+bool tc_project_supported(const mla_dims& d, int64_t q_rank, int64_t n_rows) {
+  const int64_t H = d.n_heads, n = d.qk_nope, dr = d.rope_dim, dc = d.kv_lora_rank, D = d.d_model;
+  return n_rows > 0 && n_rows < (1LL << 30) && D % 64 == 0 && q_rank % 64 == 0 && q_rank < (1LL << 30) &&
+         n > 0 && (H * n) % 4 == 0 && (H * dr) % 4 == 0 && (dc + dr) % 4 == 0 && H * n < (1LL << 30) &&
+         D < (1LL << 30);
+}
+
+static void project_gemm_dims(const mla_dims& d, int64_t q_rank, int64_t n_rows, int dims[4][3]) {
+  const int64_t H = d.n_heads;
+  const int64_t rows[4] = {q_rank, H * d.qk_nope, H * d.rope_dim, (int64_t)d.kv_lora_rank + d.rope_dim};
+  const int64_t ks[4] = {d.d_model, q_rank, q_rank, d.d_model};
+  for (int i = 0; i < 4; ++i) {
+    dims[i][0] = (int)rows[i]; dims[i][1] = (int)n_rows; dims[i][2] = (int)ks[i];
+  }
+}
+
+size_t tc_project_partial_bytes(const mla_dims& d, int64_t q_rank, int64_t n_rows) {
+  int g[4][3];
+  project_gemm_dims(d, q_rank, n_rows, g);
+  size_t b = 0;
+  for (int i = 0; i < 4; ++i)
+    if (g[i][0] > 0) b = std::max(b, gemm_partial_bytes(g[i][0], g[i][1], g[i][2], 1));
+  return b;
+}
+
+int tc_project(const mla_dims& d, int64_t q_rank, const void* x, const void* w_cq, const void* w_qc,
+               const void* w_qr, const void* w_dkv, int64_t n_rows, void* c_q, void* q_nope, float* q_r,
+               float* kv, void* partial, cudaStream_t s) {
+  int g[4][3];
+  project_gemm_dims(d, q_rank, n_rows, g);
+  const int64_t D = d.d_model;
+  auto weight = [](const void* w, int64_t rows, int64_t k) {
+    return GemmOperand{const_cast<void*>(w), (uint64_t)k, (uint64_t)rows, 1, (uint64_t)(k * 2),
+                       (uint64_t)(rows * k * 2)};
+  };
+  const GemmOperand bx{const_cast<void*>(x), (uint64_t)D, (uint64_t)n_rows, 1, (uint64_t)(D * 2),
+                       (uint64_t)(n_rows * D * 2)};
+  const GemmOperand bq{c_q, (uint64_t)q_rank, (uint64_t)n_rows, 1, (uint64_t)(q_rank * 2),
+                       (uint64_t)(n_rows * q_rank * 2)};
+  // the KV down-projection, then the query chain (c_q feeds the last two products)
+  int st = tc_gemm(weight(w_dkv, g[3][0], D), false, bx, g[3][0], g[3][1], g[3][2], 1, kv, 0, g[3][0], true,
+                   nullptr, 0, 0, false, partial, s);
+  if (st) return st;
+  if ((st = tc_gemm(weight(w_cq, g[0][0], D), false, bx, g[0][0], g[0][1], g[0][2], 1, c_q, 0, g[0][0], false,
+                    nullptr, 0, 0, false, partial, s)))
+    return st;
+  if ((st = tc_gemm(weight(w_qc, g[1][0], q_rank), false, bq, g[1][0], g[1][1], g[1][2], 1, q_nope, 0, g[1][0],
+                    false, nullptr, 0, 0, false, partial, s)))
+    return st;
+  if (g[2][0] > 0)
+    st = tc_gemm(weight(w_qr, g[2][0], q_rank), false, bq, g[2][0], g[2][1], g[2][2], 1, q_r, 0, g[2][0], true,
+                 nullptr, 0, 0, false, partial, s);
+  return st;
 }
 
 bool tc_linear_supported(int64_t m, int64_t n, int64_t k) {

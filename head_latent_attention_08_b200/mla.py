@@ -24,12 +24,14 @@ MLA_APPEND_NORM, MLA_APPEND_ROPE = 1, 2
 MLA_DECODE_CAUSAL = 1
 MLA_LINEAR_SIGMOID, MLA_LINEAR_W_KN = 1, 2
 MLA_ERR_SHAPE, MLA_ERR_TIMEOUT = 2, 7
+MLA_IO_DEVICE, MLA_IO_HOST = 0, 1
 
 EXPORTED = (
     "mla_status_string", "mla_abi_version", "mla_append_latent", "mla_absorb_weights",
     "mla_decode_workspace_size", "mla_decode_absorbed", "mla_out_project_workspace_size",
     "mla_out_project", "mla_linear", "mla_check_status", "mla_set_wait_limit", "mla_launch_count",
     "mla_set_decode_clusters", "mla_wait_selftest", "mla_decode_absorbed_noalloc",
+    "mla_project_workspace_size", "mla_project_inputs", "mla_decode_step_workspace_size", "mla_decode_step",
 )
 
 
@@ -48,6 +50,10 @@ class mla_dims(ctypes.Structure):
 
 def dims(n_heads, kv_lora_rank, rope_dim=0, qk_nope=0, v_head=0, d_model=0, kq_scale=0.0):
     return mla_dims(n_heads, kv_lora_rank, rope_dim, qk_nope, v_head, d_model, kq_scale)
+
+
+class mla_step_weights(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in ("w_cq", "w_qc", "w_qr", "w_dkv", "w_uk", "w_uv", "w_o")]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -73,6 +79,12 @@ _SIGS = {
     "mla_wait_selftest": (_I32, [_P]),
     "mla_decode_absorbed_noalloc": (_I32, [_DIMS, _I32, _P, _P, _P, _I32, _I32, _I64, _I64, _U32, _P, _P,
                                            _P]),
+    "mla_project_workspace_size": (_I32, [_DIMS, _I32, _I32, _I64, ctypes.POINTER(_SZ)]),
+    "mla_project_inputs": (_I32, [_DIMS, _I32, _I32, _P, _P, _P, _P, _P, _I64, _P, _P, _P, _P, _I64, _P, _U32,
+                                  _F, _F, _P, _SZ, _P]),
+    "mla_decode_step_workspace_size": (_I32, [_DIMS, _I32, _I32, _I32, _I64, _I64, ctypes.POINTER(_SZ)]),
+    "mla_decode_step": (_I32, [_DIMS, _I32, _I32, ctypes.POINTER(mla_step_weights), _P, _P, _P, _I32, _I64,
+                               _I64, _P, _P, _U32, _F, _F, _P, _I32, _P, _SZ, _P]),
 }
 
 
@@ -117,6 +129,16 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
         return None
     if not t.is_cuda:
         raise ValueError("tensors passed to the library must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return t.data_ptr()
+
+
+def _host_ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError("this argument is host memory")
     if not t.is_contiguous():
         raise ValueError("tensors passed to the library must be contiguous")
     return t.data_ptr()
@@ -205,6 +227,49 @@ def mla_linear(x: torch.Tensor, w: torch.Tensor, m: int, n: int, k: int, flags: 
                             _stream(stream)), "mla_linear")
 
 
+def mla_project_workspace_size(d: mla_dims, dtype: torch.dtype, q_rank: int, n_rows: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().mla_project_workspace_size(ctypes.byref(d), _dtype_code(dtype), q_rank, n_rows, ctypes.byref(n)),
+           "mla_project_workspace_size")
+    return int(n.value)
+
+
+def mla_project_inputs(d: mla_dims, q_rank: int, x: torch.Tensor, w_cq: torch.Tensor, w_qc: torch.Tensor,
+                       w_qr: Optional[torch.Tensor], w_dkv: torch.Tensor, positions: Optional[torch.Tensor],
+                       q_nope: torch.Tensor, q_pe: Optional[torch.Tensor], cache: torch.Tensor,
+                       row_idx: torch.Tensor, flags: int, workspace: torch.Tensor, eps: float = 1e-6,
+                       rope_theta: float = 10000.0, stream=None) -> None:
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().mla_project_inputs(ctypes.byref(d), _dtype_code(x.dtype), q_rank, _ptr(x), _ptr(w_cq), _ptr(w_qc),
+                                    _ptr(w_qr), _ptr(w_dkv), x.shape[0], _ptr(positions), _ptr(q_nope),
+                                    _ptr(q_pe), _ptr(cache), cache.shape[0], _ptr(row_idx), flags, eps,
+                                    rope_theta, _ptr(workspace), ws_bytes, _stream(stream)),
+           "mla_project_inputs")
+
+
+def mla_decode_step_workspace_size(d: mla_dims, dtype: torch.dtype, q_rank: int, batch: int, max_seqlen: int,
+                                   total_rows: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().mla_decode_step_workspace_size(ctypes.byref(d), _dtype_code(dtype), q_rank, batch, max_seqlen,
+                                                total_rows, ctypes.byref(n)), "mla_decode_step_workspace_size")
+    return int(n.value)
+
+
+def mla_decode_step(d: mla_dims, q_rank: int, w: mla_step_weights, x: torch.Tensor, cache: torch.Tensor,
+                    cu_seqlens: torch.Tensor, batch: int, max_seqlen: int, row_idx: torch.Tensor,
+                    positions: Optional[torch.Tensor], flags: int, y: torch.Tensor, io: int,
+                    workspace: torch.Tensor, eps: float = 1e-6, rope_theta: float = 10000.0, stream=None) -> None:
+    """One decode step through the C ABI. With io == MLA_IO_HOST, x, y, cu_seqlens, row_idx and
+    positions are host tensors (page-locked for asynchronous copies)."""
+    p = _host_ptr if io == MLA_IO_HOST else _ptr
+    assert cu_seqlens.dtype == torch.int32 and row_idx.dtype == torch.int64
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().mla_decode_step(ctypes.byref(d), _dtype_code(cache.dtype), q_rank, ctypes.byref(w), p(x),
+                                 _ptr(cache), p(cu_seqlens), batch, max_seqlen, cache.shape[0], p(row_idx),
+                                 p(positions), flags, eps, rope_theta, p(y), io, _ptr(workspace), ws_bytes,
+                                 _stream(stream)), "mla_decode_step")
+
+
 def mla_check_status(stream=None) -> int:
     v = ctypes.c_int32(0)
     _check(lib().mla_check_status(_stream(stream), ctypes.byref(v)), "mla_check_status")
@@ -272,6 +337,37 @@ class DecodeStep:
                             self.flags, self.out_lat, self.lse, self.ws_dec, stream=stream)
         mla_out_project(d, self.out_lat, self.w_uv, self.w_o, None, nq, y, self.ws_out,
                         stream=stream)
+        return y
+
+
+class DecodeLayerStep:
+    """One decode step of the attention layer from hidden states to outputs through the library's
+    single step call (mla_decode_step): input projections with the append, query absorption,
+    decode over the latent cache, value and output projection. One new token per sequence."""
+
+    def __init__(self, d: mla_dims, q_rank: int, batch: int, max_seqlen: int, cache: torch.Tensor,
+                 cu_seqlens: torch.Tensor, w_cq, w_qc, w_qr, w_dkv, w_uk, w_uv, w_o,
+                 append_flags: int = MLA_APPEND_NORM | MLA_APPEND_ROPE):
+        self.d, self.q_rank, self.batch, self.max_seqlen = d, q_rank, batch, max_seqlen
+        self.cache, self.cu, self.append_flags = cache, cu_seqlens, append_flags
+        self.tensors = (w_cq, w_qc, w_qr, w_dkv, w_uk, w_uv, w_o)     # kept alive with the struct
+        self.w = mla_step_weights(*[None if t is None else _ptr(t) for t in self.tensors])
+        self.y = torch.empty(batch, d.d_model, dtype=cache.dtype, device=cache.device)
+        self.ws = workspace(mla_decode_step_workspace_size(d, cache.dtype, q_rank, batch, max_seqlen,
+                                                           cache.shape[0]), cache.device)
+
+    def __call__(self, x, row_idx, positions, y=None, io: int = MLA_IO_DEVICE, cu_seqlens=None, stream=None):
+        """Device io: every tensor on the GPU. Host io: x, y, row_idx, positions and cu_seqlens
+        (defaulting to the step's, copied to the host once) are host tensors."""
+        y = self.y if y is None else y
+        cu = self.cu if cu_seqlens is None else cu_seqlens
+        if io == MLA_IO_HOST and cu.is_cuda:
+            self.cu_host = getattr(self, "cu_host", None)
+            if self.cu_host is None:
+                self.cu_host = cu.cpu().pin_memory()
+            cu = self.cu_host
+        mla_decode_step(self.d, self.q_rank, self.w, x, self.cache, cu, self.batch, self.max_seqlen, row_idx,
+                        positions, self.append_flags, y, io, self.ws, stream=stream)
         return y
 
 

@@ -13,13 +13,16 @@
  *   [lab] "Lab 01 - Ejercicio matematico de MLA" (lynx-cortex), Bloque B: the matmul identity
  *         q^T W_UK c = (W_UK^T q)^T c.
  *   [fm]  "preacher-1/MLA_tutorial formula.md", Part 3, inference-form equation: o_t is the
- *         concatenation of o^(s) W_v^(s), followed by the output projection.
+ *         concatenation of o^(s) W_v^(s), followed by the output projection; the query comes from
+ *         the low-rank latent c'_i = x_i W'_c as [c'_i W_qc^(s) W_kc^(s)T, c'_i W_qr^(s) R_i] and the
+ *         key from c_i = x_i W_c and the rotary part x_i W_kr R_i (from x_i, not c_i).
  *   [gm]  "Gated MLA" (tensortonic, Kimi K3 step 2 of 11): Y = [sigmoid(X Wg^T) * O] Wo^T,
  *         causal mask removing later positions, the Requirements (inputs are not mutated).
  *
  * Conventions shared by every entry point
  *   - All tensors are caller-owned DEVICE memory, dense, row-major, in the dtype named by the call
- *     (MLA_F32 or MLA_BF16), except where a parameter says float / int32 / int64 explicitly.
+ *     (MLA_F32 or MLA_BF16), except where a parameter says float / int32 / int64 explicitly, and
+ *     except the host buffers of mla_decode_step with MLA_IO_HOST.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Every call is asynchronous
  *     with respect to the host and enqueues its kernels on that stream only.
  *   - Inputs are never written. Outputs are written only where documented.
@@ -81,6 +84,20 @@ enum { MLA_APPEND_NORM = 1u, MLA_APPEND_ROPE = 2u };
 enum { MLA_DECODE_CAUSAL = 1u };
 /* flags of mla_linear */
 enum { MLA_LINEAR_SIGMOID = 1u, MLA_LINEAR_W_KN = 2u };
+/* where the step's x, y and index arrays live (mla_decode_step) */
+enum { MLA_IO_DEVICE = 0, MLA_IO_HOST = 1 };
+
+/* The weights of one decode step, all DEVICE memory in the step's dtype, PyTorch Linear convention
+ * ([out, in], row-major) for the dense projections. */
+typedef struct mla_step_weights {
+  const void* w_cq;   /* W'_c^T  [q_rank, d_model]                       query down-projection     */
+  const void* w_qc;   /* W_qc^T  [n_heads * qk_nope, q_rank]             head h: rows h*qk_nope..  */
+  const void* w_qr;   /* W_qr^T  [n_heads * rope_dim, q_rank]            head h: rows h*rope_dim.. */
+  const void* w_dkv;  /* [W_c, W_kr]^T [kv_lora_rank + rope_dim, d_model] latent rows, then rotary */
+  const void* w_uk;   /* W_UK    [n_heads, qk_nope, kv_lora_rank]        (W_kc^(h) transposed)     */
+  const void* w_uv;   /* W_UV    [n_heads, v_head, kv_lora_rank]                                   */
+  const void* w_o;    /* W_O     [d_model, n_heads * v_head]                                       */
+} mla_step_weights;
 
 /* Human-readable name of a status code (static string, never NULL). */
 MLA_API const char* mla_status_string(int32_t status);
@@ -188,6 +205,65 @@ MLA_API int32_t mla_out_project(const mla_dims* dims, int32_t dtype, const float
  */
 MLA_API int32_t mla_linear(int32_t dtype, const void* x, const void* w, int64_t m, int64_t n, int64_t k,
                    uint32_t flags, void* y, void* stream);
+
+/* Bytes of scratch mla_project_inputs needs for n_rows tokens. */
+MLA_API int32_t mla_project_workspace_size(const mla_dims* dims, int32_t dtype, int32_t q_rank, int64_t n_rows,
+                                           size_t* bytes);
+
+/*
+ * mla_project_inputs -- the input projections of n_rows new tokens ([fm] Part 3, inference-form
+ * equation, the terms computed from x), fused with the latent append:
+ *     c'_t         = x_t W'_c                        (q_rank wide; scratch, in `dtype`)
+ *     q_nope[t, h] = c'_t W_qc^(h)                   (absorbed next by MLA_ABSORB_QUERY)
+ *     q_pe[t, h]   = c'_t W_qr^(h), turned by R_{positions[t]} when flags has MLA_APPEND_ROPE
+ *     c_t, k_t     = x_t W_c, x_t W_kr               (fp32 scratch; never rounded before the append)
+ *     cache row row_idx[t] = concat(c_t, k_t) with mla_append_latent's flags (norm of c_t, rotation
+ *     of k_t at positions[t]).
+ *   x        [n_rows, d_model]; w_cq, w_qc, w_qr, w_dkv as in mla_step_weights (w_qr may be NULL
+ *            when rope_dim == 0); q_nope [n_rows, H, qk_nope] and q_pe [n_rows, H, rope_dim] written;
+ *   cache, cache_rows, row_idx, positions, eps, rope_theta: as mla_append_latent, with the cache in
+ *   `dtype`. The rotation is the append's: pair (2i, 2i+1) turns by pos * rope_theta^(-2i/rope_dim).
+ *   Products accumulate in fp32; bf16 operands go through the tensor cores when d_model and q_rank
+ *   are multiples of 64 (c'_t is then rounded to bf16 once, as the next product's operand).
+ * Errors: MLA_ERR_NULL, MLA_ERR_SHAPE (q_rank <= 0, qk_nope <= 0, d_model <= 0, rope_dim odd with
+ * ROPE), MLA_ERR_DTYPE, MLA_ERR_MODE (unknown flag), MLA_ERR_ALIGN (16 B for bf16 tensors, 256 B for
+ * the workspace), MLA_ERR_WORKSPACE; a row index outside the cache is skipped and reported through
+ * mla_check_status (MLA_ERR_SHAPE).
+ */
+MLA_API int32_t mla_project_inputs(const mla_dims* dims, int32_t dtype, int32_t q_rank, const void* x,
+                                   const void* w_cq, const void* w_qc, const void* w_qr, const void* w_dkv,
+                                   int64_t n_rows, const int32_t* positions, void* q_nope, void* q_pe, void* cache,
+                                   int64_t cache_rows, const int64_t* row_idx, uint32_t flags, float eps,
+                                   float rope_theta, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of scratch mla_decode_step needs (the same for both io modes). */
+MLA_API int32_t mla_decode_step_workspace_size(const mla_dims* dims, int32_t dtype, int32_t q_rank,
+                                               int32_t batch, int64_t max_seqlen, int64_t total_rows,
+                                               size_t* bytes);
+
+/*
+ * mla_decode_step -- one whole decode step for `batch` sequences with one new token each:
+ * mla_project_inputs (append included) -> MLA_ABSORB_QUERY -> mla_decode_absorbed (n_q = 1) ->
+ * mla_out_project without a gate ([fm] Part 3, inference form, end to end: y_t from x_t).
+ *   x [batch, d_model] -> y [batch, d_model], both in `dtype`;
+ *   cache [total_rows, d_c + d_r] (sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1], which
+ *   already count the new token; row_idx[b] is where its latent goes, normally the last of those);
+ *   cu_seqlens int32 [batch + 1], row_idx int64 [batch], positions int32 [batch] (read with
+ *   MLA_APPEND_ROPE), append_flags / eps / rope_theta as mla_append_latent.
+ *   io = MLA_IO_DEVICE: every pointer is device memory.
+ *   io = MLA_IO_HOST: x, y, cu_seqlens, row_idx and positions are HOST memory; the call copies the
+ *   inputs into the workspace and y back with cudaMemcpyAsync on `stream`. With page-locked host
+ *   memory it returns once all is enqueued: the host buffers must then stay untouched until the
+ *   stream has passed this step (y holds the result after a synchronisation). The weights and the
+ *   cache are device memory in both modes.
+ * Errors: those of the four stages, checked before the first launch where they concern sizes;
+ * MLA_ERR_MODE for an unknown io; MLA_ERR_CUDA when a copy cannot be enqueued.
+ */
+MLA_API int32_t mla_decode_step(const mla_dims* dims, int32_t dtype, int32_t q_rank, const mla_step_weights* w,
+                                const void* x, void* cache, const int32_t* cu_seqlens, int32_t batch,
+                                int64_t max_seqlen, int64_t total_rows, const int64_t* row_idx,
+                                const int32_t* positions, uint32_t append_flags, float eps, float rope_theta,
+                                void* y, int32_t io, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * mla_check_status -- synchronise `stream`, then report and clear the library's device status
