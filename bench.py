@@ -1,11 +1,13 @@
 """Benchmark of one absorbed-MLA decode step on the DeepSeek-V2-scale workload.
 
-A step is the whole hot path over one batch: append the new token's latent (RMSNorm + RoPE), absorb
-the queries into the latent (W_UK), attend over the latent cache (fused split-KV decode), project
-(W_UV, W_O). Workload: batch 64, 128 heads, d_c 512, d_r 64, qk_nope 128, v_head 128, d_model
-5120, 4096 cached positions per sequence, bf16 storage, fp32 accumulation. Inputs are seeded and
-synthetic; the per-step traffic (302 MB of cache + 201 MB of weights) is larger than the 126 MB L2,
-so no separate flush is needed between steps.
+A step is the whole hot path over one batch, from the new tokens' hidden states x to the layer
+output y: the input projections (query latent c' = x W'_c, the per-head query halves, the latent and
+rotary key x [W_c, W_kr]) with the append of the new latent (RMSNorm + RoPE), the absorption of the
+queries into the latent (W_UK), attention over the latent cache (fused split-KV decode), and the
+value and output projections (W_UV, W_O). Workload: batch 64, 128 heads, d_c 512, d_r 64, qk_nope
+128, v_head 128, d_model 5120, q_rank 1536, 4096 cached positions per sequence, bf16 storage, fp32
+accumulation. Inputs are seeded and synthetic; the per-step traffic (302 MB of cache + 298 MB of
+weights) is larger than the 126 MB L2, so no separate flush is needed between steps.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
 
@@ -35,12 +37,13 @@ WORKLOAD = dict(batch=64, n_heads=128, kv_lora_rank=512, rope_dim=64, qk_nope=12
                 d_model=5120, seqlen=4096, q_lora_rank=1536)
 SEED = 1003
 CONFIG = {
-    "workload": "DeepSeek-V2-scale absorbed MLA decode step: append + absorb + split-KV decode + "
+    "workload": "DeepSeek-V2-scale absorbed MLA decode step from hidden states: input projections "
+                "(query latent q_rank 1536, KV down-projection) + append + absorb + split-KV decode + "
                 "W_UV/W_O projection; B64 H128 d_c512 d_r64 qk_nope128 v_head128 d_model5120 "
                 "T4096 per sequence, bf16 storage, fp32 accumulate",
     "batch": 64, "n_heads": 128, "kv_lora_rank": 512, "rope_dim": 64, "qk_nope": 128,
-    "v_head": 128, "d_model": 5120, "seq_len": 4096, "n_q": 1,
-    "l2": "no flush: every step streams 302 MB of latent cache + 201 MB of weights (> 126 MB L2)",
+    "v_head": 128, "d_model": 5120, "q_lora_rank": 1536, "seq_len": 4096, "n_q": 1,
+    "l2": "no flush: every step streams 302 MB of latent cache + 298 MB of weights (> 126 MB L2)",
     "parallelism": "replicas (one independent decode per GPU, no collective)",
 }
 DECODE_SOURCES = ("head_latent_attention_08_b200/csrc/tc_decode.cu",
@@ -235,8 +238,20 @@ def oracle_problem(n_seqs: int, seed: int = SEED):
                          rope_dim=w["rope_dim"], qk_nope=w["qk_nope"], v_head=w["v_head"],
                          d_model=w["d_model"], seqlens=[w["seqlen"]] * n_seqs, dtype="bf16",
                          seed=seed)
-    for name in ("q_nope", "q_pe", "w_uk", "w_uv", "w_o", "cache", "c_new", "kpe_new"):
+    for name in ("w_uk", "w_uv", "w_o", "cache"):
         setattr(p, name, np.ascontiguousarray(getattr(p, name), dtype=np.float64))
+    pw = I.projection_weights(n_tokens=n_seqs, d_model=w["d_model"], q_rank=w["q_lora_rank"],
+                              n_heads=w["n_heads"], qk_nope=w["qk_nope"], rope_dim=w["rope_dim"],
+                              kv_lora_rank=w["kv_lora_rank"], dtype="bf16", seed=seed + 100)
+    H, n, dr, dc, q_rank = w["n_heads"], w["qk_nope"], w["rope_dim"], w["kv_lora_rank"], w["q_lora_rank"]
+
+    def f64(a):
+        return np.ascontiguousarray(a, dtype=np.float64)
+
+    # the page's row-vector layout of the Linear-convention weights (reshape / transpose only)
+    p.proj = dict(x=f64(pw.x), w_cq=f64(pw.w_cq.T), w_qc=f64(pw.w_qc.reshape(H, n, q_rank).transpose(0, 2, 1)),
+                  w_qr=f64(pw.w_qr.reshape(H, dr, q_rank).transpose(0, 2, 1)), w_c=f64(pw.w_dkv[:dc].T),
+                  w_kr=f64(pw.w_dkv[dc:].T))
     return p
 
 
@@ -269,17 +284,19 @@ def oracle_sample(p) -> float:
     """The full step of the sequences of ``p`` through the oracle; returns seconds."""
     from oracle import mla_oracle as O
     t0 = time.perf_counter()
-    cache = O.append_latent(p.cache, p.row_idx, p.c_new, p.kpe_new, p.positions, norm=True, rope=True,
-                            dtype="bf16")
-    q_abs = O.absorb_query(p.q_nope, p.q_pe, p.w_uk)
+    w = p.proj
+    q_nope, q_pe, c, k_r = O.project_inputs(w["x"], w["w_cq"], w["w_qc"], w["w_qr"], w["w_c"], w["w_kr"],
+                                            p.positions)
+    cache = O.append_latent(p.cache, p.row_idx, c, k_r, p.positions, norm=True, rope=True, dtype="bf16")
+    q_abs = O.absorb_query(q_nope, q_pe, p.w_uk)
     out_lat, _ = O.decode_absorbed(q_abs, cache, p.cu_seqlens, 1, p.kv_lora_rank, p.kq_scale, True)
     O.out_project(out_lat, p.w_uv, p.w_o)
     return time.perf_counter() - t0
 
 
-CPU_SAMPLE = ("full step (append, absorb, decode, W_UV/W_O) of one sequence of the workload per "
-              "oracle call, float64 numpy oracle, inputs widened to float64 before timing, one "
-              "thread pinned to one core")
+CPU_SAMPLE = ("full step (input projections, append, absorb, decode, W_UV/W_O) of one sequence of "
+              "the workload per oracle call, float64 numpy oracle, inputs widened to float64 before "
+              "timing, one thread pinned to one core")
 
 
 def cpu_baseline(target_s: float = 12.0):
@@ -349,9 +366,11 @@ def run_ours(args):
 
     w = WORKLOAD
     B, H, dc, dr, T = w["batch"], w["n_heads"], w["kv_lora_rank"], w["rope_dim"], w["seqlen"]
-    p = I.decode_problem(batch=B, n_heads=H, kv_lora_rank=dc, rope_dim=dr, qk_nope=w["qk_nope"],
-                         v_head=w["v_head"], d_model=w["d_model"], seqlens=[T] * B, dtype="bf16",
-                         seed=replica_seed(rank))
+    n, dv, D, QR = w["qk_nope"], w["v_head"], w["d_model"], w["q_lora_rank"]
+    p = I.decode_problem(batch=B, n_heads=H, kv_lora_rank=dc, rope_dim=dr, qk_nope=n, v_head=dv, d_model=D,
+                         seqlens=[T] * B, dtype="bf16", seed=replica_seed(rank))
+    pw = I.projection_weights(n_tokens=B, d_model=D, q_rank=QR, n_heads=H, qk_nope=n, rope_dim=dr,
+                              kv_lora_rank=dc, dtype="bf16", seed=replica_seed(rank) + 100)
     bf = torch.bfloat16
     dev = torch.device("cuda", local)
 
@@ -360,18 +379,41 @@ def run_ours(args):
 
     cache = d_(p.cache)
     cu = torch.from_numpy(p.cu_seqlens.astype(np.int32)).to(dev)
-    d = M.dims(H, dc, dr, w["qk_nope"], w["v_head"], w["d_model"])
-    step = M.DecodeStep(d, bf, B, 1, T, cache, cu, d_(p.w_uk), d_(p.w_uv), d_(p.w_o))
-    q_nope, q_pe = d_(p.q_nope), d_(p.q_pe)
-    c_new, kpe_new = d_(p.c_new, torch.float32), d_(p.kpe_new, torch.float32)
+    d = M.dims(H, dc, dr, n, dv, D)
+    wts = dict(w_cq=d_(pw.w_cq), w_qc=d_(pw.w_qc), w_qr=d_(pw.w_qr), w_dkv=d_(pw.w_dkv), w_uk=d_(p.w_uk),
+               w_uv=d_(p.w_uv), w_o=d_(p.w_o))
+    layer = M.DecodeLayerStep(d, QR, B, T, cache, cu, **wts)
+    x = d_(pw.x)
     row_idx = torch.from_numpy(p.row_idx).to(dev)
     positions = torch.from_numpy(p.positions).to(dev)
-    del p
+    flags = M.MLA_APPEND_NORM | M.MLA_APPEND_ROPE
+    # the step call by call (the same calls mla_decode_step makes), so that the decode can be timed alone
+    q_nope = torch.empty(B, H, n, dtype=bf, device=dev)
+    q_pe = torch.empty(B, H, dr, dtype=bf, device=dev)
+    q_abs = torch.empty(B, H, dc + dr, dtype=bf, device=dev)
+    out_lat = torch.empty(B, H, dc, dtype=torch.float32, device=dev)
+    y = torch.empty(B, D, dtype=bf, device=dev)
+    ws_proj = M.workspace(M.mla_project_workspace_size(d, bf, QR, B), dev)
+    ws_dec = M.workspace(M.mla_decode_workspace_size(d, bf, B, 1, T, cache.shape[0], M.MLA_DECODE_CAUSAL), dev)
+    ws_out = M.workspace(M.mla_out_project_workspace_size(d, bf, B), dev)
+    h_x = torch.from_numpy(pw.x).to(bf).pin_memory()
+    del p, pw
     stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        M.mla_project_inputs(d, QR, x, wts["w_cq"], wts["w_qc"], wts["w_qr"], wts["w_dkv"], positions, q_nope,
+                             q_pe, cache, row_idx, flags, ws_proj)
+        M.mla_absorb_weights(d, M.MLA_ABSORB_QUERY, q_nope, q_pe, wts["w_uk"], B, q_abs)
+        if ev:
+            ev[0].record(stream)
+        M.mla_decode_absorbed(d, q_abs, cache, cu, B, 1, T, M.MLA_DECODE_CAUSAL, out_lat, None, ws_dec)
+        if ev:
+            ev[1].record(stream)
+        M.mla_out_project(d, out_lat, wts["w_uv"], wts["w_o"], None, B, y, ws_out)
 
     # ---- device-resident timing -------------------------------------------------------------
     for _ in range(args.warmup):
-        step(q_nope, q_pe, c_new, kpe_new, row_idx, positions)
+        step()
     torch.cuda.synchronize()
     if M.mla_check_status() != 0:
         raise SystemExit("device status word reports a timeout")
@@ -386,19 +428,13 @@ def run_ours(args):
         clk.wait_first()
         # keep the GPU busy until the sampler has seen it under load, then time
         for _ in range(args.warmup):
-            step(q_nope, q_pe, c_new, kpe_new, row_idx, positions)
+            step()
         torch.cuda.synchronize()
         t_wall0 = time.time()
         launches0 = M.mla_launch_count()
         start.record(stream)
         for k in range(args.steps):
-            M.mla_append_latent(d, cache, row_idx, c_new, kpe_new, positions, step.append_flags)
-            M.mla_absorb_weights(d, M.MLA_ABSORB_QUERY, q_nope, q_pe, step.w_uk, nq, step.q_abs)
-            ev_dec[k][0].record(stream)
-            M.mla_decode_absorbed(d, step.q_abs, cache, cu, B, 1, T, step.flags, step.out_lat, step.lse,
-                                  step.ws_dec)
-            ev_dec[k][1].record(stream)
-            M.mla_out_project(d, step.out_lat, step.w_uv, step.w_o, None, nq, step.y, step.ws_out)
+            step(ev_dec[k])
         stop.record(stream)
         torch.cuda.synchronize()
         clk.mark(t_wall0, time.time())
@@ -408,7 +444,7 @@ def run_ours(args):
         t_x0 = time.time()
         while time.time() - t_x0 < 0.3:
             for _ in range(20):
-                step(q_nope, q_pe, c_new, kpe_new, row_idx, positions)
+                step()
             torch.cuda.synchronize()
         clk.mark_extra(t_x0, time.time())
     if world > 1:
@@ -417,25 +453,19 @@ def run_ours(args):
     dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
     status = M.mla_check_status()
 
-    # ---- end to end through the public API with host buffers --------------------------------
-    h_q_nope = q_nope.cpu().pin_memory()
-    h_q_pe = q_pe.cpu().pin_memory()
-    h_c_new = c_new.cpu().pin_memory()
-    h_kpe = kpe_new.cpu().pin_memory()
-    h_y = torch.empty(step.y.shape, dtype=bf).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (h_q_nope, h_q_pe, h_c_new, h_kpe))
+    # ---- end to end through the C ABI's step call with host buffers -------------------------
+    # every step copies x, cu_seqlens, row_idx and positions host -> device and y device -> host
+    # (mla_decode_step with MLA_IO_HOST, page-locked host memory), all inside the timed region
+    h_y = torch.empty(B, D, dtype=bf).pin_memory()
+    h_rows, h_pos, h_cu = row_idx.cpu().pin_memory(), positions.cpu().pin_memory(), cu.cpu().pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_x, h_rows, h_pos, h_cu))
     d2h = h_y.numel() * h_y.element_size()
 
-    # every step's inputs go host -> device and its output device -> host inside the timed region;
-    # HostStream overlaps those transfers with the neighbouring steps' compute (a serving loop)
-    hs = M.HostStream(step, stream)
-
     def e2e_step():
-        hs.submit(h_q_nope, h_q_pe, h_c_new, h_kpe, row_idx, positions, h_y)
+        layer(h_x, h_rows, h_pos, y=h_y, io=M.MLA_IO_HOST, cu_seqlens=h_cu)
 
     for _ in range(args.warmup):
         e2e_step()
-    hs.wait(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -443,10 +473,13 @@ def run_ours(args):
     e0.record(stream)
     for _ in range(args.steps):
         e2e_step()
-    hs.wait(stream)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
+    # the two routes run the same kernels on the same inputs: their outputs agree bit for bit
+    step()
+    torch.cuda.synchronize()
+    same_output = bool(torch.equal(h_y, y.cpu()))
 
     cpu = cpu_baseline() if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
     if world > 1:
@@ -475,7 +508,9 @@ def run_ours(args):
             },
             "cpu_baseline": cpu,
             "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps,
+                    "route": "C ABI mla_decode_step with MLA_IO_HOST (page-locked host x, y, index arrays)",
+                    "same_output_as_device_route": same_output},
             "gpu_launches": int(launches),
             "clocks": clk.summary(),
             "device_status": status,
@@ -568,7 +603,25 @@ def run_rows(args):
     report("a1..a5 whole decode step", c3, ms,
            B * T * (dc + dr) * 2 + 2 * (H * n * dc + H * dv * dc + D * H * dv),
            B * H * T * (2 * (dc + dr) + 2 * dc) + 2 * B * H * (n * dc + dv * dc) + 2 * B * D * H * dv)
-    del cache, step, w_o
+    # ---- f2: the input projections fused with the append, and the whole step from x -----------------
+    QR = 1536
+    w_cq, w_qc = rnd(QR, D, scale=D ** -0.5), rnd(H * n, QR, scale=QR ** -0.5)
+    w_qr, w_dkv = rnd(H * dr, QR, scale=QR ** -0.5), rnd(dc + dr, D, scale=D ** -0.5)
+    x = rnd(B, D)
+    qn2, qp2 = torch.empty(B, H, n, dtype=bf, device=dev), torch.empty(B, H, dr, dtype=bf, device=dev)
+    ws_p = M.workspace(M.mla_project_workspace_size(d, bf, QR, B), dev)
+    proj_w = QR * D + H * n * QR + H * dr * QR + (dc + dr) * D
+    ms = timed(lambda: M.mla_project_inputs(d, QR, x, w_cq, w_qc, w_qr, w_dkv, positions, qn2, qp2, cache, row_idx,
+                                            step.append_flags, ws_p))
+    report("f2 input projections + append", c3 + " q_rank1536 d_model5120", ms,
+           2 * (proj_w + B * D + B * H * (n + dr) + B * (dc + dr)), 2 * B * proj_w,
+           "weight-read bound: 97 MB of projection weights for 64 tokens")
+    layer = M.DecodeLayerStep(d, QR, B, T, cache, cu, w_cq, w_qc, w_qr, w_dkv, w_uk, w_uv, w_o)
+    ms = timed(lambda: layer(x, row_idx, positions))
+    report("f2 + a1..a5 whole step from x (mla_decode_step)", c3 + " q_rank1536 d_model5120", ms,
+           B * T * (dc + dr) * 2 + 2 * (proj_w + H * n * dc + H * dv * dc + D * H * dv),
+           B * H * T * (2 * (dc + dr) + 2 * dc) + 2 * B * (proj_w + H * (n * dc + dv * dc) + D * H * dv))
+    del cache, step, w_o, layer, w_qc, w_qr
     torch.cuda.empty_cache()
     # ---- C4: B16, T ~ U[1024, 32768], n_q 1 and 4 (causal) -----------------------------------------
     Bs = 16

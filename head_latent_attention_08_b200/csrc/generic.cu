@@ -301,16 +301,19 @@ int append_latent_strided(const mla_dims& d, int32_t cache_dtype, void* cache, i
 
 // ---------------------------------------------------------------------------------------------
 // rotary part of the queries: out[t, h, :] = R_{pos_t} src[t, h, :] (or a plain copy), fp32 in, the
-// storage dtype out. One CTA per token: the d_r/2 angles once into shared memory, then every head.
+// storage dtype out. Grid (token, chunk of 1024 pairs): the d_r/2 angles of the token once into shared
+// memory, then 4 pairs per thread (two 16-byte loads, one 16-byte bf16 store when the row allows).
 // ---------------------------------------------------------------------------------------------
+constexpr int ROPE_PAIRS_PER_CTA = 1024;
+
 template <typename T>
-__global__ void __launch_bounds__(128) rope_rows_kernel(const float* __restrict__ src, T* __restrict__ out,
+__global__ void __launch_bounds__(256) rope_rows_kernel(const float* __restrict__ src, T* __restrict__ out,
                                                         const int32_t* __restrict__ positions, int H, int dr,
-                                                        int rotate, double log2_theta) {
+                                                        int rotate, int vec, double log2_theta) {
   extern __shared__ float2 sc[];   // (sin, cos) of pair i
   griddep_wait();
   griddep_launch_dependents();
-  const int t = blockIdx.x, half = dr / 2;
+  const int t = blockIdx.x, half = dr / 2, pairs = H * half;
   if (rotate) {
     const int32_t pos = positions[t];
     for (int i = threadIdx.x; i < half; i += blockDim.x) {
@@ -322,16 +325,34 @@ __global__ void __launch_bounds__(128) rope_rows_kernel(const float* __restrict_
   }
   const float2* row = reinterpret_cast<const float2*>(src + (int64_t)t * H * dr);
   T* o = out + (int64_t)t * H * dr;
-  for (int e = threadIdx.x; e < H * half; e += blockDim.x) {
-    const float2 v = row[e];
-    float r0 = v.x, r1 = v.y;
-    if (rotate) {
-      const float2 a = sc[e % half];
-      r0 = fmaf(v.x, a.y, -v.y * a.x);
-      r1 = fmaf(v.x, a.x, v.y * a.y);
+  const int e0 = blockIdx.y * ROPE_PAIRS_PER_CTA + threadIdx.x * 4;
+  auto turn = [&](float2 v, int e) {
+    if (!rotate) return v;
+    const float2 a = sc[e % half];
+    return make_float2(fmaf(v.x, a.y, -v.y * a.x), fmaf(v.x, a.x, v.y * a.y));
+  };
+  if (vec && e0 + 3 < pairs) {
+    const float4 u0 = reinterpret_cast<const float4*>(row + e0)[0];
+    const float4 u1 = reinterpret_cast<const float4*>(row + e0)[1];
+    const float2 r0 = turn(make_float2(u0.x, u0.y), e0), r1 = turn(make_float2(u0.z, u0.w), e0 + 1);
+    const float2 r2 = turn(make_float2(u1.x, u1.y), e0 + 2), r3 = turn(make_float2(u1.z, u1.w), e0 + 3);
+    if constexpr (sizeof(T) == 2) {
+      __nv_bfloat162 b0 = __floats2bfloat162_rn(r0.x, r0.y), b1 = __floats2bfloat162_rn(r1.x, r1.y);
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(r2.x, r2.y), b3 = __floats2bfloat162_rn(r3.x, r3.y);
+      uint4 w;
+      w.x = *reinterpret_cast<uint32_t*>(&b0); w.y = *reinterpret_cast<uint32_t*>(&b1);
+      w.z = *reinterpret_cast<uint32_t*>(&b2); w.w = *reinterpret_cast<uint32_t*>(&b3);
+      *reinterpret_cast<uint4*>(o + 2 * e0) = w;
+    } else {
+      reinterpret_cast<float4*>(o + 2 * e0)[0] = make_float4(r0.x, r0.y, r1.x, r1.y);
+      reinterpret_cast<float4*>(o + 2 * e0)[1] = make_float4(r2.x, r2.y, r3.x, r3.y);
     }
-    o[2 * e] = from_f32<T>(r0);
-    o[2 * e + 1] = from_f32<T>(r1);
+    return;
+  }
+  for (int e = e0; e < min(e0 + 4, pairs); ++e) {
+    const float2 r = turn(row[e], e);
+    o[2 * e] = from_f32<T>(r.x);
+    o[2 * e + 1] = from_f32<T>(r.y);
   }
 }
 
@@ -341,12 +362,18 @@ int rope_rows_launch(int32_t dtype, const float* src, void* out, const int32_t* 
   if (n_rows > 0x7fffffff || dr % 2) return MLA_ERR_SHAPE;
   const size_t smem = (size_t)(dr / 2) * sizeof(float2);
   if (smem > 48 * 1024) return MLA_ERR_UNSUPPORTED;
+  const int64_t pairs = (int64_t)H * (dr / 2);
+  const dim3 grid((unsigned)n_rows, (unsigned)ceil_div(pairs, ROPE_PAIRS_PER_CTA));
+  if (grid.y > 65535u) return MLA_ERR_UNSUPPORTED;
+  // 16-byte accesses: every row starts on 16 bytes in both buffers (src fp32 rows of H*dr floats; out
+  // rows of H*dr elements) and each thread's 4 pairs do too
+  const int vec = ((int64_t)H * dr) % 8 == 0 && aligned16(src) && aligned16(out);
   const double l2t = log2((double)theta);
   if (dtype == MLA_BF16)
-    return launch_pdl(rope_rows_kernel<__nv_bfloat16>, dim3((unsigned)n_rows), dim3(128), smem, s, src,
-                      static_cast<__nv_bfloat16*>(out), positions, H, dr, rotate ? 1 : 0, l2t);
-  return launch_pdl(rope_rows_kernel<float>, dim3((unsigned)n_rows), dim3(128), smem, s, src,
-                    static_cast<float*>(out), positions, H, dr, rotate ? 1 : 0, l2t);
+    return launch_pdl(rope_rows_kernel<__nv_bfloat16>, grid, dim3(256), smem, s, src,
+                      static_cast<__nv_bfloat16*>(out), positions, H, dr, rotate ? 1 : 0, vec, l2t);
+  return launch_pdl(rope_rows_kernel<float>, grid, dim3(256), smem, s, src, static_cast<float*>(out), positions,
+                    H, dr, rotate ? 1 : 0, vec, l2t);
 }
 
 // ---------------------------------------------------------------------------------------------

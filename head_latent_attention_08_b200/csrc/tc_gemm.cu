@@ -81,6 +81,8 @@ struct TcGemmParams {
   unsigned long long wait_ns;
 };
 
+constexpr int GEMM_PRODUCERS = 3;   // warps issuing the TMA loads (0, 2 and 3; warp 1 issues the MMAs)
+
 template <int BN>
 struct GemmCfg {
   static constexpr int A_BYTES = 128 * 64 * 2;
@@ -91,12 +93,6 @@ struct GemmCfg {
   static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
   static constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;
 };
-
-__device__ __forceinline__ float apply_epilogue(float v, int sigmoid, const __nv_bfloat16* gate, int64_t gidx) {
-  if (sigmoid) v = 1.f / (1.f + expf(-v));
-  if (gate) v *= __bfloat162float(gate[gidx]);
-  return v;
-}
 
 template <int BN, bool A_MN>
 __global__ void __launch_bounds__(128, 1)
@@ -111,6 +107,7 @@ __global__ void __launch_bounds__(128, 1)
   uint64_t* done = empty + STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_load = abort_flag + 1;   // [STAGES]: the last K chunk loaded into each stage
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * 128;
@@ -127,6 +124,7 @@ __global__ void __launch_bounds__(128, 1)
     }
     mbar_init(done, 1);
     *abort_flag = 0;
+    for (int s = 0; s < STAGES; ++s) last_load[s] = -1;
     fence_mbar_init();
     prefetch_tmap(&ta);
     prefetch_tmap(&tb);
@@ -138,23 +136,20 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  griddep_wait();                // the operands may come from the previous kernel of the stream
+  const bool producer = warp != 1 && lane == 0;
+  // the activations (B), the gate and the tail may come from the previous kernel of the stream, and the
+  // output may still be read by it: everyone waits for it, the producers after their weight prefetch
+  if (!producer) griddep_wait();
   griddep_launch_dependents();
   const uint32_t tmem_d = *tmem_slot;
-  int issued = 0;
 
-  if (warp == 0 && lane == 0) {
-    // TMA producer (stage s of round ph: the previous round's MMAs must have released it)
-    int s = 0, ph = 0;
-    for (int i = 0; i < nk; ++i) {
-      if (i >= STAGES && !mbar_wait(&empty[s], (uint32_t)(ph ^ 1), p.wait_ns, p.status)) {
-        *abort_flag = 1;
-        break;
-      }
-      if (*abort_flag) break;
+  if (producer) {
+    // TMA producers, lane 0 of warps 0, 2 and 3: producer j loads K chunks j, j + P, j + 2P, ... (an
+    // SM moves more bytes with bulk copies issued from several warps than from one thread). Chunk i
+    // goes to stage i % STAGES, whose previous round the MMAs must have released first.
+    const int j = warp == 0 ? 0 : warp - 1;
+    auto load_a = [&](int i, int s) {
       uint8_t* a_dst = smem + s * Cfg::STAGE;
-      uint8_t* b_dst = a_dst + Cfg::A_BYTES;
-      mbar_arrive_expect_tx(&full[s], Cfg::STAGE);
       const int kx = (kc0 + i) * 64;
       if (A_MN) {
         tma_load_3d(a_dst, &ta, &full[s], m0, kx, bz);
@@ -162,9 +157,29 @@ __global__ void __launch_bounds__(128, 1)
       } else {
         tma_load_3d(a_dst, &ta, &full[s], kx, m0, bz);
       }
-      tma_load_3d(b_dst, &tb, &full[s], kx, n0, bz);
-      ++issued;
-      if (++s == STAGES) { s = 0; ph ^= 1; }
+    };
+    // The weights (A) are never written by the library's kernels: the first ring's weight tiles are
+    // requested before the wait, so that their latency overlaps the previous kernel's tail.
+    const int pre = min(nk, STAGES);
+    for (int i = j; i < pre; i += GEMM_PRODUCERS) {
+      mbar_arrive_expect_tx(&full[i], Cfg::STAGE);
+      load_a(i, i);
+      last_load[i] = i;
+    }
+    griddep_wait();
+    for (int i = j; i < nk; i += GEMM_PRODUCERS) {
+      const int s = i % STAGES;
+      if (i >= STAGES) {      // (a prefetched stage always gets its B tile, so that its barrier completes)
+        if (!mbar_wait(&empty[s], (uint32_t)(((i / STAGES) - 1) & 1), p.wait_ns, p.status)) {
+          *abort_flag = 1;
+          break;
+        }
+        if (*abort_flag) break;
+        mbar_arrive_expect_tx(&full[s], Cfg::STAGE);
+        load_a(i, s);
+        last_load[s] = i;
+      }
+      tma_load_3d(smem + s * Cfg::STAGE + Cfg::A_BYTES, &tb, &full[s], (kc0 + i) * 64, n0, bz);
     }
   } else if (warp == 1 && lane == 0) {
     // MMA issuer
@@ -262,10 +277,13 @@ __global__ void __launch_bounds__(128, 1)
   if (warp == 0 && lane == 0 && *abort_flag) {
     // Abandoned work: neither TMA writes nor MMAs may be left in flight behind the CTA or its tensor
     // memory. Every load issued and the MMA issuer's final commit (made on both of its paths, before
-    // the barrier above) complete by themselves; the limit here only bounds the wait.
+    // the barrier above) complete by themselves; the limit here only bounds the wait. Only the last
+    // load of a stage can still be in flight (a later one waited for the MMAs to read the earlier).
     const uint64_t drain_ns = p.wait_ns > 100000000ull ? p.wait_ns : 100000000ull;
-    for (int i = max(0, issued - STAGES); i < issued; ++i)
-      (void)mbar_wait(&full[i % STAGES], (i / STAGES) & 1, drain_ns, p.status);
+    for (int s = 0; s < STAGES; ++s) {
+      const int i = last_load[s];
+      if (i >= 0) (void)mbar_wait(&full[s], (uint32_t)((i / STAGES) & 1), drain_ns, p.status);
+    }
     (void)mbar_wait(done, 0, drain_ns, p.status);
   }
   __syncthreads();
@@ -275,26 +293,46 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
-// fixed-order sum of split-K partials + epilogue
+// fixed-order sum of split-K partials + epilogue, 4 consecutive outputs per thread (M % 4 == 0; the
+// host checks the 16-byte alignment of out and the 8-byte alignment of the gate)
 __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int n_splits, int batch, int N, int M,
                                      void* out, int64_t out_sb, int64_t out_st, int out_f32,
                                      const __nv_bfloat16* gate, int64_t gate_sb, int64_t gate_st, int sigmoid) {
   griddep_wait();
   griddep_launch_dependents();
   const int64_t per = (int64_t)batch * N * M;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < per; e += (int64_t)gridDim.x * blockDim.x) {
-    float v = 0.f;
-    for (int s = 0; s < n_splits; ++s) v += partial[s * per + e];
+  for (int64_t e = 4 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); e < per;
+       e += 4 * (int64_t)gridDim.x * blockDim.x) {
+    float4 v = *reinterpret_cast<const float4*>(partial + e);
+#pragma unroll 4
+    for (int s = 1; s < n_splits; ++s) {
+      const float4 u = *reinterpret_cast<const float4*>(partial + s * per + e);
+      v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+    }
     const int m = (int)(e % M);
     const int64_t bt = e / M;
     const int t = (int)(bt % N);
     const int bz = (int)(bt / N);
-    v = apply_epilogue(v, sigmoid, gate, bz * gate_sb + (int64_t)t * gate_st + m);
+    if (sigmoid) {
+      v.x = 1.f / (1.f + expf(-v.x)); v.y = 1.f / (1.f + expf(-v.y));
+      v.z = 1.f / (1.f + expf(-v.z)); v.w = 1.f / (1.f + expf(-v.w));
+    }
+    if (gate) {
+      const uint2 gv = *reinterpret_cast<const uint2*>(gate + bz * gate_sb + (int64_t)t * gate_st + m);
+      const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv.x));
+      const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv.y));
+      v.x *= g0.x; v.y *= g0.y; v.z *= g1.x; v.w *= g1.y;
+    }
     const int64_t o = bz * out_sb + (int64_t)t * out_st + m;
-    if (out_f32)
-      static_cast<float*>(out)[o] = v;
-    else
-      static_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(v);
+    if (out_f32) {
+      *reinterpret_cast<float4*>(static_cast<float*>(out) + o) = v;
+    } else {
+      __nv_bfloat162 b0 = __floats2bfloat162_rn(v.x, v.y), b1 = __floats2bfloat162_rn(v.z, v.w);
+      uint2 w;
+      w.x = *reinterpret_cast<uint32_t*>(&b0);
+      w.y = *reinterpret_cast<uint32_t*>(&b1);
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + o) = w;
+    }
   }
 }
 
@@ -313,9 +351,6 @@ __global__ void f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __rest
   }
 }
 
-// ---------------------------------------------------------------------------------------------
-// host: one GEMM
-// ---------------------------------------------------------------------------------------------
 struct GemmOperand {
   // a 3-D bf16 tensor seen as [batch][rows][k] (K-major) or [batch][k][rows] (MN-major)
   void* base;
@@ -426,8 +461,8 @@ static int tc_gemm(const GemmOperand& A, bool a_mn, const GemmOperand& Bop, int 
   if (st) return st;
   if (g.splits > 1) {
     const int64_t per = (int64_t)batch * N * M;
-    const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(per, 256), 8 * sm_count());
-    st = launch_pdl(splitk_reduce_kernel, dim3(blocks), dim3(256), 0, s, (const float*)p.partial, g.splits, batch,
+    const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(per / 4, 128), 16 * sm_count());
+    st = launch_pdl(splitk_reduce_kernel, dim3(blocks), dim3(128), 0, s, (const float*)p.partial, g.splits, batch,
                     N, M, out, (int64_t)out_sb, (int64_t)out_st, p.out_f32, p.gate, (int64_t)gate_sb,
                     (int64_t)gate_st, p.sigmoid);
     if (st) return st;
