@@ -124,6 +124,10 @@ int append_latent_strided(const mla_dims& d, int32_t cache_dtype, void* cache, i
                           int64_t kpe_stride, const int32_t* positions, int64_t n_new, uint32_t flags,
                           float eps, float theta, cudaStream_t stream);
 
+// log-sum-exp merge of n_parts partial decode results (rows row0 .. row0 + n_rows of each part)
+int lse_merge_launch(int n_parts, const float* const* o_parts, const float* const* l_parts, int64_t row0,
+                     int64_t n_rows, int H, int dc, float* out_lat, float* lse, cudaStream_t stream);
+
 // out[t, h, :] = R_{positions[t]} src[t, h, :] (rotate) or src[t, h, :]: src fp32 [n_rows, H, dr],
 // out in dtype
 int rope_rows_launch(int32_t dtype, const float* src, void* out, const int32_t* positions, int64_t n_rows, int H,

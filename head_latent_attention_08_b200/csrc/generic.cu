@@ -377,6 +377,87 @@ int rope_rows_launch(int32_t dtype, const float* src, void* out, const int32_t* 
 }
 
 // ---------------------------------------------------------------------------------------------
+// merge of partial decode results by their log-sum-exp (split-KV across devices): part r holds the
+// attention output O_r and lse_r of one query row and head over a disjoint slice of the positions;
+//   m = max_r lse_r,  w_r = exp(lse_r - m),  O = sum_r w_r O_r / sum_r w_r,  lse = m + log sum_r w_r.
+// One warp per (row, head); sums run over r in index order, so the result does not depend on timing.
+// The parts may live in other devices' memory (peer pointers): the kernel only loads from them.
+// ---------------------------------------------------------------------------------------------
+struct MergeParts {
+  const float* o[MLA_MERGE_MAX_PARTS];
+  const float* l[MLA_MERGE_MAX_PARTS];
+};
+
+__global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ MergeParts parts, int n_parts,
+                                                        int64_t row0, int64_t n_rh, int H, int dc, int vec4,
+                                                        float* __restrict__ out_lat, float* __restrict__ lse) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int64_t x = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);   // local row * H + h
+  if (x >= n_rh) return;
+  const int64_t g = row0 * H + x;                                                    // global row * H + h
+  float lr = -INFINITY;
+  if (lane < n_parts) lr = parts.l[lane][g];
+  float m = lr;
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float* dst = out_lat + x * dc;
+  if (m == -INFINITY) {                      // no part saw a position: empty attention
+    for (int d = lane; d < dc; d += 32) dst[d] = 0.f;
+    if (lane == 0 && lse) lse[x] = -INFINITY;
+    return;
+  }
+  const float w_lane = lr == -INFINITY ? 0.f : expf(lr - m);
+  float w[MLA_MERGE_MAX_PARTS];
+  float wsum = 0.f;
+#pragma unroll
+  for (int r = 0; r < MLA_MERGE_MAX_PARTS; ++r) {
+    w[r] = __shfl_sync(0xffffffffu, w_lane, r);
+    if (r < n_parts) wsum += w[r];
+  }
+  const float inv = 1.f / wsum;
+  if (vec4) {
+    for (int d = 4 * lane; d < dc; d += 128) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int r = 0; r < MLA_MERGE_MAX_PARTS; ++r) {
+        if (r >= n_parts) break;
+        if (w[r] == 0.f) continue;               // (an empty part's output is not read)
+        const float4 v = *reinterpret_cast<const float4*>(parts.o[r] + g * dc + d);
+        acc.x = fmaf(w[r], v.x, acc.x); acc.y = fmaf(w[r], v.y, acc.y);
+        acc.z = fmaf(w[r], v.z, acc.z); acc.w = fmaf(w[r], v.w, acc.w);
+      }
+      *reinterpret_cast<float4*>(dst + d) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
+  } else {
+    for (int d = lane; d < dc; d += 32) {
+      float acc = 0.f;
+      for (int r = 0; r < n_parts; ++r)
+        if (w[r] != 0.f) acc = fmaf(w[r], parts.o[r][g * dc + d], acc);
+      dst[d] = acc * inv;
+    }
+  }
+  if (lane == 0 && lse) lse[x] = m + logf(wsum);
+}
+
+int lse_merge_launch(int n_parts, const float* const* o_parts, const float* const* l_parts, int64_t row0,
+                     int64_t n_rows, int H, int dc, float* out_lat, float* lse, cudaStream_t s) {
+  if (n_rows <= 0) return MLA_OK;
+  MergeParts mp{};
+  bool aligned = aligned16(out_lat) && dc % 4 == 0;
+  for (int r = 0; r < n_parts; ++r) {
+    mp.o[r] = o_parts[r];
+    mp.l[r] = l_parts[r];
+    aligned = aligned && aligned16(o_parts[r]);
+  }
+  const int64_t n_rh = n_rows * H;
+  const int64_t blocks = ceil_div(n_rh, 8);
+  if (blocks > 0x7fffffffLL) return MLA_ERR_SHAPE;
+  return launch_pdl(lse_merge_kernel, dim3((unsigned)blocks), dim3(256), 0, s, mp, n_parts, row0, n_rh, H, dc,
+                    aligned ? 1 : 0, out_lat, lse);
+}
+
+// ---------------------------------------------------------------------------------------------
 // split-KV absorbed decode on CUDA cores
 //   grid: x = split of the positions, y = group of HG heads, z = query row (b * n_q + j)
 //   per tile of DG_TP positions: stage the rows in shared memory (fp32), scores for every

@@ -492,6 +492,24 @@ int32_t mla_decode_step(const mla_dims* dims, int32_t dtype, int32_t q_rank, con
   return MLA_OK;
 }
 
+int32_t mla_lse_merge(const mla_dims* dims, int32_t n_parts, const float* const* out_lat_parts,
+                      const float* const* lse_parts, int64_t row_begin, int64_t n_rows, float* out_lat, float* lse,
+                      void* stream) {
+  int st = check_dims(dims);
+  if (st) return st;
+  if (n_parts < 1 || n_parts > MLA_MERGE_MAX_PARTS || row_begin < 0 || n_rows < 0) return MLA_ERR_SHAPE;
+  if (n_rows == 0) return MLA_OK;
+  if (!out_lat_parts || !lse_parts || !out_lat) return MLA_ERR_NULL;
+  for (int r = 0; r < n_parts; ++r) {
+    if (!out_lat_parts[r] || !lse_parts[r]) return MLA_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(out_lat_parts[r]) & 15u) return MLA_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(lse_parts[r]) & 3u) return MLA_ERR_ALIGN;
+  }
+  if ((reinterpret_cast<uintptr_t>(out_lat) & 15u) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return MLA_ERR_ALIGN;
+  return lse_merge_launch(n_parts, out_lat_parts, lse_parts, row_begin, n_rows, dims->n_heads, dims->kv_lora_rank,
+                          out_lat, lse, as_stream(stream));
+}
+
 int32_t mla_check_status(void* stream, int32_t* device_status) {
   if (!device_status) return MLA_ERR_NULL;
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return MLA_ERR_CUDA;

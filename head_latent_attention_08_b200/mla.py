@@ -32,6 +32,7 @@ EXPORTED = (
     "mla_out_project", "mla_linear", "mla_check_status", "mla_set_wait_limit", "mla_launch_count",
     "mla_set_decode_clusters", "mla_wait_selftest", "mla_decode_absorbed_noalloc",
     "mla_project_workspace_size", "mla_project_inputs", "mla_decode_step_workspace_size", "mla_decode_step",
+    "mla_lse_merge",
 )
 
 
@@ -85,6 +86,7 @@ _SIGS = {
     "mla_decode_step_workspace_size": (_I32, [_DIMS, _I32, _I32, _I32, _I64, _I64, ctypes.POINTER(_SZ)]),
     "mla_decode_step": (_I32, [_DIMS, _I32, _I32, ctypes.POINTER(mla_step_weights), _P, _P, _P, _I32, _I64,
                                _I64, _P, _P, _U32, _F, _F, _P, _I32, _P, _SZ, _P]),
+    "mla_lse_merge": (_I32, [_DIMS, _I32, ctypes.POINTER(_P), ctypes.POINTER(_P), _I64, _I64, _P, _P, _P]),
 }
 
 
@@ -268,6 +270,24 @@ def mla_decode_step(d: mla_dims, q_rank: int, w: mla_step_weights, x: torch.Tens
                                  _ptr(cache), p(cu_seqlens), batch, max_seqlen, cache.shape[0], p(row_idx),
                                  p(positions), flags, eps, rope_theta, p(y), io, _ptr(workspace), ws_bytes,
                                  _stream(stream)), "mla_decode_step")
+
+
+MLA_MERGE_MAX_PARTS = 16
+
+
+def mla_lse_merge(d: mla_dims, out_lat_parts, lse_parts, row_begin: int, n_rows: int, out_lat: torch.Tensor,
+                  lse: Optional[torch.Tensor], stream=None) -> None:
+    """Merge partial decode results by their log-sum-exp. The parts are device tensors or raw device
+    addresses (e.g. peers' symmetric-memory buffers)."""
+    def addr(x):
+        return x if isinstance(x, int) else _ptr(x)
+    n = len(out_lat_parts)
+    if len(lse_parts) != n:
+        raise ValueError("one lse part per out_lat part")
+    po = (_P * n)(*[addr(x) for x in out_lat_parts])
+    pl = (_P * n)(*[addr(x) for x in lse_parts])
+    _check(lib().mla_lse_merge(ctypes.byref(d), n, po, pl, row_begin, n_rows, _ptr(out_lat), _ptr(lse),
+                               _stream(stream)), "mla_lse_merge")
 
 
 def mla_check_status(stream=None) -> int:

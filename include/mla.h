@@ -266,6 +266,29 @@ MLA_API int32_t mla_decode_step(const mla_dims* dims, int32_t dtype, int32_t q_r
                                 void* y, int32_t io, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * mla_lse_merge -- merge partial decode results computed over disjoint slices of every sequence's
+ * positions (split-KV across devices: each device holds a contiguous slice of the latent cache and runs
+ * mla_decode_absorbed on it). For each query row and head, with m = max_r lse_r and
+ * w_r = exp(lse_r - m):  out_lat = sum_r w_r out_lat_r / sum_r w_r,  lse = m + log(sum_r w_r); the
+ * softmax over the union of the slices, restated by its log-sum-exp ([rs] fn body: max-subtracted
+ * exponentials, their sum and the weighted sum of latent rows). Parts whose lse is -inf (a slice
+ * with no visible position) take no part; if every part is -inf the row is 0 and its lse -inf.
+ *   n_parts         1 .. MLA_MERGE_MAX_PARTS;
+ *   out_lat_parts   HOST array of n_parts pointers, each to float [rows_total, H, d_c] (16-byte
+ *                   aligned); lse_parts likewise to float [rows_total, H]. They may point into other
+ *                   devices' memory that this device can load from (peer access or symmetric memory):
+ *                   the kernel only reads them, so the merge is also the exchange;
+ *   row_begin, n_rows  the query rows merged: rows row_begin .. row_begin + n_rows of every part;
+ *   out_lat float [n_rows, H, d_c] and lse float [n_rows, H] (lse may be NULL) receive them.
+ * Sums run over r in index order: the result does not depend on timing or on the device that runs it.
+ * Errors: MLA_ERR_NULL, MLA_ERR_SHAPE (n_parts out of range, n_rows or row_begin < 0), MLA_ERR_ALIGN.
+ */
+#define MLA_MERGE_MAX_PARTS 16
+MLA_API int32_t mla_lse_merge(const mla_dims* dims, int32_t n_parts, const float* const* out_lat_parts,
+                              const float* const* lse_parts, int64_t row_begin, int64_t n_rows, float* out_lat,
+                              float* lse, void* stream);
+
+/*
  * mla_check_status -- synchronise `stream`, then report and clear the library's device status
  * word: MLA_OK, or MLA_ERR_TIMEOUT when a bounded device wait gave up, or MLA_ERR_SHAPE when a kernel skipped an out-of-range row index, since the last check.
  */
