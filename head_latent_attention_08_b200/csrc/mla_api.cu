@@ -492,6 +492,23 @@ int32_t mla_decode_step(const mla_dims* dims, int32_t dtype, int32_t q_rank, con
   return MLA_OK;
 }
 
+int32_t mla_prefill_attention(int32_t dtype, const void* q, const void* k, const void* v, const void* gate,
+                              int32_t batch, int32_t seq, int32_t n_heads, int32_t head_dim, float scale,
+                              uint32_t flags, void* out, void* stream) {
+  if (!dtype_ok(dtype)) return MLA_ERR_DTYPE;
+  if (flags & ~(uint32_t)MLA_DECODE_CAUSAL) return MLA_ERR_MODE;
+  if (batch < 0 || seq < 0 || n_heads <= 0 || head_dim <= 0) return MLA_ERR_SHAPE;
+  if (!(scale >= 0.f) || isinf(scale)) return MLA_ERR_SHAPE;
+  if (batch == 0 || seq == 0) return MLA_OK;
+  if (!q || !k || !v || !out) return MLA_ERR_NULL;
+  if (dtype != MLA_BF16 || !tc_prefill_supported(batch, seq, n_heads, head_dim)) return MLA_ERR_UNSUPPORTED;
+  int st = check_align(dtype, {q, k, v, gate, out});
+  if (st) return st;
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)head_dim);
+  return tc_prefill_launch(q, k, v, gate, batch, seq, n_heads, sc, (flags & MLA_DECODE_CAUSAL) != 0, out,
+                           as_stream(stream));
+}
+
 int32_t mla_lse_merge(const mla_dims* dims, int32_t n_parts, const float* const* out_lat_parts,
                       const float* const* lse_parts, int64_t row_begin, int64_t n_rows, float* out_lat, float* lse,
                       void* stream) {

@@ -31,6 +31,11 @@ size_t tc_project_partial_bytes(const mla_dims& d, int64_t q_rank, int64_t n_row
 int tc_project(const mla_dims& d, int64_t q_rank, const void* x, const void* w_cq, const void* w_qc,
                const void* w_qr, const void* w_dkv, int64_t n_rows, void* c_q, void* q_nope, float* q_r,
                float* kv, void* partial, cudaStream_t s);
+// attention of un-absorbed heads over whole prompts (bf16, head width 128): q, k, v, out and the
+// optional gate are [B*S, H*128]; out = softmax(scale q k^T, causal or full) v (times the gate)
+bool tc_prefill_supported(int64_t B, int64_t S, int64_t H, int64_t D);
+int tc_prefill_launch(const void* q, const void* k, const void* v, const void* gate, int64_t B, int64_t S, int64_t H,
+                      float scale, bool causal, void* out, cudaStream_t s);
 // dense linear Y = X W^T
 bool tc_linear_supported(int64_t m, int64_t n, int64_t k);
 int tc_linear(const void* x, const void* w, int64_t m, int64_t n, int64_t k, int sigmoid, void* y,

@@ -32,7 +32,7 @@ EXPORTED = (
     "mla_out_project", "mla_linear", "mla_check_status", "mla_set_wait_limit", "mla_launch_count",
     "mla_set_decode_clusters", "mla_wait_selftest", "mla_decode_absorbed_noalloc",
     "mla_project_workspace_size", "mla_project_inputs", "mla_decode_step_workspace_size", "mla_decode_step",
-    "mla_lse_merge",
+    "mla_lse_merge", "mla_prefill_attention",
 )
 
 
@@ -87,6 +87,7 @@ _SIGS = {
     "mla_decode_step": (_I32, [_DIMS, _I32, _I32, ctypes.POINTER(mla_step_weights), _P, _P, _P, _I32, _I64,
                                _I64, _P, _P, _U32, _F, _F, _P, _I32, _P, _SZ, _P]),
     "mla_lse_merge": (_I32, [_DIMS, _I32, ctypes.POINTER(_P), ctypes.POINTER(_P), _I64, _I64, _P, _P, _P]),
+    "mla_prefill_attention": (_I32, [_I32, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _F, _U32, _P, _P]),
 }
 
 
@@ -290,6 +291,14 @@ def mla_lse_merge(d: mla_dims, out_lat_parts, lse_parts, row_begin: int, n_rows:
                                _stream(stream)), "mla_lse_merge")
 
 
+def mla_prefill_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[torch.Tensor],
+                          batch: int, seq: int, n_heads: int, head_dim: int, scale: float, flags: int,
+                          out: torch.Tensor, stream=None) -> None:
+    _check(lib().mla_prefill_attention(_dtype_code(q.dtype), _ptr(q), _ptr(k), _ptr(v), _ptr(gate), batch, seq,
+                                       n_heads, head_dim, scale, flags, _ptr(out), _stream(stream)),
+           "mla_prefill_attention")
+
+
 def mla_check_status(stream=None) -> int:
     v = ctypes.c_int32(0)
     _check(lib().mla_check_status(_stream(stream), ctypes.byref(v)), "mla_check_status")
@@ -455,10 +464,14 @@ class HostStream:
 
 
 def gated_mla(x: torch.Tensor, wq: torch.Tensor, wc: torch.Tensor, wk: torch.Tensor, wv: torch.Tensor,
-              wg: torch.Tensor, wo: torch.Tensor, num_heads: int, causal: bool = True, stream=None):
-    """Gated MLA prefill through the absorbed route: Q, C and sigmoid(X Wg^T) by mla_linear, the
-    query absorbed into the latent per head (W_UK[h] = rows h*D_h.. of Wk), attention over the latent
-    C, then W_UV[h] = rows of Wv, the gate and Wo by mla_out_project. Returns
+              wg: torch.Tensor, wo: torch.Tensor, num_heads: int, causal: bool = True, stream=None,
+              route: str = "auto"):
+    """Gated MLA prefill. Q, C and sigmoid(X Wg^T) come from mla_linear; then either
+    * route "unabsorbed": K = C Wk^T and V = C Wv^T by mla_linear, attention of the D_h-wide heads with
+      the gate by mla_prefill_attention, Y = O Wo^T by mla_linear; or
+    * route "absorbed": the query absorbed into the latent per head (W_UK[h] = rows h*D_h.. of Wk),
+      attention over the latent C, then W_UV[h] = rows of Wv, the gate and Wo by mla_out_project.
+    "auto" takes the un-absorbed route where its tensor-core kernel applies (bf16, D_h = 128). Returns
     {"output": [B, S, D], "latent_cache": [B, S, L]}; the inputs are not modified."""
     B, S, D = x.shape
     L = wc.shape[0]
@@ -467,6 +480,10 @@ def gated_mla(x: torch.Tensor, wq: torch.Tensor, wc: torch.Tensor, wk: torch.Ten
         raise ValueError("model width must be divisible by the head count")
     Dh = D // H
     dev, dt = x.device, x.dtype
+    if route == "auto":
+        route = "unabsorbed" if (dt == torch.bfloat16 and Dh == 128) else "absorbed"
+    if route not in ("absorbed", "unabsorbed"):
+        raise ValueError("route is 'auto', 'absorbed' or 'unabsorbed'")
     x2 = x.reshape(B * S, D)
     q = torch.empty(B * S, D, dtype=dt, device=dev)
     c = torch.empty(B * S, L, dtype=dt, device=dev)
@@ -474,6 +491,17 @@ def gated_mla(x: torch.Tensor, wq: torch.Tensor, wc: torch.Tensor, wk: torch.Ten
     mla_linear(x2, wq, B * S, D, D, 0, q, stream)
     mla_linear(x2, wc, B * S, L, D, 0, c, stream)
     mla_linear(x2, wg, B * S, D, D, MLA_LINEAR_SIGMOID, g, stream)
+    if route == "unabsorbed":
+        k = torch.empty(B * S, D, dtype=dt, device=dev)
+        v = torch.empty(B * S, D, dtype=dt, device=dev)
+        mla_linear(c, wk, B * S, D, L, 0, k, stream)
+        mla_linear(c, wv, B * S, D, L, 0, v, stream)
+        o = torch.empty(B * S, D, dtype=dt, device=dev)
+        mla_prefill_attention(q, k, v, g, B, S, H, Dh, 1.0 / math.sqrt(Dh), MLA_DECODE_CAUSAL if causal else 0, o,
+                              stream)
+        y = torch.empty(B * S, D, dtype=dt, device=dev)
+        mla_linear(o, wo, B * S, D, D, 0, y, stream)
+        return {"output": y.reshape(B, S, D), "latent_cache": c.reshape(B, S, L)}
     d = dims(H, L, 0, Dh, Dh, D, 1.0 / math.sqrt(Dh))
     q_abs = torch.empty(B * S, H, L, dtype=dt, device=dev)
     mla_absorb_weights(d, MLA_ABSORB_QUERY, q, None, wk, B * S, q_abs, stream)

@@ -266,6 +266,27 @@ MLA_API int32_t mla_decode_step(const mla_dims* dims, int32_t dtype, int32_t q_r
                                 void* y, int32_t io, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * mla_prefill_attention -- attention of UN-absorbed heads over whole prompts (prefill): per sequence b
+ * and head h, O = softmax(scale * Q K^T) V with the causal mask under MLA_DECODE_CAUSAL (query s
+ * sees keys t <= s), optionally times a gate ([gm] problem equations: Q = X Wq^T, K = C Wk^T,
+ * V = C Wv^T, heads of D_h, causal mask, Y = [sigmoid(X Wg^T) * O] Wo^T; [fm] Part 3, training-form
+ * equation). With every query of a prompt present, materialising K and V per head costs less than the
+ * absorbed route, whose heads are d_c wide ([fm] Part 3, the note after the inference form).
+ *   q, k, v, out  [batch * seq, n_heads * head_dim] row-major in `dtype` (sequence b owns rows
+ *                 b*seq .. b*seq + seq - 1; head h owns columns h*head_dim ..);
+ *   gate          same shape, multiplied into out (pass sigmoid(X Wg^T)), or NULL;
+ *   scale         0 => 1/sqrt(head_dim).
+ * Tensor cores: bf16 with head_dim 128; other requests return MLA_ERR_UNSUPPORTED (the absorbed route,
+ * mla_decode_absorbed with n_q = seq, computes the same attention for any width). P is rounded to bf16
+ * for the P V product; scores, the softmax and the output accumulate in fp32.
+ * Errors: MLA_ERR_NULL, MLA_ERR_SHAPE, MLA_ERR_DTYPE, MLA_ERR_MODE, MLA_ERR_ALIGN (16 B),
+ * MLA_ERR_UNSUPPORTED; a bounded device wait that gives up reports MLA_ERR_TIMEOUT (mla_check_status).
+ */
+MLA_API int32_t mla_prefill_attention(int32_t dtype, const void* q, const void* k, const void* v, const void* gate,
+                                      int32_t batch, int32_t seq, int32_t n_heads, int32_t head_dim, float scale,
+                                      uint32_t flags, void* out, void* stream);
+
+/*
  * mla_lse_merge -- merge partial decode results computed over disjoint slices of every sequence's
  * positions (split-KV across devices: each device holds a contiguous slice of the latent cache and runs
  * mla_decode_absorbed on it). For each query row and head, with m = max_r lse_r and

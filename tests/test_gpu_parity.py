@@ -238,12 +238,13 @@ def test_config4_ragged_long_context_sampled(n_q):
         assert_close(y[rows], ref_y, "bf16", f"y b={b}")
 
 
-def test_config5_gated_prefill_full_sampled():
+@pytest.mark.parametrize("route", ["unabsorbed", "absorbed"])
+def test_config5_gated_prefill_full_sampled(route):
     gp = I.gated_problem(batch=4, seq=2048, d_model=2048, num_heads=16, latent=512, causal=True,
                          dtype="bf16", seed=I.CONFIG_SEEDS[5])
     args = [dev(a, "bf16") for a in (gp.x, gp.wq, gp.wc, gp.wk, gp.wv, gp.wg, gp.wo)]
     x_before = args[0].clone()
-    r = M.gated_mla(*args, num_heads=16, causal=True)
+    r = M.gated_mla(*args, num_heads=16, causal=True, route=route)
     torch.cuda.synchronize()
     assert set(r) == {"output", "latent_cache"}
     assert r["output"].shape == (4, 2048, 2048) and r["output"].dtype == torch.bfloat16
