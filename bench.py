@@ -660,6 +660,23 @@ def run_rows(args):
     seen5 = B5 * H5 * S5 * (S5 + 1) // 2
     report("a3+a4 split-KV decode + combine", c5 + " (n_q = S, rows = (token, head))", ms,
            B5 * S5 * L5 * 2 + B5 * S5 * H5 * L5 * (2 + 4), seen5 * (2 * L5 + 2 * L5))
+    del q5, out5, ws5
+    # ---- f4: the same prompt through the un-absorbed route -----------------------------------------
+    Dh5 = D5 // H5
+    k5, v5, g5, o5 = (rnd(B5 * S5, D5) for _ in range(4))
+    ms = timed(lambda: M.mla_prefill_attention(yq, k5, v5, g5, B5, S5, H5, Dh5, 0.0, M.MLA_DECODE_CAUSAL, o5))
+    report("f4 un-absorbed prefill attention (causal, gated)", c5 + " (heads of 128)", ms,
+           4 * B5 * S5 * D5 * 2, seen5 * 4 * Dh5)
+    wc5, wk5, wv5, wg5, wo5 = (rnd(L5, D5, scale=D5 ** -0.5), rnd(D5, L5, scale=L5 ** -0.5),
+                               rnd(D5, L5, scale=L5 ** -0.5), rnd(D5, D5, scale=D5 ** -0.5),
+                               rnd(D5, D5, scale=D5 ** -0.5))
+    x5 = x.reshape(B5, S5, D5)
+    lin_flops = 2 * B5 * S5 * (3 * D5 * D5 + D5 * L5 + 2 * L5 * D5)
+    for route in ("unabsorbed", "absorbed"):
+        attn = seen5 * 4 * (Dh5 if route == "unabsorbed" else L5)
+        ms = timed(lambda: M.gated_mla(x5, wq, wc5, wk5, wv5, wg5, wo5, H5, True, route=route), reps=5)
+        report(f"whole gated MLA prefill, {route} route", c5, ms, 2 * (B5 * S5 * (2 * D5 + L5) + 3 * D5 * D5),
+               lin_flops + attn)
     clk.__exit__(None, None, None)
     print(json.dumps({"clocks": clk.summary(), "device_status": M.mla_check_status()}), flush=True)
     return 0

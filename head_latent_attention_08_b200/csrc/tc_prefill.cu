@@ -39,6 +39,12 @@ constexpr int PF_SMEM = 5 * PF_TILE + 1024 + 512;
 constexpr uint32_t PF_TMEM_COLS = 512;
 constexpr float PF_REF_SLACK = 8.f;        // log2 units a row maximum may exceed m_ref before it moves
 
+__device__ __forceinline__ float pf_ex2(float x) {   // 2^x on the special-function unit (flushes tiny results)
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 struct PfParams {
   int B, S, H, n_qt;
   float scale_log2;                        // softmax scale times log2(e)
@@ -220,13 +226,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->s_free[s]);
       const int kmax = k_end - j * PF_BN;
-      float mt = -INFINITY;
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
 #pragma unroll
       for (int c = 0; c < PF_BN; ++c) {
         const float v = c < kmax ? __uint_as_float(xr[c]) * p.scale_log2 : -INFINITY;
         xr[c] = __float_as_uint(v);
-        mt = fmaxf(mt, v);
+        mx[c & 3] = fmaxf(mx[c & 3], v);
       }
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       // P buffer s is free once P_{j-2} V_{j-2} is done
       if (j >= 2 && !warp_wait(&bars->p_free[s], (uint32_t)((j >> 1) - 1) & 1u)) { ok = false; break; }
       if (j == 0) {
@@ -239,7 +246,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           const int sp = (j - 1) & 1;
           if (!warp_wait(&bars->p_free[sp], (uint32_t)((j - 1) >> 1) & 1u)) { ok = false; break; }
           tc_fence_after();
-          const float f = move ? exp2f(m_ref - mt) : 1.f;
+          const float f = move ? pf_ex2(m_ref - mt) : 1.f;
 #pragma unroll 1
           for (int c = 0; c < PF_D / 32; ++c) {
             uint32_t r[32];
@@ -258,16 +265,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       }
       // probabilities, rounded to bf16 once; the row sum adds the rounded values the MMA will use
       uint32_t pk[PF_BN / 2];
-      float rs = 0.f;
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < PF_BN / 2; ++c) {
-        const __nv_bfloat162 b2 = __floats2bfloat162_rn(exp2f(__uint_as_float(xr[2 * c]) - m_ref),
-                                                        exp2f(__uint_as_float(xr[2 * c + 1]) - m_ref));
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(pf_ex2(__uint_as_float(xr[2 * c]) - m_ref),
+                                                        pf_ex2(__uint_as_float(xr[2 * c + 1]) - m_ref));
         const float2 back = __bfloat1622float2(b2);
-        rs += back.x + back.y;
+        rs[c & 3] += back.x + back.y;
         pk[c] = *reinterpret_cast<const uint32_t*>(&b2);
       }
-      l += rs;
+      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
       tc_fence_after();
       tmem_st32(tP + s * 64 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
       tmem_st32(tP + s * 64 + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
