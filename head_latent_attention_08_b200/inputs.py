@@ -44,12 +44,15 @@ CONFIG_SEEDS = {k: 1000 + k for k in range(1, 6)}
 
 
 def round_to(x: np.ndarray, dtype: str) -> np.ndarray:
-    """Round ``x`` to the storage dtype ('f32' or 'bf16') and return it as float32 values."""
+    """Round ``x`` to the storage dtype ('f32', 'bf16' or 'e4m3') and return it as float32 values.
+    'e4m3' saturates at +-448 (the format's largest finite value) before torch's cast."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     if dtype == "f32":
         return x
     if dtype == "bf16":
         return torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy()
+    if dtype == "e4m3":
+        return torch.from_numpy(np.clip(x, -448.0, 448.0)).to(torch.float8_e4m3fn).to(torch.float32).numpy()
     raise ValueError(f"unknown dtype {dtype!r}")
 
 
@@ -114,7 +117,7 @@ class DecodeProblem:
 
 def decode_problem(*, batch: int, n_heads: int, kv_lora_rank: int, rope_dim: int, qk_nope: int,
                    v_head: int, d_model: int, seqlens, n_q: int = 1, dtype: str = "f32",
-                   seed: int = 7, with_weights: bool = True) -> DecodeProblem:
+                   seed: int = 7, with_weights: bool = True, cache_dtype: str = "") -> DecodeProblem:
     seqlens = np.asarray(seqlens, dtype=np.int64).reshape(-1)
     if seqlens.shape[0] != batch:
         raise ValueError("seqlens must have one entry per sequence")
@@ -136,7 +139,7 @@ def decode_problem(*, batch: int, n_heads: int, kv_lora_rank: int, rope_dim: int
         w_uk = np.zeros((0,), np.float32)
         w_uv = np.zeros((0,), np.float32)
         w_o = np.zeros((0,), np.float32)
-    cache = round_to(_normal(rng, (total, dc + dr)), dtype)
+    cache = round_to(_normal(rng, (total, dc + dr)), cache_dtype or dtype)
     c_new = _normal(rng, (nq_tot, dc))
     kpe_new = _normal(rng, (nq_tot, dr))
     # the n_q newest tokens of sequence b sit at its last n_q rows, at positions T_b - n_q .. T_b - 1

@@ -46,6 +46,8 @@ Pins (what fixes each function independently of this file; see tests/test_oracle
   Part 3's training-form equation (per-head keys c_i W_kc^(s) and x_i W_kr R_i, rotations built
   as explicit block-diagonal matrices in torch), at sizes where d = d_c' = d_c so that feeding the
   wrong latent to a weight still runs.
+* store_e4m3: hand-worked e4m3 roundings (tests/golden/e4m3_rounding.json: ties to even at several
+  binades, subnormals, saturation), and a planted round-toward-zero must fail them.
 No function here is "parity unpinned".
 """
 from __future__ import annotations
@@ -60,6 +62,21 @@ F64 = np.float64
 
 def _f64(x) -> np.ndarray:
     return np.asarray(x, dtype=F64)
+
+
+def store_e4m3(x: np.ndarray, scale: float = 1.0) -> np.ndarray:
+    """Value an fp8 (e4m3) latent-cache element stands for, as float64: the e4m3 value nearest to
+    fp32(x) / scale (an fp32 division; ties to the even code), saturated at +-448, times scale.
+
+    The pages fix no fp8 format (the lab's "<5 GB at 128k" needs at most one byte per value); the
+    reading taken is E4M3 as published for 8-bit floating point (bias 7, 3 mantissa bits, no
+    infinities, largest finite value 448) with one scale per cache. The code is decided in fp32,
+    the precision the append kernel decides it in; torch's cast serves as the rounding step.
+    """
+    v = _f64(x).astype(np.float32) / np.float32(scale)
+    v = np.clip(v, -448.0, 448.0).astype(np.float32)
+    code = torch.from_numpy(np.ascontiguousarray(v)).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    return code * float(scale)
 
 
 def store_as(x: np.ndarray, dtype: str) -> np.ndarray:

@@ -677,3 +677,35 @@ def test_planted_query_rotated_one_position_late(monkeypatch):
             orig(x, w_cq, w_qc, w_qr, w_c, w_kr, positions, theta)[2:]
     _plant_projection(monkeypatch, bad)
     assert not _projection_pin_passes()
+
+
+# ------------------------------------------------------------------------------------------
+# fp8 (e4m3) cache values
+# ------------------------------------------------------------------------------------------
+
+def _e4m3_golden_passes(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "e4m3_rounding.json")))
+    for x, want, _ in g["cases"]:
+        if O.store_e4m3(np.array([x]))[0] != want:
+            return False
+    for x, scale, want, _ in g["scaled_cases"]:
+        if O.store_e4m3(np.array([x]), scale)[0] != want:
+            return False
+    return True
+
+
+def test_e4m3_rounding_golden(golden_dir):
+    assert _e4m3_golden_passes(golden_dir)
+
+
+def test_planted_e4m3_round_toward_zero(monkeypatch, golden_dir):
+    # every finite e4m3 magnitude, then the largest one not above |x| (truncation instead of nearest)
+    mags = sorted({m * 2.0 ** -9 for m in range(8)} |
+                  {(1 + m / 8) * 2.0 ** (e - 7) for e in range(1, 16) for m in range(8) if (e, m) != (15, 7)})
+
+    def bad(x, scale=1.0):
+        v = np.asarray(x, np.float64) / scale
+        out = np.array([math.copysign(max(m for m in mags if m <= min(abs(t), 448.0)), t) for t in v.ravel()])
+        return out.reshape(v.shape) * scale
+    monkeypatch.setattr(O, "store_e4m3", bad)
+    assert not _e4m3_golden_passes(golden_dir)
