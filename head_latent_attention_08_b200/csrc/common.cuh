@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 #include "../../include/mla.h"
@@ -14,11 +15,18 @@ namespace mla {
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f32(__nv_fp8_e4m3 x) { return static_cast<float>(x); }
 
 template <typename T> __device__ __forceinline__ T from_f32(float x);
 template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
+}
+// e4m3: round to nearest even, saturating to +-448 (the format has no infinity)
+template <> __device__ __forceinline__ __nv_fp8_e4m3 from_f32<__nv_fp8_e4m3>(float x) {
+  __nv_fp8_e4m3 r;
+  r.__x = __nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+  return r;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -39,7 +47,7 @@ __device__ __forceinline__ void report_timeout(int* status) {
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t round_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
-inline size_t dtype_bytes(int32_t dt) { return dt == MLA_BF16 ? 2 : 4; }
+inline size_t dtype_bytes(int32_t dt) { return dt == MLA_BF16 ? 2 : (dt == MLA_FP8_E4M3 ? 1 : 4); }
 
 int sm_count();          // multiprocessors of the current device (cached per device)
 int current_device();
@@ -122,7 +130,7 @@ int append_latent_launch(const mla_dims& d, int32_t cache_dtype, void* cache, in
 int append_latent_strided(const mla_dims& d, int32_t cache_dtype, void* cache, int64_t cache_rows,
                           const int64_t* row_idx, const float* c_new, int64_t c_stride, const float* kpe_new,
                           int64_t kpe_stride, const int32_t* positions, int64_t n_new, uint32_t flags,
-                          float eps, float theta, cudaStream_t stream);
+                          float eps, float theta, cudaStream_t stream, float cache_scale = 1.f);
 
 // log-sum-exp merge of n_parts partial decode results (rows row0 .. row0 + n_rows of each part)
 int lse_merge_launch(int n_parts, const float* const* o_parts, const float* const* l_parts, int64_t row0,
@@ -139,9 +147,12 @@ struct DecodeArgs {
   float scale; bool causal;
   float* out_lat; float* lse;
   void* workspace; size_t workspace_bytes;
+  float cache_scale = 1.f;               // an e4m3 cache holds value / cache_scale
 };
 
 size_t decode_generic_workspace(const DecodeArgs& a);
-int decode_generic_launch(const DecodeArgs& a, int32_t dtype, cudaStream_t stream);
+// dtype: of q_abs and the cache (MLA_F32 or MLA_BF16); cache_dtype MLA_FP8_E4M3 takes an e4m3 cache
+// with a bf16 or fp32 query
+int decode_generic_launch(const DecodeArgs& a, int32_t dtype, cudaStream_t stream, int32_t cache_dtype = -1);
 
 }  // namespace mla

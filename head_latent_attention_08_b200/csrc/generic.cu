@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(128) append_latent_kernel(
     T* __restrict__ cache, const int64_t* __restrict__ row_idx, const float* __restrict__ c_new,
     int64_t c_stride, const float* __restrict__ kpe_new, int64_t kpe_stride,
     const int32_t* __restrict__ positions, int dc, int dr,
-    uint32_t flags, float eps, double log2_theta, int vec8, int64_t cache_rows, int* status) {
+    uint32_t flags, float eps, double log2_theta, int vec8, int64_t cache_rows, int* status, float cache_scale) {
   extern __shared__ float row[];
   __shared__ float red[4];
   griddep_wait();
@@ -260,6 +260,10 @@ __global__ void __launch_bounds__(128) append_latent_kernel(
         *reinterpret_cast<float4*>(dst + i + 4) = make_float4(row[i + 4], row[i + 5], row[i + 6], row[i + 7]);
       }
     }
+  } else if constexpr (sizeof(T) == 1) {
+    // e4m3: the stored code is round-to-nearest-even of value / cache_scale (an IEEE fp32 division),
+    // saturated to +-448
+    for (int i = threadIdx.x; i < W; i += blockDim.x) dst[i] = from_f32<T>(row[i] / cache_scale);
   } else {
     for (int i = threadIdx.x; i < W; i += blockDim.x) dst[i] = from_f32<T>(row[i]);
   }
@@ -276,25 +280,29 @@ int append_latent_launch(const mla_dims& d, int32_t cache_dtype, void* cache, in
 int append_latent_strided(const mla_dims& d, int32_t cache_dtype, void* cache, int64_t cache_rows,
                           const int64_t* row_idx, const float* c_new, int64_t c_stride, const float* kpe_new,
                           int64_t kpe_stride, const int32_t* positions, int64_t n_new, uint32_t flags,
-                          float eps, float theta, cudaStream_t s) {
+                          float eps, float theta, cudaStream_t s, float cache_scale) {
   int* status = device_status_ptr();
   if (!status) return MLA_ERR_CUDA;
   if (n_new == 0) return MLA_OK;
   if (n_new > 0x7fffffff) return MLA_ERR_SHAPE;
   const int W = d.kv_lora_rank + d.rope_dim;
   const size_t es = dtype_bytes(cache_dtype);
-  const int vec8 = (W % 8 == 0) && aligned16(cache) && ((size_t)W * es) % 16 == 0;
+  const int vec8 = cache_dtype != MLA_FP8_E4M3 && (W % 8 == 0) && aligned16(cache) && ((size_t)W * es) % 16 == 0;
   const size_t smem = (size_t)W * sizeof(float);
   if (smem > 48 * 1024) return MLA_ERR_UNSUPPORTED;
   if (cache_dtype == MLA_BF16)
     return launch_pdl(append_latent_kernel<__nv_bfloat16>, dim3((unsigned)n_new), dim3(128), smem, s,
                       static_cast<__nv_bfloat16*>(cache), row_idx, c_new, c_stride, kpe_new, kpe_stride,
                       positions, d.kv_lora_rank, d.rope_dim, flags, eps, log2((double)theta), vec8, cache_rows,
-                      status);
-  else
-    append_latent_kernel<float><<<(unsigned)n_new, 128, smem, s>>>(
-        static_cast<float*>(cache), row_idx, c_new, c_stride, kpe_new, kpe_stride, positions, d.kv_lora_rank,
-        d.rope_dim, flags, eps, log2((double)theta), vec8, cache_rows, status);
+                      status, 1.f);
+  if (cache_dtype == MLA_FP8_E4M3)
+    return launch_pdl(append_latent_kernel<__nv_fp8_e4m3>, dim3((unsigned)n_new), dim3(128), smem, s,
+                      static_cast<__nv_fp8_e4m3*>(cache), row_idx, c_new, c_stride, kpe_new, kpe_stride,
+                      positions, d.kv_lora_rank, d.rope_dim, flags, eps, log2((double)theta), 0, cache_rows,
+                      status, cache_scale);
+  append_latent_kernel<float><<<(unsigned)n_new, 128, smem, s>>>(
+      static_cast<float*>(cache), row_idx, c_new, c_stride, kpe_new, kpe_stride, positions, d.kv_lora_rank,
+      d.rope_dim, flags, eps, log2((double)theta), vec8, cache_rows, status, 1.f);
   MLA_LAUNCH_CHECK();
   return MLA_OK;
 }
@@ -476,9 +484,10 @@ struct DecodeGenericParams {
   float* o_part; float* m_part; float* l_part;   // [split][row][H](*dc)
   int64_t rows;
   int64_t total_rows;
+  float cache_scale;                     // cache element times this = the value (1 unless e4m3)
 };
 
-template <typename T>
+template <typename T, typename TC = T>
 __global__ void __launch_bounds__(DG_THREADS) decode_generic_kernel(DecodeGenericParams p) {
   extern __shared__ float sm[];
   const int W = p.W, HG = p.HG;
@@ -513,13 +522,13 @@ __global__ void __launch_bounds__(DG_THREADS) decode_generic_kernel(DecodeGeneri
   const int n_el = hg * p.dc;
   __syncthreads();
 
-  const T* cache = static_cast<const T*>(p.cache);
+  const TC* cache = static_cast<const TC*>(p.cache);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int t0 = lo; t0 < hi; t0 += DG_TP) {
     const int nt = min(DG_TP, hi - t0);
     for (int e = threadIdx.x; e < nt * W; e += DG_THREADS) {
       const int tt = e / W, k = e - tt * W;
-      Ks[tt * (W + 1) + k] = to_f32(cache[(start + t0 + tt) * (int64_t)W + k]);
+      Ks[tt * (W + 1) + k] = to_f32(cache[(start + t0 + tt) * (int64_t)W + k]) * p.cache_scale;
     }
     __syncthreads();
     for (int e = threadIdx.x; e < hg * DG_TP; e += DG_THREADS) {
@@ -653,7 +662,17 @@ static GenericPlan plan_generic(const DecodeArgs& a) {
 
 size_t decode_generic_workspace(const DecodeArgs& a) { return plan_generic(a).ws; }
 
-int decode_generic_launch(const DecodeArgs& a, int32_t dtype, cudaStream_t s) {
+template <typename T, typename TC>
+static int decode_generic_run(const DecodeGenericParams& p, dim3 grid, size_t smem, cudaStream_t s) {
+  if (cudaFuncSetAttribute(decode_generic_kernel<T, TC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return MLA_ERR_CUDA;
+  decode_generic_kernel<T, TC><<<grid, DG_THREADS, smem, s>>>(p);
+  MLA_LAUNCH_CHECK();
+  return MLA_OK;
+}
+
+int decode_generic_launch(const DecodeArgs& a, int32_t dtype, cudaStream_t s, int32_t cache_dtype) {
   const GenericPlan g = plan_generic(a);
   const int64_t rows = (int64_t)a.batch * a.n_q;
   if (rows == 0) return MLA_OK;
@@ -664,6 +683,7 @@ int decode_generic_launch(const DecodeArgs& a, int32_t dtype, cudaStream_t s) {
   p.n_q = a.n_q; p.H = a.H; p.dc = a.dc; p.W = a.dc + a.dr; p.HG = g.HG;
   p.chunk = g.chunk; p.n_splits = g.n_splits; p.scale = a.scale; p.causal = a.causal ? 1 : 0;
   p.out_lat = a.out_lat; p.lse = a.lse; p.rows = rows; p.total_rows = a.total_rows;
+  p.cache_scale = cache_dtype == MLA_FP8_E4M3 ? a.cache_scale : 1.f;
   const size_t rh = (size_t)rows * a.H;
   char* ws = static_cast<char*>(a.workspace);
   p.o_part = reinterpret_cast<float*>(ws);
@@ -671,18 +691,14 @@ int decode_generic_launch(const DecodeArgs& a, int32_t dtype, cudaStream_t s) {
   p.l_part = p.m_part + round_up(sizeof(float) * (size_t)g.n_splits * rh, 256) / sizeof(float);
   dim3 grid((unsigned)g.n_splits, (unsigned)ceil_div(a.H, g.HG), (unsigned)rows);
   if (grid.y > 65535u || grid.z > 65535u) return MLA_ERR_UNSUPPORTED;
-  if (dtype == MLA_BF16) {
-    if (cudaFuncSetAttribute(decode_generic_kernel<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem) != cudaSuccess)
-      return MLA_ERR_CUDA;
-    decode_generic_kernel<__nv_bfloat16><<<grid, DG_THREADS, g.smem, s>>>(p);
-  } else {
-    if (cudaFuncSetAttribute(decode_generic_kernel<float>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem) != cudaSuccess)
-      return MLA_ERR_CUDA;
-    decode_generic_kernel<float><<<grid, DG_THREADS, g.smem, s>>>(p);
-  }
-  MLA_LAUNCH_CHECK();
+  int st;
+  if (cache_dtype == MLA_FP8_E4M3)
+    st = dtype == MLA_BF16 ? decode_generic_run<__nv_bfloat16, __nv_fp8_e4m3>(p, grid, g.smem, s)
+                           : decode_generic_run<float, __nv_fp8_e4m3>(p, grid, g.smem, s);
+  else
+    st = dtype == MLA_BF16 ? decode_generic_run<__nv_bfloat16, __nv_bfloat16>(p, grid, g.smem, s)
+                           : decode_generic_run<float, float>(p, grid, g.smem, s);
+  if (st) return st;
   if (g.n_splits > 1) {
     decode_combine_kernel<<<(unsigned)rh, 128, 0, s>>>(p.o_part, p.m_part, p.l_part, g.n_splits,
                                                        (int64_t)rh, a.dc, a.out_lat, a.lse);

@@ -86,6 +86,28 @@ int32_t mla_append_latent(const mla_dims* dims, int32_t cache_dtype, void* cache
                               flags, eps, rope_theta, as_stream(stream));
 }
 
+int32_t mla_append_latent_fp8(const mla_dims* dims, uint8_t* cache, int64_t cache_rows, const int64_t* row_idx,
+                              const float* c_new, const float* kpe_new, const int32_t* positions, int64_t n_new,
+                              uint32_t flags, float eps, float rope_theta, float cache_scale, void* stream) {
+  int st = check_dims(dims);
+  if (st) return st;
+  if (flags & ~(uint32_t)(MLA_APPEND_NORM | MLA_APPEND_ROPE)) return MLA_ERR_MODE;
+  if (n_new < 0 || cache_rows < 0) return MLA_ERR_SHAPE;
+  if (!(cache_scale > 0.f) || isinf(cache_scale)) return MLA_ERR_SHAPE;
+  if (n_new == 0) return MLA_OK;
+  if (!cache || !row_idx || !c_new) return MLA_ERR_NULL;
+  if (dims->rope_dim > 0 && !kpe_new) return MLA_ERR_NULL;
+  if ((flags & MLA_APPEND_ROPE) && dims->rope_dim > 0) {
+    if (!positions) return MLA_ERR_NULL;
+    if (dims->rope_dim % 2) return MLA_ERR_SHAPE;
+    if (!(rope_theta > 0.f)) return MLA_ERR_SHAPE;
+  }
+  if ((flags & MLA_APPEND_NORM) && !(eps >= 0.f)) return MLA_ERR_SHAPE;
+  return append_latent_strided(*dims, MLA_FP8_E4M3, cache, cache_rows, row_idx, c_new, dims->kv_lora_rank, kpe_new,
+                               dims->rope_dim, positions, n_new, flags, eps, rope_theta, as_stream(stream),
+                               cache_scale);
+}
+
 int32_t mla_absorb_weights(const mla_dims* dims, int32_t dtype, int32_t mode, const void* x,
                            const void* x_pe, const void* w, int64_t n_rows, void* out, void* stream) {
   int st = check_dims(dims);
@@ -171,10 +193,14 @@ int32_t mla_decode_workspace_size(const mla_dims* dims, int32_t dtype, int32_t b
                                   int64_t max_seqlen, int64_t total_rows, uint32_t flags,
                                   size_t* bytes) {
   if (!bytes) return MLA_ERR_NULL;
-  int st = check_decode_sizes(dims, dtype, batch, n_q, max_seqlen, total_rows, flags);
+  // MLA_FP8_E4M3: the scratch of mla_decode_absorbed_fp8 (whatever the query's dtype)
+  const bool fp8 = dtype == MLA_FP8_E4M3;
+  int st = check_decode_sizes(dims, fp8 ? MLA_F32 : dtype, batch, n_q, max_seqlen, total_rows, flags);
   if (st) return st;
   DecodeArgs a = make_decode_args(dims, batch, n_q, max_seqlen, total_rows, flags);
-  if (dtype == MLA_BF16 && tc_decode_supported(a))
+  if (fp8)
+    *bytes = decode_generic_workspace(a);
+  else if (dtype == MLA_BF16 && tc_decode_supported(a))
     *bytes = tc_decode_workspace(a);
   else
     *bytes = decode_generic_workspace(a);
@@ -201,6 +227,26 @@ int32_t mla_decode_absorbed(const mla_dims* dims, int32_t dtype, const void* q_a
   }
   if (workspace_bytes < decode_generic_workspace(a)) return MLA_ERR_WORKSPACE;
   return decode_generic_launch(a, dtype, s);
+}
+
+int32_t mla_decode_absorbed_fp8(const mla_dims* dims, int32_t q_dtype, const void* q_abs, const uint8_t* cache,
+                                float cache_scale, const int32_t* cu_seqlens, int32_t batch, int32_t n_q,
+                                int64_t max_seqlen, int64_t total_rows, uint32_t flags, float* out_lat, float* lse,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_decode_sizes(dims, q_dtype, batch, n_q, max_seqlen, total_rows, flags);
+  if (st) return st;
+  if (!(cache_scale > 0.f) || isinf(cache_scale)) return MLA_ERR_SHAPE;
+  if (batch == 0) return MLA_OK;
+  if (!q_abs || !cu_seqlens || !out_lat || (total_rows > 0 && !cache)) return MLA_ERR_NULL;
+  if ((st = check_align(q_dtype, {q_abs})) || (reinterpret_cast<uintptr_t>(out_lat) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return st ? st : MLA_ERR_ALIGN;
+  DecodeArgs a = make_decode_args(dims, batch, n_q, max_seqlen, total_rows, flags);
+  a.q_abs = q_abs; a.cache = cache; a.cu_seqlens = cu_seqlens;
+  a.out_lat = out_lat; a.lse = lse; a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+  a.cache_scale = cache_scale;
+  if (workspace_bytes < decode_generic_workspace(a)) return MLA_ERR_WORKSPACE;
+  return decode_generic_launch(a, q_dtype, as_stream(stream), MLA_FP8_E4M3);
 }
 
 int32_t mla_out_project_workspace_size(const mla_dims* dims, int32_t dtype, int64_t n_rows,

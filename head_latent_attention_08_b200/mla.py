@@ -18,7 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmla_b200.so")
 
 MLA_OK = 0
-MLA_F32, MLA_BF16 = 0, 1
+MLA_F32, MLA_BF16, MLA_FP8_E4M3 = 0, 1, 2
 MLA_ABSORB_QUERY, MLA_FOLD_QK, MLA_FOLD_VO = 0, 1, 2
 MLA_APPEND_NORM, MLA_APPEND_ROPE = 1, 2
 MLA_DECODE_CAUSAL = 1
@@ -32,7 +32,7 @@ EXPORTED = (
     "mla_out_project", "mla_linear", "mla_check_status", "mla_set_wait_limit", "mla_launch_count",
     "mla_set_decode_clusters", "mla_wait_selftest", "mla_decode_absorbed_noalloc",
     "mla_project_workspace_size", "mla_project_inputs", "mla_decode_step_workspace_size", "mla_decode_step",
-    "mla_lse_merge", "mla_prefill_attention",
+    "mla_lse_merge", "mla_prefill_attention", "mla_append_latent_fp8", "mla_decode_absorbed_fp8",
 )
 
 
@@ -88,6 +88,9 @@ _SIGS = {
                                _I64, _P, _P, _U32, _F, _F, _P, _I32, _P, _SZ, _P]),
     "mla_lse_merge": (_I32, [_DIMS, _I32, ctypes.POINTER(_P), ctypes.POINTER(_P), _I64, _I64, _P, _P, _P]),
     "mla_prefill_attention": (_I32, [_I32, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _F, _U32, _P, _P]),
+    "mla_append_latent_fp8": (_I32, [_DIMS, _P, _I64, _P, _P, _P, _P, _I64, _U32, _F, _F, _F, _P]),
+    "mla_decode_absorbed_fp8": (_I32, [_DIMS, _I32, _P, _P, _F, _P, _I32, _I32, _I64, _I64, _U32, _P, _P, _P, _SZ,
+                                       _P]),
 }
 
 
@@ -124,6 +127,8 @@ def _dtype_code(t: torch.dtype) -> int:
         return MLA_F32
     if t == torch.bfloat16:
         return MLA_BF16
+    if t in (torch.uint8, torch.float8_e4m3fn):
+        return MLA_FP8_E4M3
     raise TypeError(f"unsupported dtype {t}")
 
 
@@ -297,6 +302,28 @@ def mla_prefill_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gat
     _check(lib().mla_prefill_attention(_dtype_code(q.dtype), _ptr(q), _ptr(k), _ptr(v), _ptr(gate), batch, seq,
                                        n_heads, head_dim, scale, flags, _ptr(out), _stream(stream)),
            "mla_prefill_attention")
+
+
+def mla_append_latent_fp8(d: mla_dims, cache: torch.Tensor, row_idx: torch.Tensor, c_new: torch.Tensor,
+                          kpe_new: Optional[torch.Tensor], positions: Optional[torch.Tensor], flags: int,
+                          cache_scale: float = 1.0, eps: float = 1e-6, rope_theta: float = 10000.0,
+                          stream=None) -> None:
+    """cache: a uint8 (or float8_e4m3fn) tensor [rows, d_c + d_r] holding e4m3 codes."""
+    _check(lib().mla_append_latent_fp8(ctypes.byref(d), _ptr(cache), cache.shape[0], _ptr(row_idx), _ptr(c_new),
+                                       _ptr(kpe_new), _ptr(positions), row_idx.numel(), flags, eps, rope_theta,
+                                       cache_scale, _stream(stream)), "mla_append_latent_fp8")
+
+
+def mla_decode_absorbed_fp8(d: mla_dims, q_abs: torch.Tensor, cache: torch.Tensor, cache_scale: float,
+                            cu_seqlens: torch.Tensor, batch: int, n_q: int, max_seqlen: int, flags: int,
+                            out_lat: torch.Tensor, lse: Optional[torch.Tensor], workspace: Optional[torch.Tensor],
+                            stream=None) -> None:
+    assert cu_seqlens.dtype == torch.int32 and out_lat.dtype == torch.float32
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().mla_decode_absorbed_fp8(ctypes.byref(d), _dtype_code(q_abs.dtype), _ptr(q_abs), _ptr(cache),
+                                         cache_scale, _ptr(cu_seqlens), batch, n_q, max_seqlen, cache.shape[0],
+                                         flags, _ptr(out_lat), _ptr(lse), _ptr(workspace), ws_bytes,
+                                         _stream(stream)), "mla_decode_absorbed_fp8")
 
 
 def mla_check_status(stream=None) -> int:

@@ -61,8 +61,10 @@ enum {
   MLA_ERR_MODE = 9         /* unknown mode or flag bit                                           */
 };
 
-/* Element types. All floating-point tensors of one call share the call's dtype ([gm] Constraints). */
-enum { MLA_F32 = 0, MLA_BF16 = 1 };
+/* Element types. All floating-point tensors of one call share the call's dtype ([gm] Constraints),
+ * except the fp8 latent cache of the *_fp8 entry points (MLA_FP8_E4M3: 1 byte, 4 exponent and 3
+ * mantissa bits, no infinities, largest finite value 448). */
+enum { MLA_F32 = 0, MLA_BF16 = 1, MLA_FP8_E4M3 = 2 };
 
 /* Model dimensions. kq_scale == 0 selects the default 1/sqrt(qk_nope + rope_dim): the width of the
  * UN-absorbed head, not of the latent ([rs] module docs, the kq_scale paragraph). */
@@ -124,6 +126,18 @@ MLA_API int32_t mla_append_latent(const mla_dims* dims, int32_t cache_dtype, voi
                           float rope_theta, void* stream);
 
 /*
+ * mla_append_latent_fp8 -- mla_append_latent into an e4m3 latent cache (cache [cache_rows, d_c + d_r]
+ * bytes). The row is built as there, in fp32; each value is then stored as the e4m3 code nearest to
+ * value / cache_scale (an fp32 division; ties to even; saturating at +-448). One scale per cache: 1
+ * suits RMS-normed latents and N(0, 1) rotary keys, whose values stay far below 448.
+ * Errors: those of mla_append_latent; MLA_ERR_SHAPE for a scale that is not positive and finite.
+ */
+MLA_API int32_t mla_append_latent_fp8(const mla_dims* dims, uint8_t* cache, int64_t cache_rows,
+                                      const int64_t* row_idx, const float* c_new, const float* kpe_new,
+                                      const int32_t* positions, int64_t n_new, uint32_t flags, float eps,
+                                      float rope_theta, float cache_scale, void* stream);
+
+/*
  * mla_absorb_weights -- per-head products of the absorbed form.
  *
  * MLA_ABSORB_QUERY ([rs] module docs: q_nope_absorbed[h] = wk_b[h] . q_nope[h]; [lab] Bloque B:
@@ -148,6 +162,7 @@ MLA_API int32_t mla_absorb_weights(const mla_dims* dims, int32_t dtype, int32_t 
  *   batch        number of sequences B;  n_q_per_seq  query tokens per sequence (>= 1);
  *   max_seqlen   an upper bound on every T_b (host-side planning only);
  *   total_rows   sum of T_b (rows of the packed cache).
+ *   dtype MLA_FP8_E4M3 returns the scratch of mla_decode_absorbed_fp8 (for either query dtype).
  */
 MLA_API int32_t mla_decode_workspace_size(const mla_dims* dims, int32_t dtype, int32_t batch,
                                   int32_t n_q_per_seq, int64_t max_seqlen, int64_t total_rows,
@@ -179,6 +194,19 @@ MLA_API int32_t mla_decode_absorbed(const mla_dims* dims, int32_t dtype, const v
                             const int32_t* cu_seqlens, int32_t batch, int32_t n_q_per_seq,
                             int64_t max_seqlen, int64_t total_rows, uint32_t flags, float* out_lat,
                             float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * mla_decode_absorbed_fp8 -- mla_decode_absorbed over an e4m3 latent cache (value = code * cache_scale,
+ * the cache of mla_append_latent_fp8) with a bf16 or fp32 absorbed query (q_dtype): half the cache bytes
+ * of a bf16 cache. Same arguments, layouts and results otherwise; scratch of at least
+ * mla_decode_workspace_size(dims, MLA_FP8_E4M3, ...) bytes. Runs on CUDA cores in fp32 arithmetic
+ * (decoded cache values, fp32 scores and softmax).
+ */
+MLA_API int32_t mla_decode_absorbed_fp8(const mla_dims* dims, int32_t q_dtype, const void* q_abs,
+                                        const uint8_t* cache, float cache_scale, const int32_t* cu_seqlens,
+                                        int32_t batch, int32_t n_q_per_seq, int64_t max_seqlen, int64_t total_rows,
+                                        uint32_t flags, float* out_lat, float* lse, void* workspace,
+                                        size_t workspace_bytes, void* stream);
 
 /* Bytes of scratch mla_out_project needs for n_rows query rows. */
 MLA_API int32_t mla_out_project_workspace_size(const mla_dims* dims, int32_t dtype, int64_t n_rows,
