@@ -11,6 +11,9 @@
 // four warps drain TMEM in the epilogue (warp w owns accumulator rows 32w..32w+31). The result is
 // stored transposed, out[t][m]: consecutive lanes write consecutive addresses. Weights wider than one
 // wave of tiles are split along K; the fp32 partials are summed in a fixed order by a second kernel.
+// Products with more tiles than SMs and long K (the dense linears of a prefill) run on a persistent
+// form instead: one CTA per SM walks several tiles, with two TMEM accumulators so that one tile's
+// epilogue (four dedicated warps) overlaps the next tile's loads and MMAs.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -65,6 +68,7 @@ bool encode_tmap_bf16(CUtensorMap* map, void* base, int rank, const uint64_t* di
 // ---------------------------------------------------------------------------------------------
 struct TcGemmParams {
   int M, N, K;
+  int m_tiles;       // 128-row tiles of the weight
   int n_tiles;       // BN-wide token tiles
   int k_chunks;      // 64-wide K chunks per split
   int n_splits;
@@ -351,6 +355,264 @@ __global__ void f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __rest
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// persistent form: G CTAs (one per SM at most) walk the units u = c, c + G, c + 2G, ... of the same
+// tiling (unit = (batch, split, token tile, 128-row tile), row tile fastest). The shared-memory ring
+// runs on across a CTA's units and two TMEM accumulators alternate, so that four epilogue warps drain
+// unit u while unit u + 1's tiles load and its MMAs run: a short unit no longer pays its own setup,
+// first-load latency and epilogue in series.
+//   warps 0, 2, 3: TMA producers (lane 0); warp 1: MMA issuer (lane 0) and TMEM owner;
+//   warps 4-7: epilogue (warp 4 + q reads TMEM lanes 32 q .. 32 q + 31 = accumulator rows).
+// ---------------------------------------------------------------------------------------------
+constexpr int GEMM_P_THREADS = 256;
+constexpr int GEMM_P_BAR_BYTES = 256;
+
+template <int BN>
+struct GemmPCfg {
+  static constexpr int STAGE = GemmCfg<BN>::STAGE;
+  static constexpr int FIXED = 1024 + GEMM_P_BAR_BYTES;
+  static constexpr int STAGES_FIT = (227 * 1024 - FIXED) / STAGE;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr uint32_t ACC_COLS = GemmCfg<BN>::TMEM_COLS;          // one accumulator
+  static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS < 32 ? 32 : 2 * ACC_COLS;
+};
+
+struct GemmUnit {
+  int m0, n0, split, bz, kc0, nk;
+};
+
+__device__ __forceinline__ GemmUnit gemm_unit(const TcGemmParams& p, int64_t u, int BN, int total_chunks) {
+  GemmUnit r;
+  int64_t x = u;
+  const int mt = (int)(x % p.m_tiles);
+  x /= p.m_tiles;
+  const int nt = (int)(x % p.n_tiles);
+  x /= p.n_tiles;
+  r.split = (int)(x % p.n_splits);
+  r.bz = (int)(x / p.n_splits);
+  r.m0 = mt * 128;
+  r.n0 = nt * BN;
+  r.kc0 = r.split * p.k_chunks;
+  r.nk = max(0, min(r.kc0 + p.k_chunks, total_chunks) - r.kc0);
+  return r;
+}
+
+template <int BN, bool A_MN>
+__global__ void __launch_bounds__(GEMM_P_THREADS, 1)
+    tc_gemm_persistent_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb,
+                              TcGemmParams p) {
+  using Cfg = GemmCfg<BN>;
+  using PCfg = GemmPCfg<BN>;
+  const int STAGES = p.stages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE);
+  uint64_t* empty = full + 8;
+  uint64_t* acc_full = empty + 8;      // [2]
+  uint64_t* acc_empty = acc_full + 2;  // [2]
+  uint64_t* done = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_load = abort_flag + 1;   // [8]: the last chunk (CTA-local count) loaded into each stage
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int total_chunks = (p.K + 63) / 64;
+  const int64_t U = (int64_t)p.m_tiles * p.n_tiles * p.n_splits * p.batch;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      last_load[s] = -1;
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&ta);
+    prefetch_tmap(&tb);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, PCfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const bool producer = warp != 1 && warp < 4 && lane == 0;
+  // the activations (B), the gate and the tail may come from the previous kernel of the stream, and the
+  // output may still be read by it: everyone waits for it, the producers after their weight prefetch
+  if (!producer) griddep_wait();
+  griddep_launch_dependents();
+  const uint32_t tmem = *tmem_slot;
+
+  auto wait_bar = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (*abort_flag) return false;
+    if (mbar_wait(bar, parity, p.wait_ns, p.status)) return true;
+    *abort_flag = 1;
+    return false;
+  };
+
+  if (producer) {
+    // producer j loads the CTA-local chunks g = j, j + P, ... (g counts the chunks of the CTA's units
+    // in order); chunk g goes to stage g % STAGES once the MMAs have read its previous round
+    const int j = warp == 0 ? 0 : warp - 1;
+    auto load_a = [&](const GemmUnit& w, int i, int s) {
+      uint8_t* a_dst = smem + s * Cfg::STAGE;
+      const int kx = (w.kc0 + i) * 64;
+      if (A_MN) {
+        tma_load_3d(a_dst, &ta, &full[s], w.m0, kx, w.bz);
+        tma_load_3d(a_dst + 8192, &ta, &full[s], w.m0 + 64, kx, w.bz);
+      } else {
+        tma_load_3d(a_dst, &ta, &full[s], kx, w.m0, w.bz);
+      }
+    };
+    // the weights (A) are never written by the library's kernels: the first ring's weight tiles are
+    // requested before the wait, so that their latency overlaps the previous kernel's tail
+    int g = 0;
+    for (int64_t u = blockIdx.x; u < U && g < STAGES; u += gridDim.x) {
+      const GemmUnit w = gemm_unit(p, u, BN, total_chunks);
+      for (int i = 0; i < w.nk && g < STAGES; ++i, ++g) {
+        if (g % GEMM_PRODUCERS != j) continue;
+        mbar_arrive_expect_tx(&full[g], Cfg::STAGE);
+        load_a(w, i, g);
+        last_load[g] = g;
+      }
+    }
+    griddep_wait();
+    g = 0;
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < U && ok; u += gridDim.x) {
+      const GemmUnit w = gemm_unit(p, u, BN, total_chunks);
+      for (int i = 0; i < w.nk; ++i, ++g) {
+        if (g % GEMM_PRODUCERS != j) continue;
+        const int s = g % STAGES;
+        if (g >= STAGES) {    // (a prefetched stage always gets its B tile, so that its barrier completes)
+          if (!wait_bar(&empty[s], (uint32_t)(((g / STAGES) - 1) & 1))) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[s], Cfg::STAGE);
+          load_a(w, i, s);
+          last_load[s] = g;
+        }
+        tma_load_3d(smem + s * Cfg::STAGE + Cfg::A_BYTES, &tb, &full[s], (w.kc0 + i) * 64, w.n0, w.bz);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // MMA issuer: unit number ui of this CTA accumulates into TMEM accumulator ui & 1, once the
+    // epilogue has drained that accumulator's previous unit
+    constexpr uint32_t idesc = idesc_bf16_f32(128, BN, A_MN, false);
+    int g = 0, ui = 0;
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < U && ok; u += gridDim.x, ++ui) {
+      const GemmUnit w = gemm_unit(p, u, BN, total_chunks);
+      const int acc = ui & 1;
+      if (ui >= 2 && !wait_bar(&acc_empty[acc], (uint32_t)(((ui >> 1) - 1) & 1))) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d = tmem + (uint32_t)acc * PCfg::ACC_COLS;
+      for (int i = 0; i < w.nk; ++i, ++g) {
+        const int s = g % STAGES;
+        if (!wait_bar(&full[s], (uint32_t)((g / STAGES) & 1))) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(smem + s * Cfg::STAGE);
+        const uint32_t b_base = a_base + Cfg::A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = A_MN ? smem_desc_sw128(a_base + kk * 2048, 8192, 1024)
+                                   : smem_desc_sw128(a_base + kk * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(b_base + kk * 32, 16, 1024);
+          mma_bf16_ss(d, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);
+      }
+      if (!ok) break;
+      mma_commit(&acc_full[acc]);
+    }
+    mma_commit(done);
+  } else if (warp >= 4) {
+    // ---- epilogue: thread = accumulator row m of unit ui (TMEM lane 32 (warp - 4) + lane); for each
+    // token t it stores out[t][m] directly: a warp's store covers 32 consecutive m of one token row
+    const int et = threadIdx.x - 128;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    int ui = 0;
+    for (int64_t u = blockIdx.x; u < U; u += gridDim.x, ++ui) {
+      const GemmUnit w = gemm_unit(p, u, BN, total_chunks);
+      const int acc = ui & 1;
+      const bool okw = wait_bar(&acc_full[acc], (uint32_t)((ui >> 1) & 1));
+      // one decision for the four warps
+      if (named_bar_or(1, 128, !okw || *abort_flag)) break;
+      tc_fence_after();
+      const uint32_t d = tmem + (uint32_t)acc * PCfg::ACC_COLS;
+      const int m = w.m0 + et;
+      const bool row_ok = m < p.M;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(d + lane_base + (uint32_t)c, r);
+        tmem_wait_ld();
+        const int nt = min(32, p.N - (w.n0 + c));
+        if (!row_ok || nt <= 0) continue;
+        if (p.n_splits > 1) {
+          float* dst = p.partial + (((int64_t)w.split * p.batch + w.bz) * p.N + w.n0 + c) * p.M + m;
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj)
+            if (jj < nt) dst[(int64_t)jj * p.M] = w.nk > 0 ? __uint_as_float(r[jj]) : 0.f;
+          continue;
+        }
+        const int64_t o0 = w.bz * p.out_sb + (int64_t)(w.n0 + c) * p.out_st + m;
+        const int64_t g0 = w.bz * p.gate_sb + (int64_t)(w.n0 + c) * p.gate_st + m;
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          if (jj >= nt) break;
+          float v = w.nk > 0 ? __uint_as_float(r[jj]) : 0.f;
+          if (p.sigmoid) v = 1.f / (1.f + expf(-v));
+          if (p.gate) v *= __bfloat162float(p.gate[g0 + (int64_t)jj * p.gate_st]);
+          if (p.out_f32)
+            static_cast<float*>(p.out)[o0 + (int64_t)jj * p.out_st] = v;
+          else
+            static_cast<__nv_bfloat16*>(p.out)[o0 + (int64_t)jj * p.out_st] = __float2bfloat16_rn(v);
+        }
+      }
+      if (p.tail && w.m0 == 0 && w.split == 0) {
+        // the tail columns of this unit's tokens (16-byte chunks; the host checks the alignment)
+        const int cpr = p.tail_cols / 8;
+        for (int idx = et; idx < BN * cpr; idx += 128) {
+          const int t = w.n0 + idx / cpr, q = idx % cpr;
+          if (t >= p.N) break;
+          const uint4 v = reinterpret_cast<const uint4*>(p.tail + w.bz * p.tail_sb + (int64_t)t * p.tail_st)[q];
+          reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + w.bz * p.out_sb + (int64_t)t * p.out_st +
+                                   p.tail_off)[q] = v;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);       // this warp's rows of the accumulator are read
+    }
+  }
+
+  // ---- teardown: nothing of this CTA's may be in flight when its tensor memory is released ----
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t drain_ns = p.wait_ns > 100000000ull ? p.wait_ns : 100000000ull;
+    if (*abort_flag) {
+      // only the last load of a stage can still be in flight (a later one waited for the MMAs to read
+      // the earlier)
+      for (int s = 0; s < STAGES; ++s) {
+        const int g = last_load[s];
+        if (g >= 0) (void)mbar_wait(&full[s], (uint32_t)((g / STAGES) & 1), drain_ns, p.status);
+      }
+    }
+    (void)mbar_wait(done, 0, drain_ns, p.status);      // the MMA issuer's final commit
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, PCfg::TMEM_COLS);
+  }
+}
+
 struct GemmOperand {
   // a 3-D bf16 tensor seen as [batch][rows][k] (K-major) or [batch][k][rows] (MN-major)
   void* base;
@@ -360,8 +622,15 @@ struct GemmOperand {
 
 struct GemmPlan {
   int BN, n_tiles, m_tiles, splits, k_chunks;
+  bool persistent;   // the persistent kernel (several units per CTA) instead of one tile per CTA
 };
 
+// Tiling of out[bz][t][m] = sum_k A[bz](m, k) B[bz](t, k): 128-row tiles of A, BN-token tiles of B,
+// and K split into `splits` ranges. Products with more tiles than SMs and at least 8 K chunks per tile
+// (the dense linears of a prefill) run on the persistent kernel, the K splits chosen by a cost in K
+// chunks on the busiest SM (a split adds the sum kernel, about 7 chunks' time, and the partials'
+// traffic). The others keep one tile (and K range) per CTA, split along K until one wave of tiles
+// covers the SMs: their CTAs are short, and several run at once on an SM.
 static GemmPlan plan_gemm(int M, int N, int K, int batch, int max_splits) {
   GemmPlan g;
   g.BN = N <= 64 ? 64 : (N <= 128 ? 128 : 256);
@@ -369,10 +638,28 @@ static GemmPlan plan_gemm(int M, int N, int K, int batch, int max_splits) {
   g.m_tiles = (int)ceil_div(M, 128);
   const int total_chunks = (int)ceil_div(K, 64);
   const int64_t base = (int64_t)g.m_tiles * g.n_tiles * batch;
-  int splits = (int)std::max<int64_t>(1, std::min<int64_t>(sm_count() / std::max<int64_t>(base, 1),
-                                                            total_chunks / 4));
-  splits = std::min(splits, std::max(1, max_splits));
-  g.k_chunks = (int)ceil_div(total_chunks, splits);
+  const int64_t G = sm_count();
+  g.persistent = base > G && total_chunks >= 8;
+  int best = 1;
+  if (g.persistent) {
+    const double stage_bytes = 128.0 * 64 * 2 + g.BN * 64.0 * 2;
+    double best_cost = (double)ceil_div(base, G) * total_chunks;
+    const int s_max = std::min(std::max(1, max_splits), std::min(total_chunks / 2, 32));
+    for (int s = 2; s <= s_max; ++s) {
+      const int kc = (int)ceil_div(total_chunks, s);
+      const int ss = (int)ceil_div(total_chunks, kc);
+      const double cost = (double)ceil_div(base * ss, G) * kc + 7.0 +
+                          2.0 * ss * batch * (double)N * M * 4.0 / ((double)G * stage_bytes);
+      if (cost < best_cost) {
+        best_cost = cost;
+        best = ss;
+      }
+    }
+  } else {
+    best = (int)std::max<int64_t>(1, std::min<int64_t>(G / std::max<int64_t>(base, 1), total_chunks / 4));
+    best = std::min(best, std::max(1, max_splits));
+  }
+  g.k_chunks = (int)ceil_div(total_chunks, best);
   g.splits = (int)ceil_div(total_chunks, g.k_chunks);
   return g;
 }
@@ -383,8 +670,7 @@ static size_t gemm_partial_bytes(int M, int N, int K, int batch) {
 }
 
 template <int BN, bool A_MN>
-static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, TcGemmParams p, dim3 grid,
-                         cudaStream_t s) {
+static int launch_gemm_wave_t(const CUtensorMap& ta, const CUtensorMap& tb, TcGemmParams p, cudaStream_t s) {
   static bool attr_set[64] = {false};
   const int dev = current_device();
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
@@ -393,10 +679,36 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, TcGemmPar
       return MLA_ERR_CUDA;
     attr_set[dev] = true;
   }
+  const dim3 grid((unsigned)p.m_tiles, (unsigned)(p.n_tiles * p.n_splits), (unsigned)p.batch);
+  if (grid.y > 65535u || grid.z > 65535u) return MLA_ERR_UNSUPPORTED;
   // a ring no deeper than the K chunks of one CTA: short-K products then fit several CTAs per SM
   p.stages = std::max(1, std::min(GemmCfg<BN>::STAGES, p.k_chunks));
   const int smem = p.stages * GemmCfg<BN>::STAGE + 1024 + 256;
   return launch_pdl(tc_gemm_kernel<BN, A_MN>, grid, dim3(128), (size_t)smem, s, ta, tb, p);
+}
+
+template <int BN, bool A_MN>
+static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, TcGemmParams p, cudaStream_t s,
+                         bool persistent) {
+  if (!persistent) return launch_gemm_wave_t<BN, A_MN>(ta, tb, p, s);
+  using PCfg = GemmPCfg<BN>;
+  static bool attr_set[64] = {false};
+  const int dev = current_device();
+  const int smem_max = PCfg::STAGES * GemmCfg<BN>::STAGE + PCfg::FIXED;
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(tc_gemm_persistent_kernel<BN, A_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem_max) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  const int64_t U = (int64_t)p.m_tiles * p.n_tiles * p.n_splits * p.batch;
+  const int64_t G = std::min<int64_t>(U, sm_count());
+  // a ring no deeper than the chunks one CTA streams
+  const int64_t chunks_per_cta = ceil_div(U, G) * p.k_chunks;
+  p.stages = (int)std::max<int64_t>(2, std::min<int64_t>(PCfg::STAGES, chunks_per_cta));
+  const int smem = p.stages * GemmCfg<BN>::STAGE + PCfg::FIXED;
+  return launch_pdl(tc_gemm_persistent_kernel<BN, A_MN>, dim3((unsigned)G), dim3(GEMM_P_THREADS), (size_t)smem, s,
+                    ta, tb, p);
 }
 
 // out[bz][t][m] = epi(sum_k A[bz](m, k) B[bz](t, k)); A MN-major when a_mn
@@ -432,7 +744,8 @@ static int tc_gemm(const GemmOperand& A, bool a_mn, const GemmOperand& Bop, int 
     if (!encode_tmap_bf16(&tb, Bop.base, 3, dims, st, box)) return MLA_ERR_CUDA;
   }
   TcGemmParams p{};
-  p.M = M; p.N = N; p.K = K; p.n_tiles = g.n_tiles; p.k_chunks = g.k_chunks; p.n_splits = g.splits;
+  p.M = M; p.N = N; p.K = K; p.m_tiles = g.m_tiles; p.n_tiles = g.n_tiles; p.k_chunks = g.k_chunks;
+  p.n_splits = g.splits;
   p.batch = batch; p.out = out; p.out_sb = out_sb; p.out_st = out_st; p.out_f32 = out_f32 ? 1 : 0;
   p.gate = static_cast<const __nv_bfloat16*>(gate); p.gate_sb = gate_sb; p.gate_st = gate_st;
   p.partial = static_cast<float*>(partial_ws); p.sigmoid = sigmoid ? 1 : 0;
@@ -446,17 +759,17 @@ static int tc_gemm(const GemmOperand& A, bool a_mn, const GemmOperand& Bop, int 
   p.status = device_status_ptr(); p.wait_ns = (unsigned long long)wait_limit();
   if (!p.status) return MLA_ERR_CUDA;
   if (g.splits > 1 && !partial_ws) return MLA_ERR_WORKSPACE;
-  dim3 grid((unsigned)g.m_tiles, (unsigned)(g.n_tiles * g.splits), (unsigned)batch);
-  if (grid.y > 65535u || grid.z > 65535u) return MLA_ERR_UNSUPPORTED;
+  if ((int64_t)g.m_tiles * g.n_tiles * g.splits * batch >= (1LL << 31)) return MLA_ERR_UNSUPPORTED;
   int st;
+  const bool pk = g.persistent;
   if (a_mn) {
-    st = g.BN == 64 ? launch_gemm_t<64, true>(ta, tb, p, grid, s)
-                    : g.BN == 128 ? launch_gemm_t<128, true>(ta, tb, p, grid, s)
-                                  : launch_gemm_t<256, true>(ta, tb, p, grid, s);
+    st = g.BN == 64 ? launch_gemm_t<64, true>(ta, tb, p, s, pk)
+                    : g.BN == 128 ? launch_gemm_t<128, true>(ta, tb, p, s, pk)
+                                  : launch_gemm_t<256, true>(ta, tb, p, s, pk);
   } else {
-    st = g.BN == 64 ? launch_gemm_t<64, false>(ta, tb, p, grid, s)
-                    : g.BN == 128 ? launch_gemm_t<128, false>(ta, tb, p, grid, s)
-                                  : launch_gemm_t<256, false>(ta, tb, p, grid, s);
+    st = g.BN == 64 ? launch_gemm_t<64, false>(ta, tb, p, s, pk)
+                    : g.BN == 128 ? launch_gemm_t<128, false>(ta, tb, p, s, pk)
+                                  : launch_gemm_t<256, false>(ta, tb, p, s, pk);
   }
   if (st) return st;
   if (g.splits > 1) {
