@@ -32,10 +32,10 @@ using namespace sm100;
 constexpr int PF_BM = 128;                 // queries per CTA (the MMA's M)
 constexpr int PF_BN = 128;                 // keys per tile (N of Q K^T, K of P V)
 constexpr int PF_D = 128;                  // head width (K of Q K^T, N of P V)
-constexpr int PF_THREADS = 256;            // warps 0 TMA, 1 MMA, 2-3 spare, 4-7 softmax
+constexpr int PF_THREADS = 384;            // warps 0 TMA, 1 MMA, 2-3 spare, 4-11 softmax (two per row window)
 constexpr int PF_TILE = PF_BM * PF_D * 2;  // 32 KB: one Q, K or V tile, two 64-column boxes
 constexpr int PF_BOX = PF_TILE / 2;        // 16 KB: one 128-row x 64-column box
-constexpr int PF_SMEM = 5 * PF_TILE + 1024 + 512;
+constexpr int PF_SMEM = 5 * PF_TILE + 1024 + 4096;
 constexpr uint32_t PF_TMEM_COLS = 512;
 constexpr float PF_REF_SLACK = 8.f;        // log2 units a row maximum may exceed m_ref before it moves
 
@@ -63,7 +63,11 @@ struct PfBars {
   uint32_t tmem;
   int abort;
   int last_k[2], last_v[2];                // the last tile loaded into each stage (abort drain)
+  float xmax[2][2][PF_BM];                 // [tile parity][column half][row]: the halves' row maxima
+  float xl[2][PF_BM];                      // [column half][row]: the halves' row sums
 };
+
+static_assert(sizeof(PfBars) <= 4096, "barrier region");
 
 __global__ void __launch_bounds__(PF_THREADS, 1)
     tc_prefill_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -94,8 +98,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       mbar_init(&bars->v_full[i], 1);
       mbar_init(&bars->v_empty[i], 1);
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->s_free[i], 4);
-      mbar_init(&bars->p_full[i], 4);
+      mbar_init(&bars->s_free[i], 8);
+      mbar_init(&bars->p_full[i], 8);
       mbar_init(&bars->p_free[i], 1);
       bars->last_k[i] = -1;
       bars->last_v[i] = -1;
@@ -206,55 +210,68 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     mma_commit(&bars->done);
   } else if (warp >= 4) {
     // ------------------------------- softmax and epilogue -------------------------------
+    // Two warps per TMEM lane window: warp 4 + q takes key columns 0-63 of rows 32 q .., warp 8 + q
+    // columns 64-127 (and the matching halves of O). The pair shares its rows' maxima and sums through
+    // shared memory at a 64-thread named barrier that also carries an abort decision, so that both
+    // warps of a pair always take the same path.
     const int quarter = warp & 3;                  // TMEM lanes 32 quarter .. (the warp's lane window)
+    const int half = (warp - 4) >> 2;              // key / head columns [64 half, 64 half + 64)
+    const uint32_t bar_id = 1 + (uint32_t)quarter;
     const int row = quarter * 32 + lane;           // query row of the tile
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int qi = q0 + row;                       // query position in its sequence
     const int k_end = min(p.S, p.causal ? qi + 1 : p.S);   // keys 0 .. k_end - 1 are visible
     float m_ref = 0.f, l = 0.f;
+    bool alive = true;                             // this warp's waits have all succeeded
     bool ok = true;
-    for (int j = 0; j < nkv && ok; ++j) {
+    for (int j = 0; j < nkv; ++j) {
       const int s = j & 1;
-      if (!warp_wait(&bars->s_full[s], (uint32_t)(j >> 1) & 1u)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t xr[PF_BN];
+      const bool okj = alive && warp_wait(&bars->s_full[s], (uint32_t)(j >> 1) & 1u);
+      uint32_t xr[PF_BN / 2];
+      float mh = -INFINITY;
+      if (okj) {
+        tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < PF_BN / 32; ++c)
-        tmem_ld32(tS + s * PF_BN + lane_off + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&xr[32 * c]));
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->s_free[s]);
-      const int kmax = k_end - j * PF_BN;
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
+        for (int c = 0; c < 2; ++c)
+          tmem_ld32(tS + s * PF_BN + lane_off + half * 64 + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&xr[32 * c]));
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free[s]);
+        const int kmax = k_end - j * PF_BN - half * 64;
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
 #pragma unroll
-      for (int c = 0; c < PF_BN; ++c) {
-        const float v = c < kmax ? __uint_as_float(xr[c]) * p.scale_log2 : -INFINITY;
-        xr[c] = __float_as_uint(v);
-        mx[c & 3] = fmaxf(mx[c & 3], v);
+        for (int c = 0; c < PF_BN / 2; ++c) {
+          const float v = c < kmax ? __uint_as_float(xr[c]) * p.scale_log2 : -INFINITY;
+          xr[c] = __float_as_uint(v);
+          mx[c & 3] = fmaxf(mx[c & 3], v);
+        }
+        mh = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        bars->xmax[j & 1][half][row] = mh;
       }
-      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      if (named_bar_or(bar_id, 64, !okj)) { ok = false; break; }
+      const float mt = fmaxf(bars->xmax[j & 1][0][row], bars->xmax[j & 1][1][row]);
       // P buffer s is free once P_{j-2} V_{j-2} is done
-      if (j >= 2 && !warp_wait(&bars->p_free[s], (uint32_t)((j >> 1) - 1) & 1u)) { ok = false; break; }
+      if (j >= 2 && !warp_wait(&bars->p_free[s], (uint32_t)((j >> 1) - 1) & 1u)) { alive = false; continue; }
       if (j == 0) {
         m_ref = mt == -INFINITY ? 0.f : mt;
       } else {
         const bool move = mt > m_ref + PF_REF_SLACK;
         if (__any_sync(0xffffffffu, move)) {
           // O (every product up to P_{j-1} V_{j-1}, done once p_free of tile j - 1 completes) and l
-          // follow the rows' new reference maxima; the other rows of the warp keep theirs (factor 1)
+          // follow the rows' new reference maxima (this warp's half of O); the other rows keep theirs
           const int sp = (j - 1) & 1;
-          if (!warp_wait(&bars->p_free[sp], (uint32_t)((j - 1) >> 1) & 1u)) { ok = false; break; }
+          if (!warp_wait(&bars->p_free[sp], (uint32_t)((j - 1) >> 1) & 1u)) { alive = false; continue; }
           tc_fence_after();
           const float f = move ? pf_ex2(m_ref - mt) : 1.f;
 #pragma unroll 1
-          for (int c = 0; c < PF_D / 32; ++c) {
+          for (int c = 0; c < 2; ++c) {
             uint32_t r[32];
-            tmem_ld32(tO + lane_off + c * 32, r);
+            tmem_ld32(tO + lane_off + half * 64 + c * 32, r);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
-            tmem_st32(tO + lane_off + c * 32, r);
+            tmem_st32(tO + lane_off + half * 64 + c * 32, r);
           }
           tmem_wait_st();
           if (move) {
@@ -264,10 +281,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         }
       }
       // probabilities, rounded to bf16 once; the row sum adds the rounded values the MMA will use
-      uint32_t pk[PF_BN / 2];
+      uint32_t pk[PF_BN / 4];
       float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < PF_BN / 2; ++c) {
+      for (int c = 0; c < PF_BN / 4; ++c) {
         const __nv_bfloat162 b2 = __floats2bfloat162_rn(pf_ex2(__uint_as_float(xr[2 * c]) - m_ref),
                                                         pf_ex2(__uint_as_float(xr[2 * c + 1]) - m_ref));
         const float2 back = __bfloat1622float2(b2);
@@ -276,51 +293,57 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       }
       l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
       tc_fence_after();
-      tmem_st32(tP + s * 64 + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tP + s * 64 + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_st32(tP + s * 64 + lane_off + half * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full[s]);
     }
-    // epilogue: O / l (times the gate), bf16, once the last P V product is done
-    if (ok && nkv > 0) ok = warp_wait(&bars->p_free[(nkv - 1) & 1], (uint32_t)((nkv - 1) >> 1) & 1u);
+    // epilogue: O / l (times the gate), bf16, once the last P V product is done; l is the sum of the
+    // pair's two halves, added in a fixed order
+    bool okf = ok && alive;
+    if (okf && nkv > 0) okf = warp_wait(&bars->p_free[(nkv - 1) & 1], (uint32_t)((nkv - 1) >> 1) & 1u);
     if (ok) {
-      tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const bool store = qi < p.S;
-      const int64_t ld = (int64_t)p.H * PF_D;
-      __nv_bfloat16* dst = p.out + (int64_t)(row0 + qi) * ld + h * PF_D;
-      const __nv_bfloat16* g = p.gate ? p.gate + (int64_t)(row0 + qi) * ld + h * PF_D : nullptr;
+      bars->xl[half][row] = l;
+      const bool bad = named_bar_or(bar_id, 64, !okf);
+      if (!bad) {
+        tc_fence_after();
+        const float lt = bars->xl[0][row] + bars->xl[1][row];
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const bool store = qi < p.S;
+        const int64_t ld = (int64_t)p.H * PF_D;
+        __nv_bfloat16* dst = p.out + (int64_t)(row0 + qi) * ld + h * PF_D + half * 64;
+        const __nv_bfloat16* g = p.gate ? p.gate + (int64_t)(row0 + qi) * ld + h * PF_D + half * 64 : nullptr;
 #pragma unroll 1
-      for (int c = 0; c < PF_D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tO + lane_off + c * 32, r);
-        tmem_wait_ld();
-        if (!store) continue;
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + lane_off + half * 64 + c * 32, r);
+          tmem_wait_ld();
+          if (!store) continue;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float v[8];
+          for (int q = 0; q < 4; ++q) {
+            float v[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * q + e]) * inv;
-          if (g) {
-            const uint4 gv = *reinterpret_cast<const uint4*>(g + c * 32 + 8 * q);
-            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * q + e]) * inv;
+            if (g) {
+              const uint4 gv = *reinterpret_cast<const uint4*>(g + c * 32 + 8 * q);
+              const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 gf = __bfloat1622float2(g2[e]);
+                v[2 * e] *= gf.x;
+                v[2 * e + 1] *= gf.y;
+              }
+            }
+            uint4 w;
+            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float2 gf = __bfloat1622float2(g2[e]);
-              v[2 * e] *= gf.x;
-              v[2 * e + 1] *= gf.y;
+              const __nv_bfloat162 o2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+              wp[e] = *reinterpret_cast<const uint32_t*>(&o2);
             }
+            *reinterpret_cast<uint4*>(dst + c * 32 + 8 * q) = w;
           }
-          uint4 w;
-          uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 o2 = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-            wp[e] = *reinterpret_cast<const uint32_t*>(&o2);
-          }
-          *reinterpret_cast<uint4*>(dst + c * 32 + 8 * q) = w;
         }
       }
     }
