@@ -14,9 +14,10 @@
 //    CLUSTER OF TWO CTAs shares a block, with different jobs:
 //      - the score CTA (rank 0) holds the block's latent query in TMEM (256 columns of bf16 pairs, the
 //        A operand of QK^T) and its rotary query in shared memory, streams every cache row whole (all
-//        576 columns, 128-position tiles by TMA), computes S = Q K^T in fp32 into one of two 128-column
-//        TMEM slots, runs the online softmax in fp32 and hands P (bf16) to the value CTA through
-//        distributed shared memory, 64 positions at a time, with per-row side data (the factor by
+//        576 columns, 256-position tiles by TMA through two 96 KB ring slots), computes S = Q K^T in
+//        fp32 into a 256-column TMEM slot with N = 256 MMAs, runs the online softmax in fp32 and hands
+//        P (bf16) to the value CTA through distributed shared memory (remote st.async stores counted
+//        by the value CTA's barrier), 64 positions at a time, with per-row side data (the factor by
 //        which O must be rescaled, and at the end of a block the row maximum and sum);
 //      - the value CTA (rank 1) holds all of O in TMEM, streams the latent columns of the same rows
 //        (read a second time, from L2, right after the score CTA brought them in) and accumulates
@@ -26,17 +27,17 @@
 //  * The score CTA rescales nothing: P is taken against a reference maximum that moves only when a
 //    row's maximum grows by more than 2^8 (exact: numerator and denominator share it); the rare move
 //    is passed on with the P of that tile, and the value CTA multiplies its O rows before that P.C.
-//  * Work: the (block, 128-position tile) units of all sequences are split evenly over the clusters
+//  * Work: the (block, 256-position tile) units of all sequences are split evenly over the clusters
 //    (persistent). A cluster that covers a whole block writes the normalised result; split blocks
 //    leave (O, max, sum) partials that a combine kernel merges.
 //  * Loads: one thread keeps about one TMA instruction in flight, so several threads issue them (three
 //    in the score CTA, two in the value CTA), and the value CTA fetches 64 positions x 256 columns per
-//    instruction (a 3-D box over 64-column groups). The score CTA also warms L2 a few tiles ahead.
-//  * Warp roles (384 threads). Score CTA: warps 0, 2, 3 lane 0 TMA, warp 1 lane 0 QK^T, warps 4-11
-//    softmax (warp w: rows 32 (w & 3) .., positions [64 h, 64 h + 64) of each tile, h = (w - 4) >> 2),
+//    instruction (a 3-D box over 64-column groups).
+//  * Warp roles (640 threads). Score CTA: warps 0, 2, 3 lane 0 TMA, warp 1 lane 0 QK^T, warps 4-19
+//    softmax (warp w: rows 32 (w & 3) .., positions [64 c, 64 c + 64) of each tile, c = (w - 4) >> 2),
 //    which also move each block's latent query into TMEM. Value CTA: warps 0 and 3 lane 0 TMA, warp 1
-//    lane 0 P.C, warp 2 lane 0 hands P slots back, warps 4-11 rescale and write O (warp w: rows
-//    32 (w & 3) .., O columns [256 h, 256 h + 256)).
+//    lane 0 P.C, warp 2 lane 0 hands P slots back, warps 4-19 rescale and write O (warp w: rows
+//    32 (w & 3) .., O columns [128 c, 128 c + 128)).
 //  * Every wait is bounded (global-timer limit); a wait that gives up sets the library's status word,
 //    and the CTA abandons its work: it issues nothing more, drains its own TMA loads, MMAs and bulk
 //    copies and leaves through the cluster barrier.
