@@ -140,7 +140,11 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const bool producer = warp != 1 && lane == 0;
+  // Producers in use: never more than the ring has stages. A producer waits for the release of its
+  // chunk's stage by parity, which is only sound while that stage's previous round has been loaded:
+  // with P producers taking every P-th chunk, that holds when STAGES >= P.
+  const int nprod = min(GEMM_PRODUCERS, STAGES);
+  const bool producer = warp != 1 && lane == 0 && (warp == 0 ? 0 : warp - 1) < nprod;
   // the activations (B), the gate and the tail may come from the previous kernel of the stream, and the
   // output may still be read by it: everyone waits for it, the producers after their weight prefetch
   if (!producer) griddep_wait();
@@ -165,13 +169,13 @@ __global__ void __launch_bounds__(128, 1)
     // The weights (A) are never written by the library's kernels: the first ring's weight tiles are
     // requested before the wait, so that their latency overlaps the previous kernel's tail.
     const int pre = min(nk, STAGES);
-    for (int i = j; i < pre; i += GEMM_PRODUCERS) {
+    for (int i = j; i < pre; i += nprod) {
       mbar_arrive_expect_tx(&full[i], Cfg::STAGE);
       load_a(i, i);
       last_load[i] = i;
     }
     griddep_wait();
-    for (int i = j; i < nk; i += GEMM_PRODUCERS) {
+    for (int i = j; i < nk; i += nprod) {
       const int s = i % STAGES;
       if (i >= STAGES) {      // (a prefetched stage always gets its B tile, so that its barrier completes)
         if (!mbar_wait(&empty[s], (uint32_t)(((i / STAGES) - 1) & 1), p.wait_ns, p.status)) {
@@ -442,7 +446,9 @@ __global__ void __launch_bounds__(GEMM_P_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const bool producer = warp != 1 && warp < 4 && lane == 0;
+  // producers in use: no more than the ring has stages (see the one-tile kernel)
+  const int nprod = min(GEMM_PRODUCERS, STAGES);
+  const bool producer = warp != 1 && warp < 4 && lane == 0 && (warp == 0 ? 0 : warp - 1) < nprod;
   // the activations (B), the gate and the tail may come from the previous kernel of the stream, and the
   // output may still be read by it: everyone waits for it, the producers after their weight prefetch
   if (!producer) griddep_wait();
@@ -476,7 +482,7 @@ __global__ void __launch_bounds__(GEMM_P_THREADS, 1)
     for (int64_t u = blockIdx.x; u < U && g < STAGES; u += gridDim.x) {
       const GemmUnit w = gemm_unit(p, u, BN, total_chunks);
       for (int i = 0; i < w.nk && g < STAGES; ++i, ++g) {
-        if (g % GEMM_PRODUCERS != j) continue;
+        if (g % nprod != j) continue;
         mbar_arrive_expect_tx(&full[g], Cfg::STAGE);
         load_a(w, i, g);
         last_load[g] = g;
@@ -488,7 +494,7 @@ __global__ void __launch_bounds__(GEMM_P_THREADS, 1)
     for (int64_t u = blockIdx.x; u < U && ok; u += gridDim.x) {
       const GemmUnit w = gemm_unit(p, u, BN, total_chunks);
       for (int i = 0; i < w.nk; ++i, ++g) {
-        if (g % GEMM_PRODUCERS != j) continue;
+        if (g % nprod != j) continue;
         const int s = g % STAGES;
         if (g >= STAGES) {    // (a prefetched stage always gets its B tile, so that its barrier completes)
           if (!wait_bar(&empty[s], (uint32_t)(((g / STAGES) - 1) & 1))) { ok = false; break; }
