@@ -104,3 +104,60 @@ def test_out_of_range_append_row_is_skipped_and_reported():
     torch.cuda.synchronize()
     assert M.mla_check_status() == M.MLA_ERR_SHAPE
     assert torch.equal(cache, before)
+
+
+def _with_tiny_wait_limit(fn):
+    """Run fn with a 1 ns wait limit; return the status word it left (MLA_OK or MLA_ERR_TIMEOUT)."""
+    assert M.mla_check_status() == M.MLA_OK
+    try:
+        M.mla_set_wait_limit(1)
+        fn()
+        torch.cuda.synchronize()
+        status = M.mla_check_status()
+    finally:
+        M.mla_set_wait_limit(0)
+    assert status in (M.MLA_OK, M.MLA_ERR_TIMEOUT)
+    return status
+
+
+def test_prefill_attention_with_a_tiny_wait_limit_abandons_cleanly():
+    # the un-absorbed prefill kernel: producer, MMA issuer and eight softmax warps in pairs that share
+    # their rows at a barrier; every path out of an abandoned CTA must meet the same barriers
+    B, S, H, Dh = 2, 640, 2, 128
+    rng = np.random.default_rng(3)
+    q, k, v = (I.round_to(rng.standard_normal((B * S, H * Dh)).astype(np.float32), "bf16") for _ in range(3))
+    out = torch.empty(B * S, H * Dh, dtype=torch.bfloat16, device="cuda")
+    qd, kd, vd = dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16")
+    status = _with_tiny_wait_limit(
+        lambda: M.mla_prefill_attention(qd, kd, vd, None, B, S, H, Dh, 0.0, M.MLA_DECODE_CAUSAL, out))
+    print(f"prefill with a 1 ns wait limit: status {status}")
+    M.mla_prefill_attention(qd, kd, vd, None, B, S, H, Dh, 0.0, M.MLA_DECODE_CAUSAL, out)
+    torch.cuda.synchronize()
+    assert M.mla_check_status() == M.MLA_OK
+    x = np.asarray(q, np.float64).reshape(B, S, H, Dh)
+    kk = np.asarray(k, np.float64).reshape(B, S, H, Dh)
+    vv = np.asarray(v, np.float64).reshape(B, S, H, Dh)
+    ref = np.zeros((B, S, H, Dh))
+    for b in range(B):
+        for h in range(H):
+            sc = x[b, :, h] @ kk[b, :, h].T / np.sqrt(Dh)
+            for i in range(S):
+                ref[b, i, h], _ = O.softmax_attend(sc[i, :i + 1], vv[b, :i + 1, h])
+    assert_close(host(out), ref.reshape(B * S, H * Dh), "bf16", "attention after recovery")
+
+
+@pytest.mark.parametrize("m,n,k", [(4096, 2048, 2048), (64, 9728, 1024)], ids=["persistent", "one-tile"])
+def test_linear_with_a_tiny_wait_limit_abandons_cleanly(m, n, k):
+    # (4096 tokens x 2048 outputs, K 2048: more tiles than SMs and long K, the persistent GEMM with
+    # its epilogue warps; 64 tokens x 9728 outputs: 76 one-tile CTAs without a K split)
+    rng = np.random.default_rng(4)
+    x = I.round_to(rng.standard_normal((m, k)).astype(np.float32), "bf16")
+    w = I.round_to((rng.standard_normal((n, k)) / np.sqrt(k)).astype(np.float32), "bf16")
+    xd, wd = dev(x, "bf16"), dev(w, "bf16")
+    y = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+    status = _with_tiny_wait_limit(lambda: M.mla_linear(xd, wd, m, n, k, 0, y))
+    print(f"linear {m}x{n}x{k} with a 1 ns wait limit: status {status}")
+    M.mla_linear(xd, wd, m, n, k, 0, y)
+    torch.cuda.synchronize()
+    assert M.mla_check_status() == M.MLA_OK
+    assert_close(host(y), O.linear(x, w), "bf16", "linear after recovery")
