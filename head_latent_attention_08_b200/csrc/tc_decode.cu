@@ -876,27 +876,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------------------------
-// combine: 16 CTAs per block (8 rows each); merges the partials of blocks split across clusters and writes
-// zeros / -inf for blocks with nothing to attend to
+// combine: 16 CTAs per block, eight rows each (a warp per row, four float4 of the 512 latent columns per
+// lane); merges the partials of blocks split across clusters and writes zeros / -inf for blocks with
+// nothing to attend to. A lane's loads for one partial slot are independent of each other and of the
+// next slot's, so several are in flight at once.
 // ---------------------------------------------------------------------------------------------
+constexpr int DEC_CB_ROWS = 8;   // rows per combine CTA
+
 __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
   __shared__ int slots[256];
-  __shared__ float wts[8][256];
+  __shared__ float wts[DEC_CB_ROWS][256];
   __shared__ int nsl;
   griddep_wait();
   griddep_launch_dependents();
   const int k = blockIdx.x;
-  const int r0 = blockIdx.y * 8;     // this CTA's 8 rows of the block (one per warp)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.y * DEC_CB_ROWS + warp;           // row within the block
   const int64_t bstart = p.prefix[k], bend = p.prefix[k + 1];
   const int b = k / p.nbps, rb = k % p.nbps;
   const int rows_seq = p.n_q * p.H;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ri = rb * DEC_ROWS + r;
+  const bool row_ok = ri < rows_seq;
+  const int64_t orow = (int64_t)b * rows_seq + ri;
+  float4* dst = reinterpret_cast<float4*>(p.out_lat + orow * DEC_DC);
   if (bend == bstart) {
-    for (int r = r0 + warp; r < r0 + 8; r += 8) {
-      const int ri = rb * DEC_ROWS + r;
-      if (ri >= rows_seq) break;
-      const int64_t orow = (int64_t)b * rows_seq + ri;
-      for (int d = lane; d < DEC_DC; d += 32) p.out_lat[orow * DEC_DC + d] = 0.f;
+    if (row_ok) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dst[lane + 32 * j] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (lane == 0 && p.lse) p.lse[orow] = -INFINITY;
     }
     return;
@@ -917,38 +923,45 @@ __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
     nsl = n;
   }
   __syncthreads();
+  if (!row_ok) return;
   const int n = nsl;
-  for (int r = r0 + warp; r < r0 + 8; r += 8) {
-    const int ri = rb * DEC_ROWS + r;
-    if (ri >= rows_seq) break;
-    float M = -INFINITY;
-    for (int i = lane; i < n; i += 32) M = fmaxf(M, p.m_part[(int64_t)slots[i] * DEC_ROWS + r]);
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float L = 0.f;
-    for (int i = lane; i < n; i += 32) {
-      const float m = p.m_part[(int64_t)slots[i] * DEC_ROWS + r];
-      const float w = m == -INFINITY ? 0.f : ex2(m - M);
-      wts[warp][i] = w;
-      L += w * p.l_part[(int64_t)slots[i] * DEC_ROWS + r];
-    }
-    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-    __syncwarp();
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    const int64_t orow = (int64_t)b * rows_seq + ri;
-    float4* dst = reinterpret_cast<float4*>(p.out_lat + orow * DEC_DC);
-    for (int d4 = lane; d4 < DEC_DC / 4; d4 += 32) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int i = 0; i < n; ++i) {
-        const float w = wts[warp][i];
-        if (w == 0.f) continue;
-        const float4 o = reinterpret_cast<const float4*>(p.o_part + ((int64_t)slots[i] * DEC_ROWS + r) * DEC_DC)[d4];
-        acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
-      }
-      dst[d4] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    }
-    if (lane == 0 && p.lse) p.lse[orow] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
-    __syncwarp();
+  // the row's weights w_i = 2^(m_i - M) and its sum L (slots in index order: the sum does not depend
+  // on timing)
+  float M = -INFINITY;
+  for (int i = lane; i < n; i += 32) M = fmaxf(M, p.m_part[(int64_t)slots[i] * DEC_ROWS + r]);
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float L = 0.f;
+  for (int i = lane; i < n; i += 32) {
+    const float m = p.m_part[(int64_t)slots[i] * DEC_ROWS + r];
+    const float w = m == -INFINITY ? 0.f : ex2(m - M);
+    wts[warp][i] = w;
+    L += w * p.l_part[(int64_t)slots[i] * DEC_ROWS + r];
   }
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+  __syncwarp();
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  float4 acc[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+  for (int i = 0; i < n; ++i) {
+    const float w = wts[warp][i];
+    const float4* src = reinterpret_cast<const float4*>(p.o_part + ((int64_t)slots[i] * DEC_ROWS + r) * DEC_DC);
+    float4 o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o[j] = src[lane + 32 * j];
+    if (w != 0.f) {   // (a slot with no visible position is not used)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc[j].x = fmaf(w, o[j].x, acc[j].x); acc[j].y = fmaf(w, o[j].y, acc[j].y);
+        acc[j].z = fmaf(w, o[j].z, acc[j].z); acc[j].w = fmaf(w, o[j].w, acc[j].w);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    dst[lane + 32 * j] = make_float4(acc[j].x * inv, acc[j].y * inv, acc[j].z * inv, acc[j].w * inv);
+  if (lane == 0 && p.lse) p.lse[orow] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -1097,8 +1110,12 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
   if (st0) return st0;
   int st = a.dr == 0 ? launch_decode_t<0>(tk, tv, tq, p, s) : launch_decode_t<64>(tk, tv, tq, p, s);
   if (st) return st;
-  // 16 CTAs per block (8 rows each): a split block's merge reads 2-3 partial slots of 256 KB
-  return launch_pdl(decode_combine_tc_kernel, dim3((unsigned)t.nblocks, DEC_ROWS / 8), dim3(256), 0, s, p);
+  // Equal-length sequences with one cluster per block and at least one position each: every block is
+  // written whole by its cluster, and nothing is left to combine.
+  const bool equal_blocks = a.total_rows == (int64_t)a.batch * a.max_seqlen && (!a.causal || t.nbps == 1);
+  if (equal_blocks && t.G == t.nblocks && a.max_seqlen > 0) return MLA_OK;
+  // 16 CTAs per block (eight rows each): a split block's merge reads its partial slots of 256 KB
+  return launch_pdl(decode_combine_tc_kernel, dim3((unsigned)t.nblocks, DEC_ROWS / DEC_CB_ROWS), dim3(256), 0, s, p);
 }
 
 }  // namespace mla
