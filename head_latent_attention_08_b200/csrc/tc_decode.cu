@@ -144,7 +144,8 @@ struct DecParams {
   int64_t total_rows;
   int causal;
   float scale_log2;           // kq_scale * log2(e)
-  const int32_t* prefix;      // [nblocks + 1] exclusive prefix of tiles per block
+  const int32_t* prefix;      // [nblocks + 1] exclusive prefix of tiles per block (unless uniform)
+  int uniform_tiles;          // > 0: every block has this many tiles (prefix[k] = k * uniform_tiles)
   int G;                      // clusters
   float* out_lat;
   float* lse;
@@ -186,12 +187,18 @@ __device__ __forceinline__ int block_tiles(int T, int n_q, int H, int rb, int ca
   return (cnt + DEC_BT - 1) / DEC_BT;
 }
 
+// exclusive prefix of tiles per block
+__device__ __forceinline__ int64_t dec_prefix(const DecParams& p, int k) {
+  return p.uniform_tiles > 0 ? (int64_t)k * p.uniform_tiles : (int64_t)p.prefix[k];
+}
+
 // largest k with prefix[k] <= u (the non-empty block that holds unit u, u < prefix[n])
-__device__ __forceinline__ int find_block(const int32_t* prefix, int n, int64_t u) {
-  int lo = 0, hi = n - 1;
+__device__ __forceinline__ int find_block(const DecParams& p, int64_t u) {
+  if (p.uniform_tiles > 0) return (int)(u / p.uniform_tiles);
+  int lo = 0, hi = p.nblocks - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if ((int64_t)prefix[mid] <= u) lo = mid; else hi = mid - 1;
+    if ((int64_t)p.prefix[mid] <= u) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
@@ -224,11 +231,11 @@ struct DecWalk {
   __device__ void begin(const DecParams& p, int64_t u0, int64_t u1_) {
     u = u0;
     u1 = u1_;
-    k = u0 < u1 ? find_block(p.prefix, p.nblocks, u0) : 0;
+    k = u0 < u1 ? find_block(p, u0) : 0;
   }
   __device__ bool next(const DecParams& p, DecSeg& s) {
     if (u >= u1) return false;
-    const int64_t bstart = p.prefix[k], bend = p.prefix[k + 1];
+    const int64_t bstart = dec_prefix(p, k), bend = dec_prefix(p, k + 1);
     const int64_t send = u1 < bend ? u1 : bend;
     s.k = k;
     s.b = k / p.nbps;
@@ -238,7 +245,7 @@ struct DecWalk {
     s.complete = (u == bstart) && (send == bend);
     seq_bounds(p, s.b, s.sstart, s.T);
     u = send;
-    if (u < u1) k = find_block(p.prefix, p.nblocks, u);
+    if (u < u1) k = find_block(p, u);
     return true;
   }
 };
@@ -353,7 +360,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
   griddep_launch_dependents();
   const uint32_t tmem = bars->tmem_base;
 
-  const int64_t U = p.prefix[p.nblocks];
+  const int64_t U = dec_prefix(p, p.nblocks);
   const int64_t u0 = range_start(U, p.G, pair), u1 = range_start(U, p.G, pair + 1);
   const int64_t drain_ns = p.wait_ns > 100000000ull ? p.wait_ns : 100000000ull;
   // a wait that gives up marks the CTA aborted; later waits of the CTA return false at once
@@ -892,7 +899,7 @@ __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
   const int k = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.y * DEC_CB_ROWS + warp;           // row within the block
-  const int64_t bstart = p.prefix[k], bend = p.prefix[k + 1];
+  const int64_t bstart = dec_prefix(p, k), bend = dec_prefix(p, k + 1);
   const int b = k / p.nbps, rb = k % p.nbps;
   const int rows_seq = p.n_q * p.H;
   const int ri = rb * DEC_ROWS + r;
@@ -907,7 +914,7 @@ __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
     }
     return;
   }
-  const int64_t U = p.prefix[p.nblocks];
+  const int64_t U = dec_prefix(p, p.nblocks);
   const int p0 = find_owner(U, p.G, bstart), p1 = find_owner(U, p.G, bend - 1);
   if (p0 == p1) return;   // written whole by one cluster
   if (threadIdx.x == 0) {
@@ -1106,13 +1113,19 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
     const uint32_t box[2] = {64, DEC_ROWS};
     if (!encode_tmap_bf16(&tq, const_cast<void*>(a.q_abs), 2, dims, st, box)) return MLA_ERR_CUDA;
   }
-  int st0 = launch_pdl(decode_plan_kernel, dim3(1), dim3(1024), 0, s, p, const_cast<int32_t*>(p.prefix));
-  if (st0) return st0;
+  // Equal-length sequences (total_rows = batch * max_seqlen with every T_b <= max_seqlen), each block
+  // reading up to the sequence's last position: every block has the same tile count, known here, and
+  // the plan kernel is not needed. With one cluster per block on top, every block is written whole by
+  // its cluster, and nothing is left to combine.
+  const bool equal_blocks = a.total_rows == (int64_t)a.batch * a.max_seqlen && (!a.causal || t.nbps == 1);
+  if (equal_blocks && a.max_seqlen > 0) {
+    p.uniform_tiles = (int)ceil_div(a.max_seqlen, DEC_BT);
+  } else {
+    const int st0 = launch_pdl(decode_plan_kernel, dim3(1), dim3(1024), 0, s, p, const_cast<int32_t*>(p.prefix));
+    if (st0) return st0;
+  }
   int st = a.dr == 0 ? launch_decode_t<0>(tk, tv, tq, p, s) : launch_decode_t<64>(tk, tv, tq, p, s);
   if (st) return st;
-  // Equal-length sequences with one cluster per block and at least one position each: every block is
-  // written whole by its cluster, and nothing is left to combine.
-  const bool equal_blocks = a.total_rows == (int64_t)a.batch * a.max_seqlen && (!a.causal || t.nbps == 1);
   if (equal_blocks && t.G == t.nblocks && a.max_seqlen > 0) return MLA_OK;
   // 16 CTAs per block (eight rows each): a split block's merge reads its partial slots of 256 KB
   return launch_pdl(decode_combine_tc_kernel, dim3((unsigned)t.nblocks, DEC_ROWS / DEC_CB_ROWS), dim3(256), 0, s, p);

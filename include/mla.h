@@ -160,7 +160,7 @@ MLA_API int32_t mla_absorb_weights(const mla_dims* dims, int32_t dtype, int32_t 
 /*
  * mla_decode_workspace_size -- bytes of scratch mla_decode_absorbed needs for these sizes.
  *   batch        number of sequences B;  n_q_per_seq  query tokens per sequence (>= 1);
- *   max_seqlen   an upper bound on every T_b (host-side planning only);
+ *   max_seqlen   an upper bound on every T_b (a requirement: see mla_decode_absorbed);
  *   total_rows   sum of T_b (rows of the packed cache).
  *   dtype MLA_FP8_E4M3 returns the scratch of mla_decode_absorbed_fp8 (for either query dtype).
  */
