@@ -197,7 +197,8 @@ __global__ void __launch_bounds__(128) append_latent_kernel(
     T* __restrict__ cache, const int64_t* __restrict__ row_idx, const float* __restrict__ c_new,
     int64_t c_stride, const float* __restrict__ kpe_new, int64_t kpe_stride,
     const int32_t* __restrict__ positions, int dc, int dr,
-    uint32_t flags, float eps, double log2_theta, int vec8, int64_t cache_rows, int* status, float cache_scale) {
+    uint32_t flags, float eps, double log2_theta, int vec8, int64_t cache_rows, int* status, float cache_scale,
+    int n_parts, int64_t part_stride) {
   extern __shared__ float row[];
   __shared__ float red[4];
   griddep_wait();
@@ -209,10 +210,16 @@ __global__ void __launch_bounds__(128) append_latent_kernel(
     return;
   }
   const int W = dc + dr;
-  const float* c = c_new + (int64_t)k * c_stride;
+  // the new row's values: one array, or the K-split partials of the projection that made them, added
+  // in split order
+  auto value = [&](const float* base, int64_t off) {
+    float v = base[off];
+    for (int q = 1; q < n_parts; ++q) v += base[q * part_stride + off];
+    return v;
+  };
   float ss = 0.f;
   for (int i = threadIdx.x; i < dc; i += blockDim.x) {
-    const float x = c[i];
+    const float x = value(c_new, (int64_t)k * c_stride + i);
     row[i] = x;
     ss = fmaf(x, x, ss);
   }
@@ -225,18 +232,18 @@ __global__ void __launch_bounds__(128) append_latent_kernel(
     for (int i = threadIdx.x; i < dc; i += blockDim.x) row[i] *= inv;
   }
   if (dr > 0) {
-    const float* kp = kpe_new + (int64_t)k * kpe_stride;
+    const int64_t kp = (int64_t)k * kpe_stride;
     if (flags & MLA_APPEND_ROPE) {
       const int32_t pos = positions[k];
       for (int i = threadIdx.x; i < dr / 2; i += blockDim.x) {
         float sn, cs;
         rope_sincos(pos, i, dr, log2_theta, &sn, &cs);
-        const float x0 = kp[2 * i], x1 = kp[2 * i + 1];
+        const float x0 = value(kpe_new, kp + 2 * i), x1 = value(kpe_new, kp + 2 * i + 1);
         row[dc + 2 * i] = fmaf(x0, cs, -x1 * sn);
         row[dc + 2 * i + 1] = fmaf(x0, sn, x1 * cs);
       }
     } else {
-      for (int i = threadIdx.x; i < dr; i += blockDim.x) row[dc + i] = kp[i];
+      for (int i = threadIdx.x; i < dr; i += blockDim.x) row[dc + i] = value(kpe_new, kp + i);
     }
   }
   __syncthreads();
@@ -281,6 +288,14 @@ int append_latent_strided(const mla_dims& d, int32_t cache_dtype, void* cache, i
                           const int64_t* row_idx, const float* c_new, int64_t c_stride, const float* kpe_new,
                           int64_t kpe_stride, const int32_t* positions, int64_t n_new, uint32_t flags,
                           float eps, float theta, cudaStream_t s, float cache_scale) {
+  return append_latent_parts(d, cache_dtype, cache, cache_rows, row_idx, c_new, c_stride, kpe_new, kpe_stride,
+                             positions, n_new, flags, eps, theta, s, cache_scale, 1, 0);
+}
+
+int append_latent_parts(const mla_dims& d, int32_t cache_dtype, void* cache, int64_t cache_rows,
+                        const int64_t* row_idx, const float* c_new, int64_t c_stride, const float* kpe_new,
+                        int64_t kpe_stride, const int32_t* positions, int64_t n_new, uint32_t flags, float eps,
+                        float theta, cudaStream_t s, float cache_scale, int n_parts, int64_t part_stride) {
   int* status = device_status_ptr();
   if (!status) return MLA_ERR_CUDA;
   if (n_new == 0) return MLA_OK;
@@ -294,15 +309,15 @@ int append_latent_strided(const mla_dims& d, int32_t cache_dtype, void* cache, i
     return launch_pdl(append_latent_kernel<__nv_bfloat16>, dim3((unsigned)n_new), dim3(128), smem, s,
                       static_cast<__nv_bfloat16*>(cache), row_idx, c_new, c_stride, kpe_new, kpe_stride,
                       positions, d.kv_lora_rank, d.rope_dim, flags, eps, log2((double)theta), vec8, cache_rows,
-                      status, 1.f);
+                      status, 1.f, n_parts, part_stride);
   if (cache_dtype == MLA_FP8_E4M3)
     return launch_pdl(append_latent_kernel<__nv_fp8_e4m3>, dim3((unsigned)n_new), dim3(128), smem, s,
                       static_cast<__nv_fp8_e4m3*>(cache), row_idx, c_new, c_stride, kpe_new, kpe_stride,
                       positions, d.kv_lora_rank, d.rope_dim, flags, eps, log2((double)theta), 0, cache_rows,
-                      status, cache_scale);
+                      status, cache_scale, n_parts, part_stride);
   append_latent_kernel<float><<<(unsigned)n_new, 128, smem, s>>>(
       static_cast<float*>(cache), row_idx, c_new, c_stride, kpe_new, kpe_stride, positions, d.kv_lora_rank,
-      d.rope_dim, flags, eps, log2((double)theta), vec8, cache_rows, status, 1.f);
+      d.rope_dim, flags, eps, log2((double)theta), vec8, cache_rows, status, 1.f, n_parts, part_stride);
   MLA_LAUNCH_CHECK();
   return MLA_OK;
 }
@@ -317,7 +332,8 @@ constexpr int ROPE_PAIRS_PER_CTA = 1024;
 template <typename T>
 __global__ void __launch_bounds__(256) rope_rows_kernel(const float* __restrict__ src, T* __restrict__ out,
                                                         const int32_t* __restrict__ positions, int H, int dr,
-                                                        int rotate, int vec, double log2_theta) {
+                                                        int rotate, int vec, double log2_theta, int n_parts,
+                                                        int64_t part_stride) {
   extern __shared__ float2 sc[];   // (sin, cos) of pair i
   griddep_wait();
   griddep_launch_dependents();
@@ -340,8 +356,15 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const float* __restrict_
     return make_float2(fmaf(v.x, a.y, -v.y * a.x), fmaf(v.x, a.x, v.y * a.y));
   };
   if (vec && e0 + 3 < pairs) {
-    const float4 u0 = reinterpret_cast<const float4*>(row + e0)[0];
-    const float4 u1 = reinterpret_cast<const float4*>(row + e0)[1];
+    // the source: one array, or the K-split partials of the projection that made it, added in order
+    float4 u0 = reinterpret_cast<const float4*>(row + e0)[0];
+    float4 u1 = reinterpret_cast<const float4*>(row + e0)[1];
+    for (int q = 1; q < n_parts; ++q) {
+      const float4* part = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(row + e0) + q * part_stride);
+      const float4 a = part[0], b = part[1];
+      u0.x += a.x; u0.y += a.y; u0.z += a.z; u0.w += a.w;
+      u1.x += b.x; u1.y += b.y; u1.z += b.z; u1.w += b.w;
+    }
     const float2 r0 = turn(make_float2(u0.x, u0.y), e0), r1 = turn(make_float2(u0.z, u0.w), e0 + 1);
     const float2 r2 = turn(make_float2(u1.x, u1.y), e0 + 2), r3 = turn(make_float2(u1.z, u1.w), e0 + 3);
     if constexpr (sizeof(T) == 2) {
@@ -358,14 +381,19 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const float* __restrict_
     return;
   }
   for (int e = e0; e < min(e0 + 4, pairs); ++e) {
-    const float2 r = turn(row[e], e);
+    float2 v = row[e];
+    for (int q = 1; q < n_parts; ++q) {
+      const float2 a = *reinterpret_cast<const float2*>(reinterpret_cast<const float*>(row + e) + q * part_stride);
+      v.x += a.x; v.y += a.y;
+    }
+    const float2 r = turn(v, e);
     o[2 * e] = from_f32<T>(r.x);
     o[2 * e + 1] = from_f32<T>(r.y);
   }
 }
 
 int rope_rows_launch(int32_t dtype, const float* src, void* out, const int32_t* positions, int64_t n_rows, int H,
-                     int dr, bool rotate, float theta, cudaStream_t s) {
+                     int dr, bool rotate, float theta, cudaStream_t s, int n_parts, int64_t part_stride) {
   if (n_rows <= 0 || dr <= 0) return MLA_OK;
   if (n_rows > 0x7fffffff || dr % 2) return MLA_ERR_SHAPE;
   const size_t smem = (size_t)(dr / 2) * sizeof(float2);
@@ -375,13 +403,14 @@ int rope_rows_launch(int32_t dtype, const float* src, void* out, const int32_t* 
   if (grid.y > 65535u) return MLA_ERR_UNSUPPORTED;
   // 16-byte accesses: every row starts on 16 bytes in both buffers (src fp32 rows of H*dr floats; out
   // rows of H*dr elements) and each thread's 4 pairs do too
-  const int vec = ((int64_t)H * dr) % 8 == 0 && aligned16(src) && aligned16(out);
+  const int vec = ((int64_t)H * dr) % 8 == 0 && aligned16(src) && aligned16(out) && (n_parts == 1 || part_stride % 4 == 0);
   const double l2t = log2((double)theta);
   if (dtype == MLA_BF16)
     return launch_pdl(rope_rows_kernel<__nv_bfloat16>, grid, dim3(256), smem, s, src,
-                      static_cast<__nv_bfloat16*>(out), positions, H, dr, rotate ? 1 : 0, vec, l2t);
+                      static_cast<__nv_bfloat16*>(out), positions, H, dr, rotate ? 1 : 0, vec, l2t, n_parts,
+                      part_stride);
   return launch_pdl(rope_rows_kernel<float>, grid, dim3(256), smem, s, src, static_cast<float*>(out), positions,
-                    H, dr, rotate ? 1 : 0, vec, l2t);
+                    H, dr, rotate ? 1 : 0, vec, l2t, n_parts, part_stride);
 }
 
 // ---------------------------------------------------------------------------------------------

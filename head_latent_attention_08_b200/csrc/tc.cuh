@@ -26,11 +26,17 @@ int tc_out_project(const mla_dims& d, const float* out_lat, const void* w_uv, co
 // input projections of new tokens (bf16 in, fp32 accumulate): c_q = x W_cq^T and q_nope = c_q W_qc^T
 // in bf16, q_r = c_q W_qr^T and kv = x W_dkv^T in fp32; partial = split-K scratch of
 // tc_project_partial_bytes() bytes
+// The KV and rotary-query products come back as `parts` fp32 arrays `stride` floats apart (their
+// K-split partials, to be added in order; one array when the product was not split).
+struct ProjectParts {
+  const float* kv; int kv_parts; int64_t kv_stride;
+  const float* qr; int qr_parts; int64_t qr_stride;
+};
 bool tc_project_supported(const mla_dims& d, int64_t q_rank, int64_t n_rows);
 size_t tc_project_partial_bytes(const mla_dims& d, int64_t q_rank, int64_t n_rows);
 int tc_project(const mla_dims& d, int64_t q_rank, const void* x, const void* w_cq, const void* w_qc,
                const void* w_qr, const void* w_dkv, int64_t n_rows, void* c_q, void* q_nope, float* q_r,
-               float* kv, void* partial, cudaStream_t s);
+               float* kv, void* partial, cudaStream_t s, ProjectParts* parts);
 // attention of un-absorbed heads over whole prompts (bf16, head width 128): q, k, v, out and the
 // optional gate are [B*S, H*128]; out = softmax(scale q k^T, causal or full) v (times the gate)
 bool tc_prefill_supported(int64_t B, int64_t S, int64_t H, int64_t D);

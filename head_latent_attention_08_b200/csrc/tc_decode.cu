@@ -99,7 +99,7 @@ struct DecCfg {
   static constexpr int OFF_BAR = dec_max(S_OFF_K + NK * SUPER, V_OFF_V + NV * UNIT);
   static constexpr int SMEM = OFF_BAR + DEC_BAR_BYTES + 1024;
   static_assert(PSLOT % 1024 == 0, "P slots must keep the 1024-byte swizzle alignment");
-  static_assert(NK >= 2, "a block's query takes two ring slots");
+  static_assert(NK >= 2, "the cache ring needs two slots");
   static_assert(NV >= 2, "the value ring needs two slots");
   static_assert(SMEM <= DEC_SMEM_LIMIT, "shared memory budget");
 };
@@ -160,6 +160,29 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 8 x 8 transpose of 16-byte chunks inside each group of eight lanes: before, lane 8 G + i holds in
+// c[0..7] the eight chunks of one row i of its group; after, c[t] holds chunk i of row t of the group.
+// Three butterfly stages (lane distance 4, 2, 1), each swapping the off-diagonal half of the chunks
+// with the partner lane. The map is its own inverse. It turns one-row-per-lane data (the TMEM
+// 32x32b layout) into stores where eight lanes cover 128 contiguous bytes of a row, and back for loads.
+__device__ __forceinline__ void group8_transpose(uint4 (&c)[8], int lane) {
+#pragma unroll
+  for (int k = 4; k >= 1; k >>= 1) {
+    const bool up = (lane & k) != 0;
+#pragma unroll
+    for (int lo = 0; lo < 8; ++lo) {
+      if (lo & k) continue;
+      const int hi = lo | k;
+      uint4 v = up ? c[lo] : c[hi];
+      v.x = __shfl_xor_sync(0xffffffffu, v.x, k);
+      v.y = __shfl_xor_sync(0xffffffffu, v.y, k);
+      v.z = __shfl_xor_sync(0xffffffffu, v.z, k);
+      v.w = __shfl_xor_sync(0xffffffffu, v.w, k);
+      if (up) c[lo] = v; else c[hi] = v;
+    }
+  }
 }
 
 // sequence bounds clamped to the cache
@@ -384,9 +407,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       // One thread keeps about one TMA instruction in flight at a time, so three threads (warps 0, 2
       // and 3) fill the ring together: a ring slot holds three 32 KB boxes, box b of every slot use is
       // loaded by producer b, and each producer arrives once per use (with its bytes, or without a box).
-      // Every block segment takes two uses for its latent query (boxes of 128 columns, two 128-row TMA
-      // loads each: three in the first use, the last one in the second), then three uses per
-      // 256-position tile: 64-column groups {0, 1, 2}, {3, 4, 5} and {6, 7, 8 (rotary)}.
+      // A 256-position tile takes three uses: 64-column groups {0, 1, 2}, {3, 4, 5} and {6, 7, 8
+      // (rotary)}. The latent query does not pass through the ring (the softmax warps read it), so the
+      // cache stream runs on across block boundaries.
       const int pid = warp == 0 ? 0 : warp - 1;
       DecWalk w;
       w.begin(p, u0, u1);
@@ -407,19 +430,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           mbar_arrive_expect_tx(&bars->qr_full, DEC_ROWS * 128);
           tma_load_2d(sQR, &tq, &bars->qr_full, DEC_DC, qrow);
           ++qr_loads;
-        }
-        for (int qu = 0; qu < 2 && ok; ++qu, ++n) {
-          const int s = take_slot(n);
-          if (s < 0) { ok = false; break; }
-          if (qu == 0 || pid == 0) {
-            const int qb = qu == 0 ? pid : 3;       // 128-column query box
-            uint8_t* dst = sK + s * Cfg::SUPER + (qu == 0 ? pid : 0) * Cfg::BOX;
-            mbar_arrive_expect_tx(&bars->k_full[s], Cfg::BOX);
-            tma_load_2d(dst, &tq, &bars->k_full[s], 128 * qb, qrow);
-            tma_load_2d(dst + Cfg::BOX / 2, &tq, &bars->k_full[s], 128 * qb + 64, qrow);
-          } else {
-            mbar_arrive(&bars->k_full[s]);
-          }
         }
         for (int tt = 0; tt < sg.ntl && ok; ++tt) {
           const int y = (int)(sg.sstart + (int64_t)(sg.tile0 + tt) * DEC_BT);
@@ -459,7 +469,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       int segi = 0;
       bool ok = true;
       while (ok && w.next(p, sg)) {
-        n += 2;               // the segment's query uses (read by the softmax warps)
         if (!wait_bar(&bars->q_tm, (uint32_t)segi & 1u)) { ok = false; break; }
         if (DR && !wait_bar(&bars->qr_full, (uint32_t)segi & 1u)) { ok = false; break; }
         for (int tt = 0; tt < sg.ntl; ++tt, ++g) {
@@ -517,36 +526,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       int segi = 0;
       while (w.next(p, sg)) {
         // ---- the block's latent query into TMEM: rows 32 q .., latent columns [128 cg, 128 cg + 128),
-        // from the segment's query uses (box cg: two 128-row x 64-column TMA boxes, swizzled), once the
-        // previous segment's last QK^T has read the old query
+        // read from global memory (eight lanes per 128-byte row piece, then a lane-group transpose gives
+        // every lane its own row), once the previous segment's last QK^T has read the old query. Rows
+        // past the end of q_abs read as zeros.
         {
-          const int64_t use0 = 2 * (int64_t)segi + 3 * g;          // the segment's first query use
-          const int64_t use = use0 + (cg < 3 ? 0 : 1);
-          const int slot = (int)(use % NK);
-          (void)wait_bar(&bars->k_full[slot], (uint32_t)(use / NK) & 1u);
           if (segi > 0) (void)wait_bar(&bars->q_empty, (uint32_t)(segi - 1) & 1u);
-          tc_fence_after();
-#pragma unroll 1
+          const int64_t r0 = (int64_t)sg.b * p.n_q * p.H + (int64_t)sg.rb * DEC_ROWS + q * 32 + (lane & ~7);
+          uint4 ch[2][8];
+#pragma unroll
+          for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+              const int64_t rr = r0 + t;
+              ch[bx][t] = rr < p.q_rows
+                              ? __ldg(reinterpret_cast<const uint4*>(p.q_abs + rr * p.W + cg * 128 + bx * 64 +
+                                                                     8 * (lane & 7)))
+                              : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
           for (int bx = 0; bx < 2; ++bx) {
-            const uint8_t* src = sK + slot * Cfg::SUPER + (cg < 3 ? cg : 0) * Cfg::BOX + bx * (Cfg::BOX / 2) + row * 128;
+            group8_transpose(ch[bx], lane);
             uint32_t r[32];
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-              const uint4 x = *reinterpret_cast<const uint4*>(src + ((c ^ (row & 7)) * 16));
-              r[4 * c] = x.x; r[4 * c + 1] = x.y; r[4 * c + 2] = x.z; r[4 * c + 3] = x.w;
+              r[4 * c] = ch[bx][c].x; r[4 * c + 1] = ch[bx][c].y; r[4 * c + 2] = ch[bx][c].z; r[4 * c + 3] = ch[bx][c].w;
             }
             tmem_st32(tQ + lane_off + cg * 64 + bx * 32, r);
           }
           tmem_wait_st();
           tc_fence_before();
-          fence_proxy_async_smem();     // these generic reads come before the slots' next TMA fills
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars->q_tm);
-          named_bar_sync(5, 32 * DEC_SW);   // every softmax warp has read its slot: the slots go back
-          if (w16 == 0 && lane == 0 && !*abort_flag) {
-            mbar_arrive(&bars->k_empty[use0 % NK]);
-            mbar_arrive(&bars->k_empty[(use0 + 1) % NK]);
-          }
         }
         const int cnt = row_count(sg.T, p.n_q, p.H, sg.rb * DEC_ROWS + row, p.causal);
         float m_ref = -INFINITY, l = 0.f;
@@ -837,19 +847,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
               const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
               const float mul = sg.complete ? inv : 1.f;
               float* dst = sg.complete ? p.out_lat + orow * DEC_DC : p.o_part + ((int64_t)slotp * DEC_ROWS + row) * DEC_DC;
-              const bool write = ok && (sg.complete ? ri < rows_seq : true);
+              // each lane scales its own row; after the lane-group transpose, store t of a lane goes to
+              // row 8 (lane / 8) + t of the warp's rows, columns 4 (lane % 8) .. of the 32 just read, so
+              // eight lanes write 128 contiguous bytes of one row
+              const int gfirst = q * 32 + (lane & ~7);               // first row of the lane's group
+              float* gdst = dst + (int64_t)(gfirst - row) * DEC_DC + cv * 128 + 4 * (lane & 7);
+              const int grows = !ok ? 0 : (sg.complete ? min(8, rows_seq - (sg.rb * DEC_ROWS + gfirst)) : 8);
 #pragma unroll 1
-              for (int cc = 0; cc < 128; cc += 16) {
-                uint32_t r[16];
-                tmem_ld16(tcol + cc, r);
+              for (int cc = 0; cc < 128; cc += 32) {
+                uint32_t r[32];
+                tmem_ld32(tcol + cc, r);
                 tmem_wait_ld();
-                if (write) {
-                  float4* d4 = reinterpret_cast<float4*>(dst + cv * 128 + cc);
+                uint4 ch[8];
 #pragma unroll
-                  for (int c = 0; c < 4; ++c)
-                    d4[c] = make_float4(__uint_as_float(r[4 * c]) * mul, __uint_as_float(r[4 * c + 1]) * mul,
-                                        __uint_as_float(r[4 * c + 2]) * mul, __uint_as_float(r[4 * c + 3]) * mul);
-                }
+                for (int c = 0; c < 8; ++c)
+                  ch[c] = make_uint4(__float_as_uint(__uint_as_float(r[4 * c]) * mul),
+                                     __float_as_uint(__uint_as_float(r[4 * c + 1]) * mul),
+                                     __float_as_uint(__uint_as_float(r[4 * c + 2]) * mul),
+                                     __float_as_uint(__uint_as_float(r[4 * c + 3]) * mul));
+                group8_transpose(ch, lane);
+#pragma unroll
+                for (int t = 0; t < 8; ++t)
+                  if (t < grows) *reinterpret_cast<uint4*>(gdst + (int64_t)t * DEC_DC + cc) = ch[t];
               }
               if (ok && cv == 0) {
                 if (sg.complete) {

@@ -724,10 +724,12 @@ struct GemmTail {
   int cols = 0;
 };
 
+// sum_partials = false: a K-split product leaves its fp32 partials [split][batch][N][M] in partial_ws for
+// the consumer to add in split order (the consumer then reads partial_ws with gemm_splits() parts)
 static int tc_gemm(const GemmOperand& A, bool a_mn, const GemmOperand& Bop, int M, int N, int K, int batch,
                    void* out, int64_t out_sb, int64_t out_st, bool out_f32, const void* gate, int64_t gate_sb,
                    int64_t gate_st, bool sigmoid, void* partial_ws, cudaStream_t s,
-                   const GemmTail& tail = GemmTail()) {
+                   const GemmTail& tail = GemmTail(), bool sum_partials = true) {
   // a K-major A may end inside its last 128-row tile (the TMA zero-fills the rows past M and the
   // epilogue skips them); an MN-major A loads its rows as 64-wide boxes and takes whole tiles only
   if (M <= 0 || M % 4 || (a_mn && M % 128) || K % 64 || N <= 0 || batch <= 0) return MLA_ERR_UNSUPPORTED;
@@ -778,7 +780,7 @@ static int tc_gemm(const GemmOperand& A, bool a_mn, const GemmOperand& Bop, int 
                                   : launch_gemm_t<256, false>(ta, tb, p, s, pk);
   }
   if (st) return st;
-  if (g.splits > 1) {
+  if (g.splits > 1 && sum_partials) {
     const int64_t per = (int64_t)batch * N * M;
     const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(per / 4, 128), 16 * sm_count());
     st = launch_pdl(splitk_reduce_kernel, dim3(blocks), dim3(128), 0, s, (const float*)p.partial, g.splits, batch,
@@ -880,20 +882,39 @@ static void project_gemm_dims(const mla_dims& d, int64_t q_rank, int64_t n_rows,
   }
 }
 
-size_t tc_project_partial_bytes(const mla_dims& d, int64_t q_rank, int64_t n_rows) {
+// split-K scratch of the four products, one region each: the KV and rotary-query partials are read
+// later, by the append and the rotation
+static void project_partial_offsets(const mla_dims& d, int64_t q_rank, int64_t n_rows, size_t off[5]) {
   int g[4][3];
   project_gemm_dims(d, q_rank, n_rows, g);
-  size_t b = 0;
-  for (int i = 0; i < 4; ++i)
-    if (g[i][0] > 0) b = std::max(b, gemm_partial_bytes(g[i][0], g[i][1], g[i][2], 1));
-  return b;
+  off[0] = 0;
+  for (int i = 0; i < 4; ++i) off[i + 1] = off[i] + (g[i][0] > 0 ? gemm_partial_bytes(g[i][0], g[i][1], g[i][2], 1) : 0);
+}
+
+size_t tc_project_partial_bytes(const mla_dims& d, int64_t q_rank, int64_t n_rows) {
+  size_t off[5];
+  project_partial_offsets(d, q_rank, n_rows, off);
+  return off[4];
 }
 
 int tc_project(const mla_dims& d, int64_t q_rank, const void* x, const void* w_cq, const void* w_qc,
                const void* w_qr, const void* w_dkv, int64_t n_rows, void* c_q, void* q_nope, float* q_r,
-               float* kv, void* partial, cudaStream_t s) {
+               float* kv, void* partial, cudaStream_t s, ProjectParts* parts) {
   int g[4][3];
   project_gemm_dims(d, q_rank, n_rows, g);
+  size_t off[5];
+  project_partial_offsets(d, q_rank, n_rows, off);
+  char* pw = static_cast<char*>(partial);
+  // the rotary-query product leaves its K-split partials to the rotation, which adds them in order
+  // (the KV product keeps its own reduce: the append runs one block per token and would read the
+  // partials with too few threads)
+  const int qr_splits = g[2][0] > 0 ? plan_gemm(g[2][0], g[2][1], g[2][2], 1, 1 << 20).splits : 1;
+  parts->kv = kv;
+  parts->kv_parts = 1;
+  parts->kv_stride = 0;
+  parts->qr = qr_splits > 1 ? reinterpret_cast<const float*>(pw + off[2]) : q_r;
+  parts->qr_parts = qr_splits;
+  parts->qr_stride = (int64_t)g[2][1] * g[2][0];
   const int64_t D = d.d_model;
   auto weight = [](const void* w, int64_t rows, int64_t k) {
     return GemmOperand{const_cast<void*>(w), (uint64_t)k, (uint64_t)rows, 1, (uint64_t)(k * 2),
@@ -905,17 +926,17 @@ int tc_project(const mla_dims& d, int64_t q_rank, const void* x, const void* w_c
                        (uint64_t)(n_rows * q_rank * 2)};
   // the KV down-projection, then the query chain (c_q feeds the last two products)
   int st = tc_gemm(weight(w_dkv, g[3][0], D), false, bx, g[3][0], g[3][1], g[3][2], 1, kv, 0, g[3][0], true,
-                   nullptr, 0, 0, false, partial, s);
+                   nullptr, 0, 0, false, pw + off[3], s);
   if (st) return st;
   if ((st = tc_gemm(weight(w_cq, g[0][0], D), false, bx, g[0][0], g[0][1], g[0][2], 1, c_q, 0, g[0][0], false,
-                    nullptr, 0, 0, false, partial, s)))
+                    nullptr, 0, 0, false, pw + off[0], s)))
     return st;
   if ((st = tc_gemm(weight(w_qc, g[1][0], q_rank), false, bq, g[1][0], g[1][1], g[1][2], 1, q_nope, 0, g[1][0],
-                    false, nullptr, 0, 0, false, partial, s)))
+                    false, nullptr, 0, 0, false, pw + off[1], s)))
     return st;
   if (g[2][0] > 0)
     st = tc_gemm(weight(w_qr, g[2][0], q_rank), false, bq, g[2][0], g[2][1], g[2][2], 1, q_r, 0, g[2][0], true,
-                 nullptr, 0, 0, false, partial, s);
+                 nullptr, 0, 0, false, pw + off[2], s, GemmTail(), false);
   return st;
 }
 
