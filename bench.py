@@ -621,14 +621,16 @@ def run_rows(args):
     report("f2 + a1..a5 whole step from x (mla_decode_step)", c3 + " q_rank1536 d_model5120", ms,
            B * T * (dc + dr) * 2 + 2 * (proj_w + H * n * dc + H * dv * dc + D * H * dv),
            B * H * T * (2 * (dc + dr) + 2 * dc) + 2 * B * (proj_w + H * (n * dc + dv * dc) + D * H * dv))
-    # ---- f1: the same decode over an e4m3 cache (half the bytes; CUDA cores) ---------------------------
+    # ---- f1: the same decode over an e4m3 cache (half the bytes; tensor cores with a bf16 query) --------
     codes = cache.view(torch.uint16)[:, : (dc + dr) // 2].contiguous().view(torch.uint8)   # any finite codes
     codes = (codes & 0x77)                                                                 # |value| <= 240
     ws8 = M.workspace(M.mla_decode_workspace_size(d, torch.uint8, B, 1, T, B * T, M.MLA_DECODE_CAUSAL), dev)
     ms = timed(lambda: M.mla_decode_absorbed_fp8(d, step.q_abs, codes, 1.0, cu, B, 1, T, M.MLA_DECODE_CAUSAL,
-                                                 step.out_lat, step.lse, ws8), reps=3)
-    report("f1 decode over an e4m3 cache (CUDA cores)", c3, ms, B * T * (dc + dr), B * H * T * (2 * (dc + dr) + 2 * dc),
-           "bf16 query, fp32 arithmetic; bytes = the e4m3 cache")
+                                                 step.out_lat, step.lse, ws8))
+    report("f1 decode over an e4m3 cache (tensor cores)", c3, ms, B * T * (dc + dr),
+           B * H * T * (2 * (dc + dr) + 2 * dc),
+           "bf16 query split into two e4m3 parts for QK^T, P.C in bf16 over the converted codes; bytes = the e4m3 "
+           "cache; FLOPs counted once (the two query parts double the QK^T MMAs at twice the bf16 rate)")
     del codes, ws8
     del cache, step, w_o, layer, w_qc, w_qr
     torch.cuda.empty_cache()

@@ -155,6 +155,7 @@ struct DecodeArgs {
   float* out_lat; float* lse;
   void* workspace; size_t workspace_bytes;
   float cache_scale = 1.f;               // an e4m3 cache holds value / cache_scale
+  bool cache_f8 = false;                 // the cache is e4m3 (tensor-core decode with a bf16 query)
 };
 
 size_t decode_generic_workspace(const DecodeArgs& a);

@@ -198,8 +198,12 @@ int32_t mla_decode_workspace_size(const mla_dims* dims, int32_t dtype, int32_t b
   int st = check_decode_sizes(dims, fp8 ? MLA_F32 : dtype, batch, n_q, max_seqlen, total_rows, flags);
   if (st) return st;
   DecodeArgs a = make_decode_args(dims, batch, n_q, max_seqlen, total_rows, flags);
-  if (fp8)
+  if (fp8) {
+    // the CUDA-core decode (an fp32 query) or the tensor-core one (a bf16 query): room for either
+    a.cache_f8 = true;
     *bytes = decode_generic_workspace(a);
+    if (tc_decode_supported(a)) *bytes = std::max(*bytes, tc_decode_workspace(a));
+  }
   else if (dtype == MLA_BF16 && tc_decode_supported(a))
     *bytes = tc_decode_workspace(a);
   else
@@ -245,6 +249,11 @@ int32_t mla_decode_absorbed_fp8(const mla_dims* dims, int32_t q_dtype, const voi
   a.q_abs = q_abs; a.cache = cache; a.cu_seqlens = cu_seqlens;
   a.out_lat = out_lat; a.lse = lse; a.workspace = workspace; a.workspace_bytes = workspace_bytes;
   a.cache_scale = cache_scale;
+  a.cache_f8 = true;
+  if (q_dtype == MLA_BF16 && tc_decode_supported(a)) {
+    if (workspace_bytes < tc_decode_workspace(a) || !workspace) return MLA_ERR_WORKSPACE;
+    return tc_decode_launch(a, as_stream(stream));
+  }
   if (workspace_bytes < decode_generic_workspace(a)) return MLA_ERR_WORKSPACE;
   return decode_generic_launch(a, q_dtype, as_stream(stream), MLA_FP8_E4M3);
 }

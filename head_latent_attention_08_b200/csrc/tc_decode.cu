@@ -70,16 +70,24 @@ constexpr int DEC_BAR_BYTES = 1024;
 __host__ __device__ constexpr int dec_round1024(int x) { return (x + 1023) / 1024 * 1024; }
 __host__ __device__ constexpr int dec_max(int a, int b) { return a > b ? a : b; }
 
-template <int DR>
+// F8: the cache holds e4m3 codes (one byte per value). The score CTA then streams 128-column boxes
+// (still 128-byte rows) and runs QK^T as e4m3 MMAs against a query split into e4m3 high and low parts;
+// the value CTA stages its 256-column units as e4m3 and converts them to bf16 (exactly) for P.C.
+template <int DR, bool F8 = false>
 struct DecCfg {
   static constexpr int DATA_LIMIT = DEC_SMEM_LIMIT - 1024 - DEC_BAR_BYTES;   // 1 KB for alignment
-  static constexpr int NB = 8 + (DR ? 1 : 0);              // 64-column boxes of a cache row
-  static constexpr int BOX = DEC_BT * 128;                 // 256 positions x 64 columns bf16: 32 KB
+  static constexpr int BOXW = F8 ? 128 : 64;               // cache columns per box (128-byte rows)
+  static constexpr int NB_LAT = DEC_DC / BOXW;             // latent boxes of a cache row
+  static constexpr int NB = NB_LAT + (DR ? 1 : 0);         // + the rotary box (e4m3: half past the row,
+                                                           // read as zeros)
+  static constexpr int PARTS = (NB + 2) / 3;               // ring uses per tile
+  static constexpr int BOX = DEC_BT * 128;                 // 256 positions x 128 bytes: 32 KB
   // score CTA
-  static constexpr int S_OFF_QR = 0;                       // rotary query [128 rows x 64 columns]
+  static constexpr int S_OFF_QR = 0;                       // rotary query [128 rows x 128 B]
   static constexpr int S_QR = DR ? DEC_ROWS * 128 : 0;
-  static constexpr int S_OFF_RED = S_OFF_QR + S_QR;        // row maxima [2][4][128], row sums [4][128]
-  static constexpr int S_OFF_K = dec_round1024(S_OFF_RED + 12 * DEC_ROWS * 4);
+  static constexpr int S_OFF_RED = S_OFF_QR + S_QR;        // row maxima [2][4][128], row sums [4][128],
+                                                           // query maxima [4][128]
+  static constexpr int S_OFF_K = dec_round1024(S_OFF_RED + 16 * DEC_ROWS * 4);
   static constexpr int SUPER = 3 * BOX;                    // ring slot: three boxes (12 MMAs per wait)
   static constexpr int NK = (DATA_LIMIT - S_OFF_K) / SUPER;  // ring slots
   // value CTA
@@ -95,12 +103,17 @@ struct DecCfg {
   static constexpr int V_OFF_P = 0;
   static constexpr int V_OFF_V = dec_round1024(DEC_NPH * PSLOT);
   static constexpr int UNIT = DEC_HT * 512;                // 64 positions x 256 latent columns bf16: 32 KB
-  static constexpr int NV = (DATA_LIMIT - V_OFF_V) / UNIT;  // value slots (256 latent columns each)
-  static constexpr int OFF_BAR = dec_max(S_OFF_K + NK * SUPER, V_OFF_V + NV * UNIT);
+  static constexpr int FUNIT = DEC_HT * 256;               // the same in e4m3: 16 KB
+  static constexpr int NV = F8 ? 2 : (DATA_LIMIT - V_OFF_V) / UNIT;   // bf16 value slots
+  static constexpr int V_OFF_F = V_OFF_V + NV * UNIT;      // e4m3 staging slots
+  static constexpr int NF = F8 ? (DATA_LIMIT - V_OFF_F) / FUNIT : 0;
+  static constexpr int OFF_BAR = dec_max(S_OFF_K + NK * SUPER, V_OFF_F + NF * FUNIT);
   static constexpr int SMEM = OFF_BAR + DEC_BAR_BYTES + 1024;
   static_assert(PSLOT % 1024 == 0, "P slots must keep the 1024-byte swizzle alignment");
   static_assert(NK >= 2, "the cache ring needs two slots");
   static_assert(NV >= 2, "the value ring needs two slots");
+  static_assert(!F8 || NF >= 2, "the e4m3 staging ring needs two slots");
+  static_assert(!F8 || NF <= 4, "barrier block");
   static_assert(SMEM <= DEC_SMEM_LIMIT, "shared memory budget");
 };
 
@@ -115,7 +128,7 @@ struct DecSide {
 };
 static_assert(sizeof(DecSide) == 512, "side record size");
 
-template <int NK, int NV>
+template <int NK, int NV, int NF>
 struct DecBars {
   // score CTA
   uint64_t k_full[NK], k_empty[NK];
@@ -123,7 +136,8 @@ struct DecBars {
   uint64_t s_full, s_empty;       // the S slot: computed (QK^T commit) / read out (softmax warps)
   uint64_t p_empty[DEC_NPH];      // arrived by the value CTA: a P slot may be written again
   // value CTA
-  uint64_t v_full[NV], v_empty[NV];
+  uint64_t v_full[NV], v_empty[NV];   // (e4m3 cache: v_full = converted to bf16 by the rescale warps)
+  uint64_t f_full[NF > 0 ? NF : 1], f_empty[NF > 0 ? NF : 1];   // e4m3 staging slots
   uint64_t p_full[DEC_NPH];       // P + side data landed (transaction count of the bulk copies)
   uint64_t pfree[DEC_NPH];        // P.C read the slot and the rescale/epilogue warps read its side data
   uint64_t o_fix, fix_done;       // rescale hand-shake (one phase per rescale)
@@ -154,6 +168,7 @@ struct DecParams {
   float* l_part;              // [2G][128] sums
   int* status;
   unsigned long long wait_ns;
+  float cache_scale;          // e4m3 cache: value = code * cache_scale
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -183,6 +198,46 @@ __device__ __forceinline__ void group8_transpose(uint4 (&c)[8], int lane) {
       if (up) c[lo] = v; else c[hi] = v;
     }
   }
+}
+
+// four e4m3 codes (consecutive bytes of x) -> four bf16 values (exact: every e4m3 value is a bf16 value)
+__device__ __forceinline__ uint2 e4m3x4_to_bf16x4(uint32_t x) {
+  const __half2_raw h0 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(x & 0xFFFFu), __NV_E4M3);
+  const __half2_raw h1 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(x >> 16), __NV_E4M3);
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+  const __nv_bfloat162 r0 = __floats2bfloat162_rn(a.x, a.y), r1 = __floats2bfloat162_rn(b.x, b.y);
+  return make_uint2(*reinterpret_cast<const uint32_t*>(&r0), *reinterpret_cast<const uint32_t*>(&r1));
+}
+
+// eight bf16 values (v) times a power of two (p2) as e4m3 high and low parts: hi = e4m3(x),
+// lo = e4m3(x - hi), so that hi + lo is x to about 2^-8 relative (both rounded to nearest, saturating);
+// four codes per 32-bit word in element order
+__device__ __forceinline__ void e4m3_split8(uint4 v, float p2, uint32_t& h0, uint32_t& h1, uint32_t& l0,
+                                            uint32_t& l1) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t hs[4], ls[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = make_float2(__uint_as_float(w[e] << 16) * p2, __uint_as_float(w[e] & 0xFFFF0000u) * p2);
+    const __nv_fp8x2_storage_t h = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(h, __NV_E4M3);
+    const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+    const __nv_fp8x2_storage_t l =
+        __nv_cvt_float2_to_fp8x2(make_float2(f.x - hf.x, f.y - hf.y), __NV_SATFINITE, __NV_E4M3);
+    hs[e] = h;
+    ls[e] = l;
+  }
+  h0 = hs[0] | (hs[1] << 16); h1 = hs[2] | (hs[3] << 16);
+  l0 = ls[0] | (ls[1] << 16); l1 = ls[2] | (ls[3] << 16);
+}
+
+__device__ __forceinline__ float bf16x8_absmax(uint4 v, float m) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[e] << 16)), fabsf(__uint_as_float(w[e] & 0xFFFF0000u))));
+  return m;
 }
 
 // sequence bounds clamped to the cache
@@ -310,16 +365,17 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecParams p, int32_t*
 // ---------------------------------------------------------------------------------------------
 // the decode kernel
 // ---------------------------------------------------------------------------------------------
-template <int DR>
+template <int DR, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                      const __grid_constant__ CUtensorMap tq, DecParams p) {
-  using Cfg = DecCfg<DR>;
+  using Cfg = DecCfg<DR, F8>;
   constexpr int NK = Cfg::NK;
   constexpr int NV = Cfg::NV;
+  constexpr int NF = Cfg::NF;
   constexpr int NB = Cfg::NB;
   constexpr int NPH = DEC_NPH;
-  using Bars = DecBars<NK, NV>;
+  using Bars = DecBars<NK, NV, NF>;
   static_assert(sizeof(Bars) <= DEC_BAR_BYTES, "barrier block");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -345,8 +401,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       for (int s = 0; s < NPH; ++s) mbar_init(&bars->p_empty[s], 1);
     } else {
       for (int s = 0; s < NV; ++s) {
-        mbar_init(&bars->v_full[s], 1);
+        mbar_init(&bars->v_full[s], F8 ? DEC_SW : 1);   // e4m3: one arrival per converting warp
         mbar_init(&bars->v_empty[s], 1);
+      }
+      for (int s = 0; s < NF; ++s) {
+        mbar_init(&bars->f_full[s], 1);
+        mbar_init(&bars->f_empty[s], DEC_SW);
       }
       for (int s = 0; s < NPH; ++s) {
         mbar_init(&bars->p_full[s], 1);
@@ -424,7 +484,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       };
       while (ok && w.next(p, sg)) {
         const int qrow = (int)((int64_t)sg.b * p.n_q * p.H + (int64_t)sg.rb * DEC_ROWS);
-        if (DR && pid == 0) {
+        if (DR && !F8 && pid == 0) {
           // the rotary query of this segment, once the previous segment's last QK^T has read the old one
           if (segi > 0 && !wait_bar(&bars->q_empty, (uint32_t)(segi - 1) & 1u)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars->qr_full, DEC_ROWS * 128);
@@ -433,13 +493,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         }
         for (int tt = 0; tt < sg.ntl && ok; ++tt) {
           const int y = (int)(sg.sstart + (int64_t)(sg.tile0 + tt) * DEC_BT);
-          for (int part = 0; part < 3; ++part, ++n) {
+          for (int part = 0; part < Cfg::PARTS; ++part, ++n) {
             const int s = take_slot(n);
             if (s < 0) { ok = false; break; }
-            const int j = 3 * part + pid;           // 64-column group of the cache row
+            const int j = 3 * part + pid;           // column box of the cache row
             if (j < NB) {
               mbar_arrive_expect_tx(&bars->k_full[s], Cfg::BOX);
-              tma_load_2d(sK + s * Cfg::SUPER + pid * Cfg::BOX, &tk, &bars->k_full[s], 64 * j, y);
+              tma_load_2d(sK + s * Cfg::SUPER + pid * Cfg::BOX, &tk, &bars->k_full[s], Cfg::BOXW * j, y);
             } else {
               mbar_arrive(&bars->k_full[s]);
             }
@@ -460,6 +520,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       // twelve MMAs) is released by one commit as soon as its MMAs complete; the next tile's QK^T waits
       // only for the softmax warps to have read the S slot out.
       constexpr uint32_t idesc = idesc_bf16_f32(128, DEC_BT, false, false);
+      constexpr uint32_t idesc8 = idesc_e4m3_f32(128, DEC_BT);
       const uint64_t kd0 = smem_desc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t qd0 = smem_desc_sw128(smem_u32(sQR), 16, 1024);
       DecWalk w;
@@ -470,11 +531,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       bool ok = true;
       while (ok && w.next(p, sg)) {
         if (!wait_bar(&bars->q_tm, (uint32_t)segi & 1u)) { ok = false; break; }
-        if (DR && !wait_bar(&bars->qr_full, (uint32_t)segi & 1u)) { ok = false; break; }
+        if (DR && !F8 && !wait_bar(&bars->qr_full, (uint32_t)segi & 1u)) { ok = false; break; }
         for (int tt = 0; tt < sg.ntl; ++tt, ++g) {
           if (g >= 1 && !wait_bar(&bars->s_empty, (uint32_t)(g - 1) & 1u)) { ok = false; break; }
           tc_fence_after();
-          for (int part = 0; part < 3; ++part, ++n) {
+          for (int part = 0; part < Cfg::PARTS; ++part, ++n) {
             const int s = (int)(n % NK);
             if (!wait_bar(&bars->k_full[s], (uint32_t)(n / NK) & 1u)) { ok = false; break; }
             tc_fence_after();
@@ -483,7 +544,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
               const int j = 3 * part + b;
               if (j >= NB) break;
               const uint64_t kd = kd0 + (uint64_t)((s * Cfg::SUPER + b * Cfg::BOX) >> 4);
-              if (j < 8) {
+              if constexpr (F8) {
+                // e4m3: K = 32 per MMA; the query's high part (TMEM columns [0, 128)) and low part
+                // (columns [128, 256)) against the same codes; the rotary tile holds the high part in bytes
+                // 0..63 of each row and the low part in bytes 64..127
+                if (j < Cfg::NB_LAT) {
+#pragma unroll
+                  for (int kk = 0; kk < 4; ++kk) {
+                    mma_e4m3_ts(tS, tQ + j * 32 + kk * 8, kd + (uint64_t)(kk * 2), idesc8, (j | kk) ? 1u : 0u);
+                    mma_e4m3_ts(tS, tQ + 128 + j * 32 + kk * 8, kd + (uint64_t)(kk * 2), idesc8, 1u);
+                  }
+                } else {
+#pragma unroll
+                  for (int kk = 0; kk < 2; ++kk) {
+                    mma_e4m3_ss(tS, qd0 + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2), idesc8, 1u);
+                    mma_e4m3_ss(tS, qd0 + (uint64_t)((kk + 2) * 2), kd + (uint64_t)(kk * 2), idesc8, 1u);
+                  }
+                }
+              } else if (j < 8) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                   mma_bf16_ts(tS, tQ + j * 32 + kk * 8, kd + (uint64_t)(kk * 2), idesc, (j | kk) ? 1u : 0u);
@@ -529,23 +607,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         // read from global memory (eight lanes per 128-byte row piece, then a lane-group transpose gives
         // every lane its own row), once the previous segment's last QK^T has read the old query. Rows
         // past the end of q_abs read as zeros.
-        {
-          if (segi > 0) (void)wait_bar(&bars->q_empty, (uint32_t)(segi - 1) & 1u);
-          const int64_t r0 = (int64_t)sg.b * p.n_q * p.H + (int64_t)sg.rb * DEC_ROWS + q * 32 + (lane & ~7);
+        float sl2 = p.scale_log2;       // score -> log2-domain logit
+        if (segi > 0) (void)wait_bar(&bars->q_empty, (uint32_t)(segi - 1) & 1u);
+        const int64_t r0 = (int64_t)sg.b * p.n_q * p.H + (int64_t)sg.rb * DEC_ROWS + q * 32 + (lane & ~7);
+        auto load_half = [&](int bx, uint4 (&ch)[8]) {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int64_t rr = r0 + t;
+            ch[t] = rr < p.q_rows ? __ldg(reinterpret_cast<const uint4*>(p.q_abs + rr * p.W + cg * 128 + bx * 64 +
+                                                                        8 * (lane & 7)))
+                                  : make_uint4(0u, 0u, 0u, 0u);
+          }
+          group8_transpose(ch, lane);
+        };
+        if constexpr (!F8) {
           uint4 ch[2][8];
-#pragma unroll
-          for (int bx = 0; bx < 2; ++bx)
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              const int64_t rr = r0 + t;
-              ch[bx][t] = rr < p.q_rows
-                              ? __ldg(reinterpret_cast<const uint4*>(p.q_abs + rr * p.W + cg * 128 + bx * 64 +
-                                                                     8 * (lane & 7)))
-                              : make_uint4(0u, 0u, 0u, 0u);
-            }
+          load_half(0, ch[0]);
+          load_half(1, ch[1]);
 #pragma unroll
           for (int bx = 0; bx < 2; ++bx) {
-            group8_transpose(ch[bx], lane);
             uint32_t r[32];
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -555,9 +635,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           }
           tmem_wait_st();
           tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->q_tm);
+        } else {
+          // e4m3 cache: the row times a power of two p2 (its largest magnitude lands in (224, 448]) as
+          // e4m3 high and low parts; latent high part into TMEM columns [32 cg, 32 cg + 32), low part
+          // 128 columns further; the warp's 16 rotary columns [16 cg, 16 cg + 16) into the rotary tile
+          // (high: 16-byte chunk cg of the row, low: chunk 4 + cg, swizzled). The scores are then in
+          // units of 1 / p2 / cache_scale.
+          const int64_t own = r0 - (lane & ~7) + lane;
+          uint4 rp[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+          if (DR && own < p.q_rows) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.q_abs + own * p.W + DEC_DC + 16 * cg);
+            rp[0] = __ldg(src);
+            rp[1] = __ldg(src + 1);
+          }
+          float amax = bf16x8_absmax(rp[1], bf16x8_absmax(rp[0], 0.f));
+#pragma unroll 1
+          for (int bx = 0; bx < 2; ++bx) {
+            uint4 ch[8];
+            load_half(bx, ch);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) amax = bf16x8_absmax(ch[c], amax);
+          }
+          float* qmx = red + 12 * DEC_ROWS;
+          qmx[cg * DEC_ROWS + row] = amax;
+          named_bar_sync(1 + q, 128);         // the four warps of these rows
+          const float rmax = fmaxf(fmaxf(qmx[row], qmx[DEC_ROWS + row]), fmaxf(qmx[2 * DEC_ROWS + row], qmx[3 * DEC_ROWS + row]));
+          // largest power of two p2 with rmax * p2 <= 448 (kept within the normal range)
+          const float p2 = rmax > 0.f ? __uint_as_float(__float_as_uint(fminf(448.f / rmax, 0x1p100f)) & 0x7F800000u)
+                                      : 1.f;
+          sl2 = p.scale_log2 * p.cache_scale / p2;
+#pragma unroll 1
+          for (int bx = 0; bx < 2; ++bx) {
+            uint4 ch[8];
+            load_half(bx, ch);
+            uint32_t hi[16], lo[16];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) e4m3_split8(ch[c], p2, hi[2 * c], hi[2 * c + 1], lo[2 * c], lo[2 * c + 1]);
+            tmem_st16(tQ + lane_off + cg * 32 + bx * 16, hi);
+            tmem_st16(tQ + lane_off + 128 + cg * 32 + bx * 16, lo);
+          }
+          if (DR) {
+            uint4 h, lw;
+            e4m3_split8(rp[0], p2, h.x, h.y, lw.x, lw.y);
+            e4m3_split8(rp[1], p2, h.z, h.w, lw.z, lw.w);
+            uint8_t* qrow = sQR + row * 128;
+            *reinterpret_cast<uint4*>(qrow + ((cg ^ (row & 7)) << 4)) = h;
+            *reinterpret_cast<uint4*>(qrow + (((4 + cg) ^ (row & 7)) << 4)) = lw;
+            fence_proxy_async_smem();   // generic stores read by the MMAs (async proxy)
+          }
+          tmem_wait_st();
+          tc_fence_before();
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->q_tm);
         const int cnt = row_count(sg.T, p.n_q, p.H, sg.rb * DEC_ROWS + row, p.causal);
         float m_ref = -INFINITY, l = 0.f;
         for (int tt = 0; tt < sg.ntl; ++tt, ++g) {
@@ -598,7 +728,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           mx[cg * DEC_ROWS + row] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
           named_bar_sync(1 + q, 128);         // the four warps of these rows
           const float mx_t = fmaxf(fmaxf(mx[row], mx[DEC_ROWS + row]), fmaxf(mx[2 * DEC_ROWS + row], mx[3 * DEC_ROWS + row])) *
-                             p.scale_log2;    // the scale is positive: the order is kept
+                             sl2;             // the scale is positive: the order is kept
           float alpha = 1.f;
           bool moved = false;
           if (mx_t > m_ref + DEC_MOVE) {
@@ -627,8 +757,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
             uint32_t pk[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(ex2(fmaf(s[8 * c + 2 * e], p.scale_log2, -mu)),
-                                                              ex2(fmaf(s[8 * c + 2 * e + 1], p.scale_log2, -mu)));
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(ex2(fmaf(s[8 * c + 2 * e], sl2, -mu)),
+                                                              ex2(fmaf(s[8 * c + 2 * e + 1], sl2, -mu)));
               pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
               sum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
             }
@@ -684,11 +814,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
     const uint32_t tO = tmem;   // all 512 columns
     uint8_t* sP = smem + Cfg::V_OFF_P;
     uint8_t* sV = smem + Cfg::V_OFF_V;
+    uint8_t* sF = smem + Cfg::V_OFF_F;
     if ((warp == 0 || warp == 3) && lane == 0) {
       // ------------------------------- TMA producers -------------------------------
       // per hand-over (64 positions): two value slot uses of 256 latent columns, each one TMA
       // instruction of four 64-column groups (a 3-D box: columns within a group, positions, groups);
-      // use m is issued by producer m % 2 (warps 0 and 3: two instructions in flight)
+      // use m is issued by producer m % 2 (warps 0 and 3: two instructions in flight). An e4m3 cache
+      // goes to the staging slots instead (two 128-column groups per instruction, unswizzled), which
+      // the rescale warps convert into the value slots.
       const int pid = warp == 0 ? 0 : 1;
       DecWalk w;
       w.begin(p, u0, u1);
@@ -701,6 +834,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
             const int y = (int)(sg.sstart + (int64_t)(sg.tile0 + tt) * DEC_BT + cg * DEC_HT);
             for (int nh = 0; nh < 2; ++nh, ++n) {
               if ((n & 1) != pid) continue;
+              if constexpr (F8) {
+                const int f = (int)(n % NF);
+                if (n >= NF && !wait_bar(&bars->f_empty[f], (uint32_t)((n / NF) - 1) & 1u)) { ok = false; break; }
+                mbar_arrive_expect_tx(&bars->f_full[f], Cfg::FUNIT);
+                tma_load_3d(sF + f * Cfg::FUNIT, &tv, &bars->f_full[f], 0, y, 2 * nh);
+                continue;
+              }
               const int s = (int)(n % NV);
               if (n >= NV && !wait_bar(&bars->v_empty[s], (uint32_t)((n / NV) - 1) & 1u)) { ok = false; break; }
               mbar_arrive_expect_tx(&bars->v_full[s], Cfg::UNIT);
@@ -710,8 +850,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         }
       }
       if (*abort_flag) {
-        for (int64_t i = (n > NV ? n - NV : 0); i < n; ++i)
-          if ((i & 1) == pid) (void)mbar_wait(&bars->v_full[i % NV], (uint32_t)(i / NV) & 1u, drain_ns, p.status);
+        if constexpr (F8) {
+          for (int64_t i = (n > NF ? n - NF : 0); i < n; ++i)
+            if ((i & 1) == pid) (void)mbar_wait(&bars->f_full[i % NF], (uint32_t)(i / NF) & 1u, drain_ns, p.status);
+        } else {
+          for (int64_t i = (n > NV ? n - NV : 0); i < n; ++i)
+            if ((i & 1) == pid) (void)mbar_wait(&bars->v_full[i % NV], (uint32_t)(i / NV) & 1u, drain_ns, p.status);
+        }
       }
     } else if (warp == 1 && lane == 0) {
       // ------------------------------- P.C issuer -------------------------------
@@ -801,6 +946,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       const int row = q * 32 + lane;
       const uint32_t lane_off = (uint32_t)(q * 32) << 16;
       const uint32_t tcol = tO + lane_off + cv * 128;
+      // e4m3 cache: value use u from its staging slot into a value slot as bf16 (the codes, exactly),
+      // each warp 64 of the 1024 16-byte chunks ([group 2][position 64][chunk 8]); a chunk's 16 codes
+      // are 16 columns of a 64-column bf16 group, two swizzled 16-byte chunks of the position's row
+      auto convert_use = [&](int64_t u) {
+        const int fs = (int)(u % (NF > 0 ? NF : 1)), vs = (int)(u % NV);
+        bool ok = wait_bar(&bars->f_full[fs], (uint32_t)(u / (NF > 0 ? NF : 1)) & 1u);
+        if (ok && u >= NV) ok = wait_bar(&bars->v_empty[vs], (uint32_t)((u / NV) - 1) & 1u);
+        if (!ok) return;
+        const uint8_t* src = sF + fs * Cfg::FUNIT;
+        uint8_t* dstu = sV + vs * Cfg::UNIT;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int id = w16 * 64 + e * 32 + lane;
+          const int g = id >> 9, pos = (id >> 3) & 63, c16 = id & 7;
+          const uint4 v = *reinterpret_cast<const uint4*>(src + id * 16);
+          const uint2 a = e4m3x4_to_bf16x4(v.x), b = e4m3x4_to_bf16x4(v.y);
+          const uint2 c = e4m3x4_to_bf16x4(v.z), d = e4m3x4_to_bf16x4(v.w);
+          const int cb = (c16 & 3) * 2;
+          uint8_t* rowp = dstu + (2 * g + (c16 >> 2)) * (DEC_HT * 128) + pos * 128;
+          *reinterpret_cast<uint4*>(rowp + ((cb ^ (pos & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
+          *reinterpret_cast<uint4*>(rowp + (((cb + 1) ^ (pos & 7)) << 4)) = make_uint4(c.x, c.y, d.x, d.y);
+        }
+        fence_proxy_async_smem();   // generic stores read by the P.C MMAs (async proxy)
+        __syncwarp();
+        if (lane == 0 && !*abort_flag) {
+          mbar_arrive(&bars->f_empty[fs]);
+          mbar_arrive(&bars->v_full[vs]);
+        }
+      };
       DecWalk w;
       w.begin(p, u0, u1);
       DecSeg sg;
@@ -810,6 +984,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         for (int tt = 0; tt < sg.ntl; ++tt) {
           for (int cg = 0; cg < DEC_QT; ++cg, ++i) {
             const int hs = (int)(i % NPH);
+            if constexpr (F8) {
+              convert_use(2 * i);
+              convert_use(2 * i + 1);
+            }
             (void)wait_bar(&bars->p_full[hs], (uint32_t)(i / NPH) & 1u);
             const DecSide* sd = reinterpret_cast<const DecSide*>(sP + hs * Cfg::PSLOT + Cfg::PH);
             const int any = sd[0].flag | sd[1].flag | sd[2].flag | sd[3].flag;
@@ -845,7 +1023,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
               const int64_t orow = (int64_t)sg.b * rows_seq + ri;
               const int slotp = 2 * pair + (segi == 0 ? 0 : 1);
               const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
-              const float mul = sg.complete ? inv : 1.f;
+              const float mul = (sg.complete ? inv : 1.f) * (F8 ? p.cache_scale : 1.f);
               float* dst = sg.complete ? p.out_lat + orow * DEC_DC : p.o_part + ((int64_t)slotp * DEC_ROWS + row) * DEC_DC;
               // each lane scales its own row; after the lane-group transpose, store t of a lane goes to
               // row 8 (lane / 8) + t of the warp's rows, columns 4 (lane % 8) .. of the 32 just read, so
@@ -1004,6 +1182,8 @@ bool tc_decode_supported(const DecodeArgs& a) {
   // the plan stores tile prefixes in int32: the units of all blocks must stay below 2^31
   const int64_t nblocks = (int64_t)a.batch * ceil_div((int64_t)a.n_q * a.H, DEC_ROWS);
   const int64_t tiles = std::max<int64_t>(1, ceil_div(a.max_seqlen, DEC_BT));
+  // an e4m3 cache is read by TMA from a 16-byte aligned base (rows of 576 or 512 bytes)
+  if (a.cache_f8 && (reinterpret_cast<uintptr_t>(a.cache) & 15u)) return false;
   return nblocks < (1LL << 31) / tiles;
 }
 
@@ -1012,7 +1192,7 @@ struct TcDecodePlan {
   size_t off_prefix, off_o, off_m, off_l, total;
 };
 
-template <int DR>
+template <int DR, bool F8>
 static int max_active_clusters_t() {
   int n = 0;
   cudaLaunchConfig_t cfg = {};
@@ -1023,11 +1203,12 @@ static int max_active_clusters_t() {
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
   cfg.blockDim = dim3(DEC_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = DecCfg<DR>::SMEM;
+  cfg.dynamicSmemBytes = DecCfg<DR, F8>::SMEM;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaFuncSetAttribute(tc_decode_kernel<DR>, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg<DR>::SMEM);
-  const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, (void*)tc_decode_kernel<DR>, &cfg);
+  cudaFuncSetAttribute(tc_decode_kernel<DR, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       DecCfg<DR, F8>::SMEM);
+  const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, (void*)tc_decode_kernel<DR, F8>, &cfg);
   if (e != cudaSuccess || n <= 0) {
     (void)cudaGetLastError();
     n = sm_count() / 2;
@@ -1037,12 +1218,14 @@ static int max_active_clusters_t() {
 
 // clusters of two CTAs that can be resident at once (the kernel is persistent: more would run as a
 // second wave); computed once per device and tile variant
-static int max_active_clusters(int dr) {
-  static int cached[64][2] = {{0}};
+static int max_active_clusters(int dr, bool f8) {
+  static int cached[64][4] = {{0}};
   const int dev = current_device();
-  const int v = dr == 0 ? 0 : 1;
+  const int v = (dr == 0 ? 0 : 1) + (f8 ? 2 : 0);
   if (dev < 0 || dev >= 64) return sm_count() / 2;
-  if (cached[dev][v] == 0) cached[dev][v] = dr == 0 ? max_active_clusters_t<0>() : max_active_clusters_t<64>();
+  if (cached[dev][v] == 0)
+    cached[dev][v] = v == 0 ? max_active_clusters_t<0, false>() : v == 1 ? max_active_clusters_t<64, false>()
+                   : v == 2 ? max_active_clusters_t<0, true>() : max_active_clusters_t<64, true>();
   return cached[dev][v];
 }
 
@@ -1051,7 +1234,7 @@ static TcDecodePlan plan_tc(const DecodeArgs& a) {
   t.nbps = (int)ceil_div((int64_t)a.n_q * a.H, DEC_ROWS);
   t.nblocks = a.batch * t.nbps;
   const int64_t units_max = (int64_t)t.nblocks * std::max<int64_t>(1, ceil_div(a.max_seqlen, DEC_BT));
-  const int maxc = max_active_clusters(a.dr);
+  const int maxc = max_active_clusters(a.dr, a.cache_f8);
   int G = maxc;
   // Equal-length sequences with one row block each: give every block the same number of clusters
   // (no block is split unevenly and, with one cluster per block, no partials are written at all).
@@ -1070,19 +1253,19 @@ static TcDecodePlan plan_tc(const DecodeArgs& a) {
 
 size_t tc_decode_workspace(const DecodeArgs& a) { return plan_tc(a).total; }
 
-template <int DR>
+template <int DR, bool F8>
 static int launch_decode_t(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
                            const DecParams& p, cudaStream_t s) {
   static bool attr_set[64] = {false};
   const int dev = current_device();
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(tc_decode_kernel<DR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DecCfg<DR>::SMEM) != cudaSuccess)
+    if (cudaFuncSetAttribute(tc_decode_kernel<DR, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DecCfg<DR, F8>::SMEM) != cudaSuccess)
       return MLA_ERR_CUDA;
     attr_set[dev] = true;
   }
-  return launch_pdl(tc_decode_kernel<DR>, dim3(2 * p.G), dim3(DEC_THREADS), (size_t)DecCfg<DR>::SMEM, s, tk, tv,
-                    tq, p);
+  return launch_pdl(tc_decode_kernel<DR, F8>, dim3(2 * p.G), dim3(DEC_THREADS), (size_t)DecCfg<DR, F8>::SMEM, s,
+                    tk, tv, tq, p);
 }
 
 int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
@@ -1097,6 +1280,7 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
   p.cu = a.cu_seqlens; p.batch = a.batch; p.n_q = a.n_q; p.H = a.H; p.nbps = t.nbps; p.nblocks = t.nblocks;
   p.total_rows = a.total_rows; p.causal = a.causal ? 1 : 0;
   p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.cache_scale = a.cache_f8 ? a.cache_scale : 1.f;
   p.prefix = reinterpret_cast<int32_t*>(ws + t.off_prefix);
   p.G = t.G;
   p.out_lat = a.out_lat; p.lse = a.lse;
@@ -1112,19 +1296,37 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
   // the value CTA; the query: 128 rows x 64 columns. All 128-byte swizzled (the MMA operand layout).
   CUtensorMap tk, tv, tq;
   const uint64_t rows = (uint64_t)std::max<int64_t>(a.total_rows, 1);
-  {
-    const uint64_t dims[2] = {(uint64_t)W, rows};
-    const uint64_t st[1] = {(uint64_t)W * 2};
-    const uint32_t box[2] = {64, DEC_BT};
-    if (!encode_tmap_bf16(&tk, const_cast<void*>(a.cache), 2, dims, st, box)) return MLA_ERR_CUDA;
-  }
-  {
-    // positions step by a row, groups by 64 columns: one box is 64 positions x 256 columns, laid out
-    // as four 64-column groups of [64 positions x 128 B] (the MN-major B operand of P.C)
-    const uint64_t dims[3] = {64, rows, (uint64_t)(W / 64)};
-    const uint64_t st[2] = {(uint64_t)W * 2, 128};
-    const uint32_t box[3] = {64, DEC_HT, 4};
-    if (!encode_tmap_bf16(&tv, const_cast<void*>(a.cache), 3, dims, st, box)) return MLA_ERR_CUDA;
+  if (a.cache_f8) {
+    // e4m3: 256-position x 128-column boxes for the score CTA (the rotary box starts at column 512 and
+    // reads its last 64 columns as zeros), 64-position x 256-column unswizzled staging boxes (two
+    // 128-column groups) for the value CTA
+    {
+      const uint64_t dims[2] = {(uint64_t)W, rows};
+      const uint64_t st[1] = {(uint64_t)W};
+      const uint32_t box[2] = {128, DEC_BT};
+      if (!encode_tmap_u8(&tk, const_cast<void*>(a.cache), 2, dims, st, box, 128)) return MLA_ERR_CUDA;
+    }
+    {
+      const uint64_t dims[3] = {128, rows, (uint64_t)(a.dc / 128)};
+      const uint64_t st[2] = {(uint64_t)W, 128};
+      const uint32_t box[3] = {128, DEC_HT, 2};
+      if (!encode_tmap_u8(&tv, const_cast<void*>(a.cache), 3, dims, st, box, 0)) return MLA_ERR_CUDA;
+    }
+  } else {
+    {
+      const uint64_t dims[2] = {(uint64_t)W, rows};
+      const uint64_t st[1] = {(uint64_t)W * 2};
+      const uint32_t box[2] = {64, DEC_BT};
+      if (!encode_tmap_bf16(&tk, const_cast<void*>(a.cache), 2, dims, st, box)) return MLA_ERR_CUDA;
+    }
+    {
+      // positions step by a row, groups by 64 columns: one box is 64 positions x 256 columns, laid out
+      // as four 64-column groups of [64 positions x 128 B] (the MN-major B operand of P.C)
+      const uint64_t dims[3] = {64, rows, (uint64_t)(W / 64)};
+      const uint64_t st[2] = {(uint64_t)W * 2, 128};
+      const uint32_t box[3] = {64, DEC_HT, 4};
+      if (!encode_tmap_bf16(&tv, const_cast<void*>(a.cache), 3, dims, st, box)) return MLA_ERR_CUDA;
+    }
   }
   {
     const uint64_t dims[2] = {(uint64_t)W, (uint64_t)a.batch * a.n_q * a.H};
@@ -1143,7 +1345,10 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
     const int st0 = launch_pdl(decode_plan_kernel, dim3(1), dim3(1024), 0, s, p, const_cast<int32_t*>(p.prefix));
     if (st0) return st0;
   }
-  int st = a.dr == 0 ? launch_decode_t<0>(tk, tv, tq, p, s) : launch_decode_t<64>(tk, tv, tq, p, s);
+  int st = a.cache_f8 ? (a.dr == 0 ? launch_decode_t<0, true>(tk, tv, tq, p, s)
+                                    : launch_decode_t<64, true>(tk, tv, tq, p, s))
+                       : (a.dr == 0 ? launch_decode_t<0, false>(tk, tv, tq, p, s)
+                                    : launch_decode_t<64, false>(tk, tv, tq, p, s));
   if (st) return st;
   if (equal_blocks && t.G == t.nblocks && a.max_seqlen > 0) return MLA_OK;
   // 16 CTAs per block (eight rows each): a split block's merge reads its partial slots of 256 KB
