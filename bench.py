@@ -629,7 +629,7 @@ def run_rows(args):
                                                  step.out_lat, step.lse, ws8))
     report("f1 decode over an e4m3 cache (tensor cores)", c3, ms, B * T * (dc + dr),
            B * H * T * (2 * (dc + dr) + 2 * dc),
-           "bf16 query split into two e4m3 parts for QK^T, P.C in bf16 over the converted codes; bytes = the e4m3 "
+           "bf16 query split into two e4m3 parts for QK^T, P.C in f16 over the converted codes; bytes = the e4m3 "
            "cache; FLOPs counted once (the two query parts double the QK^T MMAs at twice the bf16 rate)")
     del codes, ws8
     del cache, step, w_o, layer, w_qc, w_qr

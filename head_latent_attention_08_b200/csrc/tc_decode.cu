@@ -200,14 +200,11 @@ __device__ __forceinline__ void group8_transpose(uint4 (&c)[8], int lane) {
   }
 }
 
-// four e4m3 codes (consecutive bytes of x) -> four bf16 values (exact: every e4m3 value is a bf16 value)
-__device__ __forceinline__ uint2 e4m3x4_to_bf16x4(uint32_t x) {
+// four e4m3 codes (consecutive bytes of x) -> four f16 values (exact: every e4m3 value is an f16 value)
+__device__ __forceinline__ uint2 e4m3x4_to_f16x4(uint32_t x) {
   const __half2_raw h0 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(x & 0xFFFFu), __NV_E4M3);
   const __half2_raw h1 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(x >> 16), __NV_E4M3);
-  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h0));
-  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-  const __nv_bfloat162 r0 = __floats2bfloat162_rn(a.x, a.y), r1 = __floats2bfloat162_rn(b.x, b.y);
-  return make_uint2(*reinterpret_cast<const uint32_t*>(&r0), *reinterpret_cast<const uint32_t*>(&r1));
+  return make_uint2((uint32_t)h0.x | ((uint32_t)h0.y << 16), (uint32_t)h1.x | ((uint32_t)h1.y << 16));
 }
 
 // eight bf16 values (v) times a power of two (p2) as e4m3 high and low parts: hi = e4m3(x),
@@ -750,17 +747,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           const uint32_t prow = dst + (uint32_t)(row * 128);
           // P in bf16 (round to nearest even), 8 positions (16 bytes, one swizzled chunk of the row) at a
           // time, and the row sum of the same rounded values, so that numerator and denominator share
-          // the rounding
+          // the rounding. Over an e4m3 cache P is f16 (the type of the converted codes; 11 bits, so the
+          // row sum takes the unrounded values)
           float sum = 0.f;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             uint32_t pk[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(ex2(fmaf(s[8 * c + 2 * e], sl2, -mu)),
-                                                              ex2(fmaf(s[8 * c + 2 * e + 1], sl2, -mu)));
-              pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
-              sum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
+              const float x0 = ex2(fmaf(s[8 * c + 2 * e], sl2, -mu)), x1 = ex2(fmaf(s[8 * c + 2 * e + 1], sl2, -mu));
+              if constexpr (F8) {
+                const __half2 h2 = __floats2half2_rn(x0, x1);
+                pk[e] = *reinterpret_cast<const uint32_t*>(&h2);
+                sum += x0 + x1;
+              } else {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
+                pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+                sum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
+              }
             }
             if (send) st_async_v4(prow + (uint32_t)((c ^ (lane & 7)) * 16), make_uint4(pk[0], pk[1], pk[2], pk[3]), bar);
           }
@@ -862,7 +866,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       // ------------------------------- P.C issuer -------------------------------
       // O[:, 256 nh + ...] += P (128 x 64, K-major, from the P slot) . C (64 x 256, MN-major, from a
       // value slot); each value slot is released by its own commit
-      constexpr uint32_t idesc = idesc_bf16_f32(128, 256, false, true);
+      // (f16 operands over an e4m3 cache)
+      constexpr uint32_t idesc = F8 ? idesc_f16_f32(128, 256, false, true) : idesc_bf16_f32(128, 256, false, true);
       const uint64_t pd0 = smem_desc_sw128(smem_u32(sP), 16, 1024);
       const uint64_t vd0 = smem_desc_sw128(smem_u32(sV), DEC_HT * 128, 1024);
       DecWalk w;
@@ -946,7 +951,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       const int row = q * 32 + lane;
       const uint32_t lane_off = (uint32_t)(q * 32) << 16;
       const uint32_t tcol = tO + lane_off + cv * 128;
-      // e4m3 cache: value use u from its staging slot into a value slot as bf16 (the codes, exactly),
+      // e4m3 cache: value use u from its staging slot into a value slot as f16 (the codes, exactly),
       // each warp 64 of the 1024 16-byte chunks ([group 2][position 64][chunk 8]); a chunk's 16 codes
       // are 16 columns of a 64-column bf16 group, two swizzled 16-byte chunks of the position's row
       auto convert_use = [&](int64_t u) {
@@ -961,8 +966,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           const int id = w16 * 64 + e * 32 + lane;
           const int g = id >> 9, pos = (id >> 3) & 63, c16 = id & 7;
           const uint4 v = *reinterpret_cast<const uint4*>(src + id * 16);
-          const uint2 a = e4m3x4_to_bf16x4(v.x), b = e4m3x4_to_bf16x4(v.y);
-          const uint2 c = e4m3x4_to_bf16x4(v.z), d = e4m3x4_to_bf16x4(v.w);
+          const uint2 a = e4m3x4_to_f16x4(v.x), b = e4m3x4_to_f16x4(v.y);
+          const uint2 c = e4m3x4_to_f16x4(v.z), d = e4m3x4_to_f16x4(v.w);
           const int cb = (c16 & 3) * 2;
           uint8_t* rowp = dstu + (2 * g + (c16 >> 2)) * (DEC_HT * 128) + pos * 128;
           *reinterpret_cast<uint4*>(rowp + ((cb ^ (pos & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);

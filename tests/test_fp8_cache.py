@@ -55,7 +55,7 @@ def test_append_latent_fp8(scale, flags):
 
 CASES = [
     # q dtype, H, dc, dr, seqlens, n_q, causal. A bf16 query at H 128, d_c 512 runs on the tensor cores
-    # (QK^T as e4m3 MMAs against the query split into e4m3 high and low parts, P.C in bf16 over the
+    # (QK^T as e4m3 MMAs against the query split into e4m3 high and low parts, P.C in f16 over the
     # codes converted exactly); the rest on CUDA cores in fp32.
     ("bf16", 128, 512, 64, [1, 63, 300, 1000], 1, True),
     ("bf16", 128, 512, 64, [4, 67, 300], 4, True),
@@ -106,7 +106,7 @@ def test_decode_absorbed_fp8(case):
     ref, ref_lse = O.decode_absorbed(O.store_as(q_abs, qdt), p.cache.astype(np.float64) * scale, p.cu_seqlens,
                                      n_q, dc, p.kq_scale, causal)
     # the CUDA-core route keeps fp32 arithmetic over the same e4m3 values; the tensor-core route rounds
-    # P to bf16 and carries the query to about 2^-8: the bf16 rule
+    # P to f16 and carries the query to about 2^-8: the bf16 rule
     tol = "bf16" if tensor_core_route(qdt, H, dc) else "f32"
     assert_close(out, ref, tol, "out_lat")
     assert_lse_close(lse, ref_lse, tol, "lse")
