@@ -693,6 +693,50 @@ def run_rows(args):
     return 0
 
 
+def run_profile_decode(args):
+    """The decode call alone on the workload's shape (--batch sequences of 4096 positions, H 128), over a
+    bf16 or an e4m3 cache: a fixed small case for profiler captures (ncu -k regex:tc_decode_kernel),
+    not a benchmark line. Prints the median CUDA-event time of --steps calls after --warmup calls."""
+    import torch
+    from head_latent_attention_08_b200 import mla as M
+    dev = torch.device("cuda")
+    B, T, H, dc, dr = WORKLOAD["batch"], WORKLOAD["seqlen"], WORKLOAD["n_heads"], WORKLOAD["kv_lora_rank"], \
+        WORKLOAD["rope_dim"]
+    d = M.dims(H, dc, dr, WORKLOAD["qk_nope"], WORKLOAD["v_head"], WORKLOAD["d_model"])
+    gen = torch.Generator(device=dev).manual_seed(SEED)
+    vals = torch.randn(B * T, dc + dr, device=dev, generator=gen)
+    q = torch.randn(B, H, dc + dr, device=dev, generator=gen).to(torch.bfloat16)
+    cu = torch.arange(0, (B + 1) * T, T, dtype=torch.int32, device=dev)
+    out = torch.empty(B, H, dc, device=dev)
+    lse = torch.empty(B, H, device=dev)
+    flags = M.MLA_DECODE_CAUSAL
+    if args.profile_decode == "e4m3":
+        cache = vals.to(torch.float8_e4m3fn).view(torch.uint8)
+        ws = M.workspace(M.mla_decode_workspace_size(d, torch.uint8, B, 1, T, B * T, flags), dev)
+
+        def call():
+            M.mla_decode_absorbed_fp8(d, q, cache, 1.0, cu, B, 1, T, flags, out, lse, ws)
+    else:
+        cache = vals.to(torch.bfloat16)
+        ws = M.workspace(M.mla_decode_workspace_size(d, torch.bfloat16, B, 1, T, B * T, flags), dev)
+
+        def call():
+            M.mla_decode_absorbed(d, q, cache, cu, B, 1, T, flags, out, lse, ws)
+    del vals
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(); call(); b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    print(json.dumps({"profile_decode": args.profile_decode, "batch": B, "seqlen": T, "ms_median": statistics.median(ts),
+                      "device_status": M.mla_check_status(), "note": "profiling case, not a benchmark line"}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -703,6 +747,8 @@ def main():
     ap.add_argument("--rows", action="store_true",
                     help="time each step of the path on its own against its roofline (one JSON line "
                          "per row) instead of the benchmark line")
+    ap.add_argument("--profile-decode", choices=["bf16", "e4m3"], default=None,
+                    help="run only the decode call over a bf16 or e4m3 cache (a profiler capture case)")
     ap.add_argument("--batch", type=int, default=WORKLOAD["batch"],
                     help="sequences per step (default 64: the benchmark workload; smaller batches "
                          "are for profiling captures and are not benchmark numbers)")
@@ -715,6 +761,8 @@ def main():
         CONFIG["workload"] += f" [batch reduced to {args.batch}: profiling case, not the benchmark]"
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_decode:
+        return run_profile_decode(args)
     if args.rows:
         return run_rows(args)
     return run_ours(args)

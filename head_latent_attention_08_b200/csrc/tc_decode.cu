@@ -60,7 +60,7 @@ constexpr int DEC_THREADS = 640;   // 4 control warps + 16 softmax (score CTA) o
 constexpr int DEC_SW = 16;         // softmax / epilogue warps
 constexpr int DEC_DC = 512;        // latent width handled by this kernel
 constexpr int DEC_ROWS = 128;      // rows per block
-constexpr int DEC_NPH = 6;         // P hand-over slots in the value CTA
+constexpr int DEC_NPH = 6;         // P hand-over slots in the value CTA (at most)
 constexpr int DEC_PF = 2;          // cache tiles warmed in L2 ahead of the tile QK^T works on
 constexpr int DEC_NPROD = 3;       // TMA-issuing threads of the score CTA
 constexpr float DEC_MOVE = 8.f;    // the reference maximum moves when a row maximum exceeds it by 2^8
@@ -100,16 +100,18 @@ struct DecCfg {
   static __host__ __device__ constexpr uint32_t slot_tx(int cg) {
     return (uint32_t)(PH + 4 * (16 + (cg == 0 ? 128 : 0) + (cg == DEC_QT - 1 ? 256 : 0)));
   }
+  static constexpr int NPH = DEC_NPH;                      // P slots
   static constexpr int V_OFF_P = 0;
-  static constexpr int V_OFF_V = dec_round1024(DEC_NPH * PSLOT);
+  static constexpr int V_OFF_V = dec_round1024(NPH * PSLOT);
   static constexpr int UNIT = DEC_HT * 512;                // 64 positions x 256 latent columns bf16: 32 KB
   static constexpr int FUNIT = DEC_HT * 256;               // the same in e4m3: 16 KB
-  static constexpr int NV = F8 ? 2 : (DATA_LIMIT - V_OFF_V) / UNIT;   // bf16 value slots
+  static constexpr int NV = F8 ? 2 : (DATA_LIMIT - V_OFF_V) / UNIT;   // bf16 (e4m3 cache: f16) value slots
   static constexpr int V_OFF_F = V_OFF_V + NV * UNIT;      // e4m3 staging slots
   static constexpr int NF = F8 ? (DATA_LIMIT - V_OFF_F) / FUNIT : 0;
   static constexpr int OFF_BAR = dec_max(S_OFF_K + NK * SUPER, V_OFF_F + NF * FUNIT);
   static constexpr int SMEM = OFF_BAR + DEC_BAR_BYTES + 1024;
   static_assert(PSLOT % 1024 == 0, "P slots must keep the 1024-byte swizzle alignment");
+  static_assert(NPH >= DEC_QT && NPH <= DEC_NPH, "P slots");
   static_assert(NK >= 2, "the cache ring needs two slots");
   static_assert(NV >= 2, "the value ring needs two slots");
   static_assert(!F8 || NF >= 2, "the e4m3 staging ring needs two slots");
@@ -371,7 +373,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
   constexpr int NV = Cfg::NV;
   constexpr int NF = Cfg::NF;
   constexpr int NB = Cfg::NB;
-  constexpr int NPH = DEC_NPH;
+  constexpr int NPH = Cfg::NPH;
   using Bars = DecBars<NK, NV, NF>;
   static_assert(sizeof(Bars) <= DEC_BAR_BYTES, "barrier block");
   extern __shared__ uint8_t smem_raw[];
@@ -607,20 +609,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         float sl2 = p.scale_log2;       // score -> log2-domain logit
         if (segi > 0) (void)wait_bar(&bars->q_empty, (uint32_t)(segi - 1) & 1u);
         const int64_t r0 = (int64_t)sg.b * p.n_q * p.H + (int64_t)sg.rb * DEC_ROWS + q * 32 + (lane & ~7);
-        auto load_half = [&](int bx, uint4 (&ch)[8]) {
+        // the row pieces of half bx (latent columns 128 cg + 64 bx ..) for the lane's group, transposed
+        auto load_half = [&](int bx, uint4 (&c8)[8]) {
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
             const int64_t rr = r0 + t;
-            ch[t] = rr < p.q_rows ? __ldg(reinterpret_cast<const uint4*>(p.q_abs + rr * p.W + cg * 128 + bx * 64 +
+            c8[t] = rr < p.q_rows ? __ldg(reinterpret_cast<const uint4*>(p.q_abs + rr * p.W + cg * 128 + bx * 64 +
                                                                         8 * (lane & 7)))
                                   : make_uint4(0u, 0u, 0u, 0u);
           }
-          group8_transpose(ch, lane);
         };
+        // all sixteen loads of a lane are issued before any is used
+        uint4 ch[2][8];
+        load_half(0, ch[0]);
+        load_half(1, ch[1]);
+        group8_transpose(ch[0], lane);
+        group8_transpose(ch[1], lane);
         if constexpr (!F8) {
-          uint4 ch[2][8];
-          load_half(0, ch[0]);
-          load_half(1, ch[1]);
 #pragma unroll
           for (int bx = 0; bx < 2; ++bx) {
             uint32_t r[32];
@@ -646,13 +651,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
             rp[1] = __ldg(src + 1);
           }
           float amax = bf16x8_absmax(rp[1], bf16x8_absmax(rp[0], 0.f));
-#pragma unroll 1
-          for (int bx = 0; bx < 2; ++bx) {
-            uint4 ch[8];
-            load_half(bx, ch);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) amax = bf16x8_absmax(ch[c], amax);
-          }
+          for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) amax = bf16x8_absmax(ch[bx][c], amax);
           float* qmx = red + 12 * DEC_ROWS;
           qmx[cg * DEC_ROWS + row] = amax;
           named_bar_sync(1 + q, 128);         // the four warps of these rows
@@ -661,13 +663,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           const float p2 = rmax > 0.f ? __uint_as_float(__float_as_uint(fminf(448.f / rmax, 0x1p100f)) & 0x7F800000u)
                                       : 1.f;
           sl2 = p.scale_log2 * p.cache_scale / p2;
+          // the pieces again (now from L2), half by half, to keep registers for the split
 #pragma unroll 1
           for (int bx = 0; bx < 2; ++bx) {
-            uint4 ch[8];
-            load_half(bx, ch);
+            uint4 c8[8];
+            load_half(bx, c8);
+            group8_transpose(c8, lane);
             uint32_t hi[16], lo[16];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) e4m3_split8(ch[c], p2, hi[2 * c], hi[2 * c + 1], lo[2 * c], lo[2 * c + 1]);
+            for (int c = 0; c < 8; ++c) e4m3_split8(c8[c], p2, hi[2 * c], hi[2 * c + 1], lo[2 * c], lo[2 * c + 1]);
             tmem_st16(tQ + lane_off + cg * 32 + bx * 16, hi);
             tmem_st16(tQ + lane_off + 128 + cg * 32 + bx * 16, lo);
           }
