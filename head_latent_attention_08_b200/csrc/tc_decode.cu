@@ -957,7 +957,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       const uint32_t tcol = tO + lane_off + cv * 128;
       // e4m3 cache: value use u from its staging slot into a value slot as f16 (the codes, exactly),
       // each warp 64 of the 1024 16-byte chunks ([group 2][position 64][chunk 8]); a chunk's 16 codes
-      // are 16 columns of a 64-column bf16 group, two swizzled 16-byte chunks of the position's row
+      // are 16 columns of a 64-column f16 group, two swizzled 16-byte chunks of the position's row.
+      // 16-byte accesses go out eight lanes at a time: the eight lanes of each phase take chunks 0..3 of
+      // one position and 4..7 of the next (or the reverse), so that both the staging reads (unswizzled)
+      // and the stores (opposite position parities) touch eight different bank quads.
       auto convert_use = [&](int64_t u) {
         const int fs = (int)(u % (NF > 0 ? NF : 1)), vs = (int)(u % NV);
         bool ok = wait_bar(&bars->f_full[fs], (uint32_t)(u / (NF > 0 ? NF : 1)) & 1u);
@@ -967,8 +970,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         uint8_t* dstu = sV + vs * Cfg::UNIT;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int id = w16 * 64 + e * 32 + lane;
-          const int g = id >> 9, pos = (id >> 3) & 63, c16 = id & 7;
+          const int base = w16 * 64 + e * 32;
+          const int k = (lane >> 2) & 1;
+          const int g = base >> 9, pos = ((base >> 3) & 63) + 2 * ((lane >> 4) & 1) + k;
+          const int c16 = 4 * (k ^ ((lane >> 3) & 1)) + (lane & 3);
+          const int id = (g << 9) | (pos << 3) | c16;
           const uint4 v = *reinterpret_cast<const uint4*>(src + id * 16);
           const uint2 a = e4m3x4_to_f16x4(v.x), b = e4m3x4_to_f16x4(v.y);
           const uint2 c = e4m3x4_to_f16x4(v.z), d = e4m3x4_to_f16x4(v.w);
