@@ -38,6 +38,10 @@
 //    which also move each block's latent query into TMEM. Value CTA: warps 0 and 3 lane 0 TMA, warp 1
 //    lane 0 P.C, warp 2 lane 0 hands P slots back, warps 4-19 rescale and write O (warp w: rows
 //    32 (w & 3) .., O columns [128 c, 128 c + 128)).
+//  * An e4m3 cache (F8; value = code * cache_scale) keeps the same structure: the score CTA streams
+//    128-column boxes and runs QK^T as kind::f8f6f4 MMAs against the query split into e4m3 high and
+//    low parts (per-row power-of-two scale, both parts in TMEM), and the value CTA stages its units
+//    as e4m3 and its rescale warps convert them exactly to f16 for an f16 P.C (P in f16).
 //  * Every wait is bounded (global-timer limit); a wait that gives up sets the library's status word,
 //    and the CTA abandons its work: it issues nothing more, drains its own TMA loads, MMAs and bulk
 //    copies and leaves through the cluster barrier.

@@ -199,8 +199,11 @@ MLA_API int32_t mla_decode_absorbed(const mla_dims* dims, int32_t dtype, const v
  * mla_decode_absorbed_fp8 -- mla_decode_absorbed over an e4m3 latent cache (value = code * cache_scale,
  * the cache of mla_append_latent_fp8) with a bf16 or fp32 absorbed query (q_dtype): half the cache bytes
  * of a bf16 cache. Same arguments, layouts and results otherwise; scratch of at least
- * mla_decode_workspace_size(dims, MLA_FP8_E4M3, ...) bytes. Runs on CUDA cores in fp32 arithmetic
- * (decoded cache values, fp32 scores and softmax).
+ * mla_decode_workspace_size(dims, MLA_FP8_E4M3, ...) bytes. With a bf16 query at d_c 512 (d_r 0 or
+ * 64) it runs on the tensor cores: QK^T as e4m3 MMAs against the query split into two e4m3 parts with
+ * a per-row power-of-two scale (about 2^-8 relative), P.C in f16 over the codes converted exactly;
+ * the cache base must then be 16-byte aligned (otherwise the CUDA-core route runs). With an fp32 query
+ * it runs on CUDA cores in fp32 arithmetic (decoded cache values, fp32 scores and softmax).
  */
 MLA_API int32_t mla_decode_absorbed_fp8(const mla_dims* dims, int32_t q_dtype, const void* q_abs,
                                         const uint8_t* cache, float cache_scale, const int32_t* cu_seqlens,
