@@ -391,7 +391,7 @@ def run_ours(args):
     q_nope = torch.empty(B, H, n, dtype=bf, device=dev)
     q_pe = torch.empty(B, H, dr, dtype=bf, device=dev)
     q_abs = torch.empty(B, H, dc + dr, dtype=bf, device=dev)
-    out_lat = torch.empty(B, H, dc, dtype=torch.float32, device=dev)
+    out_lat = torch.empty(B, H, dc, dtype=bf, device=dev)     # the decode writes the W_UV operand in bf16
     y = torch.empty(B, D, dtype=bf, device=dev)
     ws_proj = M.workspace(M.mla_project_workspace_size(d, bf, QR, B), dev)
     ws_dec = M.workspace(M.mla_decode_workspace_size(d, bf, B, 1, T, cache.shape[0], M.MLA_DECODE_CAUSAL), dev)
@@ -406,10 +406,11 @@ def run_ours(args):
         M.mla_absorb_weights(d, M.MLA_ABSORB_QUERY, q_nope, q_pe, wts["w_uk"], B, q_abs)
         if ev:
             ev[0].record(stream)
-        M.mla_decode_absorbed(d, q_abs, cache, cu, B, 1, T, M.MLA_DECODE_CAUSAL, out_lat, None, ws_dec)
+        M.mla_decode_absorbed(d, q_abs, cache, cu, B, 1, T, M.MLA_DECODE_CAUSAL | M.MLA_DECODE_OUT_BF16, out_lat,
+                              None, ws_dec)
         if ev:
             ev[1].record(stream)
-        M.mla_out_project(d, out_lat, wts["w_uv"], wts["w_o"], None, B, y, ws_out)
+        M.mla_out_project_bf16(d, out_lat, wts["w_uv"], wts["w_o"], None, B, y, ws_out)
 
     # ---- device-resident timing -------------------------------------------------------------
     for _ in range(args.warmup):

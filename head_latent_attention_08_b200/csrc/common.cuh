@@ -156,6 +156,7 @@ struct DecodeArgs {
   void* workspace; size_t workspace_bytes;
   float cache_scale = 1.f;               // an e4m3 cache holds value / cache_scale
   bool cache_f8 = false;                 // the cache is e4m3 (tensor-core decode with a bf16 query)
+  void* out_lat_bf16 = nullptr;          // tensor-core decode: write out_lat here in bf16 instead
 };
 
 size_t decode_generic_workspace(const DecodeArgs& a);

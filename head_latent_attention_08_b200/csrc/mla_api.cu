@@ -62,7 +62,7 @@ const char* mla_status_string(int32_t s) {
   }
 }
 
-int32_t mla_abi_version(void) { return 2; }
+int32_t mla_abi_version(void) { return 3; }
 
 int32_t mla_append_latent(const mla_dims* dims, int32_t cache_dtype, void* cache, int64_t cache_rows,
                           const int64_t* row_idx, const float* c_new, const float* kpe_new,
@@ -181,7 +181,7 @@ static int check_decode_sizes(const mla_dims* dims, int32_t dtype, int32_t batch
   int st = check_dims(dims);
   if (st) return st;
   if (!dtype_ok(dtype)) return MLA_ERR_DTYPE;
-  if (flags & ~(uint32_t)MLA_DECODE_CAUSAL) return MLA_ERR_MODE;
+  if (flags & ~(uint32_t)(MLA_DECODE_CAUSAL | MLA_DECODE_OUT_BF16)) return MLA_ERR_MODE;
   if (batch < 0 || n_q <= 0 || max_seqlen < 0 || total_rows < 0) return MLA_ERR_SHAPE;
   if (max_seqlen > 0x7fffffffLL || total_rows > 0x7fffffffLL) return MLA_ERR_SHAPE;
   if ((int64_t)batch * max_seqlen < total_rows) return MLA_ERR_SHAPE;
@@ -225,10 +225,12 @@ int32_t mla_decode_absorbed(const mla_dims* dims, int32_t dtype, const void* q_a
   a.q_abs = q_abs; a.cache = cache; a.cu_seqlens = cu_seqlens;
   a.out_lat = out_lat; a.lse = lse; a.workspace = workspace; a.workspace_bytes = workspace_bytes;
   cudaStream_t s = as_stream(stream);
+  if (flags & MLA_DECODE_OUT_BF16) a.out_lat_bf16 = out_lat;
   if (dtype == MLA_BF16 && tc_decode_supported(a)) {
     if (workspace_bytes < tc_decode_workspace(a) || !workspace) return MLA_ERR_WORKSPACE;
     return tc_decode_launch(a, s);
   }
+  if (flags & MLA_DECODE_OUT_BF16) return MLA_ERR_UNSUPPORTED;   // the tensor-core route only
   if (workspace_bytes < decode_generic_workspace(a)) return MLA_ERR_WORKSPACE;
   return decode_generic_launch(a, dtype, s);
 }
@@ -250,10 +252,15 @@ int32_t mla_decode_absorbed_fp8(const mla_dims* dims, int32_t q_dtype, const voi
   a.out_lat = out_lat; a.lse = lse; a.workspace = workspace; a.workspace_bytes = workspace_bytes;
   a.cache_scale = cache_scale;
   a.cache_f8 = true;
+  if (flags & MLA_DECODE_OUT_BF16) {
+    if (reinterpret_cast<uintptr_t>(out_lat) & 15u) return MLA_ERR_ALIGN;
+    a.out_lat_bf16 = out_lat;
+  }
   if (q_dtype == MLA_BF16 && tc_decode_supported(a)) {
     if (workspace_bytes < tc_decode_workspace(a) || !workspace) return MLA_ERR_WORKSPACE;
     return tc_decode_launch(a, as_stream(stream));
   }
+  if (flags & MLA_DECODE_OUT_BF16) return MLA_ERR_UNSUPPORTED;   // the tensor-core route only
   if (workspace_bytes < decode_generic_workspace(a)) return MLA_ERR_WORKSPACE;
   return decode_generic_launch(a, q_dtype, as_stream(stream), MLA_FP8_E4M3);
 }
@@ -272,9 +279,12 @@ int32_t mla_out_project_workspace_size(const mla_dims* dims, int32_t dtype, int6
   return MLA_OK;
 }
 
-int32_t mla_out_project(const mla_dims* dims, int32_t dtype, const float* out_lat, const void* w_uv,
-                        const void* w_o, const void* gate, int64_t n_rows, void* y, void* workspace,
-                        size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+// out_lat in fp32 (lat_bf16 false) or bf16 (the tensor-core decode's MLA_DECODE_OUT_BF16 output)
+static int32_t out_project_impl(const mla_dims* dims, int32_t dtype, const void* out_lat, bool lat_bf16,
+                                const void* w_uv, const void* w_o, const void* gate, int64_t n_rows, void* y,
+                                void* workspace, size_t workspace_bytes, void* stream) {
   int st = check_dims(dims);
   if (st) return st;
   if (!dtype_ok(dtype)) return MLA_ERR_DTYPE;
@@ -292,7 +302,7 @@ int32_t mla_out_project(const mla_dims* dims, int32_t dtype, const float* out_la
   cudaStream_t s = as_stream(stream);
   void* v = workspace;
   if (dtype == MLA_BF16 && tc_out_project_supported(*dims, n_rows))
-    return tc_out_project(*dims, out_lat, w_uv, w_o, gate, n_rows, y, workspace, workspace_bytes, s);
+    return tc_out_project(*dims, out_lat, lat_bf16, w_uv, w_o, gate, n_rows, y, workspace, workspace_bytes, s);
   // stage 1: v[t, h, i] = gate * sum_j out_lat[t, h, j] W_UV[h, i, j]; batch = h, M = t, N = i
   GemmArgs g{};
   g.A = out_lat; g.sa_b = dc; g.sa_m = H * dc; g.sa_k = 1;
@@ -300,7 +310,7 @@ int32_t mla_out_project(const mla_dims* dims, int32_t dtype, const float* out_la
   g.C = v;       g.sc_b = dv; g.sc_m = H * dv; g.sc_n = 1;
   g.G = gate;    g.sg_b = dv; g.sg_m = H * dv; g.sg_n = 1;
   g.M = n_rows; g.N = dv; g.K = dc; g.batch = H;
-  if ((st = gemm_generic(g, MLA_F32, dtype, dtype, dtype, s))) return st;
+  if ((st = gemm_generic(g, lat_bf16 ? MLA_BF16 : MLA_F32, dtype, dtype, dtype, s))) return st;
   // stage 2: y[t, d] = sum_k v[t, k] W_O[d, k]
   GemmArgs o{};
   o.A = v;   o.sa_b = 0; o.sa_m = H * dv; o.sa_k = 1;
@@ -308,6 +318,22 @@ int32_t mla_out_project(const mla_dims* dims, int32_t dtype, const float* out_la
   o.C = y;   o.sc_b = 0; o.sc_m = D; o.sc_n = 1;
   o.M = n_rows; o.N = D; o.K = H * dv; o.batch = 1;
   return gemm_generic(o, dtype, dtype, dtype, dtype, s);
+}
+
+extern "C" {
+
+int32_t mla_out_project(const mla_dims* dims, int32_t dtype, const float* out_lat, const void* w_uv,
+                        const void* w_o, const void* gate, int64_t n_rows, void* y, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  return out_project_impl(dims, dtype, out_lat, false, w_uv, w_o, gate, n_rows, y, workspace, workspace_bytes,
+                          stream);
+}
+
+int32_t mla_out_project_bf16(const mla_dims* dims, const void* out_lat, const void* w_uv, const void* w_o,
+                             const void* gate, int64_t n_rows, void* y, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  return out_project_impl(dims, MLA_BF16, out_lat, true, w_uv, w_o, gate, n_rows, y, workspace, workspace_bytes,
+                          stream);
 }
 
 int32_t mla_linear(int32_t dtype, const void* x, const void* w, int64_t m, int64_t n, int64_t k,
@@ -540,12 +566,20 @@ int32_t mla_decode_step(const mla_dims* dims, int32_t dtype, int32_t q_rank, con
     return st;
   if ((st = mla_absorb_weights(dims, dtype, MLA_ABSORB_QUERY, q_nope, q_pe, w->w_uk, batch, q_abs, stream)))
     return st;
-  if ((st = mla_decode_absorbed(dims, dtype, q_abs, cache, cu_seqlens, batch, 1, max_seqlen, total_rows,
-                                MLA_DECODE_CAUSAL, out_lat, nullptr, scratch, L.dec_bytes, stream)))
-    return st;
-  if ((st = mla_out_project(dims, dtype, out_lat, w->w_uv, w->w_o, nullptr, batch, y_dev, scratch, L.out_bytes,
-                            stream)))
-    return st;
+  // on the tensor-core route the decode writes out_lat in bf16, the W_UV operand, directly
+  st = dtype == MLA_BF16 ? mla_decode_absorbed(dims, dtype, q_abs, cache, cu_seqlens, batch, 1, max_seqlen, total_rows,
+                                               MLA_DECODE_CAUSAL | MLA_DECODE_OUT_BF16, out_lat, nullptr, scratch,
+                                               L.dec_bytes, stream)
+                         : MLA_ERR_UNSUPPORTED;
+  if (st == MLA_OK) {
+    st = mla_out_project_bf16(dims, out_lat, w->w_uv, w->w_o, nullptr, batch, y_dev, scratch, L.out_bytes, stream);
+  } else if (st == MLA_ERR_UNSUPPORTED) {
+    if ((st = mla_decode_absorbed(dims, dtype, q_abs, cache, cu_seqlens, batch, 1, max_seqlen, total_rows,
+                                  MLA_DECODE_CAUSAL, out_lat, nullptr, scratch, L.dec_bytes, stream)))
+      return st;
+    st = mla_out_project(dims, dtype, out_lat, w->w_uv, w->w_o, nullptr, batch, y_dev, scratch, L.out_bytes, stream);
+  }
+  if (st) return st;
   if (io == MLA_IO_HOST && cudaMemcpyAsync(y, y_dev, x_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return MLA_ERR_CUDA;
   return MLA_OK;

@@ -19,9 +19,8 @@ void set_decode_clusters(int n);   // 0 = one cluster per SM pair
 // value + output projection
 bool tc_out_project_supported(const mla_dims& d, int64_t n_rows);
 size_t tc_out_project_extra_workspace(const mla_dims& d, int64_t n_rows);
-int tc_out_project(const mla_dims& d, const float* out_lat, const void* w_uv, const void* w_o,
-                   const void* gate, int64_t n_rows, void* y, void* workspace, size_t ws_bytes,
-                   cudaStream_t s);
+int tc_out_project(const mla_dims& d, const void* out_lat, bool lat_bf16, const void* w_uv, const void* w_o,
+                   const void* gate, int64_t n_rows, void* y, void* workspace, size_t ws_bytes, cudaStream_t s);
 
 // input projections of new tokens (bf16 in, fp32 accumulate): c_q = x W_cq^T and q_nope = c_q W_qc^T
 // in bf16, q_r = c_q W_qr^T and kv = x W_dkv^T in fp32; partial = split-K scratch of

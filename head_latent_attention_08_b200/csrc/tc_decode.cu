@@ -168,6 +168,7 @@ struct DecParams {
   int uniform_tiles;          // > 0: every block has this many tiles (prefix[k] = k * uniform_tiles)
   int G;                      // clusters
   float* out_lat;
+  __nv_bfloat16* out16;        // non-null: out_lat is written here in bf16 instead (whole blocks, combine)
   float* lse;
   float* o_part;              // [2G][128][512]
   float* m_part;              // [2G][128] reference maxima (log2 domain)
@@ -1049,6 +1050,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
               // eight lanes write 128 contiguous bytes of one row
               const int gfirst = q * 32 + (lane & ~7);               // first row of the lane's group
               float* gdst = dst + (int64_t)(gfirst - row) * DEC_DC + cv * 128 + 4 * (lane & 7);
+              const bool bf_out = sg.complete && p.out16 != nullptr;
+              __nv_bfloat16* g16 = bf_out ? p.out16 + ((int64_t)sg.b * rows_seq + sg.rb * DEC_ROWS + gfirst) * DEC_DC +
+                                                cv * 128 + 4 * (lane & 7)
+                                          : nullptr;
               const int grows = !ok ? 0 : (sg.complete ? min(8, rows_seq - (sg.rb * DEC_ROWS + gfirst)) : 8);
 #pragma unroll 1
               for (int cc = 0; cc < 128; cc += 32) {
@@ -1063,9 +1068,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
                                      __float_as_uint(__uint_as_float(r[4 * c + 2]) * mul),
                                      __float_as_uint(__uint_as_float(r[4 * c + 3]) * mul));
                 group8_transpose(ch, lane);
+                if (bf_out) {
+                  // bf16 out_lat: eight lanes write 64 contiguous bytes of a row
 #pragma unroll
-                for (int t = 0; t < 8; ++t)
-                  if (t < grows) *reinterpret_cast<uint4*>(gdst + (int64_t)t * DEC_DC + cc) = ch[t];
+                  for (int t = 0; t < 8; ++t) {
+                    const __nv_bfloat162 lo = __floats2bfloat162_rn(__uint_as_float(ch[t].x), __uint_as_float(ch[t].y));
+                    const __nv_bfloat162 hi = __floats2bfloat162_rn(__uint_as_float(ch[t].z), __uint_as_float(ch[t].w));
+                    if (t < grows)
+                      *reinterpret_cast<uint2*>(g16 + (int64_t)t * DEC_DC + cc) =
+                          make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+                  }
+                } else {
+#pragma unroll
+                  for (int t = 0; t < 8; ++t)
+                    if (t < grows) *reinterpret_cast<uint4*>(gdst + (int64_t)t * DEC_DC + cc) = ch[t];
+                }
               }
               if (ok && cv == 0) {
                 if (sg.complete) {
@@ -1122,10 +1139,20 @@ __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
   const bool row_ok = ri < rows_seq;
   const int64_t orow = (int64_t)b * rows_seq + ri;
   float4* dst = reinterpret_cast<float4*>(p.out_lat + orow * DEC_DC);
+  uint2* dst16 = p.out16 ? reinterpret_cast<uint2*>(p.out16 + orow * DEC_DC) : nullptr;
+  // four consecutive out_lat values (a float4) at float4 index j of the row, in the output's type
+  auto put = [&](int j, float4 v) {
+    if (dst16) {
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+      dst16[j] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+    } else {
+      dst[j] = v;
+    }
+  };
   if (bend == bstart) {
     if (row_ok) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) dst[lane + 32 * j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < 4; ++j) put(lane + 32 * j, make_float4(0.f, 0.f, 0.f, 0.f));
       if (lane == 0 && p.lse) p.lse[orow] = -INFINITY;
     }
     return;
@@ -1182,8 +1209,7 @@ __global__ void __launch_bounds__(256) decode_combine_tc_kernel(DecParams p) {
     }
   }
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
-    dst[lane + 32 * j] = make_float4(acc[j].x * inv, acc[j].y * inv, acc[j].z * inv, acc[j].w * inv);
+  for (int j = 0; j < 4; ++j) put(lane + 32 * j, make_float4(acc[j].x * inv, acc[j].y * inv, acc[j].z * inv, acc[j].w * inv));
   if (lane == 0 && p.lse) p.lse[orow] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
@@ -1303,6 +1329,7 @@ int tc_decode_launch(const DecodeArgs& a, cudaStream_t s) {
   p.prefix = reinterpret_cast<int32_t*>(ws + t.off_prefix);
   p.G = t.G;
   p.out_lat = a.out_lat; p.lse = a.lse;
+  p.out16 = static_cast<__nv_bfloat16*>(a.out_lat_bf16);
   p.o_part = reinterpret_cast<float*>(ws + t.off_o);
   p.m_part = reinterpret_cast<float*>(ws + t.off_m);
   p.l_part = reinterpret_cast<float*>(ws + t.off_l);

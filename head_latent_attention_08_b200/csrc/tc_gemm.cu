@@ -841,21 +841,22 @@ size_t tc_out_project_extra_workspace(const mla_dims& d, int64_t n_rows) {
   return round_up((size_t)n_rows * H * dc * 2, 256) + gemm_partial_bytes((int)D, (int)n_rows, (int)(H * dv), 1);
 }
 
-int tc_out_project(const mla_dims& d, const float* out_lat, const void* w_uv, const void* w_o, const void* gate,
-                   int64_t n_rows, void* y, void* workspace, size_t ws_bytes, cudaStream_t s) {
+int tc_out_project(const mla_dims& d, const void* out_lat, bool lat_bf16, const void* w_uv, const void* w_o,
+                   const void* gate, int64_t n_rows, void* y, void* workspace, size_t ws_bytes, cudaStream_t s) {
   const int64_t H = d.n_heads, dc = d.kv_lora_rank, dv = d.v_head, D = d.d_model;
   char* ws = static_cast<char*>(workspace);
   void* v = ws;
   const size_t v_bytes = round_up((size_t)n_rows * H * dv * 2, 256);
-  void* lat16 = ws + v_bytes;
+  void* lat16 = lat_bf16 ? const_cast<void*>(out_lat) : static_cast<void*>(ws + v_bytes);
   const size_t lat_bytes = round_up((size_t)n_rows * H * dc * 2, 256);
   void* partial = ws + v_bytes + lat_bytes;
   if (ws_bytes < v_bytes + tc_out_project_extra_workspace(d, n_rows)) return MLA_ERR_WORKSPACE;
-  {
+  if (!lat_bf16) {
+    // the W_UV GEMM reads out_lat as its bf16 B operand
     const int64_t n4 = n_rows * H * dc / 4;
     const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(n4, 256), 8 * sm_count());
     const int st0 = launch_pdl(f32_to_bf16_kernel, dim3(blocks), dim3(256), 0, s,
-                               reinterpret_cast<const float4*>(out_lat), static_cast<uint2*>(lat16), n4);
+                               static_cast<const float4*>(out_lat), static_cast<uint2*>(lat16), n4);
     if (st0) return st0;
   }
   // v[t, h, i] = gate * sum_j W_UV[h, i, j] lat[t, h, j]: A = W_UV[h] K-major, B = lat[:, h, :]

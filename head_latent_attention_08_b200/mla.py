@@ -21,7 +21,7 @@ MLA_OK = 0
 MLA_F32, MLA_BF16, MLA_FP8_E4M3 = 0, 1, 2
 MLA_ABSORB_QUERY, MLA_FOLD_QK, MLA_FOLD_VO = 0, 1, 2
 MLA_APPEND_NORM, MLA_APPEND_ROPE = 1, 2
-MLA_DECODE_CAUSAL = 1
+MLA_DECODE_CAUSAL, MLA_DECODE_OUT_BF16 = 1, 2
 MLA_LINEAR_SIGMOID, MLA_LINEAR_W_KN = 1, 2
 MLA_ERR_SHAPE, MLA_ERR_TIMEOUT = 2, 7
 MLA_IO_DEVICE, MLA_IO_HOST = 0, 1
@@ -33,6 +33,7 @@ EXPORTED = (
     "mla_set_decode_clusters", "mla_wait_selftest", "mla_decode_absorbed_noalloc",
     "mla_project_workspace_size", "mla_project_inputs", "mla_decode_step_workspace_size", "mla_decode_step",
     "mla_lse_merge", "mla_prefill_attention", "mla_append_latent_fp8", "mla_decode_absorbed_fp8",
+    "mla_out_project_bf16",
 )
 
 
@@ -72,6 +73,7 @@ _SIGS = {
                                    _SZ, _P]),
     "mla_out_project_workspace_size": (_I32, [_DIMS, _I32, _I64, ctypes.POINTER(_SZ)]),
     "mla_out_project": (_I32, [_DIMS, _I32, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
+    "mla_out_project_bf16": (_I32, [_DIMS, _P, _P, _P, _P, _I64, _P, _P, _SZ, _P]),
     "mla_linear": (_I32, [_I32, _P, _P, _I64, _I64, _I64, _U32, _P, _P]),
     "mla_check_status": (_I32, [_P, ctypes.POINTER(_I32)]),
     "mla_set_wait_limit": (_I32, [_I64]),
@@ -192,7 +194,8 @@ def mla_decode_absorbed(d: mla_dims, q_abs: torch.Tensor, cache: torch.Tensor, c
                         batch: int, n_q: int, max_seqlen: int, flags: int, out_lat: torch.Tensor,
                         lse: Optional[torch.Tensor], workspace: Optional[torch.Tensor],
                         stream=None) -> None:
-    assert cu_seqlens.dtype == torch.int32 and out_lat.dtype == torch.float32
+    assert cu_seqlens.dtype == torch.int32
+    assert out_lat.dtype == (torch.bfloat16 if flags & MLA_DECODE_OUT_BF16 else torch.float32)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().mla_decode_absorbed(ctypes.byref(d), _dtype_code(q_abs.dtype), _ptr(q_abs), _ptr(cache),
                                      _ptr(cu_seqlens), batch, n_q, max_seqlen, cache.shape[0], flags,
@@ -227,6 +230,16 @@ def mla_out_project(d: mla_dims, out_lat: torch.Tensor, w_uv: torch.Tensor, w_o:
     _check(lib().mla_out_project(ctypes.byref(d), _dtype_code(w_uv.dtype), _ptr(out_lat), _ptr(w_uv),
                                  _ptr(w_o), _ptr(gate), n_rows, _ptr(y), _ptr(workspace), ws_bytes,
                                  _stream(stream)), "mla_out_project")
+
+
+def mla_out_project_bf16(d: mla_dims, out_lat: torch.Tensor, w_uv: torch.Tensor, w_o: torch.Tensor,
+                         gate: Optional[torch.Tensor], n_rows: int, y: torch.Tensor,
+                         workspace: torch.Tensor, stream=None) -> None:
+    """mla_out_project with a bf16 out_lat (the decode's MLA_DECODE_OUT_BF16 output)."""
+    assert out_lat.dtype == torch.bfloat16
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().mla_out_project_bf16(ctypes.byref(d), _ptr(out_lat), _ptr(w_uv), _ptr(w_o), _ptr(gate), n_rows,
+                                      _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)), "mla_out_project_bf16")
 
 
 def mla_linear(x: torch.Tensor, w: torch.Tensor, m: int, n: int, k: int, flags: int, y: torch.Tensor,
@@ -318,7 +331,8 @@ def mla_decode_absorbed_fp8(d: mla_dims, q_abs: torch.Tensor, cache: torch.Tenso
                             cu_seqlens: torch.Tensor, batch: int, n_q: int, max_seqlen: int, flags: int,
                             out_lat: torch.Tensor, lse: Optional[torch.Tensor], workspace: Optional[torch.Tensor],
                             stream=None) -> None:
-    assert cu_seqlens.dtype == torch.int32 and out_lat.dtype == torch.float32
+    assert cu_seqlens.dtype == torch.int32
+    assert out_lat.dtype == (torch.bfloat16 if flags & MLA_DECODE_OUT_BF16 else torch.float32)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().mla_decode_absorbed_fp8(ctypes.byref(d), _dtype_code(q_abs.dtype), _ptr(q_abs), _ptr(cache),
                                          cache_scale, _ptr(cu_seqlens), batch, n_q, max_seqlen, cache.shape[0],

@@ -83,7 +83,7 @@ enum { MLA_ABSORB_QUERY = 0, MLA_FOLD_QK = 1, MLA_FOLD_VO = 2 };
 /* flags of mla_append_latent */
 enum { MLA_APPEND_NORM = 1u, MLA_APPEND_ROPE = 2u };
 /* flags of mla_decode_absorbed */
-enum { MLA_DECODE_CAUSAL = 1u };
+enum { MLA_DECODE_CAUSAL = 1u, MLA_DECODE_OUT_BF16 = 2u };
 /* flags of mla_linear */
 enum { MLA_LINEAR_SIGMOID = 1u, MLA_LINEAR_W_KN = 2u };
 /* where the step's x, y and index arrays live (mla_decode_step) */
@@ -178,7 +178,10 @@ MLA_API int32_t mla_decode_workspace_size(const mla_dims* dims, int32_t dtype, i
  *   cu_seqlens  DEVICE int32 [B + 1], non-decreasing, cu_seqlens[0] = 0, cu_seqlens[B] = total_rows.
  *   flags       MLA_DECODE_CAUSAL: query j of sequence b (the n_q newest tokens sit at its last
  *               n_q rows) sees positions t <= T_b - n_q + j; otherwise it sees all T_b positions.
- *   out_lat     float [B * n_q, H, d_c]: the softmax-weighted latent (zeros when nothing is seen).
+ *               MLA_DECODE_OUT_BF16: out_lat is written in bf16 instead (the operand of
+ *               mla_out_project_bf16); tensor-core route only, else MLA_ERR_UNSUPPORTED.
+ *   out_lat     float [B * n_q, H, d_c] (bf16 under MLA_DECODE_OUT_BF16): the softmax-weighted latent
+ *               (zeros when nothing is seen).
  *   lse         float [B * n_q, H] or NULL: natural-log sum-exp of the scaled scores (-inf if empty).
  *   workspace   caller scratch of at least mla_decode_workspace_size() bytes, 256-byte aligned.
  * Requirements: T_b <= max_seqlen for every b (not checked on the device: the plan assumes it
@@ -228,6 +231,15 @@ MLA_API int32_t mla_out_project_workspace_size(const mla_dims* dims, int32_t dty
 MLA_API int32_t mla_out_project(const mla_dims* dims, int32_t dtype, const float* out_lat, const void* w_uv,
                         const void* w_o, const void* gate, int64_t n_rows, void* y,
                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * mla_out_project_bf16 -- mla_out_project (dtype MLA_BF16) with out_lat in bf16 [n_rows, H, d_c], as
+ * mla_decode_absorbed writes it under MLA_DECODE_OUT_BF16: the W_UV product reads it directly (no
+ * fp32 -> bf16 conversion pass). out_lat 16-byte aligned; scratch as for mla_out_project.
+ */
+MLA_API int32_t mla_out_project_bf16(const mla_dims* dims, const void* out_lat, const void* w_uv, const void* w_o,
+                                     const void* gate, int64_t n_rows, void* y, void* workspace,
+                                     size_t workspace_bytes, void* stream);
 
 /*
  * mla_linear -- Y = X W^T ([gm] problem equations, PyTorch Linear convention W = [n, k]).

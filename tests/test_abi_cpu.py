@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mla_abi_version() == 2
+    assert lib.mla_abi_version() == 3
     for s in range(10):
         assert lib.mla_status_string(s)
     assert b"unknown" in lib.mla_status_string(1234)
@@ -55,7 +55,7 @@ def test_validation_errors_return_before_launch(lib):
     assert lib.mla_absorb_weights(ctypes.byref(d), 7, 0, FAKE, FAKE, FAKE, 1, FAKE, None) == 3
     assert lib.mla_absorb_weights(ctypes.byref(d), 0, 42, FAKE, FAKE, FAKE, 1, FAKE, None) == 9
     assert lib.mla_append_latent(ctypes.byref(d), 1, FAKE, 10, FAKE, FAKE, FAKE, FAKE, 1, 8, 1e-6, 1e4, None) == 9
-    assert lib.mla_decode_absorbed(ctypes.byref(d), 1, FAKE, FAKE, FAKE, 1, 1, 4, 4, 2, FAKE, None,
+    assert lib.mla_decode_absorbed(ctypes.byref(d), 1, FAKE, FAKE, FAKE, 1, 1, 4, 4, 4, FAKE, None,
                                    FAKE, 1 << 20, None) == 9
     assert lib.mla_linear(0, FAKE, FAKE, 2, 2, 2, 4, FAKE, None) == 9
     # NULL operands
