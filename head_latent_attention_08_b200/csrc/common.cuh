@@ -131,13 +131,6 @@ int append_latent_strided(const mla_dims& d, int32_t cache_dtype, void* cache, i
                           const int64_t* row_idx, const float* c_new, int64_t c_stride, const float* kpe_new,
                           int64_t kpe_stride, const int32_t* positions, int64_t n_new, uint32_t flags,
                           float eps, float theta, cudaStream_t stream, float cache_scale = 1.f);
-// the same, with c_new and kpe_new given as n_parts arrays part_stride floats apart, added in order
-// (the K-split partials of the projection that made them)
-int append_latent_parts(const mla_dims& d, int32_t cache_dtype, void* cache, int64_t cache_rows,
-                        const int64_t* row_idx, const float* c_new, int64_t c_stride, const float* kpe_new,
-                        int64_t kpe_stride, const int32_t* positions, int64_t n_new, uint32_t flags, float eps,
-                        float theta, cudaStream_t stream, float cache_scale, int n_parts, int64_t part_stride);
-
 // log-sum-exp merge of n_parts partial decode results (rows row0 .. row0 + n_rows of each part)
 int lse_merge_launch(int n_parts, const float* const* o_parts, const float* const* l_parts, int64_t row0,
                      int64_t n_rows, int H, int dc, float* out_lat, float* lse, cudaStream_t stream);

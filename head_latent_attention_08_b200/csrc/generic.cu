@@ -197,8 +197,7 @@ __global__ void __launch_bounds__(128) append_latent_kernel(
     T* __restrict__ cache, const int64_t* __restrict__ row_idx, const float* __restrict__ c_new,
     int64_t c_stride, const float* __restrict__ kpe_new, int64_t kpe_stride,
     const int32_t* __restrict__ positions, int dc, int dr,
-    uint32_t flags, float eps, double log2_theta, int vec8, int64_t cache_rows, int* status, float cache_scale,
-    int n_parts, int64_t part_stride) {
+    uint32_t flags, float eps, double log2_theta, int vec8, int64_t cache_rows, int* status, float cache_scale) {
   extern __shared__ float row[];
   __shared__ float red[4];
   griddep_wait();
@@ -210,16 +209,9 @@ __global__ void __launch_bounds__(128) append_latent_kernel(
     return;
   }
   const int W = dc + dr;
-  // the new row's values: one array, or the K-split partials of the projection that made them, added
-  // in split order
-  auto value = [&](const float* base, int64_t off) {
-    float v = base[off];
-    for (int q = 1; q < n_parts; ++q) v += base[q * part_stride + off];
-    return v;
-  };
   float ss = 0.f;
   for (int i = threadIdx.x; i < dc; i += blockDim.x) {
-    const float x = value(c_new, (int64_t)k * c_stride + i);
+    const float x = c_new[(int64_t)k * c_stride + i];
     row[i] = x;
     ss = fmaf(x, x, ss);
   }
@@ -238,12 +230,12 @@ __global__ void __launch_bounds__(128) append_latent_kernel(
       for (int i = threadIdx.x; i < dr / 2; i += blockDim.x) {
         float sn, cs;
         rope_sincos(pos, i, dr, log2_theta, &sn, &cs);
-        const float x0 = value(kpe_new, kp + 2 * i), x1 = value(kpe_new, kp + 2 * i + 1);
+        const float x0 = kpe_new[kp + 2 * i], x1 = kpe_new[kp + 2 * i + 1];
         row[dc + 2 * i] = fmaf(x0, cs, -x1 * sn);
         row[dc + 2 * i + 1] = fmaf(x0, sn, x1 * cs);
       }
     } else {
-      for (int i = threadIdx.x; i < dr; i += blockDim.x) row[dc + i] = value(kpe_new, kp + i);
+      for (int i = threadIdx.x; i < dr; i += blockDim.x) row[dc + i] = kpe_new[kp + i];
     }
   }
   __syncthreads();
@@ -288,14 +280,6 @@ int append_latent_strided(const mla_dims& d, int32_t cache_dtype, void* cache, i
                           const int64_t* row_idx, const float* c_new, int64_t c_stride, const float* kpe_new,
                           int64_t kpe_stride, const int32_t* positions, int64_t n_new, uint32_t flags,
                           float eps, float theta, cudaStream_t s, float cache_scale) {
-  return append_latent_parts(d, cache_dtype, cache, cache_rows, row_idx, c_new, c_stride, kpe_new, kpe_stride,
-                             positions, n_new, flags, eps, theta, s, cache_scale, 1, 0);
-}
-
-int append_latent_parts(const mla_dims& d, int32_t cache_dtype, void* cache, int64_t cache_rows,
-                        const int64_t* row_idx, const float* c_new, int64_t c_stride, const float* kpe_new,
-                        int64_t kpe_stride, const int32_t* positions, int64_t n_new, uint32_t flags, float eps,
-                        float theta, cudaStream_t s, float cache_scale, int n_parts, int64_t part_stride) {
   int* status = device_status_ptr();
   if (!status) return MLA_ERR_CUDA;
   if (n_new == 0) return MLA_OK;
@@ -309,15 +293,15 @@ int append_latent_parts(const mla_dims& d, int32_t cache_dtype, void* cache, int
     return launch_pdl(append_latent_kernel<__nv_bfloat16>, dim3((unsigned)n_new), dim3(128), smem, s,
                       static_cast<__nv_bfloat16*>(cache), row_idx, c_new, c_stride, kpe_new, kpe_stride,
                       positions, d.kv_lora_rank, d.rope_dim, flags, eps, log2((double)theta), vec8, cache_rows,
-                      status, 1.f, n_parts, part_stride);
+                      status, 1.f);
   if (cache_dtype == MLA_FP8_E4M3)
     return launch_pdl(append_latent_kernel<__nv_fp8_e4m3>, dim3((unsigned)n_new), dim3(128), smem, s,
                       static_cast<__nv_fp8_e4m3*>(cache), row_idx, c_new, c_stride, kpe_new, kpe_stride,
                       positions, d.kv_lora_rank, d.rope_dim, flags, eps, log2((double)theta), 0, cache_rows,
-                      status, cache_scale, n_parts, part_stride);
+                      status, cache_scale);
   append_latent_kernel<float><<<(unsigned)n_new, 128, smem, s>>>(
       static_cast<float*>(cache), row_idx, c_new, c_stride, kpe_new, kpe_stride, positions, d.kv_lora_rank,
-      d.rope_dim, flags, eps, log2((double)theta), vec8, cache_rows, status, 1.f, n_parts, part_stride);
+      d.rope_dim, flags, eps, log2((double)theta), vec8, cache_rows, status, 1.f);
   MLA_LAUNCH_CHECK();
   return MLA_OK;
 }

@@ -446,9 +446,8 @@ int32_t mla_project_inputs(const mla_dims* dims, int32_t dtype, int32_t q_rank, 
   float* q_r = reinterpret_cast<float*>(ws + L.q_r);
   float* kv = reinterpret_cast<float*>(ws + L.kv);
   cudaStream_t s = as_stream(stream);
-  // the KV and rotary-query products may come back as K-split partials, which their consumers (the
-  // append and the rotation) add in order
-  ProjectParts parts{kv, 1, 0, q_r, 1, 0};
+  // the rotary-query product may come back as K-split partials, which the rotation adds in order
+  ProjectParts parts{q_r, 1, 0};
   if (dtype == MLA_BF16 && tc_project_supported(*dims, q_rank, n_rows))
     st = tc_project(*dims, q_rank, x, w_cq, w_qc, w_qr, w_dkv, n_rows, c_q, q_nope, q_r, kv, ws + L.partial, s,
                     &parts);
@@ -460,8 +459,8 @@ int32_t mla_project_inputs(const mla_dims* dims, int32_t dtype, int32_t q_rank, 
                                        rope_theta, s, parts.qr_parts, parts.qr_stride)))
     return st;
   const int64_t W = dims->kv_lora_rank + dr;
-  return append_latent_parts(*dims, dtype, cache, cache_rows, row_idx, parts.kv, W, parts.kv + dims->kv_lora_rank, W,
-                             positions, n_rows, flags, eps, rope_theta, s, 1.f, parts.kv_parts, parts.kv_stride);
+  return append_latent_strided(*dims, dtype, cache, cache_rows, row_idx, kv, W, kv + dims->kv_lora_rank, W, positions,
+                               n_rows, flags, eps, rope_theta, s);
 }
 
 // ---------------------------------------------------------------------------------------------

@@ -28,8 +28,9 @@ int tc_out_project(const mla_dims& d, const void* out_lat, bool lat_bf16, const 
 // The KV and rotary-query products come back as `parts` fp32 arrays `stride` floats apart (their
 // K-split partials, to be added in order; one array when the product was not split).
 struct ProjectParts {
-  const float* kv; int kv_parts; int64_t kv_stride;
-  const float* qr; int qr_parts; int64_t qr_stride;
+  const float* qr;     // the rotary query product q_r, or its first K-split partial
+  int qr_parts;        // partials to add in order (1: q_r itself)
+  int64_t qr_stride;   // floats between partials
 };
 bool tc_project_supported(const mla_dims& d, int64_t q_rank, int64_t n_rows);
 size_t tc_project_partial_bytes(const mla_dims& d, int64_t q_rank, int64_t n_rows);

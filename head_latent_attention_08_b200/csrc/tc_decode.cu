@@ -65,7 +65,6 @@ constexpr int DEC_SW = 16;         // softmax / epilogue warps
 constexpr int DEC_DC = 512;        // latent width handled by this kernel
 constexpr int DEC_ROWS = 128;      // rows per block
 constexpr int DEC_NPH = 6;         // P hand-over slots in the value CTA (at most)
-constexpr int DEC_PF = 2;          // cache tiles warmed in L2 ahead of the tile QK^T works on
 constexpr int DEC_NPROD = 3;       // TMA-issuing threads of the score CTA
 constexpr float DEC_MOVE = 8.f;    // the reference maximum moves when a row maximum exceeds it by 2^8
 constexpr int DEC_SMEM_LIMIT = 232448;   // dynamic shared memory per CTA (227 KB)

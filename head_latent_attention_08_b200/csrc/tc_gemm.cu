@@ -893,8 +893,8 @@ static void project_gemm_dims(const mla_dims& d, int64_t q_rank, int64_t n_rows,
   }
 }
 
-// split-K scratch of the four products, one region each: the KV and rotary-query partials are read
-// later, by the append and the rotation
+// split-K scratch of the four products, one region each: the rotary-query partials are read
+// later, by the rotation kernel
 static void project_partial_offsets(const mla_dims& d, int64_t q_rank, int64_t n_rows, size_t off[5]) {
   int g[4][3];
   project_gemm_dims(d, q_rank, n_rows, g);
@@ -920,9 +920,6 @@ int tc_project(const mla_dims& d, int64_t q_rank, const void* x, const void* w_c
   // (the KV product keeps its own reduce: the append runs one block per token and would read the
   // partials with too few threads)
   const int qr_splits = g[2][0] > 0 ? plan_gemm(g[2][0], g[2][1], g[2][2], 1, 1 << 20).splits : 1;
-  parts->kv = kv;
-  parts->kv_parts = 1;
-  parts->kv_stride = 0;
   parts->qr = qr_splits > 1 ? reinterpret_cast<const float*>(pw + off[2]) : q_r;
   parts->qr_parts = qr_splits;
   parts->qr_stride = (int64_t)g[2][1] * g[2][0];
