@@ -209,7 +209,8 @@ MLA_DECODE_NOALLOC_MAX_BYTES = 40 << 20
 def mla_decode_absorbed_noalloc(d: mla_dims, q_abs: torch.Tensor, cache: torch.Tensor,
                                 cu_seqlens: torch.Tensor, batch: int, n_q: int, max_seqlen: int, flags: int,
                                 out_lat: torch.Tensor, lse: Optional[torch.Tensor], stream=None) -> None:
-    assert cu_seqlens.dtype == torch.int32 and out_lat.dtype == torch.float32
+    assert cu_seqlens.dtype == torch.int32
+    assert out_lat.dtype == (torch.bfloat16 if flags & MLA_DECODE_OUT_BF16 else torch.float32)
     _check(lib().mla_decode_absorbed_noalloc(ctypes.byref(d), _dtype_code(q_abs.dtype), _ptr(q_abs),
                                              _ptr(cache), _ptr(cu_seqlens), batch, n_q, max_seqlen,
                                              cache.shape[0], flags, _ptr(out_lat), _ptr(lse),

@@ -178,3 +178,28 @@ def test_decode_fp8_deepseek_scale_sampled():
         ref, ref_lse = O.decode_absorbed(q[b:b + 1], rows, np.array([0, T]), 1, 512, kq, True)
         assert_close(out[b:b + 1], ref, "bf16", f"out_lat b={b}")
         assert_lse_close(lse[b:b + 1], ref_lse, "bf16", f"lse b={b}")
+
+
+def test_decode_fp8_empty_and_short_sequences():
+    """Tensor-core route over an e4m3 cache with an empty sequence (zeros and -inf lse), a one-position
+    sequence and one that ends one position into a second tile (ragged: plan and combine run)."""
+    p = I.decode_problem(batch=3, n_heads=128, kv_lora_rank=512, rope_dim=64, qk_nope=64, v_head=64,
+                         d_model=64, seqlens=[1, 257, 40], n_q=1, dtype="bf16", seed=96, cache_dtype="e4m3")
+    rng = np.random.default_rng(96)
+    q_abs = O.store_as(np.concatenate([rng.standard_normal((1, 128, 576)),
+                                       O.absorb_query(p.q_nope, p.q_pe, p.w_uk)]), "bf16")
+    cu = np.concatenate([[0], p.cu_seqlens]).astype(np.int64)          # sequence 0 holds no positions
+    d = M.dims(128, 512, 64, 64, 64, 64)
+    out = torch.empty(4, 128, 512, device="cuda")
+    lse = torch.empty(4, 128, device="cuda")
+    codes = to_codes(p.cache)
+    ws = M.workspace(M.mla_decode_workspace_size(d, torch.uint8, 4, 1, 257, codes.shape[0], 0), "cuda")
+    M.mla_decode_absorbed_fp8(d, dev(q_abs, "bf16"), codes, 2.0, torch.from_numpy(cu.astype(np.int32)).cuda(), 4, 1,
+                              257, 0, out, lse, ws)
+    torch.cuda.synchronize()
+    assert M.mla_check_status() == M.MLA_OK
+    out, lse = host(out), host(lse)
+    ref, ref_lse = O.decode_absorbed(q_abs, p.cache.astype(np.float64) * 2.0, cu, 1, 512, p.kq_scale, False)
+    assert np.all(out[0] == 0) and np.all(np.isneginf(lse[0]))
+    assert_close(out, ref, "bf16", "out_lat")
+    assert_lse_close(lse, ref_lse, "bf16", "lse")
