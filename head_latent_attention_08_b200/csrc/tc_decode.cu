@@ -68,7 +68,7 @@ constexpr int DEC_NPH = 6;         // P hand-over slots in the value CTA (at mos
 constexpr int DEC_NPROD = 3;       // TMA-issuing threads of the score CTA
 constexpr float DEC_MOVE = 8.f;    // the reference maximum moves when a row maximum exceeds it by 2^8
 constexpr int DEC_SMEM_LIMIT = 232448;   // dynamic shared memory per CTA (227 KB)
-constexpr int DEC_BAR_BYTES = 1024;
+constexpr int DEC_BAR_BYTES = 4096;
 
 __host__ __device__ constexpr int dec_round1024(int x) { return (x + 1023) / 1024 * 1024; }
 __host__ __device__ constexpr int dec_max(int a, int b) { return a > b ? a : b; }
@@ -98,10 +98,12 @@ struct DecCfg {
   static constexpr int SIDE = 4 * 512;                     // side data of a hand-over: 4 quarters x 512 B
   static constexpr int PSLOT = PH + SIDE;                  // 18 KB (a multiple of 1024)
   // bytes that land in a P slot for hand-over cg of a tile: P, then per warp a 16-byte header (the
-  // flag), the row factors on the tile's first hand-over and the row maxima and sums on its last
-  // (read at the last tile of a block segment)
+  // flag), the row factors on the tile's first hand-over and the row maxima on its last (read at the
+  // last tile of a block segment), over an e4m3 cache the row sums with them. (With a bf16 cache the
+  // value CTA's rescale warps add the row sums up from the P slots themselves; the value CTA of the
+  // e4m3 path is bound by its shared-memory traffic, so there the score CTA keeps them.)
   static __host__ __device__ constexpr uint32_t slot_tx(int cg) {
-    return (uint32_t)(PH + 4 * (16 + (cg == 0 ? 128 : 0) + (cg == DEC_QT - 1 ? 256 : 0)));
+    return (uint32_t)(PH + 4 * (16 + (cg == 0 ? 128 : 0) + (cg == DEC_QT - 1 ? (F8 ? 256 : 128) : 0)));
   }
   static constexpr int NPH = DEC_NPH;                      // P slots
   static constexpr int V_OFF_P = 0;
@@ -128,7 +130,7 @@ struct DecSide {
   int pad[3];
   float alpha[32];   // factor for O of each row (1 where the reference did not move)
   float m[32];       // reference maximum (log2 units) after this tile
-  float l[32];       // row sum after this tile (whole row at the last tile of a block)
+  float l[32];       // e4m3 cache: row sum after this tile (whole row at the last tile of a block)
   float pad2[28];
 };
 static_assert(sizeof(DecSide) == 512, "side record size");
@@ -147,6 +149,7 @@ struct DecBars {
   uint64_t pfree[DEC_NPH];        // P.C read the slot and the rescale/epilogue warps read its side data
   uint64_t o_fix, fix_done;       // rescale hand-shake (one phase per rescale)
   uint64_t o_fin, o_free;         // epilogue hand-shake (one phase per block segment)
+  float lsum[4][DEC_ROWS];        // the rescale warps' partial row sums at a segment's end
   // both
   uint64_t drain[2];
   uint32_t tmem_base;
@@ -694,7 +697,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->q_tm);
         const int cnt = row_count(sg.T, p.n_q, p.H, sg.rb * DEC_ROWS + row, p.causal);
-        float m_ref = -INFINITY, l = 0.f;
+        float m_ref = -INFINITY, l = 0.f;   // (l: e4m3 cache only)
         for (int tt = 0; tt < sg.ntl; ++tt, ++g) {
           const bool last = tt + 1 == sg.ntl;
           float s[64];
@@ -754,9 +757,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
           const uint32_t bar = pf_remote + (uint32_t)(hs * 8);
           const uint32_t prow = dst + (uint32_t)(row * 128);
           // P in bf16 (round to nearest even), 8 positions (16 bytes, one swizzled chunk of the row) at a
-          // time, and the row sum of the same rounded values, so that numerator and denominator share
-          // the rounding. Over an e4m3 cache P is f16 (the type of the converted codes; 11 bits, so the
-          // row sum takes the unrounded values)
+          // time; the value CTA adds the row sums up from the same stored values. Over an e4m3 cache P is
+          // f16 (the type of the converted codes; 11 bits) and the row sum, of the unrounded values, is
+          // kept here.
           float sum = 0.f;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -771,24 +774,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
               } else {
                 const __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
                 pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
-                sum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
               }
             }
             if (send) st_async_v4(prow + (uint32_t)((c ^ (lane & 7)) * 16), make_uint4(pk[0], pk[1], pk[2], pk[3]), bar);
           }
-          l += sum;
-          float lsend = l;
-          if (last) {
-            // the block's row sum is the sum of the four warps' sums: the last warp of the row sends it
-            float* ls = red + 8 * DEC_ROWS;
-            ls[cg * DEC_ROWS + row] = l;
-            named_bar_sync(1 + q, 128);
-            if (cg == DEC_QT - 1)
-              lsend = (ls[row] + ls[DEC_ROWS + row]) + (ls[2 * DEC_ROWS + row] + ls[3 * DEC_ROWS + row]);
+          float lsend = 0.f;
+          if constexpr (F8) {
+            l += sum;
+            lsend = l;
+            if (last) {
+              // the block's row sum is the sum of the four warps' sums: the last warp of the row sends it
+              float* ls = red + 8 * DEC_ROWS;
+              ls[cg * DEC_ROWS + row] = l;
+              named_bar_sync(1 + q, 128);
+              if (cg == DEC_QT - 1)
+                lsend = (ls[row] + ls[DEC_ROWS + row]) + (ls[2 * DEC_ROWS + row] + ls[3 * DEC_ROWS + row]);
+            }
           }
           const int flag = (cg == 0) ? (__any_sync(0xffffffffu, moved) ? 1 : 0) : 0;
           // side data in 16-byte stores: the flag on every hand-over, the row factors on the tile's
-          // first, the maxima and sums on its last (the value CTA reads them at a segment's end)
+          // first, the maxima on its last (the value CTA reads them at a segment's end)
           const uint32_t sd = dst + (uint32_t)(Cfg::PH + q * 512);
           const int src4 = (4 * lane) & 31;     // lanes 0..7 gather rows 4 lane .. 4 lane + 3
           if (send && lane == 0) st_async_v4(sd + offsetof(DecSide, flag), make_uint4((uint32_t)flag, 0u, 0u, 0u), bar);
@@ -801,18 +806,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
             if (send && lane < 8) st_async_v4(sd + offsetof(DecSide, alpha) + 16 * lane, v, bar);
           }
           if (cg == DEC_QT - 1) {
-            uint4 vm, vl;
+            uint4 vm;
             vm.x = __float_as_uint(__shfl_sync(0xffffffffu, m_ref, src4));
             vm.y = __float_as_uint(__shfl_sync(0xffffffffu, m_ref, src4 + 1));
             vm.z = __float_as_uint(__shfl_sync(0xffffffffu, m_ref, src4 + 2));
             vm.w = __float_as_uint(__shfl_sync(0xffffffffu, m_ref, src4 + 3));
-            vl.x = __float_as_uint(__shfl_sync(0xffffffffu, lsend, src4));
-            vl.y = __float_as_uint(__shfl_sync(0xffffffffu, lsend, src4 + 1));
-            vl.z = __float_as_uint(__shfl_sync(0xffffffffu, lsend, src4 + 2));
-            vl.w = __float_as_uint(__shfl_sync(0xffffffffu, lsend, src4 + 3));
-            if (send && lane < 8) {
-              st_async_v4(sd + offsetof(DecSide, m) + 16 * lane, vm, bar);
-              st_async_v4(sd + offsetof(DecSide, l) + 16 * lane, vl, bar);
+            if (send && lane < 8) st_async_v4(sd + offsetof(DecSide, m) + 16 * lane, vm, bar);
+            if constexpr (F8) {
+              uint4 vl;
+              vl.x = __float_as_uint(__shfl_sync(0xffffffffu, lsend, src4));
+              vl.y = __float_as_uint(__shfl_sync(0xffffffffu, lsend, src4 + 1));
+              vl.z = __float_as_uint(__shfl_sync(0xffffffffu, lsend, src4 + 2));
+              vl.w = __float_as_uint(__shfl_sync(0xffffffffu, lsend, src4 + 3));
+              if (send && lane < 8) st_async_v4(sd + offsetof(DecSide, l) + 16 * lane, vl, bar);
             }
           }
         }
@@ -1000,6 +1006,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
       int64_t i = 0;
       int segi = 0, fixes = 0;
       while (w.next(p, sg)) {
+        float lp = 0.f;   // the row's sum over positions 16 cv .. 16 cv + 15 of every hand-over so far
         for (int tt = 0; tt < sg.ntl; ++tt) {
           for (int cg = 0; cg < DEC_QT; ++cg, ++i) {
             const int hs = (int)(i % NPH);
@@ -1027,14 +1034,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DEC_THREADS, 1)
                 }
                 tmem_wait_st();
               }
+              if (sd[q].flag) lp *= sd[q].alpha[lane];   // the row sum follows the reference as O does
               tc_fence_before();
               __syncwarp();
               if (lane == 0 && !*abort_flag) mbar_arrive(&bars->fix_done);
             }
+            if constexpr (!F8) {
+              // this hand-over's P (the values the P.C MMAs read), positions 16 cv .. 16 cv + 15 of the
+              // row (two swizzled 16-byte chunks), into the row sum
+              const uint8_t* prow = sP + hs * Cfg::PSLOT + row * 128;
+              const uint4 pa = *reinterpret_cast<const uint4*>(prow + (((2 * cv) ^ (row & 7)) << 4));
+              const uint4 pb = *reinterpret_cast<const uint4*>(prow + (((2 * cv + 1) ^ (row & 7)) << 4));
+              const uint32_t pw[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+              float ps = 0.f;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) ps += __uint_as_float(pw[e] << 16) + __uint_as_float(pw[e] & 0xFFFF0000u);
+              lp += ps;
+            }
             if (tt + 1 == sg.ntl && cg == DEC_QT - 1) {
               // ---- epilogue of the segment: O / l (whole block) or the partial (O, m, l)
               const float m_ref = sd[q].m[lane];
-              const float ltot = sd[q].l[lane];
+              // the row sum: the four warps' parts of the row, added in a fixed order (e4m3 cache: sent
+              // by the score CTA)
+              float ltot;
+              if constexpr (F8) {
+                ltot = sd[q].l[lane];
+              } else {
+                bars->lsum[cv][row] = lp;
+                named_bar_sync(1 + q, 128);
+                ltot = (bars->lsum[0][row] + bars->lsum[1][row]) + (bars->lsum[2][row] + bars->lsum[3][row]);
+              }
               const bool ok = wait_bar(&bars->o_fin, (uint32_t)segi & 1u);
               tc_fence_after();
               const int ri = sg.rb * DEC_ROWS + row;
