@@ -18,10 +18,11 @@
 //        fp32 into a 256-column TMEM slot with N = 256 MMAs, runs the online softmax in fp32 and hands
 //        P (bf16) to the value CTA through distributed shared memory (remote st.async stores counted
 //        by the value CTA's barrier), 64 positions at a time, with per-row side data (the factor by
-//        which O must be rescaled, and at the end of a block the row maximum and sum);
+//        which O must be rescaled, and the row maxima at the end of each tile);
 //      - the value CTA (rank 1) holds all of O in TMEM, streams the latent columns of the same rows
 //        (read a second time, from L2, right after the score CTA brought them in) and accumulates
-//        O += P . C with 128 x 256 x 16 MMAs, rescales O rows when told to, and writes the result.
+//        O += P . C with 128 x 256 x 16 MMAs, rescales O rows when told to, adds the row sums up from
+//        the P it receives, and writes the result.
 //    The scores never leave the score CTA, and they are never rounded below fp32 before the
 //    exponential: the hand-over is one-way (P and side data forward, "slot free" back).
 //  * The score CTA rescales nothing: P is taken against a reference maximum that moves only when a
@@ -36,12 +37,14 @@
 //  * Warp roles (640 threads). Score CTA: warps 0, 2, 3 lane 0 TMA, warp 1 lane 0 QK^T, warps 4-19
 //    softmax (warp w: rows 32 (w & 3) .., positions [64 c, 64 c + 64) of each tile, c = (w - 4) >> 2),
 //    which also move each block's latent query into TMEM. Value CTA: warps 0 and 3 lane 0 TMA, warp 1
-//    lane 0 P.C, warp 2 lane 0 hands P slots back, warps 4-19 rescale and write O (warp w: rows
-//    32 (w & 3) .., O columns [128 c, 128 c + 128)).
+//    lane 0 P.C, warp 2 lane 0 hands P slots back, warps 4-19 rescale O, add the row sums up (16
+//    positions of every hand-over each) and write O (warp w: rows 32 (w & 3) .., O columns
+//    [128 c, 128 c + 128)).
 //  * An e4m3 cache (F8; value = code * cache_scale) keeps the same structure: the score CTA streams
 //    128-column boxes and runs QK^T as kind::f8f6f4 MMAs against the query split into e4m3 high and
 //    low parts (per-row power-of-two scale, both parts in TMEM), and the value CTA stages its units
-//    as e4m3 and its rescale warps convert them exactly to f16 for an f16 P.C (P in f16).
+//    as e4m3 and its rescale warps convert them exactly to f16 for an f16 P.C (P in f16); there the
+//    score CTA keeps the row sums and sends them with the maxima.
 //  * Every wait is bounded (global-timer limit); a wait that gives up sets the library's status word,
 //    and the CTA abandons its work: it issues nothing more, drains its own TMA loads, MMAs and bulk
 //    copies and leaves through the cluster barrier.
