@@ -3,6 +3,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "tc.cuh"
@@ -29,6 +30,40 @@ float effective_scale(const mla_dims* d) {
 }
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// A second stream per device for work of a call that may overlap the rest of it, with the two events
+// that fork it from the caller's stream and join it back; the mutex keeps the record / wait pairs of
+// concurrent calls on one device from interleaving. Created on first use, kept for the process.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  std::mutex m;
+};
+
+SideStream* side_stream() {
+  static SideStream sides[64];
+  static std::mutex create;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  SideStream* x = &sides[dev];
+  std::lock_guard<std::mutex> lock(create);
+  if (!x->s) {
+    cudaStream_t st = nullptr;
+    cudaEvent_t f = nullptr, j = nullptr;
+    if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
+      (void)cudaGetLastError();
+      if (f) cudaEventDestroy(f);
+      if (st) cudaStreamDestroy(st);
+      return nullptr;
+    }
+    x->fork = f;
+    x->join = j;
+    x->s = st;
+  }
+  return x;
+}
 
 // bf16 operands of the tensor-core kernels are read with 16-byte vector or TMA accesses
 int check_align(int32_t dt, std::initializer_list<const void*> ptrs) {
@@ -446,19 +481,37 @@ int32_t mla_project_inputs(const mla_dims* dims, int32_t dtype, int32_t q_rank, 
   float* q_r = reinterpret_cast<float*>(ws + L.q_r);
   float* kv = reinterpret_cast<float*>(ws + L.kv);
   cudaStream_t s = as_stream(stream);
+  const bool rotate = (flags & MLA_APPEND_ROPE) != 0;
+  const int64_t W = dims->kv_lora_rank + dr;
   // the rotary-query product may come back as K-split partials, which the rotation adds in order
   ProjectParts parts{q_r, 1, 0};
-  if (dtype == MLA_BF16 && tc_project_supported(*dims, q_rank, n_rows))
+  if (dtype == MLA_BF16 && tc_project_supported(*dims, q_rank, n_rows)) {
+    // The KV branch (down-projection, its split-K sum, the append) does not depend on the query chain:
+    // it runs on the library's side stream of this device, forked from and joined back to the caller's
+    // stream, so that its short kernels overlap the query products.
+    SideStream* side = side_stream();
+    if (!side) return MLA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(side->m);
+    if (cudaEventRecord(side->fork, s) != cudaSuccess || cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
+      return MLA_ERR_CUDA;
     st = tc_project(*dims, q_rank, x, w_cq, w_qc, w_qr, w_dkv, n_rows, c_q, q_nope, q_r, kv, ws + L.partial, s,
-                    &parts);
-  else
-    st = project_generic(dims, dtype, q_rank, x, w_cq, w_qc, w_qr, w_dkv, n_rows, c_q, q_nope, q_r, kv, s);
+                    &parts, side->s);
+    if (!st)
+      st = append_latent_strided(*dims, dtype, cache, cache_rows, row_idx, kv, W, kv + dims->kv_lora_rank, W,
+                                 positions, n_rows, flags, eps, rope_theta, side->s);
+    if (!st && dr > 0)
+      st = rope_rows_launch(dtype, parts.qr, q_pe, positions, n_rows, dims->n_heads, (int)dr, rotate, rope_theta, s,
+                            parts.qr_parts, parts.qr_stride);
+    // join (also after an error, so that the caller's stream never runs ahead of the side stream's work)
+    if (cudaEventRecord(side->join, side->s) != cudaSuccess || cudaStreamWaitEvent(s, side->join, 0) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    return st;
+  }
+  st = project_generic(dims, dtype, q_rank, x, w_cq, w_qc, w_qr, w_dkv, n_rows, c_q, q_nope, q_r, kv, s);
   if (st) return st;
-  const bool rotate = (flags & MLA_APPEND_ROPE) != 0;
   if (dr > 0 && (st = rope_rows_launch(dtype, parts.qr, q_pe, positions, n_rows, dims->n_heads, (int)dr, rotate,
                                        rope_theta, s, parts.qr_parts, parts.qr_stride)))
     return st;
-  const int64_t W = dims->kv_lora_rank + dr;
   return append_latent_strided(*dims, dtype, cache, cache_rows, row_idx, kv, W, kv + dims->kv_lora_rank, W, positions,
                                n_rows, flags, eps, rope_theta, s);
 }

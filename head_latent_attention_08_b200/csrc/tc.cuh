@@ -34,9 +34,10 @@ struct ProjectParts {
 };
 bool tc_project_supported(const mla_dims& d, int64_t q_rank, int64_t n_rows);
 size_t tc_project_partial_bytes(const mla_dims& d, int64_t q_rank, int64_t n_rows);
+// the KV down-projection runs on s_kv (may be s), the query chain on s
 int tc_project(const mla_dims& d, int64_t q_rank, const void* x, const void* w_cq, const void* w_qc,
                const void* w_qr, const void* w_dkv, int64_t n_rows, void* c_q, void* q_nope, float* q_r,
-               float* kv, void* partial, cudaStream_t s, ProjectParts* parts);
+               float* kv, void* partial, cudaStream_t s, ProjectParts* parts, cudaStream_t s_kv);
 // attention of un-absorbed heads over whole prompts (bf16, head width 128): q, k, v, out and the
 // optional gate are [B*S, H*128]; out = softmax(scale q k^T, causal or full) v (times the gate)
 bool tc_prefill_supported(int64_t B, int64_t S, int64_t H, int64_t D);

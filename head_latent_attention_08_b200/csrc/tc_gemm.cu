@@ -910,7 +910,7 @@ size_t tc_project_partial_bytes(const mla_dims& d, int64_t q_rank, int64_t n_row
 
 int tc_project(const mla_dims& d, int64_t q_rank, const void* x, const void* w_cq, const void* w_qc,
                const void* w_qr, const void* w_dkv, int64_t n_rows, void* c_q, void* q_nope, float* q_r,
-               float* kv, void* partial, cudaStream_t s, ProjectParts* parts) {
+               float* kv, void* partial, cudaStream_t s, ProjectParts* parts, cudaStream_t s_kv) {
   int g[4][3];
   project_gemm_dims(d, q_rank, n_rows, g);
   size_t off[5];
@@ -932,9 +932,9 @@ int tc_project(const mla_dims& d, int64_t q_rank, const void* x, const void* w_c
                        (uint64_t)(n_rows * D * 2)};
   const GemmOperand bq{c_q, (uint64_t)q_rank, (uint64_t)n_rows, 1, (uint64_t)(q_rank * 2),
                        (uint64_t)(n_rows * q_rank * 2)};
-  // the KV down-projection, then the query chain (c_q feeds the last two products)
+  // the KV down-projection (on s_kv), then the query chain (c_q feeds the last two products)
   int st = tc_gemm(weight(w_dkv, g[3][0], D), false, bx, g[3][0], g[3][1], g[3][2], 1, kv, 0, g[3][0], true,
-                   nullptr, 0, 0, false, pw + off[3], s);
+                   nullptr, 0, 0, false, pw + off[3], s_kv);
   if (st) return st;
   if ((st = tc_gemm(weight(w_cq, g[0][0], D), false, bx, g[0][0], g[0][1], g[0][2], 1, c_q, 0, g[0][0], false,
                     nullptr, 0, 0, false, pw + off[0], s)))
