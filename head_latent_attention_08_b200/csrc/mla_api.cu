@@ -489,21 +489,26 @@ int32_t mla_project_inputs(const mla_dims* dims, int32_t dtype, int32_t q_rank, 
     // The KV branch (down-projection, its split-K sum, the append) does not depend on the query chain:
     // it runs on the library's side stream of this device, forked from and joined back to the caller's
     // stream, so that its short kernels overlap the query products.
+    // (Without a side stream, e.g. when none can be made, the branch runs on the caller's stream.)
     SideStream* side = side_stream();
-    if (!side) return MLA_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(side->m);
-    if (cudaEventRecord(side->fork, s) != cudaSuccess || cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
-      return MLA_ERR_CUDA;
+    std::unique_lock<std::mutex> lock;
+    cudaStream_t s_kv = s;
+    if (side) {
+      lock = std::unique_lock<std::mutex>(side->m);
+      if (cudaEventRecord(side->fork, s) != cudaSuccess || cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
+        return MLA_ERR_CUDA;
+      s_kv = side->s;
+    }
     st = tc_project(*dims, q_rank, x, w_cq, w_qc, w_qr, w_dkv, n_rows, c_q, q_nope, q_r, kv, ws + L.partial, s,
-                    &parts, side->s);
+                    &parts, s_kv);
     if (!st)
       st = append_latent_strided(*dims, dtype, cache, cache_rows, row_idx, kv, W, kv + dims->kv_lora_rank, W,
-                                 positions, n_rows, flags, eps, rope_theta, side->s);
+                                 positions, n_rows, flags, eps, rope_theta, s_kv);
     if (!st && dr > 0)
       st = rope_rows_launch(dtype, parts.qr, q_pe, positions, n_rows, dims->n_heads, (int)dr, rotate, rope_theta, s,
                             parts.qr_parts, parts.qr_stride);
     // join (also after an error, so that the caller's stream never runs ahead of the side stream's work)
-    if (cudaEventRecord(side->join, side->s) != cudaSuccess || cudaStreamWaitEvent(s, side->join, 0) != cudaSuccess)
+    if (side && (cudaEventRecord(side->join, side->s) != cudaSuccess || cudaStreamWaitEvent(s, side->join, 0) != cudaSuccess))
       return MLA_ERR_CUDA;
     return st;
   }
