@@ -633,6 +633,15 @@ def run_rows(args):
            "bf16 query split into two e4m3 parts for QK^T, P.C in f16 over the converted codes; bytes = the e4m3 "
            "cache; FLOPs counted once (the two query parts double the QK^T MMAs at twice the bf16 rate)")
     del codes, ws8
+    # ---- f3: the context-parallel merge of R partial (out_lat, lse) pairs, parts local to this GPU -------
+    for R in (2, 4):
+        parts = [rnd(B, H, dc, dtype=f32) for _ in range(R)]
+        lses = [rnd(B, H, dtype=f32) for _ in range(R)]
+        ms = timed(lambda: M.mla_lse_merge(d, parts, lses, 0, B, step.out_lat, step.lse))
+        report("f3 context-parallel merge (log-sum-exp)", c3 + f" R={R} parts", ms, 4 * (R + 1) * B * H * (dc + 1), 0,
+               "every part read once, the result written once; across GPUs the parts are peers' buffers read "
+               "over NVLink")
+        del parts, lses
     del cache, step, w_o, layer, w_qc, w_qr
     torch.cuda.empty_cache()
     # ---- C4: B16, T ~ U[1024, 32768], n_q 1 and 4 (causal) -----------------------------------------

@@ -418,6 +418,20 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ 
   const int64_t x = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);   // local row * H + h
   if (x >= n_rh) return;
   const int64_t g = row0 * H + x;                                                    // global row * H + h
+  // float4 rows of at most 512 columns: this lane's columns of the first four parts are requested
+  // before the weights are known (every part is a whole [rows, H, d_c] buffer; an empty part's values
+  // are loaded but never used), so that the weights' load and these overlap
+  const bool fast = vec4 && dc % 128 == 0 && dc <= 512;
+  const int ni = dc / 128;
+  float4 v[4][4];
+  if (fast) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        v[j][i] = j < n_parts && i < ni ? *reinterpret_cast<const float4*>(parts.o[j] + g * dc + 4 * lane + 128 * i)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   float lr = -INFINITY;
   if (lane < n_parts) lr = parts.l[lane][g];
   float m = lr;
@@ -437,7 +451,42 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ 
     if (r < n_parts) wsum += w[r];
   }
   const float inv = 1.f / wsum;
-  if (vec4) {
+  if (fast) {
+    // the lane's dc / 128 float4 columns, four parts at a time (one memory latency per four parts),
+    // added up in part order as below
+    float4 acc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r0 = 0; r0 < n_parts; r0 += 4) {
+      if (r0 > 0) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int r = r0 + j;
+          const bool use = r < n_parts && __shfl_sync(0xffffffffu, w_lane, r & 31) != 0.f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            v[j][i] = use && i < ni ? *reinterpret_cast<const float4*>(parts.o[r] + g * dc + 4 * lane + 128 * i)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = r0 + j;
+        const float wr = __shfl_sync(0xffffffffu, w_lane, r & 31);
+        if (r >= n_parts || wr == 0.f) continue;   // (an empty part's values take no part)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[i].x = fmaf(wr, v[j][i].x, acc[i].x); acc[i].y = fmaf(wr, v[j][i].y, acc[i].y);
+          acc[i].z = fmaf(wr, v[j][i].z, acc[i].z); acc[i].w = fmaf(wr, v[j][i].w, acc[i].w);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (i < ni)
+        *reinterpret_cast<float4*>(dst + 4 * lane + 128 * i) =
+            make_float4(acc[i].x * inv, acc[i].y * inv, acc[i].z * inv, acc[i].w * inv);
+  } else if (vec4) {
     for (int d = 4 * lane; d < dc; d += 128) {
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll

@@ -339,7 +339,8 @@ MLA_API int32_t mla_prefill_attention(int32_t dtype, const void* q, const void* 
  * with no visible position) take no part; if every part is -inf the row is 0 and its lse -inf.
  *   n_parts         1 .. MLA_MERGE_MAX_PARTS;
  *   out_lat_parts   HOST array of n_parts pointers, each to float [rows_total, H, d_c] (16-byte
- *                   aligned); lse_parts likewise to float [rows_total, H]. They may point into other
+ *                   aligned; a whole buffer even for a part whose slice is empty: its values may be
+ *                   read, never used); lse_parts likewise to float [rows_total, H]. They may point into other
  *                   devices' memory that this device can load from (peer access or symmetric memory):
  *                   the kernel only reads them, so the merge is also the exchange;
  *   row_begin, n_rows  the query rows merged: rows row_begin .. row_begin + n_rows of every part;

@@ -50,7 +50,7 @@ CASES = {
 }
 
 
-@pytest.mark.parametrize("world", [2, 3, 4])
+@pytest.mark.parametrize("world", [2, 3, 4, 6])
 @pytest.mark.parametrize("name", list(CASES))
 def test_context_parallel_decode(name, world):
     dtype, H, dc, dr, seqlens, n_q, causal = CASES[name]
