@@ -8,6 +8,7 @@
 //   * decode_generic_kernel + decode_combine_kernel: split-KV absorbed decode with an online
 //     softmax held per head by one warp (shuffle max/sum), and the log-sum-exp merge of splits.
 #include <math.h>
+#include <string.h>
 
 #include <atomic>
 
@@ -508,6 +509,44 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ 
     }
   }
   if (lane == 0 && lse) lse[x] = m + logf(wsum);
+}
+
+// ---------------------------------------------------------------------------------------------
+// the index arrays of a decode step from host memory, carried in one launch's parameters (a kernel
+// launch costs less than three small host-to-device copies, about 5 us each)
+// ---------------------------------------------------------------------------------------------
+constexpr int STEP_PARAM_BATCH = 240;   // keeps the parameter block under 4 KB
+struct StepIndices {
+  int32_t batch, has_pos;
+  int32_t cu[STEP_PARAM_BATCH + 1];
+  int32_t pos[STEP_PARAM_BATCH];
+  int64_t rows[STEP_PARAM_BATCH];
+};
+static_assert(sizeof(StepIndices) <= 4000, "kernel parameter block");
+
+__global__ void __launch_bounds__(256) put_step_indices_kernel(const __grid_constant__ StepIndices ix, int32_t* cu,
+                                                               int64_t* rows, int32_t* pos) {
+  griddep_wait();            // the previous step's kernels may still read these arrays
+  griddep_launch_dependents();
+  for (int i = threadIdx.x; i <= ix.batch; i += blockDim.x) cu[i] = ix.cu[i];
+  for (int i = threadIdx.x; i < ix.batch; i += blockDim.x) {
+    rows[i] = ix.rows[i];
+    if (ix.has_pos) pos[i] = ix.pos[i];
+  }
+}
+
+// MLA_ERR_UNSUPPORTED (nothing launched) above STEP_PARAM_BATCH sequences
+int put_step_indices(const int32_t* cu_h, const int64_t* rows_h, const int32_t* pos_h, int batch, int32_t* cu,
+                     int64_t* rows, int32_t* pos, cudaStream_t s) {
+  if (batch < 0 || batch > STEP_PARAM_BATCH) return MLA_ERR_UNSUPPORTED;
+  StepIndices ix;
+  memset(&ix, 0, sizeof(ix));
+  ix.batch = batch;
+  ix.has_pos = pos_h ? 1 : 0;
+  memcpy(ix.cu, cu_h, (size_t)(batch + 1) * sizeof(int32_t));
+  memcpy(ix.rows, rows_h, (size_t)batch * sizeof(int64_t));
+  if (pos_h) memcpy(ix.pos, pos_h, (size_t)batch * sizeof(int32_t));
+  return launch_pdl(put_step_indices_kernel, dim3(1), dim3(256), 0, s, ix, cu, rows, pos);
 }
 
 int lse_merge_launch(int n_parts, const float* const* o_parts, const float* const* l_parts, int64_t row0,

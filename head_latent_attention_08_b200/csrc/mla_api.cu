@@ -8,6 +8,13 @@
 #include "common.cuh"
 #include "tc.cuh"
 
+namespace mla {
+// generic.cu: the step's index arrays written into the workspace by one kernel whose launch parameters
+// carry them (MLA_ERR_UNSUPPORTED, nothing launched, for more sequences than that kernel takes)
+int put_step_indices(const int32_t* cu_h, const int64_t* rows_h, const int32_t* pos_h, int batch, int32_t* cu,
+                     int64_t* rows, int32_t* pos, cudaStream_t s);
+}  // namespace mla
+
 using namespace mla;
 
 namespace {
@@ -598,14 +605,23 @@ int32_t mla_decode_step(const mla_dims* dims, int32_t dtype, int32_t q_rank, con
     // are asynchronous and the call returns once everything is enqueued on `stream`
     const bool need_pos = (append_flags & MLA_APPEND_ROPE) && dims->rope_dim > 0;
     if (need_pos && !positions) return MLA_ERR_NULL;
-    if (cudaMemcpyAsync(ws + L.x_in, x, x_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(ws + L.cu, cu_seqlens, (size_t)(batch + 1) * sizeof(int32_t), cudaMemcpyHostToDevice,
-                        s) != cudaSuccess ||
-        cudaMemcpyAsync(ws + L.rows, row_idx, (size_t)batch * sizeof(int64_t), cudaMemcpyHostToDevice, s) !=
-            cudaSuccess ||
-        (need_pos && cudaMemcpyAsync(ws + L.pos, positions, (size_t)batch * sizeof(int32_t),
-                                     cudaMemcpyHostToDevice, s) != cudaSuccess))
-      return MLA_ERR_CUDA;
+    if (cudaMemcpyAsync(ws + L.x_in, x, x_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return MLA_ERR_CUDA;
+    // the small index arrays travel in one kernel's launch parameters (read now); beyond that kernel's
+    // capacity, by copies of their own
+    st = put_step_indices(cu_seqlens, row_idx, need_pos ? positions : nullptr, batch,
+                          reinterpret_cast<int32_t*>(ws + L.cu), reinterpret_cast<int64_t*>(ws + L.rows),
+                          reinterpret_cast<int32_t*>(ws + L.pos), s);
+    if (st == MLA_ERR_UNSUPPORTED) {
+      if (cudaMemcpyAsync(ws + L.cu, cu_seqlens, (size_t)(batch + 1) * sizeof(int32_t), cudaMemcpyHostToDevice,
+                          s) != cudaSuccess ||
+          cudaMemcpyAsync(ws + L.rows, row_idx, (size_t)batch * sizeof(int64_t), cudaMemcpyHostToDevice, s) !=
+              cudaSuccess ||
+          (need_pos && cudaMemcpyAsync(ws + L.pos, positions, (size_t)batch * sizeof(int32_t),
+                                       cudaMemcpyHostToDevice, s) != cudaSuccess))
+        return MLA_ERR_CUDA;
+    } else if (st) {
+      return st;
+    }
     x = ws + L.x_in;
     cu_seqlens = reinterpret_cast<const int32_t*>(ws + L.cu);
     row_idx = reinterpret_cast<const int64_t*>(ws + L.rows);

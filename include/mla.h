@@ -294,11 +294,12 @@ MLA_API int32_t mla_decode_step_workspace_size(const mla_dims* dims, int32_t dty
  *   cu_seqlens int32 [batch + 1], row_idx int64 [batch], positions int32 [batch] (read with
  *   MLA_APPEND_ROPE), append_flags / eps / rope_theta as mla_append_latent.
  *   io = MLA_IO_DEVICE: every pointer is device memory.
- *   io = MLA_IO_HOST: x, y, cu_seqlens, row_idx and positions are HOST memory; the call copies the
- *   inputs into the workspace and y back with cudaMemcpyAsync on `stream`. With page-locked host
- *   memory it returns once all is enqueued: the host buffers must then stay untouched until the
- *   stream has passed this step (y holds the result after a synchronisation). The weights and the
- *   cache are device memory in both modes.
+ *   io = MLA_IO_HOST: x, y, cu_seqlens, row_idx and positions are HOST memory. The call copies x
+ *   into the workspace and y back with cudaMemcpyAsync on `stream`. The index arrays are read when
+ *   the call is made, and passed on in a kernel's launch parameters (up to 240 sequences; beyond
+ *   that they are copied like x). With page-locked host memory the call returns once all is
+ *   enqueued: x and y must then stay untouched until the stream has passed this step (y holds the
+ *   result after a synchronisation). The weights and the cache are device memory in both modes.
  * Errors: those of the four stages, checked before the first launch where they concern sizes;
  * MLA_ERR_MODE for an unknown io; MLA_ERR_CUDA when a copy cannot be enqueued.
  */

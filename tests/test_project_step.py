@@ -194,6 +194,16 @@ def test_decode_step_host_io_equals_device_io():
     np.testing.assert_array_equal(cache_host, cache_dev)
 
 
+def test_decode_step_host_io_many_sequences():
+    # 250 sequences: more than the index arrays' launch-parameter route takes, so they are copied
+    rng = np.random.default_rng(64)
+    s = Step("bf16", 128, 512, 64, 128, 128, 256, 256, [int(t) for t in rng.integers(1, 40, 250)], 63)
+    y_dev, cache_dev = s.run(M.MLA_IO_DEVICE)
+    y_host, cache_host = s.run(M.MLA_IO_HOST)
+    np.testing.assert_array_equal(y_host, y_dev)
+    np.testing.assert_array_equal(cache_host, cache_dev)
+
+
 def test_decode_step_deepseek_scale_sampled():
     # the benchmark's workload: 64 sequences of 4096 positions, d_model 5120, q_rank 1536; four
     # sequences computed by the oracle
