@@ -405,6 +405,8 @@ int rope_rows_launch(int32_t dtype, const float* src, void* out, const int32_t* 
 // One warp per (row, head); sums run over r in index order, so the result does not depend on timing.
 // The parts may live in other devices' memory (peer pointers): the kernel only loads from them.
 // ---------------------------------------------------------------------------------------------
+constexpr int MERGE_GROUP = 2;   // parts whose columns one lane loads at once (64 registers: four blocks per SM)
+
 struct MergeParts {
   const float* o[MLA_MERGE_MAX_PARTS];
   const float* l[MLA_MERGE_MAX_PARTS];
@@ -419,15 +421,15 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ 
   const int64_t x = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);   // local row * H + h
   if (x >= n_rh) return;
   const int64_t g = row0 * H + x;                                                    // global row * H + h
-  // float4 rows of at most 512 columns: this lane's columns of the first four parts are requested
+  // float4 rows of at most 512 columns: this lane's columns of the first MERGE_GROUP parts are requested
   // before the weights are known (every part is a whole [rows, H, d_c] buffer; an empty part's values
   // are loaded but never used), so that the weights' load and these overlap
   const bool fast = vec4 && dc % 128 == 0 && dc <= 512;
   const int ni = dc / 128;
-  float4 v[4][4];
+  float4 v[MERGE_GROUP][4];
   if (fast) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < MERGE_GROUP; ++j)
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         v[j][i] = j < n_parts && i < ni ? *reinterpret_cast<const float4*>(parts.o[j] + g * dc + 4 * lane + 128 * i)
@@ -453,15 +455,15 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ 
   }
   const float inv = 1.f / wsum;
   if (fast) {
-    // the lane's dc / 128 float4 columns, four parts at a time (one memory latency per four parts),
+    // the lane's dc / 128 float4 columns, MERGE_GROUP parts at a time (one memory latency per group),
     // added up in part order as below
     float4 acc[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int r0 = 0; r0 < n_parts; r0 += 4) {
+    for (int r0 = 0; r0 < n_parts; r0 += MERGE_GROUP) {
       if (r0 > 0) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < MERGE_GROUP; ++j) {
           const int r = r0 + j;
           const bool use = r < n_parts && __shfl_sync(0xffffffffu, w_lane, r & 31) != 0.f;
 #pragma unroll
@@ -471,7 +473,7 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const __grid_constant__ 
         }
       }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < MERGE_GROUP; ++j) {
         const int r = r0 + j;
         const float wr = __shfl_sync(0xffffffffu, w_lane, r & 31);
         if (r >= n_parts || wr == 0.f) continue;   // (an empty part's values take no part)
