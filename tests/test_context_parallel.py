@@ -47,6 +47,12 @@ CASES = {
     "bf16_nq4": ("bf16", 128, 512, 64, [4, 70, 517, 900], 4, True),
     # CUDA-core decode, non-causal multi-query
     "f32_nq3": ("f32", 16, 128, 32, [5, 64, 65, 200], 3, False),
+    # latent widths the merge takes by its other routes: float4 columns not a multiple of 128, and more
+    # than 512 columns
+    "f32_dc96": ("f32", 8, 96, 16, [5, 40, 90], 2, True),
+    "f32_dc1024": ("f32", 4, 1024, 16, [7, 33, 60], 1, False),
+    # rows that are not a whole number of 16-byte chunks: the element-wise route
+    "f32_dc42": ("f32", 4, 42, 16, [5, 40, 61], 1, True),
 }
 
 
@@ -100,3 +106,7 @@ def test_merge_rejects_bad_arguments():
         M.mla_lse_merge(d, [o] * 17, [l] * 17, 0, 2, o.clone(), l.clone())
     with pytest.raises(M.MLAError):
         M.mla_lse_merge(d, [], [], 0, 2, o.clone(), l.clone())
+    # a part that does not start on a 16-byte boundary
+    shifted = torch.zeros(o.numel() + 1, device="cuda")[1:].view_as(o)
+    with pytest.raises(M.MLAError):
+        M.mla_lse_merge(d, [o, shifted], [l, l], 0, 2, o.clone(), l.clone())

@@ -194,10 +194,11 @@ def test_decode_step_host_io_equals_device_io():
     np.testing.assert_array_equal(cache_host, cache_dev)
 
 
-def test_decode_step_host_io_many_sequences():
-    # 250 sequences: more than the index arrays' launch-parameter route takes, so they are copied
+@pytest.mark.parametrize("n_seq", [240, 241])
+def test_decode_step_host_io_many_sequences(n_seq):
+    # 240 sequences: the most the index arrays' launch-parameter route takes; 241: they are copied
     rng = np.random.default_rng(64)
-    s = Step("bf16", 128, 512, 64, 128, 128, 256, 256, [int(t) for t in rng.integers(1, 40, 250)], 63)
+    s = Step("bf16", 128, 512, 64, 128, 128, 256, 256, [int(t) for t in rng.integers(1, 40, n_seq)], 63)
     y_dev, cache_dev = s.run(M.MLA_IO_DEVICE)
     y_host, cache_host = s.run(M.MLA_IO_HOST)
     np.testing.assert_array_equal(y_host, y_dev)
