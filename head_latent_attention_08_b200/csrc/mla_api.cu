@@ -607,10 +607,15 @@ int32_t mla_decode_step(const mla_dims* dims, int32_t dtype, int32_t q_rank, con
     if (need_pos && !positions) return MLA_ERR_NULL;
     if (cudaMemcpyAsync(ws + L.x_in, x, x_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return MLA_ERR_CUDA;
     // the small index arrays travel in one kernel's launch parameters (read now); beyond that kernel's
-    // capacity, by copies of their own
-    st = put_step_indices(cu_seqlens, row_idx, need_pos ? positions : nullptr, batch,
-                          reinterpret_cast<int32_t*>(ws + L.cu), reinterpret_cast<int64_t*>(ws + L.rows),
-                          reinterpret_cast<int32_t*>(ws + L.pos), s);
+    // capacity, or while the stream is being captured into a graph (whose replays must read the host
+    // buffers again, as a captured copy does), by copies of their own
+    cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &capture) != cudaSuccess) return MLA_ERR_CUDA;
+    st = capture != cudaStreamCaptureStatusNone
+             ? MLA_ERR_UNSUPPORTED
+             : put_step_indices(cu_seqlens, row_idx, need_pos ? positions : nullptr, batch,
+                                reinterpret_cast<int32_t*>(ws + L.cu), reinterpret_cast<int64_t*>(ws + L.rows),
+                                reinterpret_cast<int32_t*>(ws + L.pos), s);
     if (st == MLA_ERR_UNSUPPORTED) {
       if (cudaMemcpyAsync(ws + L.cu, cu_seqlens, (size_t)(batch + 1) * sizeof(int32_t), cudaMemcpyHostToDevice,
                           s) != cudaSuccess ||

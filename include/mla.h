@@ -297,7 +297,8 @@ MLA_API int32_t mla_decode_step_workspace_size(const mla_dims* dims, int32_t dty
  *   io = MLA_IO_HOST: x, y, cu_seqlens, row_idx and positions are HOST memory. The call copies x
  *   into the workspace and y back with cudaMemcpyAsync on `stream`. The index arrays are read when
  *   the call is made, and passed on in a kernel's launch parameters (up to 240 sequences; beyond
- *   that they are copied like x). With page-locked host memory the call returns once all is
+ *   that, or while `stream` is being captured into a CUDA graph, they are copied like x, so that a
+ *   graph's replays read them again). With page-locked host memory the call returns once all is
  *   enqueued: x and y must then stay untouched until the stream has passed this step (y holds the
  *   result after a synchronisation). The weights and the cache are device memory in both modes.
  * Errors: those of the four stages, checked before the first launch where they concern sizes;

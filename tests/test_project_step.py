@@ -194,6 +194,40 @@ def test_decode_step_host_io_equals_device_io():
     np.testing.assert_array_equal(cache_host, cache_dev)
 
 
+def test_decode_step_host_io_captured_in_a_cuda_graph():
+    # the whole step from host buffers, captured once and replayed: a replay reads x, the index arrays
+    # and writes y as they are at replay time, like a direct call with the same buffers
+    s = Step(*STEP_CASES["bf16_tc"])
+    layer = s.layer()
+    p, dt = s.p, s.dtype
+    x_h = torch.from_numpy(s.w.x).to(TORCH_DT[dt]).pin_memory()
+    rows_h = torch.from_numpy(p.row_idx).pin_memory()
+    pos_h = torch.from_numpy(p.positions).pin_memory()
+    y_h = torch.empty(p.batch, p.d_model, dtype=TORCH_DT[dt]).pin_memory()
+    layer(x_h, rows_h, pos_h, y=y_h, io=M.MLA_IO_HOST)       # first call: one-time set-up outside capture
+    torch.cuda.synchronize()
+    y_first = y_h.clone()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    with torch.cuda.graph(g, stream=side):
+        layer(x_h, rows_h, pos_h, y=y_h, io=M.MLA_IO_HOST)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y_h, y_first)
+    # new inputs in the same host buffers: the replay must see them
+    x_h.copy_(torch.from_numpy(s.w.x[::-1].copy()).to(TORCH_DT[dt]))
+    pos_h.add_(3)
+    g.replay()
+    torch.cuda.synchronize()
+    y_replay = y_h.clone()
+    assert not torch.equal(y_replay, y_first)
+    layer(x_h, rows_h, pos_h, y=y_h, io=M.MLA_IO_HOST)
+    torch.cuda.synchronize()
+    assert M.mla_check_status() == M.MLA_OK
+    assert torch.equal(y_replay, y_h)
+    del g
+
+
 @pytest.mark.parametrize("n_seq", [240, 241])
 def test_decode_step_host_io_many_sequences(n_seq):
     # 240 sequences: the most the index arrays' launch-parameter route takes; 241: they are copied
