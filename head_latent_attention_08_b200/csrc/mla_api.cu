@@ -511,12 +511,15 @@ int32_t mla_project_inputs(const mla_dims* dims, int32_t dtype, int32_t q_rank, 
     if (!st)
       st = append_latent_strided(*dims, dtype, cache, cache_rows, row_idx, kv, W, kv + dims->kv_lora_rank, W,
                                  positions, n_rows, flags, eps, rope_theta, s_kv);
+    // join (also after an error, so that the caller's stream never runs ahead of the side stream's work),
+    // before the rotation: a wait between two kernels ends their programmatic overlap, and the rotation
+    // gains less from it than the caller's next kernel (which prefetches its weights during the
+    // rotation's tail)
+    if (side && (cudaEventRecord(side->join, side->s) != cudaSuccess || cudaStreamWaitEvent(s, side->join, 0) != cudaSuccess))
+      return MLA_ERR_CUDA;
     if (!st && dr > 0)
       st = rope_rows_launch(dtype, parts.qr, q_pe, positions, n_rows, dims->n_heads, (int)dr, rotate, rope_theta, s,
                             parts.qr_parts, parts.qr_stride);
-    // join (also after an error, so that the caller's stream never runs ahead of the side stream's work)
-    if (side && (cudaEventRecord(side->join, side->s) != cudaSuccess || cudaStreamWaitEvent(s, side->join, 0) != cudaSuccess))
-      return MLA_ERR_CUDA;
     return st;
   }
   st = project_generic(dims, dtype, q_rank, x, w_cq, w_qc, w_qr, w_dkv, n_rows, c_q, q_nope, q_r, kv, s);
