@@ -323,6 +323,23 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const float* __restrict_
   griddep_wait();
   griddep_launch_dependents();
   const int t = blockIdx.x, half = dr / 2, pairs = H * half;
+  const float2* row = reinterpret_cast<const float2*>(src + (int64_t)t * H * dr);
+  T* o = out + (int64_t)t * H * dr;
+  const int e0 = blockIdx.y * ROPE_PAIRS_PER_CTA + threadIdx.x * 4;
+  // the source values are requested before the angles are formed (the two do not depend on each other)
+  const bool vfast = vec && e0 + 3 < pairs;
+  float4 u0 = make_float4(0.f, 0.f, 0.f, 0.f), u1 = u0;
+  if (vfast) {
+    // the source: one array, or the K-split partials of the projection that made it, added in order
+    u0 = reinterpret_cast<const float4*>(row + e0)[0];
+    u1 = reinterpret_cast<const float4*>(row + e0)[1];
+    for (int q = 1; q < n_parts; ++q) {
+      const float4* part = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(row + e0) + q * part_stride);
+      const float4 a = part[0], b = part[1];
+      u0.x += a.x; u0.y += a.y; u0.z += a.z; u0.w += a.w;
+      u1.x += b.x; u1.y += b.y; u1.z += b.z; u1.w += b.w;
+    }
+  }
   if (rotate) {
     const int32_t pos = positions[t];
     for (int i = threadIdx.x; i < half; i += blockDim.x) {
@@ -332,24 +349,12 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const float* __restrict_
     }
     __syncthreads();
   }
-  const float2* row = reinterpret_cast<const float2*>(src + (int64_t)t * H * dr);
-  T* o = out + (int64_t)t * H * dr;
-  const int e0 = blockIdx.y * ROPE_PAIRS_PER_CTA + threadIdx.x * 4;
   auto turn = [&](float2 v, int e) {
     if (!rotate) return v;
     const float2 a = sc[e % half];
     return make_float2(fmaf(v.x, a.y, -v.y * a.x), fmaf(v.x, a.x, v.y * a.y));
   };
-  if (vec && e0 + 3 < pairs) {
-    // the source: one array, or the K-split partials of the projection that made it, added in order
-    float4 u0 = reinterpret_cast<const float4*>(row + e0)[0];
-    float4 u1 = reinterpret_cast<const float4*>(row + e0)[1];
-    for (int q = 1; q < n_parts; ++q) {
-      const float4* part = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(row + e0) + q * part_stride);
-      const float4 a = part[0], b = part[1];
-      u0.x += a.x; u0.y += a.y; u0.z += a.z; u0.w += a.w;
-      u1.x += b.x; u1.y += b.y; u1.z += b.z; u1.w += b.w;
-    }
+  if (vfast) {
     const float2 r0 = turn(make_float2(u0.x, u0.y), e0), r1 = turn(make_float2(u0.z, u0.w), e0 + 1);
     const float2 r2 = turn(make_float2(u1.x, u1.y), e0 + 2), r3 = turn(make_float2(u1.z, u1.w), e0 + 3);
     if constexpr (sizeof(T) == 2) {
